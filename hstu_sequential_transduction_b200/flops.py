@@ -1,0 +1,51 @@
+"""Algorithmic FLOP and byte accounting for the HSTU hot path.
+
+Follows "DLRMv4 Brings Sequence-Based Recommendation Training to MLPerf",
+section "Computation Cost Analysis" (Tables 6 and 7): the attention forward
+is two GEMM-shaped contractions (Q K^T and P V), the backward roughly five,
+and only the visible (lower-triangle) pairs are counted.  Bias gathers, SiLU
+and the mask are not counted.  Weight GEMMs cost 2*m*n*k per pass.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def attn_pairs_per_seq(L: int, n_t: int = 0) -> int:
+    """Visible (query, key) pairs of one sequence: history rows see j <= i,
+    each candidate row sees the whole history and itself."""
+    L, n_t = int(L), int(n_t)
+    hist = L - n_t
+    return hist * (hist + 1) // 2 + n_t * (hist + 1)
+
+
+def attn_pairs(lengths, num_targets=None) -> int:
+    lengths = np.asarray(lengths, dtype=np.int64)
+    if num_targets is None:
+        nts = np.zeros_like(lengths)
+    else:
+        nts = np.asarray(num_targets, dtype=np.int64)
+    return int(sum(attn_pairs_per_seq(L, n) for L, n in zip(lengths, nts)))
+
+
+def attn_fwd_flops(pairs: float, num_heads: int, d_qk: int, d_v: int) -> float:
+    return 2.0 * (d_qk + d_v) * pairs * num_heads
+
+
+def attn_bwd_flops(pairs: float, num_heads: int, d_qk: int, d_v: int) -> float:
+    # recompute S (d_qk), dP = dO V^T (d_v), dV = P^T dO (d_v), dQ, dK (d_qk each)
+    return 2.0 * (3 * d_qk + 2 * d_v) * pairs * num_heads
+
+
+def f1_flops(tokens: int, d_model: int, num_heads: int, d_qk: int, d_v: int) -> float:
+    return 2.0 * tokens * d_model * num_heads * (2 * d_qk + 2 * d_v)
+
+
+def f2_flops(tokens: int, d_model: int, num_heads: int, d_v: int, width_factor: int = 1) -> float:
+    return 2.0 * tokens * width_factor * num_heads * d_v * d_model
+
+
+def gate_bytes(tokens: int, num_heads: int, d_v: int, elem_bytes: int = 2) -> float:
+    """LayerNorm(O) * U: read O and U, write G (one pass each)."""
+    return 3.0 * tokens * num_heads * d_v * elem_bytes

@@ -1,0 +1,233 @@
+"""CPU oracle for HSTU jagged attention and the transduction layer (fp64).
+
+TEST INFRASTRUCTURE ONLY.  The library and its binding never import this
+package; only `tests/`, the smoke check in `__graft_entry__` and the CPU
+baseline leg of `bench.py` may.  It shares no code with the CUDA path.
+
+The arithmetic lives in `hstu_oracle.c` (plain loops, double accumulation);
+this module builds it with gcc when needed and marshals numpy arrays.
+Inputs in bf16 are widened exactly to float64 before the call.
+
+Pins (tests/test_oracle_pins.py): a hand-worked three-token example, a dense
+brute-force formulation, torch float64 autograd, central finite differences,
+causality / independence / linearity invariants, the exhaustive bucket check
+and the cost formulas of the DLRMv4 page's Table 7.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hstu_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_f64p = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP) into oracle/liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11",
+                               _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_time_bucket.restype = ctypes.c_int
+            lib.oracle_time_bucket.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+            lib.oracle_pos_index.restype = ctypes.c_int
+            lib.oracle_pos_index.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+            lib.oracle_visible.restype = ctypes.c_int
+            lib.oracle_visible.argtypes = [ctypes.c_int64] * 4
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return int(os.environ.get("HSTU_ORACLE_THREADS", os.cpu_count() or 1))
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor (any float dtype): widen exactly
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i64(a):
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def _i32_or_none(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _p(a, kind):
+    if a is None:
+        return ctypes.cast(None, kind)
+    return a.ctypes.data_as(kind)
+
+
+def time_bucket(t_i: int, t_j: int, num_buckets: int) -> int:
+    return _load().oracle_time_bucket(int(t_i), int(t_j), int(num_buckets))
+
+
+def pos_index(p_i: int, p_j: int, pos_lo: int, pos_hi: int) -> int:
+    return _load().oracle_pos_index(int(p_i), int(p_j), int(pos_lo), int(pos_hi))
+
+
+def visible(i: int, j: int, L: int, n_t: int) -> bool:
+    return bool(_load().oracle_visible(int(i), int(j), int(L), int(n_t)))
+
+
+class _Attn:
+    """Marshalled common attention arguments."""
+
+    def __init__(self, seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time,
+                 pos_lo, pos_hi, inv_n):
+        self.off = _i64(seq_offsets)
+        self.ts = _i64(timestamps)
+        self.nt = _i32_or_none(num_targets)
+        self.B = len(self.off) - 1
+        self.T = int(self.off[-1]) if self.B >= 0 else 0
+        self.q, self.k, self.v = _f64(q), _f64(k), _f64(v)
+        self.H = self.q.shape[1]
+        self.dqk = self.q.shape[2]
+        self.dv = self.v.shape[2]
+        self.rp, self.rt = _f64(rab_pos), _f64(rab_time)
+        self.lo, self.hi = int(pos_lo), int(pos_hi)
+        assert len(self.rp) == self.hi - self.lo + 1
+        self.nb = len(self.rt)
+        self.inv_n = float(inv_n)
+
+    def head(self):
+        return [ctypes.c_int(self.B), _p(self.off, _i64p), _p(self.nt, _i32p), ctypes.c_int(self.H),
+                ctypes.c_int(self.dqk), ctypes.c_int(self.dv), _p(self.q, _f64p), _p(self.k, _f64p),
+                _p(self.v, _f64p), _p(self.ts, _i64p), _p(self.rp, _f64p), ctypes.c_int(self.lo),
+                ctypes.c_int(self.hi), _p(self.rt, _f64p), ctypes.c_int(self.nb),
+                ctypes.c_double(self.inv_n)]
+
+
+def attn_fwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
+             inv_n, threads=None):
+    """O[T, H, dv] of the jagged SiLU attention (float64)."""
+    a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
+    out = np.zeros((a.T, a.H, a.dv), dtype=np.float64)
+    _load().oracle_attn_fwd(*a.head(), _p(out, _f64p), ctypes.c_int(threads or default_threads()))
+    return out
+
+
+def attn_fwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
+                  pos_hi, inv_n, rows, threads=None):
+    """O rows for the given global token indices: [n, H, dv]."""
+    a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
+    rows = _i64(rows)
+    out = np.zeros((len(rows), a.H, a.dv), dtype=np.float64)
+    _load().oracle_attn_fwd_rows(*a.head(), ctypes.c_int64(len(rows)), _p(rows, _i64p),
+                                 _p(out, _f64p), ctypes.c_int(threads or default_threads()))
+    return out
+
+
+def attn_bwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
+             inv_n, dout, threads=None):
+    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
+    a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
+    do = _f64(dout)
+    dq = np.zeros_like(a.q)
+    dk = np.zeros_like(a.k)
+    dv = np.zeros_like(a.v)
+    drp = np.zeros_like(a.rp)
+    drt = np.zeros_like(a.rt)
+    _load().oracle_attn_bwd(*a.head(), _p(do, _f64p), _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p),
+                            _p(drp, _f64p), _p(drt, _f64p), ctypes.c_int(threads or default_threads()))
+    return dq, dk, dv, drp, drt
+
+
+def attn_bwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
+                  pos_hi, inv_n, dout, q_rows, k_rows, threads=None):
+    """dq for query rows `q_rows`; dk, dv for key rows `k_rows`."""
+    a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
+    do = _f64(dout)
+    qr, kr = _i64(q_rows), _i64(k_rows)
+    dq = np.zeros((len(qr), a.H, a.dqk))
+    dk = np.zeros((len(kr), a.H, a.dqk))
+    dv = np.zeros((len(kr), a.H, a.dv))
+    _load().oracle_attn_bwd_rows(*a.head(), _p(do, _f64p), ctypes.c_int64(len(qr)), _p(qr, _i64p),
+                                 _p(dq, _f64p), ctypes.c_int64(len(kr)), _p(kr, _i64p),
+                                 _p(dk, _f64p), _p(dv, _f64p),
+                                 ctypes.c_int(threads or default_threads()))
+    return dq, dk, dv
+
+
+def linear(x, w, bias=None, apply_silu=False, threads=None):
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    T, m = x.shape
+    n = w.shape[1]
+    out = np.zeros((T, n))
+    _load().oracle_linear(ctypes.c_int64(T), ctypes.c_int(m), ctypes.c_int(n), _p(x, _f64p),
+                          _p(w, _f64p), _p(bias, _f64p), ctypes.c_int(int(apply_silu)),
+                          _p(out, _f64p), ctypes.c_int(threads or default_threads()))
+    return out
+
+
+def norm_gate(o, u, gamma, beta, eps=1e-5, threads=None):
+    o, u, gamma, beta = _f64(o), _f64(u), _f64(gamma), _f64(beta)
+    T, F = o.shape
+    g = np.zeros((T, F))
+    _load().oracle_norm_gate(ctypes.c_int64(T), ctypes.c_int(F), _p(o, _f64p), _p(u, _f64p),
+                             _p(gamma, _f64p), _p(beta, _f64p), ctypes.c_double(eps), _p(g, _f64p),
+                             ctypes.c_int(threads or default_threads()))
+    return g
+
+
+def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma, ln_beta,
+              rab_pos, rab_time, pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, ln_eps=1e-5,
+              threads=None, want_intermediates=False):
+    """Y[T, D] of one transduction layer (and optionally uvqk, O)."""
+    off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
+    x, w1, b1, w2, b2 = _f64(x), _f64(w1), _f64(b1), _f64(w2), _f64(b2)
+    g, be, rp, rt = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time)
+    T, D = x.shape
+    W = num_heads * (2 * d_v + 2 * d_qk)
+    y = np.zeros((T, D))
+    uvqk = np.zeros((T, W)) if want_intermediates else None
+    o = np.zeros((T, num_heads * d_v)) if want_intermediates else None
+    _load().oracle_layer_fwd(
+        ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
+        ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
+        _p(b1, _f64p), _p(w2, _f64p), _p(b2, _f64p), _p(g, _f64p), _p(be, _f64p),
+        ctypes.c_double(ln_eps), _p(ts, _i64p), _p(rp, _f64p), ctypes.c_int(int(pos_lo)),
+        ctypes.c_int(int(pos_hi)), _p(rt, _f64p), ctypes.c_int(len(rt)), ctypes.c_double(inv_n),
+        _p(y, _f64p), _p(uvqk, _f64p), _p(o, _f64p), ctypes.c_int(threads or default_threads()))
+    if want_intermediates:
+        return y, uvqk, o
+    return y
+
+
+def attn_inputs_fwd(inp, threads=None):
+    """Oracle forward over a `workloads.AttnInputs`-like object."""
+    return attn_fwd(inp.seq_offsets, inp.timestamps, inp.num_targets, inp.q, inp.k, inp.v,
+                    inp.rab_pos, inp.rab_time, inp.pos_lo, inp.pos_hi, inp.inv_n, threads)

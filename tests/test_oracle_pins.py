@@ -1,0 +1,466 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test states what fixes the expected value: the hand-worked example in
+tests/golden (derived from the definition on the "HSTU Architecture" and
+"Model Architecture" sections), a dense formulation written independently
+with numpy, torch float64 autograd, central finite differences, invariants,
+exhaustive integer checks and the DLRMv4 page's Table 7 cost formulas.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hstu_sequential_transduction_b200 import flops
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _parse_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line or "=" not in line:
+                continue
+            key, val = [s.strip() for s in line.split("=", 1)]
+            vals[key] = [float(x) for x in val.split()]
+    return vals
+
+
+# ---- independent dense formulation (numpy) ---------------------------------
+
+def dense_bias_and_mask(L, n_t, t, lo, hi, rab_pos, rab_time):
+    hist = L - n_t
+    idx = np.arange(L)
+    p = np.where(idx < hist, idx, hist)
+    rel = np.clip(p[:, None] - p[None, :], lo, hi) - lo
+    nb = len(rab_time)
+    dt = np.maximum(t[:, None].astype(object) - t[None, :].astype(object), 0)
+    bkt = np.vectorize(lambda x: min(nb - 1, (int(x) + 1).bit_length() - 1), otypes=[np.int64])(dt)
+    bias = np.asarray(rab_pos)[rel] + np.asarray(rab_time)[bkt]
+    I, J = idx[:, None], idx[None, :]
+    vis = np.where(I < hist, J <= I, (J < hist) | (J == I))
+    return bias, vis
+
+
+def dense_fwd(off, ts, nt, q, k, v, rab_pos, rab_time, lo, hi, inv_n):
+    T, H, dv = v.shape
+    out = np.zeros((T, H, dv))
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        bias, vis = dense_bias_and_mask(L, n_t, ts[s0:s1], lo, hi, rab_pos, rab_time)
+        S = np.einsum("ihc,jhc->hij", q[s0:s1], k[s0:s1]) + bias[None]
+        P = S / (1.0 + np.exp(-S)) * inv_n * vis[None]
+        out[s0:s1] = np.einsum("hij,jhc->ihc", P, v[s0:s1])
+    return out
+
+
+def rand_case(rng, lengths, H=2, dqk=3, dv=2, nt=None, lo=-3, hi=4, nb=5, gap=3.0, inv_n=0.5):
+    lengths = np.asarray(lengths)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(off[-1])
+    ts = []
+    for b, L in enumerate(lengths):
+        ts.append(np.cumsum(rng.integers(0, int(2 * gap) + 1, size=L)))
+    ts = np.concatenate(ts).astype(np.int64) if T else np.zeros(0, np.int64)
+    q = rng.standard_normal((T, H, dqk))
+    k = rng.standard_normal((T, H, dqk))
+    v = rng.standard_normal((T, H, dv))
+    rp = rng.standard_normal(hi - lo + 1) * 0.3
+    rt = rng.standard_normal(nb) * 0.3
+    nta = None if nt is None else np.asarray(nt, dtype=np.int32)
+    return dict(seq_offsets=off, timestamps=ts, num_targets=nta, q=q, k=k, v=v, rab_pos=rp,
+                rab_time=rt, pos_lo=lo, pos_hi=hi, inv_n=inv_n)
+
+
+def ofwd(c, **kw):
+    d = dict(c)
+    d.update(kw)
+    return oracle.attn_fwd(d["seq_offsets"], d["timestamps"], d["num_targets"], d["q"], d["k"],
+                           d["v"], d["rab_pos"], d["rab_time"], d["pos_lo"], d["pos_hi"], d["inv_n"])
+
+
+def dfwd(c):
+    return dense_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                     c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+
+
+# ---- 1. hand-worked example -------------------------------------------------
+
+def test_hand_worked_three_tokens():
+    g = _parse_golden("hand_3token.txt")
+    q = np.array(g["q"]).reshape(3, 1, 1)
+    k = np.array(g["k"]).reshape(3, 1, 1)
+    v = np.array(g["v"]).reshape(3, 1, 1)
+    t = np.array(g["t"], dtype=np.int64)
+    out = oracle.attn_fwd([0, 3], t, None, q, k, v, g["rab_pos"], g["rab_time"],
+                          int(g["pos_lo"][0]), int(g["pos_hi"][0]), 1.0 / g["N"][0])
+    np.testing.assert_allclose(out.reshape(3), g["O"], rtol=0, atol=g["tolerance"][0])
+
+
+def test_hand_worked_buckets():
+    # the example's buckets: dt = 0, 3, 7, 10 -> 0, 2, 3, 3 (capped at 3)
+    assert [oracle.time_bucket(dt, 0, 4) for dt in (0, 3, 7, 10)] == [0, 2, 3, 3]
+
+
+# ---- 2. brute force: dense formulation --------------------------------------
+
+@pytest.mark.parametrize("seed", range(6))
+def test_loops_match_dense(seed):
+    rng = np.random.default_rng(seed)
+    lengths = rng.integers(0, 9, size=4)
+    nt = None
+    if seed % 2:
+        nt = [int(rng.integers(0, L + 1)) for L in lengths]
+    c = rand_case(rng, lengths, nt=nt, lo=-2 - seed, hi=3, nb=3 + seed)
+    np.testing.assert_allclose(ofwd(c), dfwd(c), rtol=0, atol=1e-12)
+
+
+def test_rows_variant_matches_full():
+    rng = np.random.default_rng(7)
+    c = rand_case(rng, [5, 0, 7, 3], nt=[1, 0, 2, 0])
+    full = ofwd(c)
+    rows = np.array([0, 4, 5, 9, 11, 14])
+    part = oracle.attn_fwd_rows(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"],
+                                c["v"], c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"],
+                                c["inv_n"], rows)
+    np.testing.assert_array_equal(part, full[rows])
+
+
+# ---- 3. invariants -------------------------------------------------------------
+
+def test_causality_future_tokens_do_not_change_past_rows():
+    rng = np.random.default_rng(11)
+    c = rand_case(rng, [9])
+    base = ofwd(c)
+    i0 = 4
+    c2 = dict(c)
+    for key in ("q", "k", "v"):
+        a = c[key].copy()
+        a[i0 + 1:] = rng.standard_normal(a[i0 + 1:].shape)
+        c2[key] = a
+    t = c["timestamps"].copy()
+    t[i0 + 1:] += 1000
+    c2["timestamps"] = t
+    out = ofwd(c2)
+    np.testing.assert_array_equal(out[: i0 + 1], base[: i0 + 1])
+    assert not np.array_equal(out[i0 + 1:], base[i0 + 1:])
+
+
+def test_sequences_are_independent():
+    rng = np.random.default_rng(12)
+    lengths = [4, 6, 3]
+    c = rand_case(rng, lengths)
+    base = ofwd(c)
+    off = c["seq_offsets"]
+    for b in range(3):
+        s0, s1 = off[b], off[b + 1]
+        alone = dict(c, seq_offsets=np.array([0, s1 - s0]), timestamps=c["timestamps"][s0:s1],
+                     q=c["q"][s0:s1], k=c["k"][s0:s1], v=c["v"][s0:s1])
+        np.testing.assert_array_equal(ofwd(alone), base[s0:s1])
+    # permuted batch: [2, 0, 1]
+    perm = [2, 0, 1]
+    sl = [slice(off[b], off[b + 1]) for b in perm]
+    pc = dict(c, seq_offsets=np.concatenate([[0], np.cumsum([lengths[b] for b in perm])]),
+              timestamps=np.concatenate([c["timestamps"][s] for s in sl]),
+              q=np.concatenate([c["q"][s] for s in sl]), k=np.concatenate([c["k"][s] for s in sl]),
+              v=np.concatenate([c["v"][s] for s in sl]))
+    np.testing.assert_array_equal(ofwd(pc), np.concatenate([base[s] for s in sl]))
+
+
+def test_zero_bias_is_plain_silu_attention():
+    rng = np.random.default_rng(13)
+    c = rand_case(rng, [7])
+    c = dict(c, rab_pos=np.zeros_like(c["rab_pos"]), rab_time=np.zeros_like(c["rab_time"]))
+    q, k, v = c["q"][:, 0], c["k"][:, 0], c["v"][:, 0]
+    S = q @ k.T
+    P = S / (1 + np.exp(-S)) * c["inv_n"] * np.tril(np.ones((7, 7)))
+    np.testing.assert_allclose(ofwd(c)[:, 0], P @ v, rtol=0, atol=1e-12)
+
+
+def test_linear_in_v():
+    rng = np.random.default_rng(14)
+    c = rand_case(rng, [6, 5])
+    v2 = rng.standard_normal(c["v"].shape)
+    lhs = ofwd(c, v=2.0 * c["v"] - 3.0 * v2)
+    rhs = 2.0 * ofwd(c) - 3.0 * ofwd(c, v=v2)
+    np.testing.assert_allclose(lhs, rhs, rtol=0, atol=1e-11)
+
+
+def test_constant_bias_shift_moves_between_tables():
+    rng = np.random.default_rng(15)
+    c = rand_case(rng, [8, 4], nt=[2, 1])
+    a = ofwd(c, rab_pos=c["rab_pos"] + 0.375)
+    b = ofwd(c, rab_time=c["rab_time"] + 0.375)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+# ---- 4. special cases ---------------------------------------------------------
+
+def test_single_token_closed_form():
+    rng = np.random.default_rng(16)
+    c = rand_case(rng, [1], H=1, dqk=4, dv=3)
+    s = float(c["q"][0, 0] @ c["k"][0, 0]) + c["rab_pos"][0 - c["pos_lo"]] + c["rab_time"][0]
+    expect = s / (1 + np.exp(-s)) * c["inv_n"] * c["v"][0, 0]
+    np.testing.assert_allclose(ofwd(c)[0, 0], expect, rtol=0, atol=1e-14)
+
+
+def test_zero_qk_and_bias_gives_zero():
+    rng = np.random.default_rng(17)
+    c = rand_case(rng, [5, 3])
+    out = ofwd(c, q=np.zeros_like(c["q"]), k=np.zeros_like(c["k"]),
+               rab_pos=np.zeros_like(c["rab_pos"]), rab_time=np.zeros_like(c["rab_time"]))
+    assert np.all(out == 0.0)
+
+
+def test_empty_batch_and_empty_sequences():
+    rng = np.random.default_rng(18)
+    c = rand_case(rng, [0, 0, 3, 0])
+    np.testing.assert_allclose(ofwd(c), dfwd(c), rtol=0, atol=1e-12)
+
+
+def test_candidate_rows_by_hand():
+    # 2 history tokens + 2 candidates; q=k=0 so s = pos bias + time bias only.
+    # candidate rows sit at position 2: they see j=0 (dist 2), j=1 (dist 1),
+    # themselves (dist 0), and not the other candidate.
+    L, nt = 4, 2
+    q = np.zeros((L, 1, 1))
+    k = np.zeros((L, 1, 1))
+    v = np.array([1.0, 10.0, 100.0, 1000.0]).reshape(L, 1, 1)
+    t = np.array([0, 0, 0, 0], dtype=np.int64)
+    rp = np.array([0.5, 1.0, 2.0])  # distances 0, 1, 2 (lo=0, hi=2)
+    rt = np.array([0.0])
+    out = oracle.attn_fwd([0, L], t, [nt], q, k, v, rp, rt, 0, 2, 1.0).reshape(L)
+    sl = lambda x: x / (1 + np.exp(-x))
+    assert out[2] == pytest.approx(sl(2.0) * 1 + sl(1.0) * 10 + sl(0.5) * 100, abs=1e-12)
+    assert out[3] == pytest.approx(sl(2.0) * 1 + sl(1.0) * 10 + sl(0.5) * 1000, abs=1e-12)
+    assert out[1] == pytest.approx(sl(1.0) * 1 + sl(0.5) * 10, abs=1e-12)
+
+
+# ---- 5. gradients: torch float64 autograd and finite differences -------------
+
+def _torch_dense_loss(c, dout):
+    off, nt = c["seq_offsets"], c["num_targets"]
+    q = torch.tensor(c["q"], requires_grad=True)
+    k = torch.tensor(c["k"], requires_grad=True)
+    v = torch.tensor(c["v"], requires_grad=True)
+    rp = torch.tensor(c["rab_pos"], requires_grad=True)
+    rt = torch.tensor(c["rab_time"], requires_grad=True)
+    loss = 0.0
+    lo, hi = c["pos_lo"], c["pos_hi"]
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        hist = L - n_t
+        idx = np.arange(L)
+        p = np.where(idx < hist, idx, hist)
+        rel = torch.tensor(np.clip(p[:, None] - p[None, :], lo, hi) - lo)
+        ts = c["timestamps"][s0:s1]
+        bkt = torch.tensor([[min(len(c["rab_time"]) - 1, (int(max(ts[i] - ts[j], 0)) + 1).bit_length() - 1)
+                             for j in range(L)] for i in range(L)])
+        I, J = idx[:, None], idx[None, :]
+        vis = torch.tensor(np.where(I < hist, J <= I, (J < hist) | (J == I)), dtype=torch.float64)
+        S = torch.einsum("ihc,jhc->hij", q[s0:s1], k[s0:s1]) + (rp[rel] + rt[bkt])[None]
+        P = torch.nn.functional.silu(S) * c["inv_n"] * vis[None]
+        O = torch.einsum("hij,jhc->ihc", P, v[s0:s1])
+        loss = loss + (O * torch.tensor(dout[s0:s1])).sum()
+    loss.backward()
+    return [x.grad.numpy() for x in (q, k, v, rp, rt)]
+
+
+def obwd(c, dout):
+    return oracle.attn_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"],
+                           c["v"], c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"],
+                           c["inv_n"], dout)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_bwd_matches_torch_autograd(seed):
+    rng = np.random.default_rng(100 + seed)
+    lengths = rng.integers(1, 8, size=3)
+    nt = [int(rng.integers(0, L)) for L in lengths] if seed % 2 else None
+    c = rand_case(rng, lengths, nt=nt)
+    dout = rng.standard_normal(c["v"].shape)
+    ours = obwd(c, dout)
+    ref = _torch_dense_loss(c, dout)
+    for a, b in zip(ours, ref):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-11)
+
+
+def test_bwd_central_finite_differences():
+    rng = np.random.default_rng(200)
+    c = rand_case(rng, [4, 3], H=2, dqk=2, dv=2, nt=[1, 0])
+    dout = rng.standard_normal(c["v"].shape)
+    grads = dict(zip(["q", "k", "v", "rab_pos", "rab_time"], obwd(c, dout)))
+    h = 1e-5
+    for key, g in grads.items():
+        flat = c[key].reshape(-1)
+        for e in range(flat.size):
+            plus, minus = flat.copy(), flat.copy()
+            plus[e] += h
+            minus[e] -= h
+            fp = np.sum(ofwd(c, **{key: plus.reshape(c[key].shape)}) * dout)
+            fm = np.sum(ofwd(c, **{key: minus.reshape(c[key].shape)}) * dout)
+            assert abs((fp - fm) / (2 * h) - g.reshape(-1)[e]) < 1e-7, (key, e)
+
+
+def test_bwd_rows_match_full():
+    rng = np.random.default_rng(201)
+    c = rand_case(rng, [6, 4, 5], nt=[0, 1, 2])
+    dout = rng.standard_normal(c["v"].shape)
+    dq, dk, dv, _, _ = obwd(c, dout)
+    qr, kr = np.array([0, 5, 7, 14]), np.array([1, 6, 9, 10, 14])
+    pq, pk, pv = oracle.attn_bwd_rows(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"],
+                                      c["k"], c["v"], c["rab_pos"], c["rab_time"], c["pos_lo"],
+                                      c["pos_hi"], c["inv_n"], dout, qr, kr)
+    np.testing.assert_allclose(pq, dq[qr], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(pk, dk[kr], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(pv, dv[kr], rtol=0, atol=1e-12)
+
+
+def test_bias_grad_tables_sum_to_the_same_total():
+    rng = np.random.default_rng(202)
+    c = rand_case(rng, [7, 5])
+    dout = rng.standard_normal(c["v"].shape)
+    _, _, _, drp, drt = obwd(c, dout)
+    assert drp.sum() == pytest.approx(drt.sum(), abs=1e-12)
+
+
+# ---- 6. bucket and position functions: exhaustive integer checks ---------------
+
+def _bucket_by_powers(dt, nb):
+    # largest b with 2**b <= 1 + max(dt, 0), capped at nb - 1
+    x = 1 + max(dt, 0)
+    b = 0
+    while (1 << (b + 1)) <= x:
+        b += 1
+    return min(b, nb - 1)
+
+
+def test_bucket_exhaustive_small_range():
+    lib = oracle._load()
+    for dt in range(0, 1 << 20, 1):
+        if dt < 4096 or dt % 97 == 0 or (dt & (dt + 1)) == 0 or (dt & (dt - 1)) == 0:
+            assert lib.oracle_time_bucket(dt, 0, 128) == _bucket_by_powers(dt, 128)
+
+
+def test_bucket_numpy_exhaustive_2_20():
+    # the whole [0, 2^20] range against powers-of-two boundaries (vectorised)
+    dt = np.arange(0, (1 << 20) + 1, dtype=np.int64)
+    expect = np.searchsorted(1 << np.arange(0, 40, dtype=np.int64), dt + 1, side="right") - 1
+    lib = oracle._load()
+    sample = dt[:: 1 << 10]
+    got = np.array([lib.oracle_time_bucket(int(x), 0, 64) for x in sample])
+    np.testing.assert_array_equal(got, np.minimum(expect[:: 1 << 10], 63))
+
+
+def test_bucket_powers_of_two_and_large_epochs():
+    for e in range(0, 63):
+        for d in (-1, 0, 1):
+            dt = (1 << e) + d - 1
+            if dt < 0:
+                continue
+            for base in (0, 1_700_000_000, (1 << 40) + 3):
+                assert oracle.time_bucket(base + dt, base, 128) == _bucket_by_powers(dt, 128)
+                assert oracle.time_bucket(base + dt, base, 16) == _bucket_by_powers(dt, 16)
+    assert oracle.time_bucket(5, 9, 32) == 0   # negative elapsed time clamps to 0
+
+
+def test_pos_index_clamps():
+    assert oracle.pos_index(10, 3, -4, 4) == 8
+    assert oracle.pos_index(3, 10, -4, 4) == 0
+    assert oracle.pos_index(5, 5, -4, 4) == 4
+    assert oracle.pos_index(127, 0, 0, 127) == 127
+    assert oracle.pos_index(0, 1, 0, 127) == 0
+
+
+def test_visibility_rule():
+    # history rows: j <= i; candidate rows: all history and themselves
+    L, nt = 6, 2
+    vis = [[oracle.visible(i, j, L, nt) for j in range(L)] for i in range(L)]
+    assert vis[3] == [True, True, True, True, False, False]
+    assert vis[4] == [True, True, True, True, True, False]
+    assert vis[5] == [True, True, True, True, False, True]
+
+
+# ---- 7. FLOP accounting: the DLRMv4 page's Table 7 ---------------------------
+
+def test_cost_table_reproduces_published_figures():
+    # Table 6 symbols: B=1024, L=3 layers, h=4, d_qk=d_v=128, D=512, S=4096
+    B, layers, h, d, D, S = 1024, 3, 4, 128, 512, 4096
+    pairs_lower_triangle = B * S * S / 2            # the page's S^2/2 per sequence
+    attn = layers * (flops.attn_fwd_flops(pairs_lower_triangle, h, d, d)
+                     + flops.attn_bwd_flops(pairs_lower_triangle, h, d, d))
+    assert round(attn / 1e12, 2) == 184.72
+    uvqk = layers * 3 * flops.f1_flops(B * S, D, h, d, d)
+    assert round(uvqk / 1e12, 2) == 79.16
+    outp = layers * 3 * flops.f2_flops(B * S, D, h, d, width_factor=3)
+    assert round(outp / 1e12, 2) == 59.37
+    assert round((attn + uvqk + outp) / 1e12, 2) == 323.26
+    # backward is 2.5x forward: the "factor 3.5" for fwd+bwd
+    assert flops.attn_bwd_flops(1, h, d, d) == 2.5 * flops.attn_fwd_flops(1, h, d, d)
+
+
+def test_pair_counter_by_brute_force():
+    for L, nt in [(1, 0), (5, 0), (9, 3), (6, 6), (4096, 0), (2560, 512)]:
+        if L <= 16:
+            brute = sum(oracle.visible(i, j, L, nt) for i in range(L) for j in range(L))
+            assert flops.attn_pairs_per_seq(L, nt) == brute
+    assert flops.attn_pairs_per_seq(4096) == 4096 * 4097 // 2
+    assert flops.attn_pairs([3, 0, 2], [1, 0, 0]) == (3 + 3) + 3  # hist 2 -> 3 pairs, 1 candidate sees 3
+
+
+# ---- 8. layer pieces against textbook / library definitions ----------------
+
+def test_linear_matches_numpy():
+    rng = np.random.default_rng(300)
+    x, w, b = rng.standard_normal((7, 5)), rng.standard_normal((5, 6)), rng.standard_normal(6)
+    np.testing.assert_allclose(oracle.linear(x, w, b), x @ w + b, rtol=0, atol=1e-12)
+    z = x @ w + b
+    np.testing.assert_allclose(oracle.linear(x, w, b, apply_silu=True), z / (1 + np.exp(-z)),
+                               rtol=0, atol=1e-12)
+
+
+def test_norm_gate_matches_torch_layer_norm():
+    rng = np.random.default_rng(301)
+    o, u = rng.standard_normal((9, 16)), rng.standard_normal((9, 16))
+    g, be = rng.standard_normal(16), rng.standard_normal(16)
+    ref = torch.nn.functional.layer_norm(torch.tensor(o), (16,), torch.tensor(g), torch.tensor(be),
+                                         eps=1e-5).numpy() * u
+    np.testing.assert_allclose(oracle.norm_gate(o, u, g, be), ref, rtol=0, atol=1e-12)
+
+
+def test_layer_matches_composition():
+    rng = np.random.default_rng(302)
+    H, dqk, dv, D = 2, 3, 2, 5
+    c = rand_case(rng, [4, 6, 1], H=H, dqk=dqk, dv=dv, nt=[0, 2, 0])
+    T = int(c["seq_offsets"][-1])
+    W = H * (2 * dv + 2 * dqk)
+    x = rng.standard_normal((T, D))
+    w1, b1 = rng.standard_normal((D, W)) * 0.5, rng.standard_normal(W) * 0.1
+    w2, b2 = rng.standard_normal((H * dv, D)), rng.standard_normal(D)
+    gam, bet = 1 + 0.1 * rng.standard_normal(H * dv), 0.1 * rng.standard_normal(H * dv)
+    y = oracle.layer_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], x, w1, b1, w2, b2,
+                         gam, bet, c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"],
+                         c["inv_n"], H, dqk, dv)
+    z = torch.nn.functional.silu(torch.tensor(x) @ torch.tensor(w1) + torch.tensor(b1)).numpy()
+    u = z[:, : H * dv]
+    vv = z[:, H * dv: 2 * H * dv].reshape(T, H, dv)
+    qq = z[:, 2 * H * dv: 2 * H * dv + H * dqk].reshape(T, H, dqk)
+    kk = z[:, 2 * H * dv + H * dqk:].reshape(T, H, dqk)
+    o = dense_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], qq, kk, vv, c["rab_pos"],
+                  c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"]).reshape(T, H * dv)
+    g = torch.nn.functional.layer_norm(torch.tensor(o), (H * dv,), torch.tensor(gam),
+                                       torch.tensor(bet), eps=1e-5).numpy() * u
+    np.testing.assert_allclose(y, g @ w2 + b2, rtol=0, atol=1e-10)
