@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark of the HSTU jagged attention training step on B200.
+
+One step = one pass of the attention hot path over one synthetic batch of the
+long-history workload (8 sequences, lengths U[8192, 16384], 4 heads,
+d_qk = d_v = 128, bf16 with fp32 accumulation): jagged tile schedule, forward
+(S = Q K^T, relative bias, SiLU, 1/N, P V) and backward (dQ, dK, dV and the
+bias-table gradients), all through the C ABI of libhstu.  With N > 1 GPUs each
+rank runs its own batch (weak scaling, one process per GPU) and the bias-table
+gradients are summed over ranks with one NCCL all-reduce, the only exchange a
+data-parallel step has.
+
+Metric: unmasked attention TFLOP/s, fwd 2(d_qk + d_v) and bwd 2(3 d_qk + 2 d_v)
+FLOPs per visible pair and head ("DLRMv4 ..." page, Table 7 accounting).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HSTU jagged attention fwd/bwd TFLOP/s (unmasked) and % of B200 bf16 dense peak"
+WORKLOAD = "long_history_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels of ours launched per step: fwd call (schedule, attention) and bwd call
+# (schedule, attention backward, dq conversion)
+LAUNCHES_PER_STEP = 5
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms (read-only)."""
+
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                if self.uuid and parts[1] != self.uuid:
+                    continue
+                rows.append((ts, parts))
+        os.unlink(self.file.name)
+        win = [p for ts, p in rows if t0 - 0.25 <= ts <= t1 + 0.25] or [p for _, p in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        sm, smax = [], []
+        for p in win:
+            try:
+                sm.append(float(p[2]))
+                smax.append(float(p[3]))
+            except ValueError:
+                pass
+            for n, v in zip(names, p[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+def attn_flops(inp):
+    from hstu_sequential_transduction_b200 import flops
+    nt = None if inp.num_targets is None else inp.num_targets.numpy()
+    pairs = flops.attn_pairs(inp.lengths, nt)
+    H, dqk, dv = inp.q.shape[1], inp.q.shape[2], inp.v.shape[2]
+    return flops.attn_fwd_flops(pairs, H, dqk, dv), flops.attn_bwd_flops(pairs, H, dqk, dv)
+
+
+def cpu_oracle_sample(inp, length: int, threads: int):
+    """Time the oracle's fwd + bwd on the first `length` tokens of sequence 0."""
+    import oracle
+    from hstu_sequential_transduction_b200 import flops
+    L = int(min(length, int(inp.lengths[0])))
+    sl = slice(0, L)
+    args = ([0, L], inp.timestamps[sl], None, inp.q[sl], inp.k[sl], inp.v[sl], inp.rab_pos,
+            inp.rab_time, inp.pos_lo, inp.pos_hi, inp.inv_n)
+    t = time.perf_counter()
+    oracle.attn_fwd(*args, threads=threads)
+    oracle.attn_bwd(*args, inp.dout[sl], threads=threads)
+    dt = time.perf_counter() - t
+    pairs = flops.attn_pairs([L])
+    H, d = inp.q.shape[1], inp.q.shape[2]
+    fl = flops.attn_fwd_flops(pairs, H, d, d) + flops.attn_bwd_flops(pairs, H, d, d)
+    return L, fl, dt
+
+
+def calibrated_length(inp, budget_s: float, threads: int, probe: int = 512):
+    _, _, dt = cpu_oracle_sample(inp, probe, threads)
+    scale = math.sqrt(max(budget_s, 0.05) / max(dt, 1e-3))
+    return int(min(int(inp.lengths[0]), max(64, probe * scale)))
+
+
+def cpu_baseline(inp):
+    import oracle
+    threads = oracle.default_threads()
+    L = calibrated_length(inp, 15.0, threads)
+    L, fl, dt = cpu_oracle_sample(inp, L, threads)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"oracle fwd+bwd, fp64, on the first {L} tokens of sequence 0 of the "
+                      f"{WORKLOAD} batch (4 heads, d=128): {fl / 1e9:.1f} GFLOP in {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from hstu_sequential_transduction_b200 import workloads
+    inp = workloads.generate(workloads.WORKLOADS[WORKLOAD])
+    threads = oracle.default_threads()
+    per_step = min(5.0, 150.0 / max(1, args.steps + args.warmup))
+    L = calibrated_length(inp, per_step, threads)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(inp, L, threads)
+    total_fl = total_t = 0.0
+    for _ in range(args.steps):
+        _, fl, dt = cpu_oracle_sample(inp, L, threads)
+        total_fl += fl
+        total_t += dt
+    value = total_fl / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_tokens": L, "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: oracle fwd+bwd on the first {L} tokens of "
+                                   f"sequence 0 (4 heads, d=128)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from hstu_sequential_transduction_b200 import ops, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ops.load_library(allow_build=(world == 1))
+
+    w = workloads.WORKLOADS[WORKLOAD]
+    inp = workloads.generate(w, seed=w.seed + rank)
+    fwd_fl, bwd_fl = attn_flops(inp)
+    T = inp.total_tokens
+    kw = dict(max_seq_len=inp.max_seq_len, inv_n=inp.inv_n, pos_lo=inp.pos_lo, pos_hi=inp.pos_hi)
+    q, k, v, dout = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.dout))
+    off, ts = inp.seq_offsets.to(dev), inp.timestamps.to(dev)
+    rp, rt = inp.rab_pos.to(dev), inp.rab_time.to(dev)
+    npos, nb = rp.numel(), rt.numel()
+    out = torch.empty_like(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bias_grads = torch.empty(npos + nb, dtype=torch.float32, device=dev)
+    grads = (dq, dk, dv, bias_grads[:npos], bias_grads[npos:])
+    desc = ops.make_attn_desc(len(inp.lengths), inp.max_seq_len, T, q.shape[1], q.shape[2],
+                              v.shape[2], ops.HSTU_BF16, inp.inv_n, inp.pos_lo, inp.pos_hi, nb)
+    ws_f = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc, False), dev)
+    ws_b = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc, True), dev)
+    stream = torch.cuda.current_stream()
+    ev_f0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_f1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None, q=q, k=k, v=v, off=off, ts=ts, rp=rp, rt=rt, dout=dout, out=out, grads=grads):
+        if i is not None:
+            ev_f0[i].record(stream)
+        ops.hstu_attn_fwd(q, k, v, off, ts, None, rp, rt, out=out, workspace=ws_f, stream=stream, **kw)
+        if i is not None:
+            ev_f1[i].record(stream)
+        ops.hstu_attn_bwd(q, k, v, off, ts, None, rp, rt, dout, grads=grads, workspace=ws_b,
+                          stream=stream, **kw)
+        if i is not None:
+            ev_b1[i].record(stream)
+        if world > 1:
+            dist.all_reduce(bias_grads)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    st, bits = ops.hstu_check_device_flag(ws_b, stream)
+    assert st == 0, f"device input check flagged {bits}"
+
+    uuid = ""
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+    ms = start.elapsed_time(end) / args.steps
+    fwd_ms = statistics.mean(ev_f0[i].elapsed_time(ev_f1[i]) for i in range(args.steps))
+    bwd_ms = statistics.mean(ev_f1[i].elapsed_time(ev_b1[i]) for i in range(args.steps))
+
+    stats = torch.tensor([ms, fwd_fl + bwd_fl, fwd_fl, bwd_fl], dtype=torch.float64, device=dev)
+    if world > 1:
+        mx = stats[:1].clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = stats[1:].clone()
+        dist.all_reduce(sm)
+        stats = torch.cat([mx, sm])
+    ms_max, total_fl = float(stats[0]), float(stats[1])
+    value = total_fl / (ms_max * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: pinned inputs copied in,
+    # every output read back, inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.dout, inp.seq_offsets,
+                                            inp.timestamps, inp.rab_pos, inp.rab_time)]
+        dev_in = [torch.empty_like(t, device=dev) for t in host_in]
+        dev_out = [out, dq, dk, dv, bias_grads]
+        host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in dev_out]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+        def e2e_step():
+            for d_, h_ in zip(dev_in, host_in):
+                d_.copy_(h_, non_blocking=True)
+            eq, ek, ev, edo, eoff, ets, erp, ert = dev_in
+            step(None, eq, ek, ev, eoff, ets, erp, ert, edo)
+            for h_, d_ in zip(host_out, dev_out):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(3, args.steps // 3)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e2e = {"value": total_fl / (float(ems) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+        fwd_tf = fwd_fl / (fwd_ms * 1e-3) / 1e12
+        bwd_tf = bwd_fl / (bwd_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, per-rank batches)",
+            "config": {"workload": WORKLOAD, "batch_per_gpu": len(inp.lengths),
+                       "seq_len": "U[8192,16384]", "tokens_per_gpu": T, "heads": q.shape[1],
+                       "d_qk": q.shape[2], "d_v": v.shape[2], "pos_clamp": 4096,
+                       "time_buckets": nb, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (q, k, v, dout = %d MB per step)"
+                             % (4 * q.numel() * 2 // 2**20)},
+            "fwd": {"tflops": fwd_tf, "ms": fwd_ms, "pct_of_bf16_peak": 100 * fwd_tf / burst},
+            "bwd": {"tflops": bwd_tf, "ms": bwd_ms, "pct_of_bf16_peak": 100 * bwd_tf / burst},
+            "pct_of_bf16_peak": 100 * (value / world) / burst,
+            "roofline": {"bound": "tensor", "kernel": "attention backward (hstu_attn_bwd call)",
+                         "achieved": bwd_tf, "peak": sustained, "unit": "TFLOP/s",
+                         "frac": bwd_tf / sustained, "traffic": None,
+                         "peak_source": f"bf16_tflops_sustained, {peak_src}"},
+            "clocks": clocks,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

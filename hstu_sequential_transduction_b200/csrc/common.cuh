@@ -1,0 +1,159 @@
+// Shared device helpers for the HSTU kernels (sm_100a).
+//
+// The index functions here are the single definition every kernel and the
+// debug entry use for the relative-bias gathers of the HSTU attention
+// ("DLRMv4 Brings Sequence-Based Recommendation Training to MLPerf", section
+// "Model Architecture": a bias from positional and temporal distance).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hstu.h"
+
+namespace hstu {
+
+// Workspace header (first 256 bytes of every attention workspace).
+struct WsHeader {
+    int flag;      // device input-check bits of the last call
+    int n_items;   // work items written by the scheduler
+    int cursor;    // work-stealing counter of persistent kernels
+    int pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+enum : int {
+    FLAG_OFFSET0 = 1,
+    FLAG_SEQ_RANGE = 2,
+    FLAG_SEQ_TOO_LONG = 4,
+    FLAG_TARGETS = 8,
+    FLAG_TOTAL = 16,
+};
+
+// Everything an attention kernel reads; strides are in elements between rows.
+struct AttnParams {
+    const void *q, *k, *v;
+    void *o;
+    int64_t sq, sk, sv, so;
+    const int64_t *seq_offsets;
+    const int64_t *timestamps;
+    const int32_t *num_targets;
+    const float *rab_pos, *rab_time;
+    int B, H, dqk, dv, max_seq_len;
+    int64_t T;
+    float inv_n;
+    int pos_lo, pos_hi, nb;
+    const int2 *items;
+    WsHeader *hdr;
+    // backward only
+    const void *dout;
+    int64_t sdo;
+    void *dq, *dk, *dvv;
+    int64_t sdq, sdk, sdv;
+    float *dq_acc;  // fp32 [T, H, dqk] accumulator (bf16 mode)
+    float *d_rab_pos, *d_rab_time;
+};
+
+// floor(log2(1 + max(dt, 0))) capped at nb - 1, exact on int64 seconds.
+__device__ __forceinline__ int time_bucket(int64_t t_i, int64_t t_j, int nb)
+{
+    int64_t dt = t_i - t_j;
+    dt = dt < 0 ? 0 : dt;
+    int b = 63 - __clzll((long long)(dt + 1));
+    return b < nb - 1 ? b : nb - 1;
+}
+
+__device__ __forceinline__ int pos_index(int p_i, int p_j, int lo, int hi)
+{
+    int d = p_i - p_j;
+    d = d < lo ? lo : (d > hi ? hi : d);
+    return d - lo;
+}
+
+// Local position of token i: candidates share the slot after the history.
+__device__ __forceinline__ int token_pos(int i, int hist) { return i < hist ? i : hist; }
+
+__device__ __forceinline__ bool visible(int i, int j, int hist)
+{
+    return i < hist ? (j <= i) : (j < hist || j == i);
+}
+
+// SiLU on the fp32 score.  The fast form uses the hardware exponential.
+__device__ __forceinline__ float silu_fast(float x)
+{
+    return x * __frcp_rn(1.0f + __expf(-x));
+}
+
+__device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
+
+__device__ __forceinline__ float silu_grad_precise(float x)
+{
+    float s = 1.0f / (1.0f + expf(-x));
+    return s * (1.0f + x * (1.0f - s));
+}
+
+// ---- bf16 / async-copy / tensor-core helpers (legacy mma.sync path) -------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte async copy; src_bytes < 16 zero-fills the rest.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+                 "l"(gmem), "r"(src_bytes));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                            const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                                  uint32_t &r3, const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ---- host helpers -----------------------------------------------------------
+
+inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+// Upper bound on the work items of a schedule with tiles of `tile` rows.
+inline int64_t max_items(int64_t T, int B, int tile) { return (T + tile - 1) / tile + B; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace hstu

@@ -1,0 +1,369 @@
+// C ABI of libhstu: argument validation, workspace carving and kernel dispatch.
+// Every check that can fail runs on the host before anything is enqueued.
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace hstu;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hstu_status check_attn_desc(const hstu_attn_desc *d)
+{
+    if (!d)
+        return HSTU_ERR_INVALID_ARG;
+    if (d->num_seqs < 0 || d->max_seq_len < 0 || d->total_tokens < 0 || d->num_heads < 1 ||
+        d->num_time_buckets < 1 || d->pos_hi < d->pos_lo || !std::isfinite(d->inv_n))
+        return HSTU_ERR_INVALID_ARG;
+    if (d->dtype != HSTU_F32 && d->dtype != HSTU_BF16)
+        return HSTU_ERR_INVALID_ARG;
+    if ((int64_t)d->pos_hi - d->pos_lo + 1 > (1 << 24))
+        return HSTU_ERR_UNSUPPORTED;
+    if (d->d_qk != d->d_v)
+        return HSTU_ERR_UNSUPPORTED;
+    if (d->dtype == HSTU_BF16 && d->d_qk != 32 && d->d_qk != 64 && d->d_qk != 128)
+        return HSTU_ERR_UNSUPPORTED;
+    if (d->dtype == HSTU_F32 && d->d_qk != 32 && d->d_qk != 64)
+        return HSTU_ERR_UNSUPPORTED;
+    if (max_items(d->total_tokens, d->num_seqs, kMmaTile) > INT_MAX / 4 ||
+        d->total_tokens * d->num_heads > ((int64_t)1 << 40))
+        return HSTU_ERR_UNSUPPORTED;
+    return HSTU_OK;
+}
+
+size_t elem_bytes(const hstu_attn_desc *d) { return d->dtype == HSTU_BF16 ? 2 : 4; }
+
+size_t items_bytes(const hstu_attn_desc *d)
+{
+    return align256(sizeof(int2) * (size_t)max_items(d->total_tokens, d->num_seqs, kMmaTile));
+}
+
+size_t attn_ws(const hstu_attn_desc *d, int is_bwd)
+{
+    size_t b = sizeof(WsHeader) + items_bytes(d);
+    if (is_bwd && d->dtype == HSTU_BF16)
+        b += align256(sizeof(float) * (size_t)d->total_tokens * d->num_heads * d->d_qk);
+    return b;
+}
+
+hstu_status check_ws(void *ws, size_t have, size_t need)
+{
+    if (need && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return HSTU_ERR_WORKSPACE;
+    return have < need ? HSTU_ERR_WORKSPACE : HSTU_OK;
+}
+
+hstu_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA; }
+
+#define HSTU_TRY(x)                        \
+    do {                                   \
+        hstu_status _s = (x);              \
+        if (_s != HSTU_OK)                 \
+            return _s;                     \
+    } while (0)
+
+#define HSTU_CUDA(x) HSTU_TRY(cuda_status(x))
+
+AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_t *ts,
+                       const int32_t *nt, const float *rp, const float *rt, void *ws)
+{
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.seq_offsets = off;
+    p.timestamps = ts;
+    p.num_targets = nt;
+    p.rab_pos = rp;
+    p.rab_time = rt;
+    p.B = d->num_seqs;
+    p.H = d->num_heads;
+    p.dqk = d->d_qk;
+    p.dv = d->d_v;
+    p.max_seq_len = d->max_seq_len;
+    p.T = d->total_tokens;
+    p.inv_n = d->inv_n;
+    p.pos_lo = d->pos_lo;
+    p.pos_hi = d->pos_hi;
+    p.nb = d->num_time_buckets;
+    p.hdr = static_cast<WsHeader *>(ws);
+    p.items = reinterpret_cast<const int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
+    return p;
+}
+
+int grid_items(const hstu_attn_desc *d) { return (int)max_items(d->total_tokens, d->num_seqs, kMmaTile); }
+
+hstu_status schedule(const hstu_attn_desc *d, const int64_t *off, const int32_t *nt, int is_bwd,
+                     void *ws, cudaStream_t stream)
+{
+    int2 *items = reinterpret_cast<int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
+    return cuda_status(launch_schedule(off, nt, d->num_seqs, d->total_tokens, d->max_seq_len,
+                                       kMmaTile, is_bwd, items, grid_items(d),
+                                       static_cast<WsHeader *>(ws), nullptr, stream));
+}
+
+// Attention forward on explicit row strides (used by the layer as well).
+hstu_status attn_fwd_strided(const hstu_attn_desc *d, const void *q, int64_t sq, const void *k,
+                             int64_t sk, const void *v, int64_t sv, const int64_t *off,
+                             const int64_t *ts, const int32_t *nt, const float *rp, const float *rt,
+                             void *out, int64_t so, void *ws, cudaStream_t stream)
+{
+    HSTU_TRY(schedule(d, off, nt, 0, ws, stream));
+    AttnParams p = base_params(d, off, ts, nt, rp, rt, ws);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = out;
+    p.sq = sq;
+    p.sk = sk;
+    p.sv = sv;
+    p.so = so;
+    if (d->dtype == HSTU_BF16)
+        return cuda_status(launch_attn_fwd_mma(p, grid_items(d), stream));
+    return cuda_status(launch_attn_fwd_f32(p, grid_items(d), stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hstu_status_string(int status)
+{
+    switch (status) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG: invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA: a CUDA runtime call failed";
+    case HSTU_ERR_DEVICE_CHECK: return "HSTU_ERR_DEVICE_CHECK: device-side input check failed";
+    default: return "unknown hstu_status";
+    }
+}
+
+int hstu_version(void) { return kVersion; }
+
+hstu_status hstu_attn_workspace_size(const hstu_attn_desc *desc, int is_bwd, size_t *bytes)
+{
+    HSTU_TRY(check_attn_desc(desc));
+    if (!bytes)
+        return HSTU_ERR_INVALID_ARG;
+    *bytes = attn_ws(desc, is_bwd);
+    return HSTU_OK;
+}
+
+hstu_status hstu_attn_fwd(const hstu_attn_desc *desc, const void *q, const void *k, const void *v,
+                          const int64_t *seq_offsets, const int64_t *timestamps,
+                          const int32_t *num_targets, const float *rab_pos, const float *rab_time,
+                          void *out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    HSTU_TRY(check_attn_desc(desc));
+    if (!seq_offsets || !rab_pos || !rab_time)
+        return HSTU_ERR_INVALID_ARG;
+    if (desc->total_tokens > 0 && (!q || !k || !v || !out || !timestamps))
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return HSTU_ERR_INVALID_ARG;
+    HSTU_TRY(check_ws(workspace, workspace_bytes, attn_ws(desc, 0)));
+    const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
+    return attn_fwd_strided(desc, q, row, k, row, v, row, seq_offsets, timestamps, num_targets,
+                            rab_pos, rab_time, out, row, workspace, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void *k, const void *v,
+                          const int64_t *seq_offsets, const int64_t *timestamps,
+                          const int32_t *num_targets, const float *rab_pos, const float *rab_time,
+                          const void *dout, void *dq, void *dk, void *dv, float *d_rab_pos,
+                          float *d_rab_time, void *workspace, size_t workspace_bytes, void *stream)
+{
+    HSTU_TRY(check_attn_desc(desc));
+    if (!seq_offsets || !rab_pos || !rab_time || !d_rab_pos || !d_rab_time)
+        return HSTU_ERR_INVALID_ARG;
+    if (desc->total_tokens > 0 &&
+        (!q || !k || !v || !dout || !dq || !dk || !dv || !timestamps))
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return HSTU_ERR_INVALID_ARG;
+    HSTU_TRY(check_ws(workspace, workspace_bytes, attn_ws(desc, 1)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int npos = desc->pos_hi - desc->pos_lo + 1;
+    HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * npos, st));
+    HSTU_CUDA(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->num_time_buckets, st));
+    const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
+    const size_t tensor_bytes = (size_t)desc->total_tokens * row * elem_bytes(desc);
+    const bool bf16 = desc->dtype == HSTU_BF16;
+    AttnParams p = base_params(desc, seq_offsets, timestamps, num_targets, rab_pos, rab_time, workspace);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.sq = p.sk = p.sv = row;
+    p.dout = dout;
+    p.sdo = row;
+    p.dq = dq;
+    p.dk = dk;
+    p.dvv = dv;
+    p.sdq = p.sdk = p.sdv = row;
+    p.d_rab_pos = d_rab_pos;
+    p.d_rab_time = d_rab_time;
+    if (bf16) {
+        p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + sizeof(WsHeader) +
+                                             items_bytes(desc));
+        HSTU_CUDA(cudaMemsetAsync(p.dq_acc, 0, sizeof(float) * (size_t)desc->total_tokens * row, st));
+        HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
+        HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
+        return cuda_status(launch_convert_dq(p.dq_acc, dq, desc->total_tokens, desc->num_heads,
+                                             desc->d_qk, row, st));
+    }
+    if (tensor_bytes) {
+        HSTU_CUDA(cudaMemsetAsync(dk, 0, tensor_bytes, st));
+        HSTU_CUDA(cudaMemsetAsync(dv, 0, tensor_bytes, st));
+        HSTU_CUDA(cudaMemsetAsync(dq, 0, tensor_bytes, st));
+    }
+    HSTU_TRY(schedule(desc, seq_offsets, num_targets, 0, workspace, st));
+    return cuda_status(launch_attn_bwd_f32(p, grid_items(desc), st));
+}
+
+static hstu_status check_layer_desc(const hstu_layer_desc *d)
+{
+    if (!d)
+        return HSTU_ERR_INVALID_ARG;
+    HSTU_TRY(check_attn_desc(&d->attn));
+    if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps))
+        return HSTU_ERR_INVALID_ARG;
+    const int F = d->attn.num_heads * d->attn.d_v;
+    if (F != 64 && F != 128 && F != 256 && F != 512 && F != 1024)
+        return HSTU_ERR_UNSUPPORTED;
+    if (d->attn.dtype == HSTU_BF16 && (d->d_model % 32 || F % 32))
+        return HSTU_ERR_UNSUPPORTED;
+    return HSTU_OK;
+}
+
+static int layer_width(const hstu_attn_desc *a) { return a->num_heads * (2 * a->d_v + 2 * a->d_qk); }
+
+static size_t layer_ws(const hstu_layer_desc *d, bool keep_uvqk, bool keep_o)
+{
+    const hstu_attn_desc *a = &d->attn;
+    const size_t eb = elem_bytes(a), T = (size_t)a->total_tokens;
+    size_t b = attn_ws(a, 0);
+    if (!keep_uvqk)
+        b += align256(T * layer_width(a) * eb);
+    if (!keep_o)
+        b += align256(T * a->num_heads * a->d_v * eb);
+    b += align256(T * a->num_heads * a->d_v * eb);  // G
+    return b;
+}
+
+hstu_status hstu_layer_workspace_size(const hstu_layer_desc *desc, size_t *bytes)
+{
+    HSTU_TRY(check_layer_desc(desc));
+    if (!bytes)
+        return HSTU_ERR_INVALID_ARG;
+    *bytes = layer_ws(desc, false, false);
+    return HSTU_OK;
+}
+
+hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const void *w1, const void *b1,
+                           const void *w2, const void *b2, const float *ln_gamma, const float *ln_beta,
+                           const int64_t *seq_offsets, const int64_t *timestamps,
+                           const int32_t *num_targets, const float *rab_pos, const float *rab_time,
+                           void *y, void *saved_uvqk, void *saved_o, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    HSTU_TRY(check_layer_desc(desc));
+    const hstu_attn_desc *a = &desc->attn;
+    if (!seq_offsets || !rab_pos || !rab_time || !w1 || !w2 || !ln_gamma || !ln_beta)
+        return HSTU_ERR_INVALID_ARG;
+    if (a->total_tokens > 0 && (!x || !y || !timestamps))
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(y) || !aligned16(saved_uvqk) ||
+        !aligned16(saved_o))
+        return HSTU_ERR_INVALID_ARG;
+    const size_t need = layer_ws(desc, saved_uvqk != nullptr, saved_o != nullptr);
+    HSTU_TRY(check_ws(workspace, workspace_bytes, need));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = a->dtype == HSTU_BF16;
+    const size_t eb = elem_bytes(a), T = (size_t)a->total_tokens;
+    const int W = layer_width(a), hv = a->num_heads * a->d_v, hq = a->num_heads * a->d_qk;
+    const int D = desc->d_model;
+
+    char *cur = static_cast<char *>(workspace) + attn_ws(a, 0);
+    char *uvqk = static_cast<char *>(saved_uvqk);
+    if (!uvqk) {
+        uvqk = cur;
+        cur += align256(T * W * eb);
+    }
+    char *o = static_cast<char *>(saved_o);
+    if (!o) {
+        o = cur;
+        cur += align256(T * hv * eb);
+    }
+    char *g = cur;
+
+    if (bf16)
+        HSTU_CUDA(launch_gemm_bf16(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, st));
+    else
+        HSTU_CUDA(launch_gemm_f32(static_cast<const float *>(x), D, static_cast<const float *>(w1),
+                                  static_cast<const float *>(b1), reinterpret_cast<float *>(uvqk), W,
+                                  (int64_t)T, W, D, true, st));
+    HSTU_TRY(attn_fwd_strided(a, uvqk + (size_t)2 * hv * eb, W, uvqk + (size_t)(2 * hv + hq) * eb, W,
+                              uvqk + (size_t)hv * eb, W, seq_offsets, timestamps, num_targets,
+                              rab_pos, rab_time, o, hv, workspace, st));
+    HSTU_CUDA(launch_norm_gate(bf16, o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv,
+                               (int64_t)T, hv, st));
+    if (bf16)
+        return cuda_status(launch_gemm_bf16(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, st));
+    return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(g), hv,
+                                       static_cast<const float *>(w2), static_cast<const float *>(b2),
+                                       static_cast<float *>(y), D, (int64_t)T, D, hv, false, st));
+}
+
+hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream)
+{
+    if (!workspace)
+        return HSTU_ERR_WORKSPACE;
+    int32_t flag = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    HSTU_CUDA(cudaMemcpyAsync(&flag, workspace, sizeof(flag), cudaMemcpyDeviceToHost, st));
+    HSTU_CUDA(cudaStreamSynchronize(st));
+    if (bits)
+        *bits = flag;
+    return flag ? HSTU_ERR_DEVICE_CHECK : HSTU_OK;
+}
+
+hstu_status hstu_debug_bias_indices(const hstu_attn_desc *desc, const int64_t *seq_offsets,
+                                    const int64_t *timestamps, const int32_t *num_targets,
+                                    const int64_t *rows, int64_t n, int32_t *pos_index,
+                                    int32_t *bucket, void *stream)
+{
+    HSTU_TRY(check_attn_desc(desc));
+    if (n < 0 || (n > 0 && (!seq_offsets || !timestamps || !rows || !pos_index || !bucket)))
+        return HSTU_ERR_INVALID_ARG;
+    return cuda_status(launch_debug_indices(seq_offsets, timestamps, num_targets, desc->num_seqs,
+                                            desc->pos_lo, desc->pos_hi, desc->num_time_buckets, rows,
+                                            n, pos_index, bucket, static_cast<cudaStream_t>(stream)));
+}
+
+hstu_status hstu_debug_schedule(const hstu_attn_desc *desc, const int64_t *seq_offsets,
+                                const int32_t *num_targets, int is_bwd, int32_t tile_rows,
+                                int32_t *items, int32_t max_items_cap, int32_t *count, int32_t *flag,
+                                void *stream)
+{
+    HSTU_TRY(check_attn_desc(desc));
+    if (!seq_offsets || !items || !count || !flag || tile_rows < 1)
+        return HSTU_ERR_INVALID_ARG;
+    if (max_items_cap < max_items(desc->total_tokens, desc->num_seqs, tile_rows))
+        return HSTU_ERR_WORKSPACE;
+    // the header lives in caller memory: `flag` must point at 256 writable bytes
+    return cuda_status(launch_schedule(seq_offsets, num_targets, desc->num_seqs, desc->total_tokens,
+                                       desc->max_seq_len, tile_rows, is_bwd,
+                                       reinterpret_cast<int2 *>(items), max_items_cap,
+                                       reinterpret_cast<WsHeader *>(flag), count,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

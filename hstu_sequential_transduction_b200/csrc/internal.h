@@ -1,0 +1,48 @@
+// Host-side launchers shared between the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hstu {
+
+struct WsHeader;
+struct AttnParams;
+
+// Tile rows of the work items each attention implementation consumes.
+constexpr int kMmaTile = 64;
+
+cudaError_t launch_schedule(const int64_t *off, const int32_t *nt, int B, int64_t T, int max_len,
+                            int tile, int is_bwd, int2 *items, int capacity, WsHeader *hdr,
+                            int32_t *count_out, cudaStream_t stream);
+
+cudaError_t launch_debug_indices(const int64_t *off, const int64_t *ts, const int32_t *nt, int B,
+                                 int lo, int hi, int nb, const int64_t *rows, int64_t n,
+                                 int32_t *pos_out, int32_t *bkt_out, cudaStream_t stream);
+
+// bf16 attention on the legacy tensor-core path (mma.sync), 64-row tiles.
+cudaError_t launch_attn_fwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
+cudaError_t launch_attn_bwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
+
+// fp32 attention on CUDA cores, 64-row tiles.
+cudaError_t launch_attn_fwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
+cudaError_t launch_attn_bwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
+
+// dq (bf16) <- dq_acc (fp32), n elements of rows with stride.
+cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int d, int64_t sdq,
+                              cudaStream_t stream);
+
+// C[M, N] = act(A[M, K] B[K, N] + bias[N]); act = SiLU if silu.  Row strides
+// lda, ldc in elements; B is dense [K, N].
+cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
+                             int64_t ldc, int64_t M, int N, int K, bool silu, cudaStream_t stream);
+cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const float *bias,
+                            float *C, int64_t ldc, int64_t M, int N, int K, bool silu,
+                            cudaStream_t stream);
+
+// G[t, :] = LayerNorm(O[t, :]) * U[t, :] over F features.
+cudaError_t launch_norm_gate(bool bf16, const void *O, int64_t ldo, const void *U, int64_t ldu,
+                             const float *gamma, const float *beta, float eps, void *G,
+                             int64_t ldg, int64_t T, int F, cudaStream_t stream);
+
+}  // namespace hstu

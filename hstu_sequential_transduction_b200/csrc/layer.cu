@@ -1,0 +1,289 @@
+// Projection GEMMs and the LayerNorm-gate of the HSTU transduction layer
+// ("DLRMv4 Brings Sequence-Based Recommendation Training to MLPerf", section
+// "Model Architecture": a projection producing the layer's internal
+// representations, then a gated transformation of the attention output).
+//
+//   f1:   [U | V | Q | K] = SiLU(X W1 + b1)   (bias + SiLU fused in the epilogue;
+//         the four blocks are column ranges of one output, so the attention
+//         reads Q, K, V in place through row strides: no split copies)
+//   gate: G = LayerNorm(O) * U                 (one warp per token, fp32 stats)
+//   f2:   Y = G W2 + b2
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hstu {
+
+namespace {
+
+// ---- bf16 GEMM on the legacy tensor-core path (mma.sync) -------------------
+constexpr int GM = 128, GN = 128, GK = 32, kGemmThreads = 256;
+constexpr int LDA = GK + 8, LDB = GN + 8;
+
+__global__ void __launch_bounds__(kGemmThreads)
+gemm_bf16_kernel(const __nv_bfloat16 *__restrict__ A, int64_t lda, const __nv_bfloat16 *__restrict__ Bm,
+                 const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ C, int64_t ldc,
+                 int64_t M, int N, int K, int silu)
+{
+    __shared__ __align__(16) __nv_bfloat16 sA[2][GM * LDA];
+    __shared__ __align__(16) __nv_bfloat16 sB[2][GK * LDB];
+    const int64_t m0 = (int64_t)blockIdx.y * GM;
+    const int n0 = blockIdx.x * GN;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wm = warp >> 2, wn = warp & 3, g = lane >> 2, t4 = lane & 3, m = lane >> 3;
+
+    auto load = [&](int buf, int k0) {
+        for (int c = threadIdx.x; c < GM * (GK / 8); c += kGemmThreads) {
+            int r = c / (GK / 8), ch = c % (GK / 8);
+            bool ok = m0 + r < M;
+            const __nv_bfloat16 *src = ok ? A + (m0 + r) * lda + k0 + ch * 8 : A;
+            cp_async16(&sA[buf][r * LDA + ch * 8], src, ok ? 16 : 0);
+        }
+        for (int c = threadIdx.x; c < GK * (GN / 8); c += kGemmThreads) {
+            int r = c / (GN / 8), ch = c % (GN / 8);
+            bool ok = n0 + ch * 8 < N;
+            const __nv_bfloat16 *src = ok ? Bm + (int64_t)(k0 + r) * N + n0 + ch * 8 : Bm;
+            cp_async16(&sB[buf][r * LDB + ch * 8], src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+
+    float acc[4][4][4];
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < 4; b++)
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                acc[a][b][e] = 0.f;
+
+    const int nk = K / GK;
+    load(0, 0);
+    for (int kt = 0; kt < nk; kt++) {
+        const int buf = kt & 1;
+        if (kt + 1 < nk) {
+            load(buf ^ 1, (kt + 1) * GK);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < GK / 16; kk++) {
+            uint32_t af[4][4];
+#pragma unroll
+            for (int mi = 0; mi < 4; mi++)
+                ldmatrix_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3],
+                            &sA[buf][(wm * 64 + mi * 16 + (lane & 7) + 8 * (m & 1)) * LDA + kk * 16 + 8 * (m >> 1)]);
+#pragma unroll
+            for (int np = 0; np < 2; np++) {
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(r0, r1, r2, r3,
+                                  &sB[buf][(kk * 16 + (lane & 7) + 8 * (m & 1)) * LDB + wn * 32 + np * 16 + 8 * (m >> 1)]);
+#pragma unroll
+                for (int mi = 0; mi < 4; mi++) {
+                    mma_bf16_16816(acc[mi][2 * np], af[mi], r0, r1);
+                    mma_bf16_16816(acc[mi][2 * np + 1], af[mi], r2, r3);
+                }
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int mi = 0; mi < 4; mi++) {
+#pragma unroll
+        for (int ni = 0; ni < 4; ni++) {
+            const int col = n0 + wn * 32 + ni * 8 + 2 * t4;
+            if (col >= N)
+                continue;
+            const float b0 = bias ? __bfloat162float(bias[col]) : 0.f;
+            const float b1 = bias ? __bfloat162float(bias[col + 1]) : 0.f;
+#pragma unroll
+            for (int a = 0; a < 2; a++) {
+                const int64_t row = m0 + wm * 64 + mi * 16 + g + 8 * a;
+                if (row >= M)
+                    continue;
+                float x0 = acc[mi][ni][2 * a] + b0, x1 = acc[mi][ni][2 * a + 1] + b1;
+                if (silu) {
+                    x0 = silu_fast(x0);
+                    x1 = silu_fast(x1);
+                }
+                *reinterpret_cast<uint32_t *>(C + row * ldc + col) = pack_bf16(x0, x1);
+            }
+        }
+    }
+}
+
+// ---- fp32 GEMM on CUDA cores ---------------------------------------------------
+constexpr int FT = 64, FK = 16;
+
+__global__ void __launch_bounds__(256)
+gemm_f32_kernel(const float *__restrict__ A, int64_t lda, const float *__restrict__ Bm,
+                const float *__restrict__ bias, float *__restrict__ C, int64_t ldc, int64_t M, int N,
+                int K, int silu)
+{
+    __shared__ float sA[FK][FT + 1];
+    __shared__ float sB[FK][FT];
+    const int64_t m0 = (int64_t)blockIdx.y * FT;
+    const int n0 = blockIdx.x * FT;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += FK) {
+        for (int e = threadIdx.x; e < FT * FK; e += 256) {
+            int r = e / FK, c = e % FK;
+            sA[c][r] = (m0 + r < M && k0 + c < K) ? A[(m0 + r) * lda + k0 + c] : 0.f;
+            int rb = e / FT, cb = e % FT;
+            sB[rb][cb] = (k0 + rb < K && n0 + cb < N) ? Bm[(int64_t)(k0 + rb) * N + n0 + cb] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < FK; kk++) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                a[i] = sA[kk][ty * 4 + i];
+                b[i] = sB[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int64_t row = m0 + ty * 4 + i;
+        if (row >= M)
+            continue;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int col = n0 + tx * 4 + j;
+            if (col >= N)
+                continue;
+            float x = acc[i][j] + (bias ? bias[col] : 0.f);
+            C[row * ldc + col] = silu ? silu_precise(x) : x;
+        }
+    }
+}
+
+// ---- LayerNorm(O) * U ----------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float ld(const T *p);
+template <>
+__device__ __forceinline__ float ld<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+template <typename T>
+__device__ __forceinline__ void st(T *p, float v);
+template <>
+__device__ __forceinline__ void st<float>(float *p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// One warp per token; lane l holds features l*VPT .. l*VPT + VPT - 1.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256)
+norm_gate_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, int64_t ldu,
+                 const float *__restrict__ gamma, const float *__restrict__ beta, float eps,
+                 T *__restrict__ G, int64_t ldg, int64_t Trows)
+{
+    constexpr int F = 32 * VPT;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (row >= Trows)
+        return;
+    const T *o = O + row * ldo + lane * VPT;
+    float x[VPT];
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < VPT; e++) {
+        x[e] = ld<T>(o + e);
+        sum += x[e];
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float mean = sum * (1.0f / F);
+    float var = 0.f;
+#pragma unroll
+    for (int e = 0; e < VPT; e++) {
+        const float d = x[e] - mean;
+        var += d * d;
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1)
+        var += __shfl_xor_sync(0xffffffffu, var, off);
+    const float rstd = rsqrtf(var * (1.0f / F) + eps);
+    const T *u = U + row * ldu + lane * VPT;
+    T *gout = G + row * ldg + lane * VPT;
+#pragma unroll
+    for (int e = 0; e < VPT; e++) {
+        const int c = lane * VPT + e;
+        const float y = ((x[e] - mean) * rstd * gamma[c] + beta[c]) * ld<T>(u + e);
+        st<T>(gout + e, y);
+    }
+}
+
+template <typename T>
+cudaError_t norm_gate_t(const T *O, int64_t ldo, const T *U, int64_t ldu, const float *gamma,
+                        const float *beta, float eps, T *G, int64_t ldg, int64_t Trows, int F,
+                        cudaStream_t stream)
+{
+    const int64_t threads = Trows * 32;
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    switch (F) {
+    case 64: norm_gate_kernel<T, 2><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 128: norm_gate_kernel<T, 4><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 256: norm_gate_kernel<T, 8><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 512: norm_gate_kernel<T, 16><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 1024: norm_gate_kernel<T, 32><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
+                             int64_t ldc, int64_t M, int N, int K, bool silu, cudaStream_t stream)
+{
+    if (M == 0)
+        return cudaSuccess;
+    if (K % GK || N % 8)
+        return cudaErrorInvalidValue;
+    dim3 grid((N + GN - 1) / GN, (unsigned)((M + GM - 1) / GM));
+    gemm_bf16_kernel<<<grid, kGemmThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(A), lda, static_cast<const __nv_bfloat16 *>(Bm),
+        static_cast<const __nv_bfloat16 *>(bias), static_cast<__nv_bfloat16 *>(C), ldc, M, N, K, silu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const float *bias,
+                            float *C, int64_t ldc, int64_t M, int N, int K, bool silu,
+                            cudaStream_t stream)
+{
+    if (M == 0)
+        return cudaSuccess;
+    dim3 grid((N + FT - 1) / FT, (unsigned)((M + FT - 1) / FT));
+    gemm_f32_kernel<<<grid, 256, 0, stream>>>(A, lda, Bm, bias, C, ldc, M, N, K, silu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_gate(bool bf16, const void *O, int64_t ldo, const void *U, int64_t ldu,
+                             const float *gamma, const float *beta, float eps, void *G,
+                             int64_t ldg, int64_t T, int F, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    if (bf16)
+        return norm_gate_t(static_cast<const __nv_bfloat16 *>(O), ldo, static_cast<const __nv_bfloat16 *>(U),
+                           ldu, gamma, beta, eps, static_cast<__nv_bfloat16 *>(G), ldg, T, F, stream);
+    return norm_gate_t(static_cast<const float *>(O), ldo, static_cast<const float *>(U), ldu, gamma,
+                       beta, eps, static_cast<float *>(G), ldg, T, F, stream);
+}
+
+}  // namespace hstu

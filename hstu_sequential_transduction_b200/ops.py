@@ -1,0 +1,253 @@
+"""Python binding of libhstu (ctypes): argument marshalling only.
+
+Every function here has the name of the C entry point it calls (include/hstu.h)
+and does no arithmetic of the method: it checks tensor placement, allocates
+outputs and workspace through PyTorch's allocator, and passes raw device
+pointers plus the current CUDA stream.  There is no fallback: if the library
+cannot be loaded or built, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+HSTU_F32, HSTU_BF16 = 0, 1
+STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3: "HSTU_ERR_WORKSPACE",
+          4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_DEVICE_CHECK"}
+
+EXPORTED = ["hstu_status_string", "hstu_version", "hstu_attn_workspace_size",
+            "hstu_layer_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd",
+            "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule"]
+
+
+class HstuError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+class hstu_attn_desc(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
+                ("total_tokens", ctypes.c_int64), ("num_heads", ctypes.c_int32),
+                ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("inv_n", ctypes.c_float), ("pos_lo", ctypes.c_int32), ("pos_hi", ctypes.c_int32),
+                ("num_time_buckets", ctypes.c_int32), ("debug_checks", ctypes.c_int32)]
+
+
+class hstu_layer_desc(ctypes.Structure):
+    _fields_ = [("attn", hstu_attn_desc), ("d_model", ctypes.c_int32), ("ln_eps", ctypes.c_float)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(allow_build: bool = True) -> ctypes.CDLL:
+    """Load libhstu.so, compiling it first when it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if allow_build and _build.needs_build():
+                _build.build()
+            if not os.path.exists(_build.LIB):
+                raise RuntimeError(f"libhstu.so not found at {_build.LIB}; build it with "
+                                   "python -m hstu_sequential_transduction_b200.build")
+            lib = ctypes.CDLL(_build.LIB)
+            lib.hstu_status_string.restype = ctypes.c_char_p
+            lib.hstu_status_string.argtypes = [ctypes.c_int]
+            lib.hstu_version.restype = ctypes.c_int
+            for name in EXPORTED[2:]:
+                getattr(lib, name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise HstuError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HSTU_BF16
+    if t.dtype == torch.float32:
+        return HSTU_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def make_attn_desc(num_seqs, max_seq_len, total_tokens, num_heads, d_qk, d_v, dtype, inv_n,
+                   pos_lo, pos_hi, num_time_buckets) -> hstu_attn_desc:
+    return hstu_attn_desc(int(num_seqs), int(max_seq_len), int(total_tokens), int(num_heads),
+                          int(d_qk), int(d_v), int(dtype), float(inv_n), int(pos_lo), int(pos_hi),
+                          int(num_time_buckets), 0)
+
+
+def hstu_status_string(status: int) -> str:
+    return load_library().hstu_status_string(int(status)).decode()
+
+
+def hstu_version() -> int:
+    return load_library().hstu_version()
+
+
+def hstu_attn_workspace_size(desc: hstu_attn_desc, is_bwd: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check("hstu_attn_workspace_size",
+           load_library().hstu_attn_workspace_size(ctypes.byref(desc), int(is_bwd), ctypes.byref(n)))
+    return n.value
+
+
+def hstu_layer_workspace_size(desc: hstu_layer_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("hstu_layer_workspace_size",
+           load_library().hstu_layer_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time):
+    return make_attn_desc(seq_offsets.numel() - 1, max_seq_len, q.shape[0], q.shape[1], q.shape[2],
+                          v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, rab_time.numel())
+
+
+def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, *,
+                  max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, out=None,
+                  workspace=None, stream=None):
+    """O = jagged SiLU attention; q, k [T, H, d_qk], v [T, H, d_v] on CUDA."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _dev(t, name, q.dtype)
+    _dev(seq_offsets, "seq_offsets", torch.int64)
+    _dev(timestamps, "timestamps", torch.int64)
+    _dev(num_targets, "num_targets", torch.int32)
+    _dev(rab_pos, "rab_pos", torch.float32)
+    _dev(rab_time, "rab_time", torch.float32)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    if out is None:
+        out = torch.empty_like(v)
+    _dev(out, "out", q.dtype)
+    need = hstu_attn_workspace_size(desc, False)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check("hstu_attn_fwd", load_library().hstu_attn_fwd(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(timestamps),
+        _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), _stream(stream)))
+    return out
+
+
+def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, dout, *,
+                  max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, grads=None,
+                  workspace=None, stream=None):
+    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _dev(t, name, q.dtype)
+    _dev(seq_offsets, "seq_offsets", torch.int64)
+    _dev(timestamps, "timestamps", torch.int64)
+    _dev(num_targets, "num_targets", torch.int32)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty_like(rab_pos), torch.empty_like(rab_time))
+    dq, dk, dv, drp, drt = grads
+    need = hstu_attn_workspace_size(desc, True)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check("hstu_attn_bwd", load_library().hstu_attn_bwd(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(timestamps),
+        _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(drp), _ptr(drt), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream)))
+    return dq, dk, dv, drp, drt
+
+
+def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets,
+                   rab_pos, rab_time, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
+                   inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, y=None,
+                   saved_uvqk=None, saved_o=None, workspace=None, stream=None):
+    """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer."""
+    for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("b2", b2)):
+        _dev(t, name, x.dtype)
+    _dev(ln_gamma, "ln_gamma", torch.float32)
+    _dev(ln_beta, "ln_beta", torch.float32)
+    T, D = x.shape
+    attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
+    desc = hstu_layer_desc(attn, int(D), float(ln_eps))
+    if y is None:
+        y = torch.empty((T, D), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(hstu_layer_workspace_size(desc), x.device)
+    _check("hstu_layer_fwd", load_library().hstu_layer_fwd(
+        ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(ln_gamma),
+        _ptr(ln_beta), _ptr(seq_offsets), _ptr(timestamps), _ptr(num_targets), _ptr(rab_pos),
+        _ptr(rab_time), _ptr(y), _ptr(saved_uvqk), _ptr(saved_o), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), _stream(stream)))
+    return y
+
+
+def hstu_check_device_flag(workspace: torch.Tensor, stream=None):
+    """(status, bits) of the device input check of the last call on `workspace`."""
+    bits = ctypes.c_int32(0)
+    st = load_library().hstu_check_device_flag(_ptr(workspace), ctypes.byref(bits), _stream(stream))
+    return st, bits.value
+
+
+def hstu_debug_bias_indices(desc: hstu_attn_desc, seq_offsets, timestamps, num_targets, rows,
+                            stream=None):
+    n = rows.shape[0]
+    pos = torch.empty(n, dtype=torch.int32, device=rows.device)
+    bkt = torch.empty(n, dtype=torch.int32, device=rows.device)
+    _check("hstu_debug_bias_indices", load_library().hstu_debug_bias_indices(
+        ctypes.byref(desc), _ptr(seq_offsets), _ptr(timestamps), _ptr(num_targets), _ptr(rows),
+        ctypes.c_int64(n), _ptr(pos), _ptr(bkt), _stream(stream)))
+    return pos, bkt
+
+
+def hstu_debug_schedule(desc: hstu_attn_desc, seq_offsets, num_targets, is_bwd: bool,
+                        tile_rows: int, stream=None):
+    T, B = desc.total_tokens, desc.num_seqs
+    cap = (T + tile_rows - 1) // tile_rows + B
+    dev = seq_offsets.device
+    items = torch.full((max(cap, 1), 2), -1, dtype=torch.int32, device=dev)
+    count = torch.zeros(1, dtype=torch.int32, device=dev)
+    hdr = torch.zeros(64, dtype=torch.int32, device=dev)
+    _check("hstu_debug_schedule", load_library().hstu_debug_schedule(
+        ctypes.byref(desc), _ptr(seq_offsets), _ptr(num_targets), int(is_bwd), int(tile_rows),
+        _ptr(items), ctypes.c_int32(cap), _ptr(count), _ptr(hdr), _stream(stream)))
+    return items, count, hdr

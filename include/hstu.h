@@ -1,0 +1,181 @@
+/*
+ * libhstu: B200 (sm_100a) HSTU jagged pointwise attention and transduction layer.
+ *
+ * What the calls compute (sources: "NVIDIA generative recommenders" summary,
+ * section "HSTU Architecture"; "DLRMv4 Brings Sequence-Based Recommendation
+ * Training to MLPerf", sections "Model Architecture", "HSTU Hyperparameters"
+ * and "Computation Cost Analysis", Table 7):
+ *
+ *   for each sequence b (rows seq_offsets[b] .. seq_offsets[b+1]-1, local i, j)
+ *   and each head:
+ *     s_ij = q_i . k_j + rab_pos[clamp(p_i - p_j, pos_lo, pos_hi) - pos_lo]
+ *                      + rab_time[min(NB-1, floor(log2(1 + max(t_i - t_j, 0))))]
+ *     P_ij = SiLU(s_ij) * inv_n   if key j is visible from query i, else 0
+ *     O_i  = sum_j P_ij v_j
+ *   visibility: with n_t = num_targets[b] (0 when num_targets is NULL) the last
+ *   n_t tokens are candidates; history rows see j <= i, candidate rows see the
+ *   whole history and themselves.  p_i = i for history tokens and
+ *   L_b - n_t for candidates.  Timestamps are integer seconds.
+ *
+ *   Layer: [U | V | Q | K] = SiLU(X W1 + b1) (column blocks in that order, each
+ *   [T, H, d] with d fastest); O = attention(Q, K, V);
+ *   G = LayerNorm_{H*d_v}(O; gamma, beta, eps) * U;  Y = G W2 + b2.
+ *
+ * Conventions for every call:
+ *  - Pointers to tensors are DEVICE pointers; descriptors and size outputs are
+ *    host memory.  The caller owns every buffer; the library allocates nothing
+ *    and keeps no state between calls.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously; no call synchronizes the host except
+ *    hstu_check_device_flag.
+ *  - Layouts: values are row-major jagged [T, H, d] (T = seq_offsets[B]),
+ *    seq_offsets int64 [B+1], timestamps int64 [T], num_targets int32 [B] or
+ *    NULL, rab_pos float32 [pos_hi - pos_lo + 1], rab_time float32 [NB].
+ *    Weights are row-major.  dtype HSTU_BF16 means bf16 values/weights with
+ *    fp32 accumulation (P is rounded to bf16 before P V); HSTU_F32 is fp32
+ *    throughout.
+ *  - Argument errors are found on the host before any launch and return
+ *    HSTU_ERR_INVALID_ARG / HSTU_ERR_UNSUPPORTED / HSTU_ERR_WORKSPACE with
+ *    nothing enqueued.  Inconsistent device data (seq_offsets not starting at 0,
+ *    decreasing, exceeding T or max_seq_len; num_targets outside [0, L_b])
+ *    never faults: the scheduler drops the offending sequences and records a
+ *    flag in the workspace, which hstu_check_device_flag reports.  Kernels
+ *    never trap.
+ */
+#ifndef HSTU_H
+#define HSTU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HSTU_OK = 0,
+    HSTU_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad range */
+    HSTU_ERR_UNSUPPORTED = 2,  /* head dims other than 32/64/128, d_qk != d_v, ... */
+    HSTU_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+    HSTU_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+    HSTU_ERR_DEVICE_CHECK = 5  /* the device-side input check flagged the last call */
+} hstu_status;
+
+typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype;
+
+typedef struct {
+    int32_t num_seqs;         /* B >= 0 */
+    int32_t max_seq_len;      /* >= every L_b; sizes the schedule */
+    int64_t total_tokens;     /* T = seq_offsets[B] */
+    int32_t num_heads;        /* H >= 1 */
+    int32_t d_qk;             /* per-head query/key width: 32, 64 or 128 */
+    int32_t d_v;              /* per-head value width: equal to d_qk */
+    int32_t dtype;            /* hstu_dtype of q, k, v, out and their gradients */
+    float inv_n;              /* the 1/N scale applied after SiLU */
+    int32_t pos_lo, pos_hi;   /* rab_pos covers distances pos_lo..pos_hi */
+    int32_t num_time_buckets; /* NB >= 1 */
+    int32_t debug_checks;     /* reserved; device input checks always run */
+} hstu_attn_desc;
+
+typedef struct {
+    hstu_attn_desc attn;      /* attention part; dtype also types x, w1, b1, w2, b2, y */
+    int32_t d_model;          /* D: width of X and Y (a multiple of 32 for bf16) */
+    float ln_eps;             /* LayerNorm epsilon (1e-5 in the workloads) */
+} hstu_layer_desc;
+
+/* Human-readable name of a status code (static string). */
+const char *hstu_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int hstu_version(void);
+
+/*
+ * Bytes of device workspace an attention call needs (is_bwd = 0 forward,
+ * 1 backward).  The workspace must be 256-byte aligned; its contents need no
+ * initialisation and are scratch between calls.
+ */
+hstu_status hstu_attn_workspace_size(const hstu_attn_desc *desc, int is_bwd, size_t *bytes);
+
+/* Bytes of device workspace hstu_layer_fwd needs. */
+hstu_status hstu_layer_workspace_size(const hstu_layer_desc *desc, size_t *bytes);
+
+/*
+ * Attention forward: out[T, H, d_v] (overwritten; rows of all sequences
+ * written, including empty-attention rows, which are zero).
+ * q, k: [T, H, d_qk]; v, out: [T, H, d_v], all of desc->dtype.
+ */
+hstu_status hstu_attn_fwd(const hstu_attn_desc *desc, const void *q, const void *k,
+                          const void *v, const int64_t *seq_offsets, const int64_t *timestamps,
+                          const int32_t *num_targets, const float *rab_pos,
+                          const float *rab_time, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * Attention backward for the loss sum(O * dout): dq, dk [T, H, d_qk],
+ * dv [T, H, d_v] (desc->dtype) and the float32 bias-table gradients
+ * d_rab_pos [pos_hi - pos_lo + 1], d_rab_time [NB], summed over all pairs and
+ * heads.  Every output is overwritten, not accumulated.  The pair
+ * gradient is dS_ij = (dout_i . v_j) * SiLU'(s_ij) * inv_n.
+ */
+hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void *k,
+                          const void *v, const int64_t *seq_offsets, const int64_t *timestamps,
+                          const int32_t *num_targets, const float *rab_pos,
+                          const float *rab_time, const void *dout, void *dq, void *dk, void *dv,
+                          float *d_rab_pos, float *d_rab_time, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * One transduction layer forward.  x [T, D]; w1 [D, H(2 d_v + 2 d_qk)];
+ * b1 [H(2 d_v + 2 d_qk)]; w2 [H d_v, D]; b2 [D] (dtype of the desc);
+ * ln_gamma, ln_beta float32 [H d_v]; y [T, D] (overwritten).
+ * saved_uvqk [T, H(2 d_v + 2 d_qk)] and saved_o [T, H d_v] are optional
+ * (NULL = not kept); when given they receive SiLU(X W1 + b1) and the
+ * attention output, as a training step would keep them.
+ */
+hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const void *w1,
+                           const void *b1, const void *w2, const void *b2,
+                           const float *ln_gamma, const float *ln_beta,
+                           const int64_t *seq_offsets, const int64_t *timestamps,
+                           const int32_t *num_targets, const float *rab_pos,
+                           const float *rab_time, void *y, void *saved_uvqk, void *saved_o,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronizes `stream` and reports the device-side input check of the most
+ * recent call that used `workspace`: HSTU_OK or HSTU_ERR_DEVICE_CHECK.  The
+ * flag's bits (1 = seq_offsets[0] != 0, 2 = a sequence decreasing or past T,
+ * 4 = a sequence longer than max_seq_len, 8 = num_targets outside [0, L_b],
+ * 16 = seq_offsets[B] != T) are stored in *bits when bits is not NULL.
+ */
+hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream);
+
+/*
+ * Test hook: the bias indices the attention kernels use for n global token
+ * pairs (rows[2e], rows[2e+1]) = (i, j) of the same sequence.  Writes
+ * pos_index[e] = clamp(p_i - p_j, lo, hi) - lo and bucket[e] (int32, device).
+ * Pairs whose rows lie in different sequences get -1 in both outputs.
+ */
+hstu_status hstu_debug_bias_indices(const hstu_attn_desc *desc, const int64_t *seq_offsets,
+                                    const int64_t *timestamps, const int32_t *num_targets,
+                                    const int64_t *rows, int64_t n, int32_t *pos_index,
+                                    int32_t *bucket, void *stream);
+
+/*
+ * Test hook: run the jagged tile scheduler alone.  Writes the work list the
+ * attention kernels consume, as int32 pairs (sequence, tile) in processing
+ * order, into items[2 * max_items] and the count into *count (device).
+ * `flag` is a device buffer of at least 256 bytes (the workspace header);
+ * its first int32 receives the input-check bits.  Forward tiles are query
+ * tiles of `tile_rows` rows; backward tiles are key tiles.  Returns
+ * HSTU_ERR_WORKSPACE if max_items is below the bound ceil(T / tile_rows) + B.
+ */
+hstu_status hstu_debug_schedule(const hstu_attn_desc *desc, const int64_t *seq_offsets,
+                                const int32_t *num_targets, int is_bwd, int32_t tile_rows,
+                                int32_t *items, int32_t max_items, int32_t *count,
+                                int32_t *flag, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H */
