@@ -122,8 +122,9 @@ def test_device_flag_reports_bad_offsets_without_fault(cuda_device):
                               inp.pos_hi, inp.rab_time.numel())
     ws = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc, False), cuda_device)
     out = torch.zeros_like(d["v"])
+    kw = dict(attn_kwargs(inp), max_seq_len=128)
     ops.hstu_attn_fwd(d["q"], d["k"], d["v"], bad_off, d["timestamps"], None, d["rab_pos"],
-                      d["rab_time"], out=out, workspace=ws, **attn_kwargs(inp))
+                      d["rab_time"], out=out, workspace=ws, **kw)
     st, bits = ops.hstu_check_device_flag(ws)
     assert st == 5 and bits & 2 and bits & 16
     # the valid first sequence was still computed
@@ -132,7 +133,7 @@ def test_device_flag_reports_bad_offsets_without_fault(cuda_device):
     assert_bf16_close(out[:80], ref, what="valid sequence")
     # a correct call clears the flag
     ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None, d["rab_pos"],
-                      d["rab_time"], out=out, workspace=ws, **attn_kwargs(inp))
+                      d["rab_time"], out=out, workspace=ws, **kw)
     assert ops.hstu_check_device_flag(ws) == (0, 0)
 
 
