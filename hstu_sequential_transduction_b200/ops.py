@@ -24,7 +24,8 @@ STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3:
 
 EXPORTED = ["hstu_status_string", "hstu_version", "hstu_attn_workspace_size",
             "hstu_layer_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd",
-            "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule"]
+            "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule",
+            "hstu_attn_fwd_noalloc"]
 
 
 class HstuError(RuntimeError):
@@ -169,6 +170,18 @@ def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(timestamps),
         _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(workspace),
         ctypes.c_size_t(workspace.numel()), _stream(stream)))
+    return out
+
+
+def hstu_attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, out,
+                          *, max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, stream=None):
+    """hstu_attn_fwd without a workspace: the library keeps the scheduler's
+    scratch in a static device array (for callers that cannot allocate).
+    `out` must be preallocated; nothing is allocated here either."""
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    _check("hstu_attn_fwd_noalloc", load_library().hstu_attn_fwd_noalloc(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(timestamps),
+        _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _stream(stream)))
     return out
 
 

@@ -141,6 +141,29 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Attention forward that allocates nothing (no counterpart on the HSTU
+ * pages; it exists for callers, not for the method).  Same computation,
+ * arguments and layouts as hstu_attn_fwd, without the workspace: some callers
+ * cannot allocate device memory at all, such as a plugin inside a host
+ * framework that owns every device allocation and passes it only input and
+ * output buffers, or a latency-critical path that may not call cudaMalloc
+ * because it can synchronize the device.  The scheduler's scratch lives in a
+ * static device array of about 512 KiB that every GPU loading this library
+ * holds until exit; problems needing more than 65536 work items
+ * (ceil(T / 64) + B) return HSTU_ERR_UNSUPPORTED before anything is enqueued.
+ * The first call on each device looks the array's address up (with that
+ * device current) and should come before any stream capture.  Calls share
+ * the array, so calls that overlap on the GPU race and must be serialized by
+ * the caller.  The device input-check flag is kept in that array and is not
+ * reported; inconsistent sequences are still dropped, never read out of range.
+ */
+hstu_status hstu_attn_fwd_noalloc(const hstu_attn_desc *desc, const void *q, const void *k,
+                                  const void *v, const int64_t *seq_offsets,
+                                  const int64_t *timestamps, const int32_t *num_targets,
+                                  const float *rab_pos, const float *rab_time, void *out,
+                                  void *stream);
+
+/*
  * Synchronizes `stream` and reports the device-side input check of the most
  * recent call that used `workspace`: HSTU_OK or HSTU_ERR_DEVICE_CHECK.  The
  * flag's bits (1 = seq_offsets[0] != 0, 2 = a sequence decreasing or past T,
