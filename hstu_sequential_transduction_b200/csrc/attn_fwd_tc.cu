@@ -1,0 +1,404 @@
+// HSTU jagged attention forward on sm_100a: TMA + tcgen05 (TMEM) kernel.
+//
+// Computes, per (sequence, 128-row query tile, head) work item,
+//   O = inv_n * sum_j SiLU(Q K_j^T + rab_pos + rab_time) V_j
+// over the visible 128-row key tiles j (the pointwise attention of the
+// "HSTU Architecture" section; causal block with appended candidates of the
+// DLRMv4 page's "Model Architecture" section).  No score matrix reaches HBM.
+//
+// Warp roles (320 threads):
+//   warp 0     TMA producer: Q once, then K_j and V_j into two-stage rings
+//              (separate K and V rings, so K_{j+2} loads as soon as S_j is done);
+//   warp 1     owns TMEM (512 columns) and issues every tcgen05.mma from one
+//              thread: S_j = Q K_j^T into one of two S buffers, O += P_j V_j;
+//   warps 2-9  epilogue: two warpgroups, each takes 64 of the 128 key columns
+//              of every S tile: tcgen05.ld, relative bias, SiLU, bf16 pack, and
+//              the swizzled store of P into shared memory (the A operand of
+//              P V); at the end they read O from TMEM and write it out.
+// TMEM columns: S buffers [0,128) and [128,256), O [256, 256 + D).
+//
+// Epilogue arithmetic on full tiles (every pair visible, timestamps of the
+// tile within 2^24 s of the query tile's first stamp):
+//   h = s/2 + rab_pos/2 + rab_time/2       (tables pre-halved, exact)
+//   SiLU(x) = x sigma(x) = h (1 + tanh h)  (one MUFU tanh per score)
+// The positional term reads a per-tile 256-entry window of the clamped table
+// (index p_i - p_j, contiguous per row).  The temporal bucket
+// floor(log2(1 + dt)) is the exponent of the fp32 difference (t_i + 1) - t_j
+// of rebased stamps, computed with round-toward-zero so the exponent is exact,
+// and a 512-entry table indexed by sign+exponent maps it to rab_time/2.
+// Diagonal, ragged and candidate tiles, and tiles whose stamps span more than
+// 2^24 s, take the general path (per-pair visibility, exact int64 bucket).
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr int TBM = 128, TBN = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreadsTc = kEpiThreads + 64;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kRegion = 16384;  // one 128-row x 128-byte swizzled region
+
+enum Bars { Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, S_FREE = 11,
+            P_FULL = 13, P_FREE = 14, O_FULL = 15, NBARS = 16 };
+
+template <int D>
+struct FwdLayout {
+    static constexpr int NREG = D / 64;
+    static constexpr int TILE = NREG * kRegion;
+    static constexpr int Q = 0;
+    static constexpr int K0 = Q + TILE;
+    static constexpr int V0 = K0 + 2 * TILE;
+    static constexpr int P = V0 + 2 * TILE;
+    static constexpr int E = P + 2 * kRegion;
+    static constexpr int W = E + 512 * 4;
+    static constexpr int TJ = W + 2 * 256 * 4;
+    static constexpr int BAR = TJ + 2 * 128 * 4;
+    static constexpr int MISC = BAR + NBARS * 8;
+    static constexpr int BYTES = MISC + 64;
+};
+
+__device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float *E)
+{
+    const float d = __fsub_rz(ti1, tj);
+    const uint32_t off = (__float_as_uint(d) >> 21) & 0x7FCu;
+    return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(E) + off);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
+                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv)
+{
+    using LY = FwdLayout<D>;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+
+    const int item = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    if (item >= p.hdr->n_items)
+        return;
+    const int2 it = p.items[item];
+    const int qt = it.y;
+    const int64_t s0 = p.seq_offsets[it.x];
+    const int L = (int)(p.seq_offsets[it.x + 1] - s0);
+    const int hist = L - (p.num_targets ? p.num_targets[it.x] : 0);
+    const int i0 = qt * TBM;
+    const int nh = (hist + TBN - 1) / TBN;
+    const int nfull = min(qt + 1, nh);
+    const int ntiles = nfull + (qt >= nh ? 1 : 0);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int i) { return base + LY::BAR + 8u * i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + LY::MISC + 8);
+    float *E = reinterpret_cast<float *>(sm + LY::E);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NBARS; i++) {
+            const bool epi = (i == S_FREE || i == S_FREE + 1 || i == P_FULL);
+            mbar_init(bar(i), epi ? kEpiWarps : 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tq);
+        tma_prefetch(&tk);
+        tma_prefetch(&tv);
+    }
+    if (warp == 1)
+        tmem_alloc(base + LY::MISC, kTmemCols);
+    if (warp >= 2) {
+        // expanded time table: index = sign:exponent of the fp32 (1 + dt)
+        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreads) {
+            const int bkt = (e >= 256 || e < 127) ? 0 : min(e - 127, p.nb - 1);
+            E[e] = 0.5f * p.rab_time[bkt];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + LY::MISC);
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            mbar_expect_tx(bar(Q_FULL), LY::TILE);
+            for (int r = 0; r < LY::NREG; r++)
+                tma_load_2d(base + LY::Q + r * kRegion, &tq, h * D + 64 * r, (int)(s0 + i0), bar(Q_FULL));
+            for (int t = 0; t < ntiles; t++) {
+                const int s = t & 1;
+                const int j0 = (t < nfull ? t : qt) * TBN;
+                if (t >= 2 && !mbar_wait(bar(K_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, p.hdr))
+                    break;
+                mbar_expect_tx(bar(K_FULL + s), LY::TILE);
+                for (int r = 0; r < LY::NREG; r++)
+                    tma_load_2d(base + LY::K0 + s * LY::TILE + r * kRegion, &tk, h * D + 64 * r,
+                                (int)(s0 + j0), bar(K_FULL + s));
+                if (t >= 2 && !mbar_wait(bar(V_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, p.hdr))
+                    break;
+                mbar_expect_tx(bar(V_FULL + s), LY::TILE);
+                for (int r = 0; r < LY::NREG; r++)
+                    tma_load_2d(base + LY::V0 + s * LY::TILE + r * kRegion, &tv, h * D + 64 * r,
+                                (int)(s0 + j0), bar(V_FULL + s));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(TBM, TBN, 0, 0);
+            constexpr uint32_t idO = idesc_bf16(TBM, D, 0, 1);
+            auto issue_S = [&](int t) {
+                const int s = t & 1;
+                for (int ks = 0; ks < D / 16; ks++) {
+                    const uint32_t off = (ks >> 2) * kRegion + (ks & 3) * 32;
+                    const uint64_t a = smem_desc_sw128(base + LY::Q + off, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(base + LY::K0 + s * LY::TILE + off, 16, 1024);
+                    umma_bf16(tmem + s * TBN, a, b, idS, ks > 0);
+                }
+                umma_commit(bar(K_EMPTY + s));
+                umma_commit(bar(S_FULL + s));
+            };
+            auto issue_PV = [&](int t) {
+                const int s = t & 1;
+                for (int ks = 0; ks < TBN / 16; ks++) {
+                    const uint64_t a = smem_desc_sw128(base + LY::P + (ks >> 2) * kRegion + (ks & 3) * 32, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(base + LY::V0 + s * LY::TILE + ks * 2048, kRegion, 1024);
+                    umma_bf16(tmem + 2 * TBN, a, b, idO, (t > 0 || ks > 0));
+                }
+                umma_commit(bar(V_EMPTY + s));
+                umma_commit(bar(P_FREE));
+            };
+            bool ok = mbar_wait(bar(Q_FULL), 0, abort_flag, p.hdr);
+            for (int t = 0; ok && t < min(2, ntiles); t++) {
+                ok = mbar_wait(bar(K_FULL + t), 0, abort_flag, p.hdr);
+                if (ok) {
+                    tc_fence_after();
+                    issue_S(t);
+                }
+            }
+            for (int j = 0; ok && j < ntiles; j++) {
+                ok = mbar_wait(bar(P_FULL), j & 1, abort_flag, p.hdr) &&
+                     mbar_wait(bar(V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                issue_PV(j);
+                if (j + 2 < ntiles) {
+                    ok = mbar_wait(bar(S_FREE + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr) &&
+                         mbar_wait(bar(K_FULL + (j & 1)), ((j + 2) >> 1) & 1, abort_flag, p.hdr);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    issue_S(j + 2);
+                }
+            }
+            umma_commit(bar(O_FULL));
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
+        const int etid = threadIdx.x - 64;
+        const int r = quarter * 32 + lane;
+        const int i = i0 + r;
+        const bool row_ok = i < L;
+        const int64_t tb = p.timestamps[s0 + i0];
+        const int64_t ti = row_ok ? p.timestamps[s0 + i] : tb;
+        const int pi = token_pos(i, hist);
+        const int pmin = token_pos(i0, hist);
+        const int64_t lim = (int64_t)1 << 24;
+        const int qbad = named_bar_or(1, kEpiThreads, (ti - tb + 1 >= lim) || (ti - tb + 1 <= -lim));
+        const float ti1f = (float)(ti - tb + 1);
+        float *Wb = reinterpret_cast<float *>(sm + LY::W);
+        float *TJb = reinterpret_cast<float *>(sm + LY::TJ);
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+
+        float wreg = 0.f;
+        int64_t treg = tb;
+        auto prep = [&](int t) {
+            const int j0 = (t < nfull ? t : qt) * TBN;
+            int d = pmin - j0 - 127 + etid;
+            d = d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d);
+            wreg = 0.5f * p.rab_pos[d - p.pos_lo];
+            if (etid < TBN) {
+                const int j = j0 + etid;
+                treg = j < L ? p.timestamps[s0 + j] : tb;
+            }
+        };
+        prep(0);
+        bool ok = true;
+        for (int t = 0; t < ntiles; t++) {
+            const int s = t & 1;
+            const int j0 = (t < nfull ? t : qt) * TBN;
+            Wb[s * 256 + etid] = wreg;
+            int kbad = 0;
+            if (etid < TBN) {
+                const int64_t dt = treg - tb;
+                kbad = dt >= lim || dt <= -lim;
+                TJb[s * TBN + etid] = (float)dt;
+            }
+            const bool slow_time = named_bar_or(1, kEpiThreads, kbad) || qbad;
+            const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0);
+            if (t + 1 < ntiles)
+                prep(t + 1);
+
+            if (!(ok = mbar_wait(bar(S_FULL + s), (t >> 1) & 1, abort_flag, p.hdr)))
+                break;
+            tc_fence_after();
+            float sv[64];
+            tmem_ld32(trow + s * TBN + 64 * g, sv);
+            tmem_ld32(trow + s * TBN + 64 * g + 32, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(S_FREE + s));
+
+            uint32_t pk[32];
+            if (full && !slow_time) {
+                const float *wr = Wb + s * 256 + (pi - pmin) + 127 - 64 * g;
+                const float *tj = TJb + s * TBN + 64 * g;
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float h0 = fmaf(sv[c], 0.5f, wr[-c]) + time_bias_fast(ti1f, tj[c], E);
+                    const float h1 = fmaf(sv[c + 1], 0.5f, wr[-(c + 1)]) + time_bias_fast(ti1f, tj[c + 1], E);
+                    pk[c >> 1] = pack_bf16(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    float pv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int j = j0 + 64 * g + c + e;
+                        pv[e] = 0.f;
+                        if (row_ok && j < L && visible(i, j, hist)) {
+                            const float bp = p.rab_pos[pos_index(pi, token_pos(j, hist), p.pos_lo, p.pos_hi)];
+                            const float bt = p.rab_time[time_bucket(ti, p.timestamps[s0 + j], p.nb)];
+                            const float hh = 0.5f * (sv[c + e] + bp + bt);
+                            pv[e] = fmaf(hh, tanh_approx(hh), hh);
+                        }
+                    }
+                    pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+                }
+            }
+            // the previous P V must have finished reading the P buffer
+            if (t > 0 && !(ok = mbar_wait(bar(P_FREE), (t - 1) & 1, abort_flag, p.hdr)))
+                break;
+            unsigned char *prow = sm + LY::P + g * kRegion + r * 128;
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+                *reinterpret_cast<uint4 *>(prow + ((u ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(P_FULL));
+        }
+        if (ok && mbar_wait(bar(O_FULL), 0, abort_flag, p.hdr)) {
+            tc_fence_after();
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (s0 + i) * p.so + (int64_t)h * D + g * (D / 2);
+#pragma unroll
+            for (int cc = 0; cc < D / 2; cc += 32) {
+                float ov[32];
+                tmem_ld32(trow + 2 * TBN + g * (D / 2) + cc, ov);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        uint4 v;
+                        v.x = pack_bf16(ov[8 * u] * p.inv_n, ov[8 * u + 1] * p.inv_n);
+                        v.y = pack_bf16(ov[8 * u + 2] * p.inv_n, ov[8 * u + 3] * p.inv_n);
+                        v.z = pack_bf16(ov[8 * u + 4] * p.inv_n, ov[8 * u + 5] * p.inv_n);
+                        v.w = pack_bf16(ov[8 * u + 6] * p.inv_n, ov[8 * u + 7] * p.inv_n);
+                        *reinterpret_cast<uint4 *>(orow + cc + 8 * u) = v;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem, kTmemCols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+template <int D>
+cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
+{
+    CUtensorMap maps[3];
+    const void *ptrs[3] = {p.q, p.k, p.v};
+    const int64_t strides[3] = {p.sq, p.sk, p.sv};
+    cudaError_t e = make_row_tensor_map(&maps[0], ptrs[0], p.T, p.H * D, strides[0]);
+    if (e == cudaSuccess)
+        e = make_row_tensor_map(&maps[1], ptrs[1], p.T, p.H * D, strides[1]);
+    if (e == cudaSuccess)
+        e = make_row_tensor_map(&maps[2], ptrs[2], p.T, p.H * D, strides[2]);
+    if (e != cudaSuccess)
+        return e;
+    const size_t bytes = FwdLayout<D>::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess)
+        return e;
+    attn_fwd_tc_kernel<D><<<(unsigned)grid_items * p.H, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
+                                int64_t row_stride_elems)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_stride_elems * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+bool attn_tc_supported(const AttnParams &p)
+{
+    return (p.dqk == 64 || p.dqk == 128) && p.dv == p.dqk && p.T > 0 && p.T < ((int64_t)1 << 31) - 256 &&
+           tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
+{
+    if (grid_items <= 0)
+        return cudaSuccess;
+    switch (p.dqk) {
+    case 64: return fwd_tc_launch<64>(p, grid_items, stream);
+    case 128: return fwd_tc_launch<128>(p, grid_items, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace hstu

@@ -96,14 +96,18 @@ AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_
     return p;
 }
 
-int grid_items(const hstu_attn_desc *d) { return (int)max_items(d->total_tokens, d->num_seqs, kMmaTile); }
+int grid_items(const hstu_attn_desc *d, int tile = kMmaTile)
+{
+    return (int)max_items(d->total_tokens, d->num_seqs, tile);
+}
 
+// The work list always has room for the 64-row bound, the largest of all tilings.
 hstu_status schedule(const hstu_attn_desc *d, const int64_t *off, const int32_t *nt, int is_bwd,
-                     void *ws, cudaStream_t stream)
+                     void *ws, cudaStream_t stream, int tile = kMmaTile)
 {
     int2 *items = reinterpret_cast<int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
     return cuda_status(launch_schedule(off, nt, d->num_seqs, d->total_tokens, d->max_seq_len,
-                                       kMmaTile, is_bwd, items, grid_items(d),
+                                       tile, is_bwd, items, grid_items(d),
                                        static_cast<WsHeader *>(ws), nullptr, stream));
 }
 
@@ -113,7 +117,6 @@ hstu_status attn_fwd_strided(const hstu_attn_desc *d, const void *q, int64_t sq,
                              const int64_t *ts, const int32_t *nt, const float *rp, const float *rt,
                              void *out, int64_t so, void *ws, cudaStream_t stream)
 {
-    HSTU_TRY(schedule(d, off, nt, 0, ws, stream));
     AttnParams p = base_params(d, off, ts, nt, rp, rt, ws);
     p.q = q;
     p.k = k;
@@ -123,6 +126,11 @@ hstu_status attn_fwd_strided(const hstu_attn_desc *d, const void *q, int64_t sq,
     p.sk = sk;
     p.sv = sv;
     p.so = so;
+    if (d->dtype == HSTU_BF16 && attn_tc_supported(p)) {
+        HSTU_TRY(schedule(d, off, nt, 0, ws, stream, kTcTile));
+        return cuda_status(launch_attn_fwd_tc(p, grid_items(d, kTcTile), stream));
+    }
+    HSTU_TRY(schedule(d, off, nt, 0, ws, stream));
     if (d->dtype == HSTU_BF16)
         return cuda_status(launch_attn_fwd_mma(p, grid_items(d), stream));
     return cuda_status(launch_attn_fwd_f32(p, grid_items(d), stream));

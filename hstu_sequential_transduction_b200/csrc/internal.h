@@ -1,6 +1,7 @@
 // Host-side launchers shared between the kernel files and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -11,6 +12,7 @@ struct AttnParams;
 
 // Tile rows of the work items each attention implementation consumes.
 constexpr int kMmaTile = 64;
+constexpr int kTcTile = 128;
 
 cudaError_t launch_schedule(const int64_t *off, const int32_t *nt, int B, int64_t T, int max_len,
                             int tile, int is_bwd, int2 *items, int capacity, WsHeader *hdr,
@@ -23,6 +25,13 @@ cudaError_t launch_debug_indices(const int64_t *off, const int64_t *ts, const in
 // bf16 attention on the legacy tensor-core path (mma.sync), 64-row tiles.
 cudaError_t launch_attn_fwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
 cudaError_t launch_attn_bwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
+
+// bf16 attention on tcgen05 / TMA (sm_100a), 128-row tiles, head dims 64 and 128.
+bool attn_tc_supported(const AttnParams &p);
+cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream);
+// 2-D bf16 tensor map over [rows, cols] with a row stride, 64 x 128 boxes, 128B swizzle.
+cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
+                                int64_t row_stride_elems);
 
 // fp32 attention on CUDA cores, 64-row tiles.
 cudaError_t launch_attn_fwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
