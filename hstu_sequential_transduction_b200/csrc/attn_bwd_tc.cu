@@ -1,0 +1,525 @@
+// HSTU jagged attention backward on sm_100a: TMA + tcgen05 (TMEM), head dim 128.
+//
+// Exact derivatives of the forward (the DLRMv4 page, text under Table 7: the
+// backward produces dQ, dK and dV through about five GEMMs), plus the
+// gradients of the shared relative-bias tables.  Per work item (sequence,
+// 128-row key tile, head) the CTA keeps K and V resident and walks the query
+// rows that see the tile in steps of 64:
+//   S^T  = K Q^T,  dP^T = V dO^T               (TMEM, 64 columns each)
+//   P = SiLU(s), dS' = dP * 2 SiLU'(s)          (epilogue, s = score + bias)
+//   dV += P^T dO,  dK += dS'^T Q                (TMEM accumulators, 128 cols each)
+//   dQ^T = K^T dS'^T                            (TMEM) -> shared staging ->
+//        TMA bulk reduce-add into an fp32 dQ accumulator in global memory
+// The constant factors (inv_n for P, inv_n / 2 for dS) are applied once at
+// the end.  With h = s / 2 and t = tanh(h):
+//   SiLU(s) = h (1 + t),  SiLU'(s) = (1 + t)(1 + h (1 - t)) / 2.
+// Bias-table gradients: every step's dS' is summed per positional index in a
+// 256-bin shared window (flushed with one global reduction per touched bin),
+// or in a register when the whole step falls on one clamped index; per time
+// bucket it is summed in run-length order (buckets are monotone along a row
+// of sorted stamps) into shared bins flushed once per CTA.
+//
+// Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
+// warps 2-9 epilogue (lane quarter = warp % 4 selects the TMEM rows, the two
+// warpgroups split each step's 64 query columns).
+// TMEM columns: dK [0,128), dV [128,256), S^T [256,320), dP^T [320,384),
+// dQ^T [384,448).
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr int KB = 128;  // key rows per CTA
+constexpr int QB = 64;   // query rows per step
+constexpr int DH = 128;  // head dim
+constexpr int kEpiThreadsB = 256;
+constexpr int kThreadsB = kEpiThreadsB + 64;
+constexpr uint32_t kTmemColsB = 512;
+constexpr int kRegK = 16384;  // 128 rows x 128 B
+constexpr int kRegQ = 8192;   // 64 rows x 128 B
+constexpr int kMaxTimeBins = 512;
+constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+
+enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 3, S_FULL = 5, S_FREE = 6, P_FULL = 7, P_FREE = 8,
+             DQ_FULL = 9, DQ_FREE = 10, ACC_FULL = 11, NBARS_B = 12 };
+
+struct BL {
+    static constexpr int K = 0;
+    static constexpr int V = K + 2 * kRegK;
+    static constexpr int Q0 = V + 2 * kRegK;       // 2 stages x 2 regions
+    static constexpr int O0 = Q0 + 4 * kRegQ;      // dO, 2 stages x 2 regions
+    static constexpr int PT = O0 + 4 * kRegQ;      // P^T  [128 keys x 64 queries]
+    static constexpr int DST = PT + kRegK;         // dS'^T
+    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32 [64 x 128]
+    static constexpr int E = DQS + QB * DH * 4;    // time bias by exponent (512)
+    static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
+    static constexpr int TG = EG + 512 * 4;        // time grads by bucket (general path)
+    static constexpr int TI = TG + kMaxTimeBins * 4;  // 2 x 64 rebased query stamps
+    static constexpr int WB = TI + 2 * QB * 4;     // 2 x 256 positional bias window
+    static constexpr int GB = WB + 2 * 256 * 4;    // 2 x 256 positional grad window
+    static constexpr int BAR = GB + 2 * 256 * 4;
+    static constexpr int MISC = BAR + NBARS_B * 8;
+    static constexpr int BYTES = MISC + 64;
+};
+
+__device__ __forceinline__ uint32_t exp_offset(float ti1, float tj)
+{
+    return (__float_as_uint(__fsub_rz(ti1, tj)) >> 21) & 0x7FCu;
+}
+
+__device__ __forceinline__ int exp_bucket(int e, int nb)
+{
+    return (e >= 256 || e < 127) ? 0 : min(e - 127, nb - 1);
+}
+
+// Step classes (uniform across the CTA for one 64-row query step).
+enum StepClass { CLS_GENERAL = 0, CLS_FAST = 1, CLS_CLAMPED = 2 };
+
+__global__ void __launch_bounds__(kThreadsB, 1)
+attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ)
+{
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sm = smem_raw + (base - raw);
+
+    const int item = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    if (item >= p.hdr->n_items)
+        return;
+    const int2 it = p.items[item];
+    const int64_t s0 = p.seq_offsets[it.x];
+    const int L = (int)(p.seq_offsets[it.x + 1] - s0);
+    const int hist = L - (p.num_targets ? p.num_targets[it.x] : 0);
+    const int j0 = it.y * KB;
+    const int q_end = j0 < hist ? L : min(j0 + KB, L);
+    const int nq = (q_end - j0 + QB - 1) / QB;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int i) { return base + BL::BAR + 8u * i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + BL::MISC + 8);
+    float *E = reinterpret_cast<float *>(sm + BL::E);
+    float *EG = reinterpret_cast<float *>(sm + BL::EG);
+    float *TG = reinterpret_cast<float *>(sm + BL::TG);
+    float *GB = reinterpret_cast<float *>(sm + BL::GB);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NBARS_B; i++) {
+            const bool epi = (i == S_FREE || i == P_FULL || i == DQ_FREE);
+            mbar_init(bar(i), epi ? 8 : 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmK);
+        tma_prefetch(&tmV);
+        tma_prefetch(&tmQ);
+        tma_prefetch(&tmO);
+        tma_prefetch(&tmDQ);
+    }
+    if (warp == 1)
+        tmem_alloc(base + BL::MISC, kTmemColsB);
+    if (warp >= 2) {
+        const int etid = threadIdx.x - 64;
+        for (int e = etid; e < 512; e += kEpiThreadsB) {
+            E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
+            EG[e] = 0.f;
+            TG[e] = 0.f;
+            GB[e] = 0.f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + BL::MISC);
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            mbar_expect_tx(bar(KV_FULL), 4 * kRegK);
+            for (int r = 0; r < 2; r++) {
+                tma_load_2d(base + BL::K + r * kRegK, &tmK, h * DH + 64 * r, (int)(s0 + j0), bar(KV_FULL));
+                tma_load_2d(base + BL::V + r * kRegK, &tmV, h * DH + 64 * r, (int)(s0 + j0), bar(KV_FULL));
+            }
+            for (int i = 0; i < nq; i++) {
+                const int s = i & 1;
+                const int y = (int)(s0 + j0 + i * QB);
+                if (i >= 2 && !mbar_wait(bar(Q_EMPTY + s), ((i - 2) >> 1) & 1, abort_flag, p.hdr))
+                    break;
+                mbar_expect_tx(bar(Q_FULL + s), 4 * kRegQ);
+                for (int r = 0; r < 2; r++) {
+                    tma_load_2d(base + BL::Q0 + s * 2 * kRegQ + r * kRegQ, &tmQ, h * DH + 64 * r, y, bar(Q_FULL + s));
+                    tma_load_2d(base + BL::O0 + s * 2 * kRegQ + r * kRegQ, &tmO, h * DH + 64 * r, y, bar(Q_FULL + s));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idSdP = idesc_bf16(KB, QB, 0, 0);
+            constexpr uint32_t idGrad = idesc_bf16(KB, DH, 0, 1);
+            constexpr uint32_t idDQ = idesc_bf16(DH, QB, 1, 1);
+            auto issue_SdP = [&](int i) {
+                const int s = i & 1;
+                for (int ks = 0; ks < DH / 16; ks++) {
+                    const uint32_t ok_ = (ks >> 2) * kRegK + (ks & 3) * 32;
+                    const uint32_t oq = s * 2 * kRegQ + (ks >> 2) * kRegQ + (ks & 3) * 32;
+                    umma_bf16(tmem + COL_S, smem_desc_sw128(base + BL::K + ok_, 16, 1024),
+                              smem_desc_sw128(base + BL::Q0 + oq, 16, 1024), idSdP, ks > 0);
+                    umma_bf16(tmem + COL_DP, smem_desc_sw128(base + BL::V + ok_, 16, 1024),
+                              smem_desc_sw128(base + BL::O0 + oq, 16, 1024), idSdP, ks > 0);
+                }
+                umma_commit(bar(S_FULL));
+            };
+            auto issue_grads = [&](int i) {
+                const int s = i & 1;
+                for (int ks = 0; ks < QB / 16; ks++) {
+                    const uint32_t acc = (i > 0 || ks > 0);
+                    umma_bf16(tmem + COL_DV, smem_desc_sw128(base + BL::PT + ks * 32, 16, 1024),
+                              smem_desc_sw128(base + BL::O0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                    umma_bf16(tmem + COL_DK, smem_desc_sw128(base + BL::DST + ks * 32, 16, 1024),
+                              smem_desc_sw128(base + BL::Q0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                }
+            };
+            auto issue_dq = [&]() {
+                for (int ks = 0; ks < KB / 16; ks++)
+                    umma_bf16(tmem + COL_DQ, smem_desc_sw128(base + BL::K + ks * 2048, kRegK, 1024),
+                              smem_desc_sw128(base + BL::DST + ks * 2048, kRegK, 1024), idDQ, ks > 0);
+            };
+            bool ok = mbar_wait(bar(KV_FULL), 0, abort_flag, p.hdr) &&
+                      mbar_wait(bar(Q_FULL), 0, abort_flag, p.hdr);
+            if (ok) {
+                tc_fence_after();
+                issue_SdP(0);
+            }
+            for (int i = 0; ok && i < nq; i++) {
+                if (i + 1 < nq) {
+                    ok = mbar_wait(bar(S_FREE), i & 1, abort_flag, p.hdr) &&
+                         mbar_wait(bar(Q_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1, abort_flag, p.hdr);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    issue_SdP(i + 1);
+                }
+                if (!(ok = mbar_wait(bar(P_FULL), i & 1, abort_flag, p.hdr)))
+                    break;
+                tc_fence_after();
+                issue_grads(i);
+                if (i > 0) {
+                    if (!(ok = mbar_wait(bar(DQ_FREE), (i - 1) & 1, abort_flag, p.hdr)))
+                        break;
+                    tc_fence_after();
+                }
+                issue_dq();
+                umma_commit(bar(Q_EMPTY + (i & 1)));
+                umma_commit(bar(P_FREE));
+                umma_commit(bar(DQ_FULL));
+            }
+            umma_commit(bar(ACC_FULL));
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
+        const int etid = threadIdx.x - 64;
+        const int r = quarter * 32 + lane;  // key row of the tile (TMEM lane); d index for dQ^T
+        const int j = j0 + r;
+        const bool krow_ok = j < L;
+        const int lo = p.pos_lo, hi = p.pos_hi;
+        const int64_t tb = p.timestamps[s0 + j0];
+        const int64_t tj = krow_ok ? p.timestamps[s0 + j] : tb;
+        const int pj = token_pos(j, hist);
+        const int64_t lim = (int64_t)1 << 24;
+        const int kbad = named_bar_or(1, kEpiThreadsB, (tj - tb >= lim) || (tj - tb <= -lim));
+        const float tjf = (float)(tj - tb);
+        const float gscale = 0.5f * p.inv_n;
+        const bool tg_smem = p.nb <= kMaxTimeBins;
+        float *TI = reinterpret_cast<float *>(sm + BL::TI);
+        float *WB = reinterpret_cast<float *>(sm + BL::WB);
+        float *DQS = reinterpret_cast<float *>(sm + BL::DQS);
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+
+        float wreg = 0.f;
+        int64_t treg = tb;
+        auto prep = [&](int i) {
+            const int i0 = j0 + i * QB;
+            int d = i0 - (j0 + KB - 1) + etid;
+            d = d < lo ? lo : (d > hi ? hi : d);
+            wreg = 0.5f * p.rab_pos[d - lo];
+            if (etid < QB) {
+                const int ii = i0 + etid;
+                treg = ii < L ? p.timestamps[s0 + ii] : tb;
+            }
+        };
+        prep(0);
+        int prev_pbase = 0;
+        bool ok = true;
+        for (int i = 0; i < nq; i++) {
+            const int buf = i & 1;
+            const int i0 = j0 + i * QB;
+            WB[buf * 256 + etid] = wreg;
+            int qbad = 0;
+            if (etid < QB) {
+                const int64_t dt = treg - tb + 1;
+                qbad = dt >= lim || dt <= -lim;
+                TI[buf * QB + etid] = (float)dt;
+            }
+            const bool time_bad = named_bar_or(1, kEpiThreadsB, qbad) || kbad;
+            if (i > 0) {
+                // every reduction of the previous step has landed: flush its window
+                float *gp = GB + (buf ^ 1) * 256;
+                const float v = gp[etid];
+                if (v != 0.f) {
+                    red_add_global(p.d_rab_pos + prev_pbase + etid, v * gscale);
+                    gp[etid] = 0.f;
+                }
+            }
+            if (i + 1 < nq)
+                prep(i + 1);
+            const int last_i = min(i0 + QB, L) - 1, last_j = min(j0 + KB, L) - 1;
+            const int dmin = token_pos(i0, hist) - token_pos(last_j, hist);
+            const int dmax = token_pos(last_i, hist) - token_pos(j0, hist);
+            const int pbase = (dmin < lo ? lo : (dmin > hi ? hi : dmin)) - lo;
+            const bool full = (i0 >= j0 + KB - 1) && (j0 + KB <= hist) && (i0 + QB <= L);
+            int cls = CLS_GENERAL;
+            if (full && !time_bad) {
+                if (dmin >= hi || dmax <= lo)
+                    cls = CLS_CLAMPED;
+                else if (dmin >= lo && dmax <= hi && i0 + QB <= hist)
+                    cls = CLS_FAST;
+            }
+            prev_pbase = pbase;
+
+            if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
+                break;
+            tc_fence_after();
+            float sv[32], dv[32];
+            tmem_ld32(trow + COL_S + 32 * g, sv);
+            tmem_ld32(trow + COL_DP + 32 * g, dv);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(S_FREE));
+
+            uint32_t pk[16], dk[16];
+            int cur = -1;
+            float tacc = 0.f;
+            if (cls != CLS_GENERAL) {
+                const bool fast = cls == CLS_FAST;
+                const int eb = (j0 + KB - 1 - j) + 32 * g;
+                const float *wrow = WB + buf * 256 + eb;
+                float *grow = GB + buf * 256 + eb;
+                const float *ti = TI + buf * QB + 32 * g;
+                const float bconst = 0.5f * p.rab_pos[pbase];
+                float pacc = 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    float pv[2], dsv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const uint32_t off = exp_offset(ti[c + e], tjf);
+                        const float bp = fast ? wrow[c + e] : bconst;
+                        const float hh = fmaf(sv[c + e], 0.5f, bp) + E[off >> 2];
+                        const float t = tanh_approx(hh);
+                        pv[e] = fmaf(hh, t, hh);
+                        const float a = 1.f + t;
+                        const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
+                        dsv[e] = ds;
+                        if (fast)
+                            red_add_shared(grow + c + e, ds);
+                        else
+                            pacc += ds;
+                        if ((int)off != cur) {
+                            if (cur >= 0)
+                                red_add_shared(EG + (cur >> 2), tacc);
+                            cur = (int)off;
+                            tacc = 0.f;
+                        }
+                        tacc += ds;
+                    }
+                    pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+                    dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
+                }
+                if (cur >= 0)
+                    red_add_shared(EG + (cur >> 2), tacc);
+                if (!fast) {
+#pragma unroll
+                    for (int o = 16; o; o >>= 1)
+                        pacc += __shfl_xor_sync(0xffffffffu, pacc, o);
+                    if (lane == 0)
+                        red_add_shared(GB + buf * 256, pacc);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    float pv[2], dsv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int ii = i0 + 32 * g + c + e;
+                        pv[e] = 0.f;
+                        dsv[e] = 0.f;
+                        if (krow_ok && ii < L && visible(ii, j, hist)) {
+                            const int idx = pos_index(token_pos(ii, hist), pj, lo, hi);
+                            const int b = time_bucket(p.timestamps[s0 + ii], tj, p.nb);
+                            const float hh = 0.5f * (sv[c + e] + p.rab_pos[idx] + p.rab_time[b]);
+                            const float t = tanh_approx(hh);
+                            pv[e] = fmaf(hh, t, hh);
+                            const float a = 1.f + t;
+                            const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
+                            dsv[e] = ds;
+                            red_add_shared(GB + buf * 256 + (idx - pbase), ds);
+                            if (tg_smem) {
+                                if (b != cur) {
+                                    if (cur >= 0)
+                                        red_add_shared(TG + cur, tacc);
+                                    cur = b;
+                                    tacc = 0.f;
+                                }
+                                tacc += ds;
+                            } else {
+                                red_add_global(p.d_rab_time + b, ds * gscale);
+                            }
+                        }
+                    }
+                    pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+                    dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
+                }
+                if (tg_smem && cur >= 0)
+                    red_add_shared(TG + cur, tacc);
+            }
+
+            // P^T and dS'^T rows of this thread (K-major, 128B swizzle) once the
+            // previous step's gradient MMAs have finished reading them
+            if (i > 0 && !(ok = mbar_wait(bar(P_FREE), (i - 1) & 1, abort_flag, p.hdr)))
+                break;
+            unsigned char *prow = sm + BL::PT + r * 128;
+            unsigned char *drow = sm + BL::DST + r * 128;
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int sw = ((4 * g + u) ^ (r & 7)) << 4;
+                *reinterpret_cast<uint4 *>(prow + sw) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                *reinterpret_cast<uint4 *>(drow + sw) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(P_FULL));
+
+            // dQ'^T of this step -> staging [64 queries x 128] -> bulk reduce-add
+            if (!(ok = mbar_wait(bar(DQ_FULL), i & 1, abort_flag, p.hdr)))
+                break;
+            tc_fence_after();
+            float qv[32];
+            tmem_ld32(trow + COL_DQ + 32 * g, qv);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(DQ_FREE));
+            if (etid == 0)
+                bulk_wait_read0();
+            named_bar(2, kEpiThreadsB);
+#pragma unroll
+            for (int c = 0; c < 32; c++)
+                DQS[(32 * g + c) * DH + r] = qv[c];
+            fence_proxy_async_smem();
+            named_bar(2, kEpiThreadsB);
+            if (etid == 0) {
+                tma_reduce_add_2d(&tmDQ, h * DH, (int)(s0 + i0), base + BL::DQS);
+                bulk_commit();
+            }
+        }
+        named_bar(1, kEpiThreadsB);
+        if (ok) {
+            const float v = GB[((nq - 1) & 1) * 256 + etid];
+            if (v != 0.f)
+                red_add_global(p.d_rab_pos + prev_pbase + etid, v * gscale);
+        }
+        for (int e = etid; e < 512; e += kEpiThreadsB) {
+            const float v = EG[e];
+            if (v != 0.f)
+                red_add_global(p.d_rab_time + exp_bucket(e, p.nb), v * gscale);
+            if (tg_smem && e < p.nb) {
+                const float w = TG[e];
+                if (w != 0.f)
+                    red_add_global(p.d_rab_time + e, w * gscale);
+            }
+        }
+        if (ok && mbar_wait(bar(ACC_FULL), 0, abort_flag, p.hdr)) {
+            tc_fence_after();
+            __nv_bfloat16 *gdk = static_cast<__nv_bfloat16 *>(p.dk) + (s0 + j) * p.sdk + (int64_t)h * DH + 64 * g;
+            __nv_bfloat16 *gdv = static_cast<__nv_bfloat16 *>(p.dvv) + (s0 + j) * p.sdv + (int64_t)h * DH + 64 * g;
+#pragma unroll
+            for (int which = 0; which < 2; which++) {
+                const uint32_t col = (which ? COL_DV : COL_DK) + 64 * g;
+                const float scale = which ? p.inv_n : gscale;
+                __nv_bfloat16 *dst = which ? gdv : gdk;
+#pragma unroll
+                for (int cc = 0; cc < 64; cc += 32) {
+                    float v[32];
+                    tmem_ld32(trow + col + cc, v);
+                    tmem_wait_ld();
+                    if (krow_ok) {
+#pragma unroll
+                        for (int u = 0; u < 4; u++) {
+                            uint4 w;
+                            w.x = pack_bf16(v[8 * u] * scale, v[8 * u + 1] * scale);
+                            w.y = pack_bf16(v[8 * u + 2] * scale, v[8 * u + 3] * scale);
+                            w.z = pack_bf16(v[8 * u + 4] * scale, v[8 * u + 5] * scale);
+                            w.w = pack_bf16(v[8 * u + 6] * scale, v[8 * u + 7] * scale);
+                            *reinterpret_cast<uint4 *>(dst + cc + 8 * u) = w;
+                        }
+                    }
+                }
+            }
+        }
+        if (etid == 0)
+            bulk_wait0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem, kTmemColsB);
+}
+
+}  // namespace
+
+bool attn_bwd_tc_supported(const AttnParams &p)
+{
+    return p.dqk == DH && p.dv == DH && attn_tc_supported(p);
+}
+
+cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
+{
+    if (grid_items <= 0)
+        return cudaSuccess;
+    CUtensorMap mk, mv, mq, mo, mdq;
+    const int cols = p.H * DH;
+    cudaError_t e = make_row_tensor_map(&mk, p.k, p.T, cols, p.sk);
+    if (e == cudaSuccess)
+        e = make_row_tensor_map(&mv, p.v, p.T, cols, p.sv);
+    if (e == cudaSuccess)
+        e = make_tensor_map_2d(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.T, cols, p.sq * 2, 64, QB,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = make_tensor_map_2d(&mo, p.dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.T, cols, p.sdo * 2, 64, QB,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = make_tensor_map_2d(&mdq, p.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.T, cols, (int64_t)cols * 4,
+                               DH, QB, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess)
+        return e;
+    const size_t bytes = BL::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess)
+        return e;
+    attn_bwd_tc_kernel<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq);
+    return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -368,20 +368,28 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
 
 }  // namespace
 
-cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
-                                int64_t row_stride_elems)
+cudaError_t make_tensor_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
+                               int64_t rows, int64_t cols, int64_t row_stride_bytes, int box_cols,
+                               int box_rows, CUtensorMapSwizzle swizzle)
 {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc)
         return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)row_stride_elems * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint64_t strides[1] = {(cuuint64_t)row_stride_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
+                                int64_t row_stride_elems)
+{
+    return make_tensor_map_2d(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rows, cols, row_stride_elems * 2,
+                              64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool attn_tc_supported(const AttnParams &p)

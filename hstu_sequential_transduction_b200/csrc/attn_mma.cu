@@ -517,14 +517,14 @@ attn_bwd_mma_kernel(const AttnParams p)
 }
 
 __global__ void convert_dq_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
-                                  int64_t T, int H, int d, int64_t sdq)
+                                  int64_t T, int H, int d, int64_t sdq, float scale)
 {
     const int64_t n = T * H * d;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
          e += (int64_t)gridDim.x * blockDim.x) {
         int64_t t = e / ((int64_t)H * d);
         int64_t r = e % ((int64_t)H * d);
-        dq[t * sdq + r] = __float2bfloat16_rn(acc[e]);
+        dq[t * sdq + r] = __float2bfloat16_rn(acc[e] * scale);
     }
 }
 
@@ -585,13 +585,14 @@ cudaError_t launch_attn_bwd_mma(const AttnParams &p, int grid_items, cudaStream_
 }
 
 cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int d, int64_t sdq,
-                              cudaStream_t stream)
+                              float scale, cudaStream_t stream)
 {
     if (T == 0)
         return cudaSuccess;
     int64_t n = T * H * d;
     int blocks = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
-    convert_dq_kernel<<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(dq), T, H, d, sdq);
+    convert_dq_kernel<<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(dq), T, H, d, sdq,
+                                                  scale);
     return cudaGetLastError();
 }
 

@@ -222,10 +222,17 @@ hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void 
         p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + sizeof(WsHeader) +
                                              items_bytes(desc));
         HSTU_CUDA(cudaMemsetAsync(p.dq_acc, 0, sizeof(float) * (size_t)desc->total_tokens * row, st));
-        HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
-        HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
+        float dq_scale = 1.0f;
+        if (attn_bwd_tc_supported(p)) {
+            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st, kTcTile));
+            HSTU_CUDA(launch_attn_bwd_tc(p, grid_items(desc, kTcTile), st));
+            dq_scale = 0.5f * desc->inv_n;
+        } else {
+            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
+            HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
+        }
         return cuda_status(launch_convert_dq(p.dq_acc, dq, desc->total_tokens, desc->num_heads,
-                                             desc->d_qk, row, st));
+                                             desc->d_qk, row, dq_scale, st));
     }
     if (tensor_bytes) {
         HSTU_CUDA(cudaMemsetAsync(dk, 0, tensor_bytes, st));

@@ -32,14 +32,22 @@ cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t
 // 2-D bf16 tensor map over [rows, cols] with a row stride, 64 x 128 boxes, 128B swizzle.
 cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
                                 int64_t row_stride_elems);
+// General 2-D tensor map (row stride in bytes, box of box_cols x box_rows elements).
+cudaError_t make_tensor_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
+                               int64_t rows, int64_t cols, int64_t row_stride_bytes, int box_cols,
+                               int box_rows, CUtensorMapSwizzle swizzle);
+// bf16 backward on tcgen05 (head dim 128), key tiles of 128 rows; dq_acc receives
+// dQ / (0.5 * inv_n) (apply that scale when converting).
+bool attn_bwd_tc_supported(const AttnParams &p);
+cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream);
 
 // fp32 attention on CUDA cores, 64-row tiles.
 cudaError_t launch_attn_fwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
 cudaError_t launch_attn_bwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
 
-// dq (bf16) <- dq_acc (fp32), n elements of rows with stride.
+// dq (bf16) <- scale * dq_acc (fp32), n elements of rows with stride.
 cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int d, int64_t sdq,
-                              cudaStream_t stream);
+                              float scale, cudaStream_t stream);
 
 // C[M, N] = act(A[M, K] B[K, N] + bias[N]); act = SiLU if silu.  Row strides
 // lda, ldc in elements; B is dense [K, N].

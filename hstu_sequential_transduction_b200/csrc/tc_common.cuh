@@ -202,3 +202,36 @@ __device__ __forceinline__ int named_bar_or(int id, int count, int pred)
 }
 
 }  // namespace hstu
+
+namespace hstu {
+
+// Bulk tensor reduce-add of a shared tile into global memory (tracked by a
+// bulk async-group of the issuing thread).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(src)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+
+// Wait until the issuing thread's bulk groups have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+
+// Wait until the issuing thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
+__device__ __forceinline__ void red_add_shared(float *addr, float v)
+{
+    asm volatile("red.shared.add.f32 [%0], %1;\n" ::"r"(smem_u32(addr)), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_global(float *addr, float v)
+{
+    asm volatile("red.global.add.f32 [%0], %1;\n" ::"l"(addr), "f"(v) : "memory");
+}
+
+}  // namespace hstu
