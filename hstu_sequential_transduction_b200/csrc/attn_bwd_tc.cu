@@ -13,11 +13,16 @@
 // The constant factors (inv_n for P, inv_n / 2 for dS) are applied once at
 // the end.  With h = s / 2 and t = tanh(h):
 //   SiLU(s) = h (1 + t),  SiLU'(s) = (1 + t)(1 + h (1 - t)) / 2.
-// Bias-table gradients: every step's dS' is summed per positional index in a
-// 256-bin shared window (flushed with one global reduction per touched bin),
-// or in a register when the whole step falls on one clamped index; per time
-// bucket it is summed in run-length order (buckets are monotone along a row
-// of sorted stamps) into shared bins flushed once per CTA.
+// Bias-table gradients without per-pair atomics: the positional index of a
+// pair is query - key, constant along diagonals, so each warp reduces its
+// 32 x 32 block of dS' along the 63 diagonals with one shuffle per column and
+// stores them to per-warp slots that are summed and flushed per step (one
+// global reduction per touched index); a step on one clamped index is a plain
+// sum.  Time buckets are monotone along a key row of sorted stamps: each step
+// splits a row into at most two buckets (else a per-column fallback), and the
+// running bucket sum is carried across steps, so shared-memory atomics happen
+// only when a row changes bucket.  Candidate rows and stamps spanning more
+// than 2^24 s take a general per-pair path.
 //
 // Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
 // warps 2-9 epilogue (lane quarter = warp % 4 selects the TMEM rows, the two
@@ -52,14 +57,15 @@ struct BL {
     static constexpr int O0 = Q0 + 4 * kRegQ;      // dO, 2 stages x 2 regions
     static constexpr int PT = O0 + 4 * kRegQ;      // P^T  [128 keys x 64 queries]
     static constexpr int DST = PT + kRegK;         // dS'^T
-    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32 [64 x 128]
+    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, 8 warps x [32 x 32]
     static constexpr int E = DQS + QB * DH * 4;    // time bias by exponent (512)
     static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
     static constexpr int TG = EG + 512 * 4;        // time grads by bucket (general path)
     static constexpr int TI = TG + kMaxTimeBins * 4;  // 2 x 64 rebased query stamps
     static constexpr int WB = TI + 2 * QB * 4;     // 2 x 256 positional bias window
-    static constexpr int GB = WB + 2 * 256 * 4;    // 2 x 256 positional grad window
-    static constexpr int BAR = GB + 2 * 256 * 4;
+    static constexpr int GB = WB + 2 * 256 * 4;    // 2 x 256 positional grad window (general path)
+    static constexpr int WG = GB + 2 * 256 * 4;    // 2 x 8 warps x 64 diagonal sums
+    static constexpr int BAR = WG + 2 * 8 * 64 * 4;
     static constexpr int MISC = BAR + NBARS_B * 8;
     static constexpr int BYTES = MISC + 64;
 };
@@ -75,7 +81,79 @@ __device__ __forceinline__ int exp_bucket(int e, int nb)
 }
 
 // Step classes (uniform across the CTA for one 64-row query step).
-enum StepClass { CLS_GENERAL = 0, CLS_FAST = 1, CLS_CLAMPED = 2 };
+//   CLAMPED  every pair visible and on one clamped positional index;
+//   WINDOW   no candidate rows: positional index = query - key, read from
+//            and reduced into a per-step window (masked when not full);
+//   GENERAL  candidate rows or stamps outside the fast-bucket range.
+enum StepClass { CLS_GENERAL = 0, CLS_WINDOW = 1, CLS_WINDOW_MASKED = 2, CLS_CLAMPED = 3 };
+
+// Result of the elementwise pass over one thread's 32 query columns.
+struct RowOut {
+    uint32_t b0, b1;  // exponent offsets of the first and last visible column
+    float all, hi;    // sum of dS' over the row segment, and over columns in bucket b1
+    bool mid;         // a visible column falls in a bucket other than b0 and b1
+};
+
+// Elementwise backward of the 32 query columns one thread owns (one key row):
+// P = SiLU, dS' = dP (1+t)(1+h(1-t)); dS' replaces dP in dv[], P is packed.
+// Columns outside [c_lo, c_hi) are masked when MASK.  No atomics, no
+// data-dependent branches.
+template <bool MASK, bool WINDOW>
+__device__ __forceinline__ RowOut bwd_row(const float *sv, float *dv, const float *ti, float tjf, const char *Eb,
+                                          const float *wrow, float bconst, int c_lo, int c_hi, uint32_t *pk)
+{
+    RowOut o;
+    const int f = MASK ? min(max(c_lo, 0), 31) : 0, l = MASK ? min(max(c_hi - 1, 0), 31) : 31;
+    o.b0 = exp_offset(ti[f], tjf);
+    o.b1 = exp_offset(ti[l], tjf);
+    o.all = 0.f;
+    o.hi = 0.f;
+    o.mid = false;
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+        float pv[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int cc = c + e;
+            const uint32_t off = exp_offset(ti[cc], tjf);
+            const float bp = WINDOW ? wrow[cc] : bconst;
+            const float hh = fmaf(sv[cc], 0.5f, bp) + *reinterpret_cast<const float *>(Eb + off);
+            const float t = tanh_approx(hh);
+            float pval = fmaf(hh, t, hh);
+            const float a = 1.f + t;
+            float ds = dv[cc] * fmaf(a, fmaf(-hh, t, hh), a);
+            bool vis = true;
+            if (MASK) {
+                vis = cc >= c_lo && cc < c_hi;
+                pval = vis ? pval : 0.f;
+                ds = vis ? ds : 0.f;
+            }
+            dv[cc] = ds;
+            pv[e] = pval;
+            o.all += ds;
+            o.hi += (off == o.b1) ? ds : 0.f;
+            o.mid |= vis && (off != o.b0) && (off != o.b1);
+        }
+        pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+    }
+    return o;
+}
+
+// Sums of dS' along the 63 diagonals of a warp's 32 x 32 block (lanes are key
+// rows, registers query columns): lane l returns diagonal l in accP and
+// diagonal l - 32 in accN, with one shuffle per column.
+__device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float &accP, float &accN)
+{
+    accP = 0.f;
+    accN = 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; k++) {
+        const float y = __shfl_sync(0xffffffffu, ds[k], (k - lane) & 31);
+        const bool pos = k >= lane;
+        accP += pos ? y : 0.f;
+        accN += pos ? 0.f : y;
+    }
+}
 
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
@@ -239,8 +317,86 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         const bool tg_smem = p.nb <= kMaxTimeBins;
         float *TI = reinterpret_cast<float *>(sm + BL::TI);
         float *WB = reinterpret_cast<float *>(sm + BL::WB);
-        float *DQS = reinterpret_cast<float *>(sm + BL::DQS);
+        float *WG = reinterpret_cast<float *>(sm + BL::WG);
+        float *DQW = reinterpret_cast<float *>(sm + BL::DQS) + ew * 1024;  // this warp's [32 x 32]
+        const uint32_t dqw_addr = base + BL::DQS + ew * 4096;
+        const char *Eb = reinterpret_cast<const char *>(E);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+
+        // time-bucket run carried across steps (buckets only grow along a key row
+        // of sorted stamps, so a thread changes bins a few dozen times per CTA)
+        uint32_t tcur = 0xFFFFFFFFu;
+        float tacc = 0.f;
+        auto time_add = [&](uint32_t off, float v) {
+            if (off == tcur) {
+                tacc += v;
+                return;
+            }
+            if (tcur != 0xFFFFFFFFu && tacc != 0.f)
+                atomicAdd(EG + (tcur >> 2), tacc);
+            tcur = off;
+            tacc = v;
+        };
+
+        // dQ'^T of step k for this warp: TMEM -> [32 queries x 32 d] staging ->
+        // bulk reduce-add (each warp its own box, no CTA-wide barrier)
+        auto handle_dq = [&](int k) -> bool {
+            if (!mbar_wait(bar(DQ_FULL), k & 1, abort_flag, p.hdr))
+                return false;
+            tc_fence_after();
+            float qv[32];
+            tmem_ld32(trow + COL_DQ + 32 * g, qv);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(DQ_FREE));
+                bulk_wait_read0();
+            }
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 32; c++)
+                DQW[c * 32 + lane] = qv[c];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_reduce_add_2d(&tmDQ, h * DH + 32 * quarter, (int)(s0 + j0 + k * QB + 32 * g), dqw_addr);
+                bulk_commit();
+            }
+            return true;
+        };
+
+        // positional gradients of a finished step -> global table
+        auto flush_pos = [&](int pb, int cls_, int dmin_w, int pbase_) {
+            float *gp = GB + pb * 256;
+            const float v = gp[etid];
+            if (v != 0.f) {
+                red_add_global(p.d_rab_pos + pbase_ + etid, v * gscale);
+                gp[etid] = 0.f;
+            }
+            if (cls_ == CLS_WINDOW || cls_ == CLS_WINDOW_MASKED) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; w++) {
+                    const int ebw = KB - 1 + 32 * ((w >> 2) - ((w + 2) & 3));
+                    const int slot = etid - ebw + 31;
+                    if (slot >= 0 && slot <= 62)
+                        sum += WG[(pb * 8 + w) * 64 + slot];
+                }
+                if (sum != 0.f) {
+                    int d = dmin_w + etid;
+                    d = d < lo ? lo : (d > hi ? hi : d);
+                    red_add_global(p.d_rab_pos + (d - lo), sum * gscale);
+                }
+            } else if (cls_ == CLS_CLAMPED && etid == 0) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; w++)
+                    sum += WG[(pb * 8 + w) * 64 + 63];
+                if (sum != 0.f)
+                    red_add_global(p.d_rab_pos + pbase_, sum * gscale);
+            }
+        };
 
         float wreg = 0.f;
         int64_t treg = tb;
@@ -255,7 +411,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             }
         };
         prep(0);
-        int prev_pbase = 0;
+        int prev_cls = CLS_GENERAL, prev_dmin = 0, prev_pbase = 0;
         bool ok = true;
         for (int i = 0; i < nq; i++) {
             const int buf = i & 1;
@@ -268,15 +424,8 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 TI[buf * QB + etid] = (float)dt;
             }
             const bool time_bad = named_bar_or(1, kEpiThreadsB, qbad) || kbad;
-            if (i > 0) {
-                // every reduction of the previous step has landed: flush its window
-                float *gp = GB + (buf ^ 1) * 256;
-                const float v = gp[etid];
-                if (v != 0.f) {
-                    red_add_global(p.d_rab_pos + prev_pbase + etid, v * gscale);
-                    gp[etid] = 0.f;
-                }
-            }
+            if (i > 0)
+                flush_pos(buf ^ 1, prev_cls, prev_dmin, prev_pbase);
             if (i + 1 < nq)
                 prep(i + 1);
             const int last_i = min(i0 + QB, L) - 1, last_j = min(j0 + KB, L) - 1;
@@ -285,12 +434,14 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             const int pbase = (dmin < lo ? lo : (dmin > hi ? hi : dmin)) - lo;
             const bool full = (i0 >= j0 + KB - 1) && (j0 + KB <= hist) && (i0 + QB <= L);
             int cls = CLS_GENERAL;
-            if (full && !time_bad) {
-                if (dmin >= hi || dmax <= lo)
+            if (!time_bad) {
+                if (full && (dmin >= hi || dmax <= lo))
                     cls = CLS_CLAMPED;
-                else if (dmin >= lo && dmax <= hi && i0 + QB <= hist)
-                    cls = CLS_FAST;
+                else if (min(i0 + QB, L) <= hist)
+                    cls = full ? CLS_WINDOW : CLS_WINDOW_MASKED;
             }
+            prev_cls = cls;
+            prev_dmin = i0 - (j0 + KB - 1);
             prev_pbase = pbase;
 
             if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
@@ -306,54 +457,51 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 mbar_arrive(bar(S_FREE));
 
             uint32_t pk[16], dk[16];
-            int cur = -1;
-            float tacc = 0.f;
             if (cls != CLS_GENERAL) {
-                const bool fast = cls == CLS_FAST;
-                const int eb = (j0 + KB - 1 - j) + 32 * g;
-                const float *wrow = WB + buf * 256 + eb;
-                float *grow = GB + buf * 256 + eb;
-                const float *ti = TI + buf * QB + 32 * g;
-                const float bconst = 0.5f * p.rab_pos[pbase];
-                float pacc = 0.f;
+                const int cb = 32 * g;
+                const float *ti = TI + buf * QB + cb;
+                const float *wrow = WB + buf * 256 + (j0 + KB - 1 - j) + cb;
+                float *wg = WG + (buf * 8 + ew) * 64;
+                RowOut o;
+                if (cls == CLS_CLAMPED) {
+                    o = bwd_row<false, false>(sv, dv, ti, tjf, Eb, nullptr, 0.5f * p.rab_pos[pbase], 0, 32, pk);
+                    float sum = o.all;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    float pv[2], dsv[2];
-#pragma unroll
-                    for (int e = 0; e < 2; e++) {
-                        const uint32_t off = exp_offset(ti[c + e], tjf);
-                        const float bp = fast ? wrow[c + e] : bconst;
-                        const float hh = fmaf(sv[c + e], 0.5f, bp) + E[off >> 2];
-                        const float t = tanh_approx(hh);
-                        pv[e] = fmaf(hh, t, hh);
-                        const float a = 1.f + t;
-                        const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
-                        dsv[e] = ds;
-                        if (fast)
-                            red_add_shared(grow + c + e, ds);
-                        else
-                            pacc += ds;
-                        if ((int)off != cur) {
-                            if (cur >= 0)
-                                red_add_shared(EG + (cur >> 2), tacc);
-                            cur = (int)off;
-                            tacc = 0.f;
-                        }
-                        tacc += ds;
-                    }
-                    pk[c >> 1] = pack_bf16(pv[0], pv[1]);
-                    dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
-                }
-                if (cur >= 0)
-                    red_add_shared(EG + (cur >> 2), tacc);
-                if (!fast) {
-#pragma unroll
-                    for (int o = 16; o; o >>= 1)
-                        pacc += __shfl_xor_sync(0xffffffffu, pacc, o);
+                    for (int s = 16; s; s >>= 1)
+                        sum += __shfl_xor_sync(0xffffffffu, sum, s);
                     if (lane == 0)
-                        red_add_shared(GB + buf * 256, pacc);
+                        wg[63] = sum;
+                } else {
+                    if (cls == CLS_WINDOW)
+                        o = bwd_row<false, true>(sv, dv, ti, tjf, Eb, wrow, 0.f, 0, 32, pk);
+                    else
+                        o = bwd_row<true, true>(sv, dv, ti, tjf, Eb, wrow, 0.f, j - i0 - cb,
+                                                krow_ok ? min(32, L - i0 - cb) : 0, pk);
+                    float accP, accN;
+                    warp_diagonals(dv, lane, accP, accN);
+                    wg[lane + 31] = accP;
+                    if (lane > 0)
+                        wg[lane - 1] = accN;
                 }
+                if (!o.mid) {
+                    if (o.b1 != o.b0) {
+                        time_add(o.b0, o.all - o.hi);
+                        time_add(o.b1, o.hi);
+                    } else {
+                        time_add(o.b0, o.all);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; c++)
+                        if (dv[c] != 0.f)
+                            time_add(exp_offset(ti[c], tjf), dv[c]);
+                }
+#pragma unroll
+                for (int c = 0; c < 32; c += 2)
+                    dk[c >> 1] = pack_bf16(dv[c], dv[c + 1]);
             } else {
+                int cur = -1;
+                float gacc = 0.f;
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     float pv[2], dsv[2];
@@ -371,15 +519,15 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                             const float a = 1.f + t;
                             const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
                             dsv[e] = ds;
-                            red_add_shared(GB + buf * 256 + (idx - pbase), ds);
+                            atomicAdd(GB + buf * 256 + (idx - pbase), ds);
                             if (tg_smem) {
                                 if (b != cur) {
                                     if (cur >= 0)
-                                        red_add_shared(TG + cur, tacc);
+                                        atomicAdd(TG + cur, gacc);
                                     cur = b;
-                                    tacc = 0.f;
+                                    gacc = 0.f;
                                 }
-                                tacc += ds;
+                                gacc += ds;
                             } else {
                                 red_add_global(p.d_rab_time + b, ds * gscale);
                             }
@@ -389,9 +537,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
                 }
                 if (tg_smem && cur >= 0)
-                    red_add_shared(TG + cur, tacc);
+                    atomicAdd(TG + cur, gacc);
             }
 
+            // the previous step's dQ, deferred so the gradient MMAs overlap this step's math
+            if (i > 0 && !(ok = handle_dq(i - 1)))
+                break;
             // P^T and dS'^T rows of this thread (K-major, 128B swizzle) once the
             // previous step's gradient MMAs have finished reading them
             if (i > 0 && !(ok = mbar_wait(bar(P_FREE), (i - 1) & 1, abort_flag, p.hdr)))
@@ -408,37 +559,14 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar(P_FULL));
-
-            // dQ'^T of this step -> staging [64 queries x 128] -> bulk reduce-add
-            if (!(ok = mbar_wait(bar(DQ_FULL), i & 1, abort_flag, p.hdr)))
-                break;
-            tc_fence_after();
-            float qv[32];
-            tmem_ld32(trow + COL_DQ + 32 * g, qv);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar(DQ_FREE));
-            if (etid == 0)
-                bulk_wait_read0();
-            named_bar(2, kEpiThreadsB);
-#pragma unroll
-            for (int c = 0; c < 32; c++)
-                DQS[(32 * g + c) * DH + r] = qv[c];
-            fence_proxy_async_smem();
-            named_bar(2, kEpiThreadsB);
-            if (etid == 0) {
-                tma_reduce_add_2d(&tmDQ, h * DH, (int)(s0 + i0), base + BL::DQS);
-                bulk_commit();
-            }
         }
+        if (ok)
+            ok = handle_dq(nq - 1);
+        if (tcur != 0xFFFFFFFFu && tacc != 0.f)
+            atomicAdd(EG + (tcur >> 2), tacc);
         named_bar(1, kEpiThreadsB);
-        if (ok) {
-            const float v = GB[((nq - 1) & 1) * 256 + etid];
-            if (v != 0.f)
-                red_add_global(p.d_rab_pos + prev_pbase + etid, v * gscale);
-        }
+        if (ok)
+            flush_pos((nq - 1) & 1, prev_cls, prev_dmin, prev_pbase);
         for (int e = etid; e < 512; e += kEpiThreadsB) {
             const float v = EG[e];
             if (v != 0.f)
@@ -477,7 +605,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 }
             }
         }
-        if (etid == 0)
+        if (lane == 0)
             bulk_wait0();
     }
     tc_fence_before();
@@ -511,7 +639,7 @@ cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t
                                CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
         e = make_tensor_map_2d(&mdq, p.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.T, cols, (int64_t)cols * 4,
-                               DH, QB, CU_TENSOR_MAP_SWIZZLE_NONE);
+                               32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess)
         return e;
     const size_t bytes = BL::BYTES + 1024;

@@ -224,9 +224,23 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 // Wait until the issuing thread's bulk groups have completed.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
+// Shared-memory float reduction.  No memory clobber: the bins it targets are
+// only read after a barrier, so the compiler may schedule it freely.
 __device__ __forceinline__ void red_add_shared(float *addr, float v)
 {
-    asm volatile("red.shared.add.f32 [%0], %1;\n" ::"r"(smem_u32(addr)), "f"(v) : "memory");
+    asm volatile("red.shared.add.f32 [%0], %1;\n" ::"r"(smem_u32(addr)), "f"(v));
+}
+
+__device__ __forceinline__ void red_add_shared_u32(uint32_t saddr, float v)
+{
+    asm volatile("red.shared.add.f32 [%0], %1;\n" ::"r"(saddr), "f"(v));
+}
+
+// Same, predicated on `pred` (no branch).
+__device__ __forceinline__ void red_add_shared_if(uint32_t saddr, float v, bool pred)
+{
+    asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %2, 0;\n @p red.shared.add.f32 [%0], %1;\n}\n" ::"r"(saddr),
+                 "f"(v), "r"((int)pred));
 }
 
 __device__ __forceinline__ void red_add_global(float *addr, float v)
