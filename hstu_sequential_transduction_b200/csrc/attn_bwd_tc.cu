@@ -39,12 +39,14 @@ namespace {
 constexpr int KB = 128;  // key rows per CTA
 constexpr int QB = 64;   // query rows per step
 constexpr int DH = 128;  // head dim
-constexpr int kEpiThreadsB = 256;
+constexpr int kEpiWarpsB = 8;                   // 2 per TMEM lane quarter
+constexpr int kEpiThreadsB = kEpiWarpsB * 32;
 constexpr int kThreadsB = kEpiThreadsB + 64;
+constexpr int kGroupsB = kEpiWarpsB / 4;         // column groups of a step
+constexpr int NC = QB / kGroupsB;                // query columns per epilogue thread
 constexpr uint32_t kTmemColsB = 512;
 constexpr int kRegK = 16384;  // 128 rows x 128 B
 constexpr int kRegQ = 8192;   // 64 rows x 128 B
-constexpr int kMaxTimeBins = 512;
 constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
 
 enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 3, S_FULL = 5, S_FREE = 6, P_FULL = 7, P_FREE = 8,
@@ -57,15 +59,12 @@ struct BL {
     static constexpr int O0 = Q0 + 4 * kRegQ;      // dO, 2 stages x 2 regions
     static constexpr int PT = O0 + 4 * kRegQ;      // P^T  [128 keys x 64 queries]
     static constexpr int DST = PT + kRegK;         // dS'^T
-    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, 8 warps x [32 x 32]
+    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, per warp [NC x 32]
     static constexpr int E = DQS + QB * DH * 4;    // time bias by exponent (512)
     static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
-    static constexpr int TG = EG + 512 * 4;        // time grads by bucket (general path)
-    static constexpr int TI = TG + kMaxTimeBins * 4;  // 2 x 64 rebased query stamps
-    static constexpr int WB = TI + 2 * QB * 4;     // 2 x 256 positional bias window
-    static constexpr int GB = WB + 2 * 256 * 4;    // 2 x 256 positional grad window (general path)
-    static constexpr int WG = GB + 2 * 256 * 4;    // 2 x 8 warps x 64 diagonal sums
-    static constexpr int BAR = WG + 2 * 8 * 64 * 4;
+    static constexpr int PW = EG + 512 * 4;        // per warp: NC query stamps + 64 bias window
+    static constexpr int PW_FLOATS = NC + 64;
+    static constexpr int BAR = PW + kEpiWarpsB * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS_B * 8;
     static constexpr int BYTES = MISC + 64;
 };
@@ -80,74 +79,98 @@ __device__ __forceinline__ int exp_bucket(int e, int nb)
     return (e >= 256 || e < 127) ? 0 : min(e - 127, nb - 1);
 }
 
-// Step classes (uniform across the CTA for one 64-row query step).
+// Block classes (uniform across one warp's 32 keys x NC queries of a step).
 //   CLAMPED  every pair visible and on one clamped positional index;
-//   WINDOW   no candidate rows: positional index = query - key, read from
-//            and reduced into a per-step window (masked when not full);
-//   GENERAL  candidate rows or stamps outside the fast-bucket range.
+//   WINDOW   no candidate queries: positional index = query - key, read from
+//            and reduced along the block's diagonals (masked when not full);
+//   GENERAL  candidate queries, unsorted stamps or stamps outside the
+//            fast-bucket range: exact per-pair path.
 enum StepClass { CLS_GENERAL = 0, CLS_WINDOW = 1, CLS_WINDOW_MASKED = 2, CLS_CLAMPED = 3 };
 
-// Result of the elementwise pass over one thread's 32 query columns.
+// NC consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld_nc(uint32_t taddr, float *v)
+{
+    if constexpr (NC == 16)
+        tmem_ld16(taddr, v);
+    else
+        tmem_ld32(taddr, v);
+}
+
+// Result of the elementwise pass over one thread's NC query columns.
 struct RowOut {
     uint32_t b0, b1;  // exponent offsets of the first and last visible column
     float all, hi;    // sum of dS' over the row segment, and over columns in bucket b1
     bool mid;         // a visible column falls in a bucket other than b0 and b1
 };
 
-// Elementwise backward of the 32 query columns one thread owns (one key row):
+// Elementwise backward of the NC query columns one thread owns (one key row):
 // P = SiLU, dS' = dP (1+t)(1+h(1-t)); dS' replaces dP in dv[], P is packed.
-// Columns outside [c_lo, c_hi) are masked when MASK.  No atomics, no
+// Columns outside [c_lo, c_hi) are masked when MASK.  TWO: the step is known
+// to put every key row in at most two time buckets (sorted stamps, narrow
+// span), so the bucket is one compare of the exact round-toward-zero
+// difference against the upper bucket's power of two.  No atomics, no
 // data-dependent branches.
-template <bool MASK, bool WINDOW>
+template <bool MASK, bool WINDOW, bool TWO>
 __device__ __forceinline__ RowOut bwd_row(const float *sv, float *dv, const float *ti, float tjf, const char *Eb,
                                           const float *wrow, float bconst, int c_lo, int c_hi, uint32_t *pk)
 {
     RowOut o;
-    const int f = MASK ? min(max(c_lo, 0), 31) : 0, l = MASK ? min(max(c_hi - 1, 0), 31) : 31;
+    const int f = MASK ? min(max(c_lo, 0), NC - 1) : 0, l = MASK ? min(max(c_hi - 1, 0), NC - 1) : NC - 1;
     o.b0 = exp_offset(ti[f], tjf);
     o.b1 = exp_offset(ti[l], tjf);
+    const float E0 = *reinterpret_cast<const float *>(Eb + o.b0);
+    const float E1 = *reinterpret_cast<const float *>(Eb + o.b1);
+    const float thr = __uint_as_float(o.b1 << 21);  // 2^(bucket of b1), exact
     o.all = 0.f;
     o.hi = 0.f;
     o.mid = false;
 #pragma unroll
-    for (int c = 0; c < 32; c += 2) {
+    for (int c = 0; c < NC; c += 2) {
         float pv[2];
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const int cc = c + e;
-            const uint32_t off = exp_offset(ti[cc], tjf);
+            float bt;
+            bool up;
+            if (TWO) {
+                up = __fsub_rz(ti[cc], tjf) >= thr;
+                bt = up ? E1 : E0;
+            } else {
+                const uint32_t off = exp_offset(ti[cc], tjf);
+                bt = *reinterpret_cast<const float *>(Eb + off);
+                up = off == o.b1;
+                o.mid |= (!MASK || (cc >= c_lo && cc < c_hi)) && (off != o.b0) && (off != o.b1);
+            }
             const float bp = WINDOW ? wrow[cc] : bconst;
-            const float hh = fmaf(sv[cc], 0.5f, bp) + *reinterpret_cast<const float *>(Eb + off);
+            const float hh = fmaf(sv[cc], 0.5f, bp) + bt;
             const float t = tanh_approx(hh);
             float pval = fmaf(hh, t, hh);
             const float a = 1.f + t;
             float ds = dv[cc] * fmaf(a, fmaf(-hh, t, hh), a);
-            bool vis = true;
             if (MASK) {
-                vis = cc >= c_lo && cc < c_hi;
+                const bool vis = cc >= c_lo && cc < c_hi;
                 pval = vis ? pval : 0.f;
                 ds = vis ? ds : 0.f;
             }
             dv[cc] = ds;
             pv[e] = pval;
             o.all += ds;
-            o.hi += (off == o.b1) ? ds : 0.f;
-            o.mid |= vis && (off != o.b0) && (off != o.b1);
+            o.hi += up ? ds : 0.f;
         }
         pk[c >> 1] = pack_bf16(pv[0], pv[1]);
     }
     return o;
 }
 
-// Sums of dS' along the 63 diagonals of a warp's 32 x 32 block (lanes are key
-// rows, registers query columns): lane l returns diagonal l in accP and
-// diagonal l - 32 in accN, with one shuffle per column.
+// Sums of dS' along the diagonals of a warp's 32 x NC block (lanes are key
+// rows, registers query columns): lane l returns diagonal l in accP (zero for
+// l >= NC) and diagonal l - 32 in accN, with one shuffle per column.
 __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float &accP, float &accN)
 {
     accP = 0.f;
     accN = 0.f;
 #pragma unroll
-    for (int k = 0; k < 32; k++) {
+    for (int k = 0; k < NC; k++) {
         const float y = __shfl_sync(0xffffffffu, ds[k], (k - lane) & 31);
         const bool pos = k >= lane;
         accP += pos ? y : 0.f;
@@ -181,13 +204,11 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + BL::MISC + 8);
     float *E = reinterpret_cast<float *>(sm + BL::E);
     float *EG = reinterpret_cast<float *>(sm + BL::EG);
-    float *TG = reinterpret_cast<float *>(sm + BL::TG);
-    float *GB = reinterpret_cast<float *>(sm + BL::GB);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS_B; i++) {
             const bool epi = (i == S_FREE || i == P_FULL || i == DQ_FREE);
-            mbar_init(bar(i), epi ? 8 : 1);
+            mbar_init(bar(i), epi ? kEpiWarpsB : 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -206,8 +227,6 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         for (int e = etid; e < 512; e += kEpiThreadsB) {
             E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
             EG[e] = 0.f;
-            TG[e] = 0.f;
-            GB[e] = 0.f;
         }
     }
     tc_fence_before();
@@ -301,8 +320,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         }
     } else {
         // ---------------- epilogue ----------------
+        // Every warp handles a 32-key x NC-query block of each step on its own:
+        // stamps, bias window, class and bias-table gradients are per warp, so
+        // the loop has no CTA-wide barrier.
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
         const int etid = threadIdx.x - 64;
+        const uint32_t full = 0xffffffffu;
         const int r = quarter * 32 + lane;  // key row of the tile (TMEM lane); d index for dQ^T
         const int j = j0 + r;
         const bool krow_ok = j < L;
@@ -311,17 +334,22 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         const int64_t tj = krow_ok ? p.timestamps[s0 + j] : tb;
         const int pj = token_pos(j, hist);
         const int64_t lim = (int64_t)1 << 24;
-        const int kbad = named_bar_or(1, kEpiThreadsB, (tj - tb >= lim) || (tj - tb <= -lim));
         const float tjf = (float)(tj - tb);
         const float gscale = 0.5f * p.inv_n;
-        const bool tg_smem = p.nb <= kMaxTimeBins;
-        float *TI = reinterpret_cast<float *>(sm + BL::TI);
-        float *WB = reinterpret_cast<float *>(sm + BL::WB);
-        float *WG = reinterpret_cast<float *>(sm + BL::WG);
-        float *DQW = reinterpret_cast<float *>(sm + BL::DQS) + ew * 1024;  // this warp's [32 x 32]
-        const uint32_t dqw_addr = base + BL::DQS + ew * 4096;
+        const int jw0 = j0 + quarter * 32;                 // first key row of the warp
+        const int jw_n = max(0, min(32, L - jw0));         // valid key rows of the warp
+        const int64_t tj_up = __shfl_up_sync(full, tj, 1);
+        const bool rows_bad = __any_sync(full, krow_ok && ((tj - tb >= lim) || (tj - tb <= -lim) ||
+                                                           (lane > 0 && tj_up > tj)));
+        const float tjf_first = __shfl_sync(full, tjf, 0);
+        const float tjf_last = __shfl_sync(full, tjf, max(jw_n - 1, 0));
+        float *TIw = reinterpret_cast<float *>(sm + BL::PW) + ew * BL::PW_FLOATS;  // NC stamps
+        float *Ww = TIw + NC;  // Ww[m]: positional bias / 2 at diagonal (query - key) = D_w + m - 31
+        float *DQW = reinterpret_cast<float *>(sm + BL::DQS) + ew * NC * 32;  // this warp's [NC x 32]
+        const uint32_t dqw_addr = base + BL::DQS + ew * NC * 128;
         const char *Eb = reinterpret_cast<const char *>(E);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        auto clamp_idx = [&](int d) { return (d < lo ? lo : (d > hi ? hi : d)) - lo; };
 
         // time-bucket run carried across steps (buckets only grow along a key row
         // of sorted stamps, so a thread changes bins a few dozen times per CTA)
@@ -338,14 +366,14 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             tacc = v;
         };
 
-        // dQ'^T of step k for this warp: TMEM -> [32 queries x 32 d] staging ->
-        // bulk reduce-add (each warp its own box, no CTA-wide barrier)
+        // dQ'^T of step k for this warp: TMEM -> [NC queries x 32 d] staging ->
+        // bulk reduce-add (each warp its own box)
         auto handle_dq = [&](int k) -> bool {
             if (!mbar_wait(bar(DQ_FULL), k & 1, abort_flag, p.hdr))
                 return false;
             tc_fence_after();
-            float qv[32];
-            tmem_ld32(trow + COL_DQ + 32 * g, qv);
+            float qv[NC];
+            tmem_ld_nc(trow + COL_DQ + NC * g, qv);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -355,133 +383,102 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             }
             __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 32; c++)
+            for (int c = 0; c < NC; c++)
                 DQW[c * 32 + lane] = qv[c];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_reduce_add_2d(&tmDQ, h * DH + 32 * quarter, (int)(s0 + j0 + k * QB + 32 * g), dqw_addr);
+                tma_reduce_add_2d(&tmDQ, h * DH + 32 * quarter, (int)(s0 + j0 + k * QB + NC * g), dqw_addr);
                 bulk_commit();
             }
             return true;
         };
 
-        // positional gradients of a finished step -> global table
-        auto flush_pos = [&](int pb, int cls_, int dmin_w, int pbase_) {
-            float *gp = GB + pb * 256;
-            const float v = gp[etid];
-            if (v != 0.f) {
-                red_add_global(p.d_rab_pos + pbase_ + etid, v * gscale);
-                gp[etid] = 0.f;
-            }
-            if (cls_ == CLS_WINDOW || cls_ == CLS_WINDOW_MASKED) {
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; w++) {
-                    const int ebw = KB - 1 + 32 * ((w >> 2) - ((w + 2) & 3));
-                    const int slot = etid - ebw + 31;
-                    if (slot >= 0 && slot <= 62)
-                        sum += WG[(pb * 8 + w) * 64 + slot];
-                }
-                if (sum != 0.f) {
-                    int d = dmin_w + etid;
-                    d = d < lo ? lo : (d > hi ? hi : d);
-                    red_add_global(p.d_rab_pos + (d - lo), sum * gscale);
-                }
-            } else if (cls_ == CLS_CLAMPED && etid == 0) {
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; w++)
-                    sum += WG[(pb * 8 + w) * 64 + 63];
-                if (sum != 0.f)
-                    red_add_global(p.d_rab_pos + pbase_, sum * gscale);
-            }
+        // per-warp inputs of step i, prefetched one step ahead
+        int64_t tq = tb;
+        float wlo = 0.f, whi = 0.f;
+        auto prefetch = [&](int i) {
+            const int iw0 = j0 + i * QB + NC * g;
+            const int dw = iw0 - jw0;
+            wlo = 0.5f * p.rab_pos[clamp_idx(dw + lane - 31)];
+            whi = 0.5f * p.rab_pos[clamp_idx(dw + lane + 1)];
+            if (lane < NC)
+                tq = iw0 + lane < L ? p.timestamps[s0 + iw0 + lane] : tb;
         };
-
-        float wreg = 0.f;
-        int64_t treg = tb;
-        auto prep = [&](int i) {
-            const int i0 = j0 + i * QB;
-            int d = i0 - (j0 + KB - 1) + etid;
-            d = d < lo ? lo : (d > hi ? hi : d);
-            wreg = 0.5f * p.rab_pos[d - lo];
-            if (etid < QB) {
-                const int ii = i0 + etid;
-                treg = ii < L ? p.timestamps[s0 + ii] : tb;
-            }
-        };
-        prep(0);
-        int prev_cls = CLS_GENERAL, prev_dmin = 0, prev_pbase = 0;
+        prefetch(0);
         bool ok = true;
         for (int i = 0; i < nq; i++) {
-            const int buf = i & 1;
             const int i0 = j0 + i * QB;
-            WB[buf * 256 + etid] = wreg;
-            int qbad = 0;
-            if (etid < QB) {
-                const int64_t dt = treg - tb + 1;
-                qbad = dt >= lim || dt <= -lim;
-                TI[buf * QB + etid] = (float)dt;
-            }
-            const bool time_bad = named_bar_or(1, kEpiThreadsB, qbad) || kbad;
-            if (i > 0)
-                flush_pos(buf ^ 1, prev_cls, prev_dmin, prev_pbase);
+            const int iw0 = i0 + NC * g;  // first query of this warp's block
+            const int dw = iw0 - jw0;     // query - key offset of the block's diagonal 0
+            const int64_t tq_up = __shfl_up_sync(full, tq, 1);
+            const bool q_ok = lane < NC && iw0 + lane < L;
+            const bool cols_bad = __any_sync(full, q_ok && ((tq - tb + 1 >= lim) || (tq - tb + 1 <= -lim) ||
+                                                            (lane > 0 && tq_up > tq)));
+            __syncwarp();
+            if (lane < NC)
+                TIw[lane] = (float)(tq - tb + 1);
+            Ww[lane] = wlo;
+            Ww[lane + 32] = whi;
+            __syncwarp();
             if (i + 1 < nq)
-                prep(i + 1);
-            const int last_i = min(i0 + QB, L) - 1, last_j = min(j0 + KB, L) - 1;
-            const int dmin = token_pos(i0, hist) - token_pos(last_j, hist);
-            const int dmax = token_pos(last_i, hist) - token_pos(j0, hist);
-            const int pbase = (dmin < lo ? lo : (dmin > hi ? hi : dmin)) - lo;
-            const bool full = (i0 >= j0 + KB - 1) && (j0 + KB <= hist) && (i0 + QB <= L);
+                prefetch(i + 1);
+
+            const int q_last = min(iw0 + NC, L) - 1;  // last valid query of the block
+            const bool full_w = (iw0 >= jw0 + 31) && (jw0 + 32 <= hist) && (iw0 + NC <= L) && (iw0 + NC <= hist);
+            const int dmin_w = dw - 31, dmax_w = dw + NC - 1;
             int cls = CLS_GENERAL;
-            if (!time_bad) {
-                if (full && (dmin >= hi || dmax <= lo))
+            if (!rows_bad && !cols_bad) {
+                if (full_w && (dmin_w >= hi || dmax_w <= lo))
                     cls = CLS_CLAMPED;
-                else if (min(i0 + QB, L) <= hist)
-                    cls = full ? CLS_WINDOW : CLS_WINDOW_MASKED;
+                else if (q_last < hist)
+                    cls = full_w ? CLS_WINDOW : CLS_WINDOW_MASKED;
             }
-            prev_cls = cls;
-            prev_dmin = i0 - (j0 + KB - 1);
-            prev_pbase = pbase;
+            bool two = false;
+            if (cls != CLS_GENERAL && q_last >= iw0 && jw_n > 0) {
+                const float dlo = __fsub_rz(TIw[0], tjf_last);
+                const float dhi = __fsub_rz(TIw[q_last - iw0], tjf_first);
+                two = dlo >= 1.f && ((__float_as_uint(dhi) >> 23) - (__float_as_uint(dlo) >> 23)) <= 1u;
+            }
 
             if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
                 break;
             tc_fence_after();
-            float sv[32], dv[32];
-            tmem_ld32(trow + COL_S + 32 * g, sv);
-            tmem_ld32(trow + COL_DP + 32 * g, dv);
+            float sv[NC], dv[NC];
+            tmem_ld_nc(trow + COL_S + NC * g, sv);
+            tmem_ld_nc(trow + COL_DP + NC * g, dv);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar(S_FREE));
 
-            uint32_t pk[16], dk[16];
+            uint32_t pk[NC / 2], dk[NC / 2];
             if (cls != CLS_GENERAL) {
-                const int cb = 32 * g;
-                const float *ti = TI + buf * QB + cb;
-                const float *wrow = WB + buf * 256 + (j0 + KB - 1 - j) + cb;
-                float *wg = WG + (buf * 8 + ew) * 64;
                 RowOut o;
                 if (cls == CLS_CLAMPED) {
-                    o = bwd_row<false, false>(sv, dv, ti, tjf, Eb, nullptr, 0.5f * p.rab_pos[pbase], 0, 32, pk);
+                    o = two ? bwd_row<false, false, true>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk)
+                            : bwd_row<false, false, false>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
                     float sum = o.all;
 #pragma unroll
                     for (int s = 16; s; s >>= 1)
-                        sum += __shfl_xor_sync(0xffffffffu, sum, s);
-                    if (lane == 0)
-                        wg[63] = sum;
+                        sum += __shfl_xor_sync(full, sum, s);
+                    if (lane == 0 && sum != 0.f)
+                        red_add_global(p.d_rab_pos + clamp_idx(dmin_w), sum * gscale);
                 } else {
+                    const float *wrow = Ww + 31 - lane;  // wrow[c]: diagonal c - lane
                     if (cls == CLS_WINDOW)
-                        o = bwd_row<false, true>(sv, dv, ti, tjf, Eb, wrow, 0.f, 0, 32, pk);
+                        o = two ? bwd_row<false, true, true>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
+                                : bwd_row<false, true, false>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk);
                     else
-                        o = bwd_row<true, true>(sv, dv, ti, tjf, Eb, wrow, 0.f, j - i0 - cb,
-                                                krow_ok ? min(32, L - i0 - cb) : 0, pk);
+                        o = bwd_row<true, true, false>(sv, dv, TIw, tjf, Eb, wrow, 0.f, j - iw0,
+                                                       krow_ok ? min(NC, L - iw0) : 0, pk);
                     float accP, accN;
                     warp_diagonals(dv, lane, accP, accN);
-                    wg[lane + 31] = accP;
-                    if (lane > 0)
-                        wg[lane - 1] = accN;
+                    if (accP != 0.f)
+                        red_add_global(p.d_rab_pos + clamp_idx(dw + lane), accP * gscale);
+                    if (accN != 0.f)
+                        red_add_global(p.d_rab_pos + clamp_idx(dw + lane - 32), accN * gscale);
                 }
                 if (!o.mid) {
                     if (o.b1 != o.b0) {
@@ -492,22 +489,21 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 32; c++)
+                    for (int c = 0; c < NC; c++)
                         if (dv[c] != 0.f)
-                            time_add(exp_offset(ti[c], tjf), dv[c]);
+                            time_add(exp_offset(TIw[c], tjf), dv[c]);
                 }
 #pragma unroll
-                for (int c = 0; c < 32; c += 2)
+                for (int c = 0; c < NC; c += 2)
                     dk[c >> 1] = pack_bf16(dv[c], dv[c + 1]);
             } else {
-                int cur = -1;
-                float gacc = 0.f;
+                // exact per-pair path: candidates, unsorted or far-apart stamps
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
+                for (int c = 0; c < NC; c += 2) {
                     float pv[2], dsv[2];
 #pragma unroll
                     for (int e = 0; e < 2; e++) {
-                        const int ii = i0 + 32 * g + c + e;
+                        const int ii = iw0 + c + e;
                         pv[e] = 0.f;
                         dsv[e] = 0.f;
                         if (krow_ok && ii < L && visible(ii, j, hist)) {
@@ -519,25 +515,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                             const float a = 1.f + t;
                             const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
                             dsv[e] = ds;
-                            atomicAdd(GB + buf * 256 + (idx - pbase), ds);
-                            if (tg_smem) {
-                                if (b != cur) {
-                                    if (cur >= 0)
-                                        atomicAdd(TG + cur, gacc);
-                                    cur = b;
-                                    gacc = 0.f;
-                                }
-                                gacc += ds;
-                            } else {
-                                red_add_global(p.d_rab_time + b, ds * gscale);
-                            }
+                            red_add_global(p.d_rab_pos + idx, ds * gscale);
+                            red_add_global(p.d_rab_time + b, ds * gscale);
                         }
                     }
                     pk[c >> 1] = pack_bf16(pv[0], pv[1]);
                     dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
                 }
-                if (tg_smem && cur >= 0)
-                    atomicAdd(TG + cur, gacc);
             }
 
             // the previous step's dQ, deferred so the gradient MMAs overlap this step's math
@@ -550,8 +534,8 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             unsigned char *prow = sm + BL::PT + r * 128;
             unsigned char *drow = sm + BL::DST + r * 128;
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int sw = ((4 * g + u) ^ (r & 7)) << 4;
+            for (int u = 0; u < NC / 8; u++) {
+                const int sw = ((NC / 8 * g + u) ^ (r & 7)) << 4;
                 *reinterpret_cast<uint4 *>(prow + sw) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                 *reinterpret_cast<uint4 *>(drow + sw) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
             }
@@ -565,29 +549,23 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         if (tcur != 0xFFFFFFFFu && tacc != 0.f)
             atomicAdd(EG + (tcur >> 2), tacc);
         named_bar(1, kEpiThreadsB);
-        if (ok)
-            flush_pos((nq - 1) & 1, prev_cls, prev_dmin, prev_pbase);
         for (int e = etid; e < 512; e += kEpiThreadsB) {
             const float v = EG[e];
             if (v != 0.f)
                 red_add_global(p.d_rab_time + exp_bucket(e, p.nb), v * gscale);
-            if (tg_smem && e < p.nb) {
-                const float w = TG[e];
-                if (w != 0.f)
-                    red_add_global(p.d_rab_time + e, w * gscale);
-            }
         }
         if (ok && mbar_wait(bar(ACC_FULL), 0, abort_flag, p.hdr)) {
             tc_fence_after();
-            __nv_bfloat16 *gdk = static_cast<__nv_bfloat16 *>(p.dk) + (s0 + j) * p.sdk + (int64_t)h * DH + 64 * g;
-            __nv_bfloat16 *gdv = static_cast<__nv_bfloat16 *>(p.dvv) + (s0 + j) * p.sdv + (int64_t)h * DH + 64 * g;
+            constexpr int DC = DH / kGroupsB;  // dK / dV columns per thread
+            __nv_bfloat16 *gdk = static_cast<__nv_bfloat16 *>(p.dk) + (s0 + j) * p.sdk + (int64_t)h * DH + DC * g;
+            __nv_bfloat16 *gdv = static_cast<__nv_bfloat16 *>(p.dvv) + (s0 + j) * p.sdv + (int64_t)h * DH + DC * g;
 #pragma unroll
             for (int which = 0; which < 2; which++) {
-                const uint32_t col = (which ? COL_DV : COL_DK) + 64 * g;
+                const uint32_t col = (which ? COL_DV : COL_DK) + DC * g;
                 const float scale = which ? p.inv_n : gscale;
                 __nv_bfloat16 *dst = which ? gdv : gdk;
 #pragma unroll
-                for (int cc = 0; cc < 64; cc += 32) {
+                for (int cc = 0; cc < DC; cc += 32) {
                     float v[32];
                     tmem_ld32(trow + col + cc, v);
                     tmem_wait_ld();
@@ -639,7 +617,7 @@ cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t
                                CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
         e = make_tensor_map_2d(&mdq, p.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.T, cols, (int64_t)cols * 4,
-                               32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+                               32, NC, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess)
         return e;
     const size_t bytes = BL::BYTES + 1024;
