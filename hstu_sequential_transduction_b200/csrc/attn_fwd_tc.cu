@@ -70,6 +70,36 @@ __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float
     return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(E) + off);
 }
 
+// P for the 64 key columns one thread owns (one query row), packed to bf16.
+// wr[-c]: positional bias / 2 of column c; tj[c]: rebased key stamp.
+// MASK: columns c >= c_lim are not visible.  TWO: the row's columns fall in
+// at most two time buckets (hi for columns whose difference reaches `thr`).
+template <bool MASK, bool TWO>
+__device__ __forceinline__ void fwd_row(const float *sv, const float *wr, const float *tj, float ti1,
+                                        const float *E, float e_hi, float e_lo, float thr, int c_lim,
+                                        uint32_t *pk)
+{
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        float pv[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int cc = c + e;
+            float bt;
+            if (TWO)
+                bt = __fsub_rz(ti1, tj[cc]) >= thr ? e_hi : e_lo;
+            else
+                bt = time_bias_fast(ti1, tj[cc], E);
+            const float hh = fmaf(sv[cc], 0.5f, wr[-cc]) + bt;
+            float v = fmaf(hh, tanh_approx(hh), hh);
+            if (MASK)
+                v = cc < c_lim ? v : 0.f;
+            pv[e] = v;
+        }
+        pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
@@ -220,7 +250,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
 
         float wreg = 0.f;
-        int64_t treg = tb;
+        int64_t treg = tb, treg_prev = tb;
         auto prep = [&](int t) {
             const int j0 = (t < nfull ? t : qt) * TBN;
             int d = pmin - j0 - 127 + etid;
@@ -229,6 +259,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             if (etid < TBN) {
                 const int j = j0 + etid;
                 treg = j < L ? p.timestamps[s0 + j] : tb;
+                treg_prev = (j < L && etid > 0) ? p.timestamps[s0 + j - 1] : treg;
             }
         };
         prep(0);
@@ -237,13 +268,15 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             const int s = t & 1;
             const int j0 = (t < nfull ? t : qt) * TBN;
             Wb[s * 256 + etid] = wreg;
-            int kbad = 0;
+            int kbad = 0, kunsorted = 0;
             if (etid < TBN) {
                 const int64_t dt = treg - tb;
                 kbad = dt >= lim || dt <= -lim;
+                kunsorted = etid > 0 && treg_prev > treg;
                 TJb[s * TBN + etid] = (float)dt;
             }
             const bool slow_time = named_bar_or(1, kEpiThreads, kbad) || qbad;
+            const bool tj_sorted = !named_bar_or(3, kEpiThreads, kunsorted);
             const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0);
             if (t + 1 < ntiles)
                 prep(t + 1);
@@ -261,14 +294,29 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 mbar_arrive(bar(S_FREE + s));
 
             uint32_t pk[32];
-            if (full && !slow_time) {
+            // diagonal / ragged tiles without candidate rows keep the fast math
+            // with a per-column mask (positions equal indices there)
+            const bool masked_fast = !full && !slow_time && min(i0 + TBM, L) <= hist;
+            if ((full && !slow_time) || masked_fast) {
                 const float *wr = Wb + s * 256 + (pi - pmin) + 127 - 64 * g;
                 const float *tj = TJb + s * TBN + 64 * g;
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float h0 = fmaf(sv[c], 0.5f, wr[-c]) + time_bias_fast(ti1f, tj[c], E);
-                    const float h1 = fmaf(sv[c + 1], 0.5f, wr[-(c + 1)]) + time_bias_fast(ti1f, tj[c + 1], E);
-                    pk[c >> 1] = pack_bf16(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
+                if (full) {
+                    // columns are sorted by time within the tile when the key
+                    // stamps are; the row spans at most two buckets if the
+                    // first and last differences are one exponent apart
+                    const float dh = __fsub_rz(ti1f, tj[0]), dl = __fsub_rz(ti1f, tj[63]);
+                    const uint32_t bh = __float_as_uint(dh) >> 23, bl = __float_as_uint(dl) >> 23;
+                    const bool two = __all_sync(0xffffffffu, !row_ok || (tj_sorted && dl >= 1.f && bh - bl <= 1u));
+                    if (two) {
+                        const float e_hi = time_bias_fast(ti1f, tj[0], E), e_lo = time_bias_fast(ti1f, tj[63], E);
+                        fwd_row<false, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, __uint_as_float(bh << 23), 64, pk);
+                    } else {
+                        fwd_row<false, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 64, pk);
+                    }
+                } else {
+                    // visible: key j <= i and j < L
+                    const int c_lim = min(i - j0 - 64 * g + 1, L - j0 - 64 * g);
+                    fwd_row<true, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lim, pk);
                 }
             } else {
 #pragma unroll
