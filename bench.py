@@ -201,7 +201,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from hstu_sequential_transduction_b200 import ops, workloads
+    from hstu_sequential_transduction_b200 import ops, parallel, workloads
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -246,7 +246,7 @@ def run_ours(args):
         if i is not None:
             ev_b1[i].record(stream)
         if world > 1:
-            dist.all_reduce(bias_grads)
+            parallel.allreduce_bias_grads(grads[3], grads[4])
 
     def barrier():
         if world > 1:
