@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer-stack", action="store_true",
+                    help="skip the secondary eight-layer forward measurement")
     return ap.parse_args()
 
 
@@ -162,6 +164,54 @@ def cpu_baseline(inp):
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"oracle fwd+bwd, fp64, on the first {L} tokens of sequence 0 of the "
                       f"{WORKLOAD} batch (4 heads, d=128): {fl / 1e9:.1f} GFLOP in {dt:.1f} s"}
+
+
+def layer_stack_timing(dev, stream, reps: int = 3):
+    """Secondary measurement: the eight-layer bf16 stack forward (Zipf lengths,
+    D=512, 4 heads, d=128) through hstu_layer_fwd, timed with CUDA events."""
+    import torch
+
+    from hstu_sequential_transduction_b200 import flops, ops, workloads
+
+    w = workloads.WORKLOADS["layer_stack_bf16"]
+    inp = workloads.generate(w)
+    a = inp.attn
+    T = a.total_tokens
+    kw = dict(num_heads=w.num_heads, d_qk=w.d_qk, d_v=w.d_v, max_seq_len=a.max_seq_len, inv_n=a.inv_n,
+              pos_lo=a.pos_lo, pos_hi=a.pos_hi)
+    off, ts = a.seq_offsets.to(dev), a.timestamps.to(dev)
+    rp, rt = a.rab_pos.to(dev), a.rab_time.to(dev)
+    layers = [tuple(t.to(dev) for t in (lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta))
+              for lw in inp.layers]
+    xs = [inp.x.to(dev)] + [torch.empty_like(inp.x, device=dev) for _ in layers]
+    attn0 = ops.make_attn_desc(len(a.lengths), a.max_seq_len, T, w.num_heads, w.d_qk, w.d_v, ops.HSTU_BF16,
+                               a.inv_n, a.pos_lo, a.pos_hi, rt.numel())
+    desc = ops.hstu_layer_desc(attn0, w.d_model, 1e-5)
+    ws = ops.alloc_workspace(ops.hstu_layer_workspace_size(desc), dev)
+
+    def forward():
+        for li, (w1, b1, w2, b2, g, be) in enumerate(layers):
+            ops.hstu_layer_fwd(xs[li], w1, b1, w2, b2, g, be, off, ts, None, rp, rt, y=xs[li + 1],
+                               workspace=ws, stream=stream, **kw)
+
+    forward()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        forward()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    pairs = flops.attn_pairs(a.lengths)
+    attn_fl = flops.attn_fwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
+    gemm_fl = flops.f1_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
+        flops.f2_flops(T, w.d_model, w.num_heads, w.d_v)
+    total = w.num_layers * (attn_fl + gemm_fl)
+    return {"workload": "layer_stack_bf16", "layers": w.num_layers, "tokens": T,
+            "ms_per_forward": ms, "tflops": total / (ms * 1e-3) / 1e12,
+            "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
+            "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v)}
 
 
 def run_reference(args):
@@ -328,6 +378,8 @@ def run_ours(args):
         e2e = {"value": total_fl / (float(ems) * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    layer = None if args.no_layer_stack else layer_stack_timing(dev, stream)
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
@@ -355,6 +407,8 @@ def run_ours(args):
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "e2e": e2e,
         }
+        if layer is not None:
+            line["layer_stack"] = layer
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(line), flush=True)

@@ -319,7 +319,10 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
     }
     char *g = cur;
 
-    if (bf16)
+    WsHeader *hdr = static_cast<WsHeader *>(workspace);
+    if (bf16 && gemm_tc_supported(x, D, w1, uvqk, W, (int64_t)T, W, D))
+        HSTU_CUDA(launch_gemm_tc(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, hdr, st));
+    else if (bf16)
         HSTU_CUDA(launch_gemm_bf16(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, st));
     else
         HSTU_CUDA(launch_gemm_f32(static_cast<const float *>(x), D, static_cast<const float *>(w1),
@@ -330,6 +333,8 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
                               rab_pos, rab_time, o, hv, workspace, st));
     HSTU_CUDA(launch_norm_gate(bf16, o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv,
                                (int64_t)T, hv, st));
+    if (bf16 && gemm_tc_supported(g, hv, w2, y, D, (int64_t)T, D, hv))
+        return cuda_status(launch_gemm_tc(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
     if (bf16)
         return cuda_status(launch_gemm_bf16(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, st));
     return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(g), hv,

@@ -53,6 +53,11 @@ cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int 
 // lda, ldc in elements; B is dense [K, N].
 cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
                              int64_t ldc, int64_t M, int N, int K, bool silu, cudaStream_t stream);
+// The same on tcgen05 / TMA (sm_100a): K a multiple of 64, N of 128; hdr receives
+// a timeout flag if a pipeline wait ever gives up.
+bool gemm_tc_supported(const void *A, int64_t lda, const void *Bm, void *C, int64_t ldc, int64_t M, int N, int K);
+cudaError_t launch_gemm_tc(const void *A, int64_t lda, const void *Bm, const void *bias, void *C, int64_t ldc,
+                           int64_t M, int N, int K, bool silu, WsHeader *hdr, cudaStream_t stream);
 cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const float *bias,
                             float *C, int64_t ldc, int64_t M, int N, int K, bool silu,
                             cudaStream_t stream);
