@@ -184,7 +184,66 @@ __device__ __forceinline__ void st<float>(float *p, float v) { *p = v; }
 template <>
 __device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
 
-// One warp per token; lane l holds features l*VPT .. l*VPT + VPT - 1.
+// VPT contiguous elements of a row as floats, with the widest aligned vector loads.
+template <typename T, int VPT>
+__device__ __forceinline__ void load_vec(const T *p, float *x)
+{
+    constexpr int BYTES = VPT * (int)sizeof(T);
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+        for (int b = 0; b < BYTES / 16; b++) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p) + b);
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&u[k]);
+                    x[8 * b + 2 * k] = __low2float(h);
+                    x[8 * b + 2 * k + 1] = __high2float(h);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    x[4 * b + k] = __uint_as_float(u[k]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            x[e] = ld<T>(p + e);
+    }
+}
+
+template <typename T, int VPT>
+__device__ __forceinline__ void store_vec(T *p, const float *y)
+{
+    constexpr int BYTES = VPT * (int)sizeof(T);
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+        for (int b = 0; b < BYTES / 16; b++) {
+            uint4 w;
+            if constexpr (sizeof(T) == 2) {
+                w.x = pack_bf16(y[8 * b], y[8 * b + 1]);
+                w.y = pack_bf16(y[8 * b + 2], y[8 * b + 3]);
+                w.z = pack_bf16(y[8 * b + 4], y[8 * b + 5]);
+                w.w = pack_bf16(y[8 * b + 6], y[8 * b + 7]);
+            } else {
+                w.x = __float_as_uint(y[4 * b]);
+                w.y = __float_as_uint(y[4 * b + 1]);
+                w.z = __float_as_uint(y[4 * b + 2]);
+                w.w = __float_as_uint(y[4 * b + 3]);
+            }
+            reinterpret_cast<uint4 *>(p)[b] = w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            st<T>(p + e, y[e]);
+    }
+}
+
+// One warp per token; lane l holds features l*VPT .. l*VPT + VPT - 1, moved
+// with 16-byte vector loads and stores (memory-bound: read O and U, write G).
 template <typename T, int VPT>
 __global__ void __launch_bounds__(256)
 norm_gate_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, int64_t ldu,
@@ -196,14 +255,15 @@ norm_gate_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, 
     const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (row >= Trows)
         return;
-    const T *o = O + row * ldo + lane * VPT;
-    float x[VPT];
+    float x[VPT], u[VPT], ga[VPT], be[VPT];
+    load_vec<T, VPT>(O + row * ldo + lane * VPT, x);
+    load_vec<T, VPT>(U + row * ldu + lane * VPT, u);
+    load_vec<float, VPT>(gamma + lane * VPT, ga);
+    load_vec<float, VPT>(beta + lane * VPT, be);
     float sum = 0.f;
 #pragma unroll
-    for (int e = 0; e < VPT; e++) {
-        x[e] = ld<T>(o + e);
+    for (int e = 0; e < VPT; e++)
         sum += x[e];
-    }
 #pragma unroll
     for (int off = 16; off; off >>= 1)
         sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -218,14 +278,11 @@ norm_gate_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, 
     for (int off = 16; off; off >>= 1)
         var += __shfl_xor_sync(0xffffffffu, var, off);
     const float rstd = rsqrtf(var * (1.0f / F) + eps);
-    const T *u = U + row * ldu + lane * VPT;
-    T *gout = G + row * ldg + lane * VPT;
+    float y[VPT];
 #pragma unroll
-    for (int e = 0; e < VPT; e++) {
-        const int c = lane * VPT + e;
-        const float y = ((x[e] - mean) * rstd * gamma[c] + beta[c]) * ld<T>(u + e);
-        st<T>(gout + e, y);
-    }
+    for (int e = 0; e < VPT; e++)
+        y[e] = ((x[e] - mean) * rstd * ga[e] + be[e]) * u[e];
+    store_vec<T, VPT>(G + row * ldg + lane * VPT, y);
 }
 
 template <typename T>
