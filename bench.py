@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-stack", action="store_true",
                     help="skip the secondary eight-layer forward measurement")
+    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer"], default=None,
+                    help="run only a small case twice (for ncu captures) and exit")
     return ap.parse_args()
 
 
@@ -417,8 +419,41 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def kernel_case(which: str):
+    """A small case of one kernel, run twice, for ncu captures: 3 sequences of
+    11k-13k tokens (long-history shapes, ~36k tokens, inputs > L2), or one
+    eight-layer stack forward."""
+    import numpy as np
+    import torch
+
+    from hstu_sequential_transduction_b200 import ops, workloads
+
+    dev = torch.device("cuda:0")
+    if which == "layer":
+        layer_stack_timing(dev, torch.cuda.current_stream(), reps=1)
+        torch.cuda.synchronize()
+        return
+    rng = np.random.default_rng(7)
+    inp = workloads.make_attn_inputs(rng, [12000, 11000, 13000], 4, 128, 128, 300.0, -4096, 4096, 128, 16384,
+                                     torch.bfloat16, with_dout=True)
+    d = {k: (getattr(inp, k).to(dev) if getattr(inp, k) is not None else None)
+         for k in ("q", "k", "v", "seq_offsets", "timestamps", "rab_pos", "rab_time", "dout")}
+    kw = dict(max_seq_len=inp.max_seq_len, inv_n=inp.inv_n, pos_lo=inp.pos_lo, pos_hi=inp.pos_hi)
+    for _ in range(2):
+        if which == "fwd":
+            ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None, d["rab_pos"],
+                              d["rab_time"], **kw)
+        else:
+            ops.hstu_attn_bwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None, d["rab_pos"],
+                              d["rab_time"], d["dout"], **kw)
+    torch.cuda.synchronize()
+
+
 def main():
     args = parse_args()
+    if args.kernel_case:
+        kernel_case(args.kernel_case)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
