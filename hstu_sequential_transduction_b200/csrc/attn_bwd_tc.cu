@@ -28,7 +28,8 @@
 // warps 2-9 epilogue (lane quarter = warp % 4 selects the TMEM rows, the two
 // warpgroups split each step's 64 query columns).
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,320), dP^T [320,384),
-// dQ^T [384,448).
+// dQ^T [384,448), and the bf16 P^T [448,480) and dS'^T [480,512) of a step,
+// which the dV and dK MMAs read as their A operands straight from TMEM.
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -47,7 +48,7 @@ constexpr int NC = QB / kGroupsB;                // query columns per epilogue t
 constexpr uint32_t kTmemColsB = 512;
 constexpr int kRegK = 16384;  // 128 rows x 128 B
 constexpr int kRegQ = 8192;   // 64 rows x 128 B
-constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384, COL_PT = 448, COL_DST = 480;
 
 enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 3, S_FULL = 5, S_FREE = 6, P_FULL = 7, P_FREE = 8,
              DQ_FULL = 9, DQ_FREE = 10, ACC_FULL = 11, NBARS_B = 12 };
@@ -57,8 +58,7 @@ struct BL {
     static constexpr int V = K + 2 * kRegK;
     static constexpr int Q0 = V + 2 * kRegK;       // 2 stages x 2 regions
     static constexpr int O0 = Q0 + 4 * kRegQ;      // dO, 2 stages x 2 regions
-    static constexpr int PT = O0 + 4 * kRegQ;      // P^T  [128 keys x 64 queries]
-    static constexpr int DST = PT + kRegK;         // dS'^T
+    static constexpr int DST = O0 + 4 * kRegQ;     // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
     static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, per warp [NC x 32]
     static constexpr int E = DQS + QB * DH * 4;    // time bias by exponent (512)
     static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
@@ -103,47 +103,76 @@ struct RowOut {
     bool mid;         // a visible column falls in a bucket other than b0 and b1
 };
 
+// Time-bucket modes of a 32 x NC block (decided per warp from the extreme
+// stamp differences of its sorted rows and columns).
+enum BucketMode { BK_ANY = 0, BK_ONE = 1, BK_TWO = 2 };
+
 // Elementwise backward of the NC query columns one thread owns (one key row):
 // P = SiLU, dS' = dP (1+t)(1+h(1-t)); dS' replaces dP in dv[], P is packed.
-// Columns outside [c_lo, c_hi) are masked when MASK.  TWO: the step is known
-// to put every key row in at most two time buckets (sorted stamps, narrow
-// span), so the bucket is one compare of the exact round-toward-zero
-// difference against the upper bucket's power of two.  No atomics, no
-// data-dependent branches.
-template <bool MASK, bool WINDOW, bool TWO>
-__device__ __forceinline__ RowOut bwd_row(const float *sv, float *dv, const float *ti, float tjf, const char *Eb,
+// Columns outside [c_lo, c_hi) are masked when MASK.  The time bucket of a
+// column: BK_ONE, the whole block is in one bucket; BK_TWO, every row spans
+// at most two buckets, so the bucket is one compare of the exact
+// round-toward-zero difference against the upper bucket's power of two;
+// BK_ANY, looked up per column.  No atomics, no data-dependent branches.
+// Written as three passes over the columns (biased half-scores, tanh,
+// products) so that the independent per-column chains are issued back to
+// back instead of one after the other.
+template <bool MASK, bool WINDOW, int MODE>
+__device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti, float tjf, const char *Eb,
                                           const float *wrow, float bconst, int c_lo, int c_hi, uint32_t *pk)
 {
     RowOut o;
     const int f = MASK ? min(max(c_lo, 0), NC - 1) : 0, l = MASK ? min(max(c_hi - 1, 0), NC - 1) : NC - 1;
     o.b0 = exp_offset(ti[f], tjf);
-    o.b1 = exp_offset(ti[l], tjf);
+    o.b1 = MODE == BK_ONE ? o.b0 : exp_offset(ti[l], tjf);
     const float E0 = *reinterpret_cast<const float *>(Eb + o.b0);
     const float E1 = *reinterpret_cast<const float *>(Eb + o.b1);
     const float thr = __uint_as_float(o.b1 << 21);  // 2^(bucket of b1), exact
-    o.all = 0.f;
-    o.hi = 0.f;
     o.mid = false;
+    float upf[NC];  // 1 where the column is in bucket b1
+#pragma unroll
+    for (int u = 0; u < NC / 4; u++) {
+        float tv[4];
+        if (MODE != BK_ONE) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(ti + 4 * u);  // stamps are shared by the warp
+            tv[0] = t4.x;
+            tv[1] = t4.y;
+            tv[2] = t4.z;
+            tv[3] = t4.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int c = 4 * u + e;
+            float bt;
+            if (MODE == BK_ONE) {
+                bt = E0;
+                upf[c] = 0.f;
+            } else if (MODE == BK_TWO) {
+                const bool up = __fsub_rz(tv[e], tjf) >= thr;
+                upf[c] = up ? 1.f : 0.f;
+                bt = up ? E1 : E0;
+            } else {
+                const uint32_t off = exp_offset(tv[e], tjf);
+                bt = *reinterpret_cast<const float *>(Eb + off);
+                upf[c] = off == o.b1 ? 1.f : 0.f;
+                o.mid |= (!MASK || (c >= c_lo && c < c_hi)) && (off != o.b0) && (off != o.b1);
+            }
+            const float bp = WINDOW ? wrow[c] : bconst;
+            sv[c] = fmaf(sv[c], 0.5f, bp) + bt;
+        }
+    }
+    float th[NC];
+#pragma unroll
+    for (int c = 0; c < NC; c++)
+        th[c] = tanh_approx(sv[c]);
+    float all = 0.f, hi = 0.f;
 #pragma unroll
     for (int c = 0; c < NC; c += 2) {
         float pv[2];
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const int cc = c + e;
-            float bt;
-            bool up;
-            if (TWO) {
-                up = __fsub_rz(ti[cc], tjf) >= thr;
-                bt = up ? E1 : E0;
-            } else {
-                const uint32_t off = exp_offset(ti[cc], tjf);
-                bt = *reinterpret_cast<const float *>(Eb + off);
-                up = off == o.b1;
-                o.mid |= (!MASK || (cc >= c_lo && cc < c_hi)) && (off != o.b0) && (off != o.b1);
-            }
-            const float bp = WINDOW ? wrow[cc] : bconst;
-            const float hh = fmaf(sv[cc], 0.5f, bp) + bt;
-            const float t = tanh_approx(hh);
+            const float hh = sv[cc], t = th[cc];
             float pval = fmaf(hh, t, hh);
             const float a = 1.f + t;
             float ds = dv[cc] * fmaf(a, fmaf(-hh, t, hh), a);
@@ -154,11 +183,14 @@ __device__ __forceinline__ RowOut bwd_row(const float *sv, float *dv, const floa
             }
             dv[cc] = ds;
             pv[e] = pval;
-            o.all += ds;
-            o.hi += up ? ds : 0.f;
+            all += ds;
+            if (MODE != BK_ONE)
+                hi = fmaf(upf[cc], ds, hi);
         }
         pk[c >> 1] = pack_bf16(pv[0], pv[1]);
     }
+    o.all = all;
+    o.hi = hi;
     return o;
 }
 
@@ -171,10 +203,12 @@ __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float 
     accN = 0.f;
 #pragma unroll
     for (int k = 0; k < NC; k++) {
-        const float y = __shfl_sync(0xffffffffu, ds[k], (k - lane) & 31);
-        const bool pos = k >= lane;
-        accP += pos ? y : 0.f;
-        accN += pos ? 0.f : y;
+        // the source lane is taken modulo 32: k - lane wraps to the row on diagonal lane or lane - 32
+        const float y = __shfl_sync(0xffffffffu, ds[k], k - lane);
+        if (k >= lane)
+            accP += y;
+        else
+            accN += y;
     }
 }
 
@@ -274,12 +308,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             };
             auto issue_grads = [&](int i) {
                 const int s = i & 1;
+                // A = P^T / dS'^T from TMEM (lane = key, column = query pair)
                 for (int ks = 0; ks < QB / 16; ks++) {
                     const uint32_t acc = (i > 0 || ks > 0);
-                    umma_bf16(tmem + COL_DV, smem_desc_sw128(base + BL::PT + ks * 32, 16, 1024),
-                              smem_desc_sw128(base + BL::O0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
-                    umma_bf16(tmem + COL_DK, smem_desc_sw128(base + BL::DST + ks * 32, 16, 1024),
-                              smem_desc_sw128(base + BL::Q0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                    umma_bf16_ts(tmem + COL_DV, tmem + COL_PT + 8 * ks,
+                                 smem_desc_sw128(base + BL::O0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                    umma_bf16_ts(tmem + COL_DK, tmem + COL_DST + 8 * ks,
+                                 smem_desc_sw128(base + BL::Q0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
                 }
             };
             auto issue_dq = [&]() {
@@ -434,11 +469,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 else if (q_last < hist)
                     cls = full_w ? CLS_WINDOW : CLS_WINDOW_MASKED;
             }
-            bool two = false;
+            int mode = BK_ANY;
             if (cls != CLS_GENERAL && q_last >= iw0 && jw_n > 0) {
                 const float dlo = __fsub_rz(TIw[0], tjf_last);
                 const float dhi = __fsub_rz(TIw[q_last - iw0], tjf_first);
-                two = dlo >= 1.f && ((__float_as_uint(dhi) >> 23) - (__float_as_uint(dlo) >> 23)) <= 1u;
+                const uint32_t de = (__float_as_uint(dhi) >> 23) - (__float_as_uint(dlo) >> 23);
+                if (dlo >= 1.f)
+                    mode = de == 0 ? BK_ONE : (de == 1 ? BK_TWO : BK_ANY);
             }
 
             if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
@@ -457,8 +494,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             if (cls != CLS_GENERAL) {
                 RowOut o;
                 if (cls == CLS_CLAMPED) {
-                    o = two ? bwd_row<false, false, true>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk)
-                            : bwd_row<false, false, false>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
+                    if (mode == BK_ONE)
+                        o = bwd_row<false, false, BK_ONE>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
+                    else if (mode == BK_TWO)
+                        o = bwd_row<false, false, BK_TWO>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
+                    else
+                        o = bwd_row<false, false, BK_ANY>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
                     float sum = o.all;
 #pragma unroll
                     for (int s = 16; s; s >>= 1)
@@ -468,10 +509,11 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 } else {
                     const float *wrow = Ww + 31 - lane;  // wrow[c]: diagonal c - lane
                     if (cls == CLS_WINDOW)
-                        o = two ? bwd_row<false, true, true>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
-                                : bwd_row<false, true, false>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk);
+                        o = mode == BK_ONE   ? bwd_row<false, true, BK_ONE>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
+                            : mode == BK_TWO ? bwd_row<false, true, BK_TWO>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
+                                             : bwd_row<false, true, BK_ANY>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk);
                     else
-                        o = bwd_row<true, true, false>(sv, dv, TIw, tjf, Eb, wrow, 0.f, j - iw0,
+                        o = bwd_row<true, true, BK_ANY>(sv, dv, TIw, tjf, Eb, wrow, 0.f, j - iw0,
                                                        krow_ok ? min(NC, L - iw0) : 0, pk);
                     float accP, accN;
                     warp_diagonals(dv, lane, accP, accN);
@@ -527,18 +569,21 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             // the previous step's dQ, deferred so the gradient MMAs overlap this step's math
             if (i > 0 && !(ok = handle_dq(i - 1)))
                 break;
-            // P^T and dS'^T rows of this thread (K-major, 128B swizzle) once the
-            // previous step's gradient MMAs have finished reading them
+            // P^T and dS'^T of this thread's row to TMEM, dS'^T also to shared
+            // memory (K-major, 128B swizzle), once the previous step's gradient
+            // and dQ MMAs have finished reading them
             if (i > 0 && !(ok = mbar_wait(bar(P_FREE), (i - 1) & 1, abort_flag, p.hdr)))
                 break;
-            unsigned char *prow = sm + BL::PT + r * 128;
+            tmem_st16(trow + COL_PT + (NC / 2) * g, pk);
+            tmem_st16(trow + COL_DST + (NC / 2) * g, dk);
             unsigned char *drow = sm + BL::DST + r * 128;
 #pragma unroll
             for (int u = 0; u < NC / 8; u++) {
                 const int sw = ((NC / 8 * g + u) ^ (r & 7)) << 4;
-                *reinterpret_cast<uint4 *>(prow + sw) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                 *reinterpret_cast<uint4 *>(drow + sw) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
             }
+            tmem_wait_st();
+            tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
