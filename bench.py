@@ -40,6 +40,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels of ours launched per step: fwd call (schedule, attention) and bwd call
 # (schedule, attention backward, dq conversion)
 LAUNCHES_PER_STEP = 5
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention-backward launch on
+# this workload, from a one-pass ncu capture of
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd_tc -c 1
+#       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
+# valid only for the kernel source it was taken on (else the line reports null)
+BWD_TRAFFIC = {"source_sha256": "3e82e0ae3d19d9d2a7a60ed1a046b44a89f3cb9d749a30c8cb3547696fb3dbf9",
+               "bytes": 5.24e9 + 2.89e9}
+
+
+def bwd_traffic():
+    import hashlib
+    path = os.path.join(ROOT, "hstu_sequential_transduction_b200", "csrc", "attn_bwd_tc.cu")
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return BWD_TRAFFIC["bytes"] if digest == BWD_TRAFFIC["source_sha256"] else None
 
 
 def parse_args():
@@ -403,7 +421,7 @@ def run_ours(args):
             "pct_of_bf16_peak": 100 * (value / world) / burst,
             "roofline": {"bound": "tensor", "kernel": "attention backward (hstu_attn_bwd call)",
                          "achieved": bwd_tf, "peak": sustained, "unit": "TFLOP/s",
-                         "frac": bwd_tf / sustained, "traffic": None,
+                         "frac": bwd_tf / sustained, "traffic": bwd_traffic(),
                          "peak_source": f"bf16_tflops_sustained, {peak_src}"},
             "clocks": clocks,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
