@@ -74,29 +74,63 @@ __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float
 // wr[-c]: positional bias / 2 of column c; tj[c]: rebased key stamp.
 // MASK: columns c >= c_lim are not visible.  TWO: the row's columns fall in
 // at most two time buckets (hi for columns whose difference reaches `thr`).
-template <bool MASK, bool TWO>
-__device__ __forceinline__ void fwd_row(const float *sv, const float *wr, const float *tj, float ti1,
+// MODE: 0 time bucket looked up per column, 1 one bucket for the whole row
+// (e_hi), 2 two buckets split at thr.  CONSTB: the positional index is clamped
+// for every column, so the positional bias is wr[0].
+template <bool MASK, int MODE, bool CONSTB>
+__device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float *tj, float ti1,
                                         const float *E, float e_hi, float e_lo, float thr, int c_lim,
                                         uint32_t *pk)
 {
+    const float bconst = CONSTB ? wr[0] + (MODE == 1 ? e_hi : 0.f) : 0.f;
+    // three passes per 32 columns (biased half-scores, tanh, products) so the
+    // independent per-column chains issue back to back
 #pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        float pv[2];
+    for (int hb = 0; hb < 64; hb += 32) {
 #pragma unroll
-        for (int e = 0; e < 2; e++) {
-            const int cc = c + e;
-            float bt;
-            if (TWO)
-                bt = __fsub_rz(ti1, tj[cc]) >= thr ? e_hi : e_lo;
-            else
-                bt = time_bias_fast(ti1, tj[cc], E);
-            const float hh = fmaf(sv[cc], 0.5f, wr[-cc]) + bt;
-            float v = fmaf(hh, tanh_approx(hh), hh);
-            if (MASK)
-                v = cc < c_lim ? v : 0.f;
-            pv[e] = v;
+        for (int u = 0; u < 8; u++) {
+            float tv[4];
+            if (MODE != 1) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(tj + hb + 4 * u);  // shared by the warp
+                tv[0] = t4.x;
+                tv[1] = t4.y;
+                tv[2] = t4.z;
+                tv[3] = t4.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int cc = hb + 4 * u + e;
+                if (CONSTB && MODE == 1) {
+                    sv[cc] = fmaf(sv[cc], 0.5f, bconst);
+                    continue;
+                }
+                float bt;
+                if (MODE == 1)
+                    bt = e_hi;
+                else if (MODE == 2)
+                    bt = __fsub_rz(ti1, tv[e]) >= thr ? e_hi : e_lo;
+                else
+                    bt = time_bias_fast(ti1, tv[e], E);
+                sv[cc] = fmaf(sv[cc], 0.5f, CONSTB ? wr[0] : wr[-cc]) + bt;
+            }
         }
-        pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+        float th[32];
+#pragma unroll
+        for (int c = 0; c < 32; c++)
+            th[c] = tanh_approx(sv[hb + c]);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+            float pv[2];
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                const int cc = hb + c + e;
+                float v = fmaf(sv[cc], th[c + e], sv[cc]);
+                if (MASK)
+                    v = cc < c_lim ? v : 0.f;
+                pv[e] = v;
+            }
+            pk[(hb + c) >> 1] = pack_bf16(pv[0], pv[1]);
+        }
     }
 }
 
@@ -306,17 +340,31 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     // first and last differences are one exponent apart
                     const float dh = __fsub_rz(ti1f, tj[0]), dl = __fsub_rz(ti1f, tj[63]);
                     const uint32_t bh = __float_as_uint(dh) >> 23, bl = __float_as_uint(dl) >> 23;
-                    const bool two = __all_sync(0xffffffffu, !row_ok || (tj_sorted && dl >= 1.f && bh - bl <= 1u));
-                    if (two) {
-                        const float e_hi = time_bias_fast(ti1f, tj[0], E), e_lo = time_bias_fast(ti1f, tj[63], E);
-                        fwd_row<false, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, __uint_as_float(bh << 23), 64, pk);
+                    const bool srt = tj_sorted && dl >= 1.f;
+                    const bool one = __all_sync(0xffffffffu, !row_ok || (srt && bh == bl));
+                    const bool two = __all_sync(0xffffffffu, !row_ok || (srt && bh - bl <= 1u));
+                    // every column past the positional clamp (full tiles hold history keys only)
+                    const int dnear = pi - (j0 + 64 * g + 63), dfar = pi - (j0 + 64 * g);
+                    const bool cst = __all_sync(0xffffffffu, !row_ok || dnear >= p.pos_hi || dfar <= p.pos_lo);
+                    const float e_hi = time_bias_fast(ti1f, tj[0], E), e_lo = time_bias_fast(ti1f, tj[63], E);
+                    const float thr = __uint_as_float(bh << 23);
+                    if (one) {
+                        if (cst)
+                            fwd_row<false, 1, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                        else
+                            fwd_row<false, 1, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                    } else if (two) {
+                        if (cst)
+                            fwd_row<false, 2, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                        else
+                            fwd_row<false, 2, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
                     } else {
-                        fwd_row<false, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 64, pk);
+                        fwd_row<false, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 64, pk);
                     }
                 } else {
                     // visible: key j <= i and j < L
                     const int c_lim = min(i - j0 - 64 * g + 1, L - j0 - 64 * g);
-                    fwd_row<true, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lim, pk);
+                    fwd_row<true, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lim, pk);
                 }
             } else {
 #pragma unroll
