@@ -283,17 +283,24 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         float *TJb = reinterpret_cast<float *>(sm + LY::TJ);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
 
+        // loads of the next tile's inputs; nothing here consumes a loaded value,
+        // so the loads stay in flight while this tile is processed
         float wreg = 0.f;
         int64_t treg = tb, treg_prev = tb;
         auto prep = [&](int t) {
             const int j0 = (t < nfull ? t : qt) * TBN;
             int d = pmin - j0 - 127 + etid;
             d = d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d);
-            wreg = 0.5f * p.rab_pos[d - p.pos_lo];
+            wreg = p.rab_pos[d - p.pos_lo];
             if (etid < TBN) {
                 const int j = j0 + etid;
-                treg = j < L ? p.timestamps[s0 + j] : tb;
-                treg_prev = (j < L && etid > 0) ? p.timestamps[s0 + j - 1] : treg;
+                treg = tb;
+                treg_prev = tb;
+                if (j < L) {
+                    treg = p.timestamps[s0 + j];
+                    if (etid > 0)
+                        treg_prev = p.timestamps[s0 + j - 1];
+                }
             }
         };
         prep(0);
@@ -301,7 +308,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         for (int t = 0; t < ntiles; t++) {
             const int s = t & 1;
             const int j0 = (t < nfull ? t : qt) * TBN;
-            Wb[s * 256 + etid] = wreg;
+            Wb[s * 256 + etid] = 0.5f * wreg;
             int kbad = 0, kunsorted = 0;
             if (etid < TBN) {
                 const int64_t dt = treg - tb;
