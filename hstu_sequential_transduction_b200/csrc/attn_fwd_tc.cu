@@ -13,9 +13,11 @@
 //              thread: S_j = Q K_j^T into one of two S buffers, O += P_j V_j;
 //   warps 2-9  epilogue: two warpgroups, each takes 64 of the 128 key columns
 //              of every S tile: tcgen05.ld, relative bias, SiLU, bf16 pack, and
-//              the swizzled store of P into shared memory (the A operand of
-//              P V); at the end they read O from TMEM and write it out.
-// TMEM columns: S buffers [0,128) and [128,256), O [256, 256 + D).
+//              tcgen05.st of P over the first 32 of its own S columns, where the
+//              P V MMA reads it as its A operand; at the end they read O from
+//              TMEM and write it out.
+// TMEM columns: S buffers [0,128) and [128,256), O [256, 256 + D).  S_{j+2}
+// reuses buffer j % 2 once P_j V_j has completed.
 //
 // Epilogue arithmetic on full tiles (every pair visible, timestamps of the
 // tile within 2^24 s of the query tile's first stamp):
@@ -44,8 +46,11 @@ constexpr int kThreadsTc = kEpiThreads + 64;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRegion = 16384;  // one 128-row x 128-byte swizzled region
 
-enum Bars { Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, S_FREE = 11,
-            P_FULL = 13, P_FREE = 14, O_FULL = 15, NBARS = 16 };
+// P_FULL + b: P of the tile in S buffer b is in TMEM (one barrier per buffer, so
+// the epilogue can never be two phases ahead of the MMA thread on one of them);
+// P_FREE: P_j V_j has completed (its A operand, P_j in TMEM, is consumed)
+enum Bars { Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, P_FULL = 11,
+            P_FREE = 13, O_FULL = 14, NBARS = 15 };
 
 template <int D>
 struct FwdLayout {
@@ -54,11 +59,11 @@ struct FwdLayout {
     static constexpr int Q = 0;
     static constexpr int K0 = Q + TILE;
     static constexpr int V0 = K0 + 2 * TILE;
-    static constexpr int P = V0 + 2 * TILE;
-    static constexpr int E = P + 2 * kRegion;
-    static constexpr int W = E + 512 * 4;
-    static constexpr int TJ = W + 2 * 256 * 4;
-    static constexpr int BAR = TJ + 2 * 128 * 4;
+    static constexpr int E = V0 + 2 * TILE;
+    // per epilogue warp: 64 key stamps + 96-entry positional-bias window of a tile
+    static constexpr int PW = E + 512 * 4;
+    static constexpr int PW_FLOATS = 64 + 96;
+    static constexpr int BAR = PW + kEpiWarps * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS * 8;
     static constexpr int BYTES = MISC + 64;
 };
@@ -165,7 +170,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS; i++) {
-            const bool epi = (i == S_FREE || i == S_FREE + 1 || i == P_FULL);
+            const bool epi = (i == P_FULL || i == P_FULL + 1);
             mbar_init(bar(i), epi ? kEpiWarps : 1);
         }
         *abort_flag = 0;
@@ -231,10 +236,11 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             };
             auto issue_PV = [&](int t) {
                 const int s = t & 1;
+                // A = P_t from TMEM: keys 16 ks .. sit in S buffer columns 64 (ks / 4) + 8 (ks % 4)
                 for (int ks = 0; ks < TBN / 16; ks++) {
-                    const uint64_t a = smem_desc_sw128(base + LY::P + (ks >> 2) * kRegion + (ks & 3) * 32, 16, 1024);
                     const uint64_t b = smem_desc_sw128(base + LY::V0 + s * LY::TILE + ks * 2048, kRegion, 1024);
-                    umma_bf16(tmem + 2 * TBN, a, b, idO, (t > 0 || ks > 0));
+                    umma_bf16_ts(tmem + 2 * TBN, tmem + s * TBN + 64 * (ks >> 2) + 8 * (ks & 3), b, idO,
+                                 (t > 0 || ks > 0));
                 }
                 umma_commit(bar(V_EMPTY + s));
                 umma_commit(bar(P_FREE));
@@ -248,14 +254,14 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 }
             }
             for (int j = 0; ok && j < ntiles; j++) {
-                ok = mbar_wait(bar(P_FULL), j & 1, abort_flag, p.hdr) &&
+                ok = mbar_wait(bar(P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr) &&
                      mbar_wait(bar(V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr);
                 if (!ok)
                     break;
                 tc_fence_after();
                 issue_PV(j);
                 if (j + 2 < ntiles) {
-                    ok = mbar_wait(bar(S_FREE + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr) &&
+                    ok = mbar_wait(bar(P_FREE), j & 1, abort_flag, p.hdr) &&
                          mbar_wait(bar(K_FULL + (j & 1)), ((j + 2) >> 1) & 1, abort_flag, p.hdr);
                     if (!ok)
                         break;
@@ -268,56 +274,62 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
     } else {
         // ---------------- epilogue ----------------
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
-        const int etid = threadIdx.x - 64;
         const int r = quarter * 32 + lane;
         const int i = i0 + r;
         const bool row_ok = i < L;
         const int64_t tb = p.timestamps[s0 + i0];
         const int64_t ti = row_ok ? p.timestamps[s0 + i] : tb;
         const int pi = token_pos(i, hist);
-        const int pmin = token_pos(i0, hist);
         const int64_t lim = (int64_t)1 << 24;
-        const int qbad = named_bar_or(1, kEpiThreads, (ti - tb + 1 >= lim) || (ti - tb + 1 <= -lim));
+        const uint32_t full_mask = 0xffffffffu;
+        const bool qbad = __any_sync(full_mask, (ti - tb + 1 >= lim) || (ti - tb + 1 <= -lim));
         const float ti1f = (float)(ti - tb + 1);
-        float *Wb = reinterpret_cast<float *>(sm + LY::W);
-        float *TJb = reinterpret_cast<float *>(sm + LY::TJ);
+        // this warp's 32 rows x 64 key columns of a tile: its own stamps and bias
+        // window, so the loop needs no barrier wider than a warp
+        float *TJw = reinterpret_cast<float *>(sm + LY::PW) + ew * LY::PW_FLOATS;  // key stamp - tb
+        // Ww[m]: positional bias / 2 at offset pw - jw - 63 + m, pw = the warp's first row position
+        // (positions grow with the row, candidates share one, so a row's pi - pw is in [0, 31])
+        float *Ww = TJw + 64;
+        const int pw = token_pos(i0 + 32 * quarter, hist);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        auto clamp_idx = [&](int d) { return (d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d)) - p.pos_lo; };
 
         // loads of the next tile's inputs; nothing here consumes a loaded value,
         // so the loads stay in flight while this tile is processed
-        float wreg = 0.f;
-        int64_t treg = tb, treg_prev = tb;
+        float w0 = 0.f, w1 = 0.f, w2 = 0.f;
+        int64_t ta = tb, tc = tb;  // stamps of key columns 2 lane, 2 lane + 1
         auto prep = [&](int t) {
-            const int j0 = (t < nfull ? t : qt) * TBN;
-            int d = pmin - j0 - 127 + etid;
-            d = d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d);
-            wreg = p.rab_pos[d - p.pos_lo];
-            if (etid < TBN) {
-                const int j = j0 + etid;
-                treg = tb;
-                treg_prev = tb;
-                if (j < L) {
-                    treg = p.timestamps[s0 + j];
-                    if (etid > 0)
-                        treg_prev = p.timestamps[s0 + j - 1];
-                }
-            }
+            const int jw = (t < nfull ? t : qt) * TBN + 64 * g;
+            const int dbase = pw - jw - 63;
+            w0 = p.rab_pos[clamp_idx(dbase + lane)];
+            w1 = p.rab_pos[clamp_idx(dbase + lane + 32)];
+            w2 = p.rab_pos[clamp_idx(dbase + lane + 64)];
+            const int j = jw + 2 * lane;
+            ta = tb;
+            tc = tb;
+            if (j < L)
+                ta = p.timestamps[s0 + j];
+            if (j + 1 < L)
+                tc = p.timestamps[s0 + j + 1];
         };
         prep(0);
         bool ok = true;
         for (int t = 0; t < ntiles; t++) {
             const int s = t & 1;
             const int j0 = (t < nfull ? t : qt) * TBN;
-            Wb[s * 256 + etid] = 0.5f * wreg;
-            int kbad = 0, kunsorted = 0;
-            if (etid < TBN) {
-                const int64_t dt = treg - tb;
-                kbad = dt >= lim || dt <= -lim;
-                kunsorted = etid > 0 && treg_prev > treg;
-                TJb[s * TBN + etid] = (float)dt;
-            }
-            const bool slow_time = named_bar_or(1, kEpiThreads, kbad) || qbad;
-            const bool tj_sorted = !named_bar_or(3, kEpiThreads, kunsorted);
+            const int j = j0 + 64 * g + 2 * lane;
+            const int64_t ta_next = __shfl_down_sync(full_mask, ta, 1);
+            const bool kbad = (j < L && (ta - tb >= lim || ta - tb <= -lim)) ||
+                              (j + 1 < L && (tc - tb >= lim || tc - tb <= -lim));
+            const bool kunsorted = (j + 1 < L && ta > tc) || (lane < 31 && j + 2 < L && tc > ta_next);
+            const bool slow_time = __any_sync(full_mask, kbad) || qbad;
+            const bool tj_sorted = !__any_sync(full_mask, kunsorted);
+            __syncwarp();
+            *reinterpret_cast<float2 *>(TJw + 2 * lane) = make_float2((float)(ta - tb), (float)(tc - tb));
+            Ww[lane] = 0.5f * w0;
+            Ww[lane + 32] = 0.5f * w1;
+            Ww[lane + 64] = 0.5f * w2;
+            __syncwarp();
             const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0);
             if (t + 1 < ntiles)
                 prep(t + 1);
@@ -329,18 +341,14 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             tmem_ld32(trow + s * TBN + 64 * g, sv);
             tmem_ld32(trow + s * TBN + 64 * g + 32, sv + 32);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar(S_FREE + s));
 
             uint32_t pk[32];
             // diagonal / ragged tiles without candidate rows keep the fast math
             // with a per-column mask (positions equal indices there)
             const bool masked_fast = !full && !slow_time && min(i0 + TBM, L) <= hist;
             if ((full && !slow_time) || masked_fast) {
-                const float *wr = Wb + s * 256 + (pi - pmin) + 127 - 64 * g;
-                const float *tj = TJb + s * TBN + 64 * g;
+                const float *wr = Ww + (pi - pw) + 63;  // wr[-c]: key column c of this row
+                const float *tj = TJw;
                 if (full) {
                     // columns are sorted by time within the tile when the key
                     // stamps are; the row spans at most two buckets if the
@@ -391,18 +399,14 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     pk[c >> 1] = pack_bf16(pv[0], pv[1]);
                 }
             }
-            // the previous P V must have finished reading the P buffer
-            if (t > 0 && !(ok = mbar_wait(bar(P_FREE), (t - 1) & 1, abort_flag, p.hdr)))
-                break;
-            unsigned char *prow = sm + LY::P + g * kRegion + r * 128;
-#pragma unroll
-            for (int u = 0; u < 8; u++)
-                *reinterpret_cast<uint4 *>(prow + ((u ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            fence_proxy_async_smem();
+            // P over the first 32 of this thread's S columns (already read)
+            tmem_st16(trow + s * TBN + 64 * g, pk);
+            tmem_st16(trow + s * TBN + 64 * g + 16, pk + 16);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(bar(P_FULL));
+                mbar_arrive(bar(P_FULL + s));
         }
         if (ok && mbar_wait(bar(O_FULL), 0, abort_flag, p.hdr)) {
             tc_fence_after();
