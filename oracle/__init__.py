@@ -227,6 +227,31 @@ def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma,
     return y
 
 
+def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_beta, rab_pos, rab_time,
+              pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None):
+    """Gradients of sum(Y * dy) for one transduction layer: a dict with dx, dw1, db1,
+    dw2, db2, d_ln_gamma, d_ln_beta, d_rab_pos, d_rab_time."""
+    off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
+    x, w1, b1, w2 = _f64(x), _f64(w1), _f64(b1), _f64(w2)
+    g, be, rp, rt, dyy = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time), _f64(dy)
+    T, D = x.shape
+    hv = num_heads * d_v
+    W = num_heads * (2 * d_v + 2 * d_qk)
+    out = {"dx": np.zeros((T, D)), "dw1": np.zeros((D, W)), "db1": np.zeros(W), "dw2": np.zeros((hv, D)),
+           "db2": np.zeros(D), "d_ln_gamma": np.zeros(hv), "d_ln_beta": np.zeros(hv),
+           "d_rab_pos": np.zeros(len(rp)), "d_rab_time": np.zeros(len(rt))}
+    _load().oracle_layer_bwd(
+        ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
+        ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
+        _p(b1, _f64p), _p(w2, _f64p), _p(g, _f64p), _p(be, _f64p), ctypes.c_double(ln_eps),
+        _p(ts, _i64p), _p(rp, _f64p), ctypes.c_int(int(pos_lo)), ctypes.c_int(int(pos_hi)), _p(rt, _f64p),
+        ctypes.c_int(len(rt)), ctypes.c_double(inv_n), _p(dyy, _f64p), _p(out["dx"], _f64p),
+        _p(out["dw1"], _f64p), _p(out["db1"], _f64p), _p(out["dw2"], _f64p), _p(out["db2"], _f64p),
+        _p(out["d_ln_gamma"], _f64p), _p(out["d_ln_beta"], _f64p), _p(out["d_rab_pos"], _f64p),
+        _p(out["d_rab_time"], _f64p), ctypes.c_int(threads or default_threads()))
+    return out
+
+
 def attn_inputs_fwd(inp, threads=None):
     """Oracle forward over a `workloads.AttnInputs`-like object."""
     return attn_fwd(inp.seq_offsets, inp.timestamps, inp.num_targets, inp.q, inp.k, inp.v,

@@ -480,3 +480,173 @@ void oracle_layer_fwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
     free(o);
     free(g);
 }
+
+/*
+ * One transduction layer, backward of the loss sum(Y * dy), by the chain rule
+ * through the forward above, step by step in reverse:
+ *   Z = X W1 + b1, A = SiLU(Z) = [U | V | Q | K];  O = attention(Q, K, V);
+ *   xh = (O - mean) rstd, G = (xh gamma + beta) * U;  Y = G W2 + b2.
+ *   dW2 = G^T dy, db2 = sum_t dy, dG = dy W2^T;
+ *   dU = dG (xh gamma + beta); dL = dG U; dgamma = sum_t dL xh; dbeta = sum_t dL;
+ *   dO = rstd (dL gamma - mean(dL gamma) - xh mean(dL gamma xh));
+ *   (dQ, dK, dV, d_rab_pos, d_rab_time) = attention backward with dout = dO;
+ *   dZ = [dU | dV | dQ | dK] * SiLU'(Z);  dW1 = X^T dZ, db1 = sum_t dZ, dX = dZ W1^T.
+ * Every output is overwritten.
+ */
+void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *num_targets,
+                      int num_heads, int d_qk, int d_v, int d_model, const double *x,
+                      const double *w1, const double *b1, const double *w2,
+                      const double *ln_gamma, const double *ln_beta, double ln_eps,
+                      const int64_t *timestamps, const double *rab_pos, int pos_lo, int pos_hi,
+                      const double *rab_time, int num_buckets, double inv_n, const double *dy,
+                      double *dx, double *dw1, double *db1, double *dw2, double *db2,
+                      double *dgamma, double *dbeta, double *d_rab_pos, double *d_rab_time,
+                      int num_threads)
+{
+    int64_t T = seq_offsets[num_seqs];
+    int hv = num_heads * d_v, hq = num_heads * d_qk;
+    int W = 2 * hv + 2 * hq, D = d_model;
+    size_t Tn = (size_t)(T > 0 ? T : 1);
+    double *z = (double *)malloc(sizeof(double) * Tn * W);
+    double *u = (double *)malloc(sizeof(double) * Tn * hv);
+    double *vv = (double *)malloc(sizeof(double) * Tn * hv);
+    double *qq = (double *)malloc(sizeof(double) * Tn * hq);
+    double *kk = (double *)malloc(sizeof(double) * Tn * hq);
+    double *o = (double *)malloc(sizeof(double) * Tn * hv);
+    double *xh = (double *)malloc(sizeof(double) * Tn * hv);
+    double *rstd = (double *)malloc(sizeof(double) * Tn);
+    double *g = (double *)malloc(sizeof(double) * Tn * hv);
+    double *dg = (double *)malloc(sizeof(double) * Tn * hv);
+    double *du = (double *)malloc(sizeof(double) * Tn * hv);
+    double *dl = (double *)malloc(sizeof(double) * Tn * hv);
+    double *dout = (double *)malloc(sizeof(double) * Tn * hv);
+    double *dq = (double *)malloc(sizeof(double) * Tn * hq);
+    double *dk = (double *)malloc(sizeof(double) * Tn * hq);
+    double *dv = (double *)malloc(sizeof(double) * Tn * hv);
+    double *dz = (double *)malloc(sizeof(double) * Tn * W);
+
+    /* forward, keeping what the backward needs */
+    oracle_linear(T, D, W, x, w1, b1, 0, z, num_threads);
+    for (int64_t t = 0; t < T; t++) {
+        for (int c = 0; c < hv; c++) {
+            u[t * hv + c] = silu(z[t * W + c]);
+            vv[t * hv + c] = silu(z[t * W + hv + c]);
+        }
+        for (int c = 0; c < hq; c++) {
+            qq[t * hq + c] = silu(z[t * W + 2 * hv + c]);
+            kk[t * hq + c] = silu(z[t * W + 2 * hv + hq + c]);
+        }
+    }
+    oracle_attn_fwd(num_seqs, seq_offsets, num_targets, num_heads, d_qk, d_v, qq, kk, vv,
+                    timestamps, rab_pos, pos_lo, pos_hi, rab_time, num_buckets, inv_n, o,
+                    num_threads);
+    for (int64_t t = 0; t < T; t++) {
+        const double *ot = o + t * hv;
+        double mean = 0.0, var = 0.0;
+        for (int c = 0; c < hv; c++)
+            mean += ot[c];
+        mean /= hv;
+        for (int c = 0; c < hv; c++)
+            var += (ot[c] - mean) * (ot[c] - mean);
+        var /= hv;
+        rstd[t] = 1.0 / sqrt(var + ln_eps);
+        for (int c = 0; c < hv; c++) {
+            xh[t * hv + c] = (ot[c] - mean) * rstd[t];
+            g[t * hv + c] = (xh[t * hv + c] * ln_gamma[c] + ln_beta[c]) * u[t * hv + c];
+        }
+    }
+
+    /* output projection: dW2 = G^T dy, db2 = sum dy, dG = dy W2^T */
+    for (int j = 0; j < hv; j++)
+        for (int c = 0; c < D; c++)
+            dw2[(int64_t)j * D + c] = 0.0;
+    for (int c = 0; c < D; c++)
+        db2[c] = 0.0;
+    for (int64_t t = 0; t < T; t++) {
+        for (int c = 0; c < D; c++)
+            db2[c] += dy[t * D + c];
+        for (int j = 0; j < hv; j++) {
+            double gj = g[t * hv + j], acc = 0.0;
+            for (int c = 0; c < D; c++) {
+                dw2[(int64_t)j * D + c] += gj * dy[t * D + c];
+                acc += dy[t * D + c] * w2[(int64_t)j * D + c];
+            }
+            dg[t * hv + j] = acc;
+        }
+    }
+
+    /* gate and LayerNorm */
+    for (int c = 0; c < hv; c++) {
+        dgamma[c] = 0.0;
+        dbeta[c] = 0.0;
+    }
+    for (int64_t t = 0; t < T; t++) {
+        double m1 = 0.0, m2 = 0.0;
+        for (int c = 0; c < hv; c++) {
+            int64_t e = t * hv + c;
+            du[e] = dg[e] * (xh[e] * ln_gamma[c] + ln_beta[c]);
+            dl[e] = dg[e] * u[e];
+            dgamma[c] += dl[e] * xh[e];
+            dbeta[c] += dl[e];
+            m1 += dl[e] * ln_gamma[c];
+            m2 += dl[e] * ln_gamma[c] * xh[e];
+        }
+        m1 /= hv;
+        m2 /= hv;
+        for (int c = 0; c < hv; c++) {
+            int64_t e = t * hv + c;
+            dout[e] = rstd[t] * (dl[e] * ln_gamma[c] - m1 - xh[e] * m2);
+        }
+    }
+
+    /* attention */
+    oracle_attn_bwd(num_seqs, seq_offsets, num_targets, num_heads, d_qk, d_v, qq, kk, vv,
+                    timestamps, rab_pos, pos_lo, pos_hi, rab_time, num_buckets, inv_n, dout, dq, dk,
+                    dv, d_rab_pos, d_rab_time, num_threads);
+
+    /* projection and SiLU: dZ = [dU | dV | dQ | dK] * SiLU'(Z) */
+    for (int64_t t = 0; t < T; t++) {
+        for (int c = 0; c < hv; c++) {
+            dz[t * W + c] = du[t * hv + c] * silu_grad(z[t * W + c]);
+            dz[t * W + hv + c] = dv[t * hv + c] * silu_grad(z[t * W + hv + c]);
+        }
+        for (int c = 0; c < hq; c++) {
+            dz[t * W + 2 * hv + c] = dq[t * hq + c] * silu_grad(z[t * W + 2 * hv + c]);
+            dz[t * W + 2 * hv + hq + c] = dk[t * hq + c] * silu_grad(z[t * W + 2 * hv + hq + c]);
+        }
+    }
+    for (int k = 0; k < D; k++)
+        for (int c = 0; c < W; c++)
+            dw1[(int64_t)k * W + c] = 0.0;
+    for (int c = 0; c < W; c++)
+        db1[c] = 0.0;
+    for (int64_t t = 0; t < T; t++) {
+        for (int c = 0; c < W; c++)
+            db1[c] += dz[t * W + c];
+        for (int k = 0; k < D; k++) {
+            double xv = x[t * D + k], acc = 0.0;
+            for (int c = 0; c < W; c++) {
+                dw1[(int64_t)k * W + c] += xv * dz[t * W + c];
+                acc += dz[t * W + c] * w1[(int64_t)k * W + c];
+            }
+            dx[t * D + k] = acc;
+        }
+    }
+    free(z);
+    free(u);
+    free(vv);
+    free(qq);
+    free(kk);
+    free(o);
+    free(xh);
+    free(rstd);
+    free(g);
+    free(dg);
+    free(du);
+    free(dl);
+    free(dout);
+    free(dq);
+    free(dk);
+    free(dv);
+    free(dz);
+}

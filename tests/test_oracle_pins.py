@@ -464,3 +464,103 @@ def test_layer_matches_composition():
     g = torch.nn.functional.layer_norm(torch.tensor(o), (H * dv,), torch.tensor(gam),
                                        torch.tensor(bet), eps=1e-5).numpy() * u
     np.testing.assert_allclose(y, g @ w2 + b2, rtol=0, atol=1e-10)
+
+
+# ---- 8. layer backward: torch float64 autograd and finite differences --------
+
+def _layer_case(seed, lengths=(4, 6, 1), nt=(0, 2, 0), H=2, dqk=3, dv=3, D=5):
+    rng = np.random.default_rng(seed)
+    c = rand_case(rng, list(lengths), H=H, dqk=dqk, dv=dv, nt=list(nt))
+    T = int(c["seq_offsets"][-1])
+    W = H * (2 * dv + 2 * dqk)
+    prm = {"x": rng.standard_normal((T, D)), "w1": rng.standard_normal((D, W)) * 0.5,
+           "b1": rng.standard_normal(W) * 0.1, "w2": rng.standard_normal((H * dv, D)),
+           "b2": rng.standard_normal(D), "ln_gamma": 1 + 0.1 * rng.standard_normal(H * dv),
+           "ln_beta": 0.1 * rng.standard_normal(H * dv), "rab_pos": c["rab_pos"], "rab_time": c["rab_time"]}
+    dy = rng.standard_normal((T, D))
+    return c, prm, dy, (H, dqk, dv)
+
+
+def _torch_layer_loss(c, prm, dy, dims):
+    """sum(Y * dy) of the layer written with torch ops (dense masked attention)."""
+    H, dqk, dv = dims
+    t = {k: torch.tensor(v, requires_grad=True) for k, v in prm.items()}
+    T = prm["x"].shape[0]
+    hv, hq = H * dv, H * dqk
+    a = torch.nn.functional.silu(t["x"] @ t["w1"] + t["b1"])
+    u = a[:, :hv]
+    vv = a[:, hv:2 * hv].reshape(T, H, dv)
+    qq = a[:, 2 * hv:2 * hv + hq].reshape(T, H, dqk)
+    kk = a[:, 2 * hv + hq:].reshape(T, H, dqk)
+    off, nt = c["seq_offsets"], c["num_targets"]
+    lo, hi = c["pos_lo"], c["pos_hi"]
+    outs = []
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        hist = L - n_t
+        idx = np.arange(L)
+        p = np.where(idx < hist, idx, hist)
+        rel = torch.tensor(np.clip(p[:, None] - p[None, :], lo, hi) - lo)
+        ts = c["timestamps"][s0:s1]
+        nbk = len(prm["rab_time"])
+        bkt = torch.tensor([[min(nbk - 1, (int(max(ts[i] - ts[j], 0)) + 1).bit_length() - 1)
+                             for j in range(L)] for i in range(L)])
+        I, J = idx[:, None], idx[None, :]
+        vis = torch.tensor(np.where(I < hist, J <= I, (J < hist) | (J == I)), dtype=torch.float64)
+        S = torch.einsum("ihc,jhc->hij", qq[s0:s1], kk[s0:s1]) + (t["rab_pos"][rel] + t["rab_time"][bkt])[None]
+        P = torch.nn.functional.silu(S) * c["inv_n"] * vis[None]
+        outs.append(torch.einsum("hij,jhc->ihc", P, vv[s0:s1]).reshape(L, hv))
+    o = torch.cat(outs)
+    g = torch.nn.functional.layer_norm(o, (hv,), t["ln_gamma"], t["ln_beta"], eps=1e-5) * u
+    y = g @ t["w2"] + t["b2"]
+    (y * torch.tensor(dy)).sum().backward()
+    return {k: v.grad.numpy() for k, v in t.items()}
+
+
+def _olayer_bwd(c, prm, dy, dims):
+    H, dqk, dv = dims
+    return oracle.layer_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], prm["x"], prm["w1"],
+                            prm["b1"], prm["w2"], prm["ln_gamma"], prm["ln_beta"], prm["rab_pos"],
+                            prm["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv, dy)
+
+
+_LAYER_GRAD_NAMES = {"x": "dx", "w1": "dw1", "b1": "db1", "w2": "dw2", "b2": "db2", "ln_gamma": "d_ln_gamma",
+                     "ln_beta": "d_ln_beta", "rab_pos": "d_rab_pos", "rab_time": "d_rab_time"}
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_layer_bwd_matches_torch_autograd(seed):
+    c, prm, dy, dims = _layer_case(400 + seed)
+    ours = _olayer_bwd(c, prm, dy, dims)
+    ref = _torch_layer_loss(c, prm, dy, dims)
+    for k, name in _LAYER_GRAD_NAMES.items():
+        np.testing.assert_allclose(ours[name], ref[k], rtol=1e-9, atol=1e-10, err_msg=name)
+
+
+def test_layer_bwd_central_finite_differences():
+    c, prm, dy, dims = _layer_case(410, lengths=(3, 2), nt=(1, 0), H=1, dqk=2, dv=2, D=3)
+    H, dqk, dv = dims
+    ours = _olayer_bwd(c, prm, dy, dims)
+
+    def loss(p):
+        y = oracle.layer_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], p["x"], p["w1"], p["b1"],
+                             p["w2"], p["b2"], p["ln_gamma"], p["ln_beta"], p["rab_pos"], p["rab_time"],
+                             c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv)
+        return float(np.sum(y * dy))
+
+    h = 1e-6
+    rng = np.random.default_rng(411)
+    for k, name in _LAYER_GRAD_NAMES.items():
+        flat = prm[k].reshape(-1)
+        for e in rng.choice(flat.size, size=min(flat.size, 6), replace=False):
+            plus, minus = dict(prm), dict(prm)
+            fp, fm = flat.copy(), flat.copy()
+            fp[e] += h
+            fm[e] -= h
+            plus[k], minus[k] = fp.reshape(prm[k].shape), fm.reshape(prm[k].shape)
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            assert abs(fd - ours[name].reshape(-1)[e]) < 1e-6 * max(1.0, abs(fd)), (name, e, fd)
