@@ -1,16 +1,27 @@
 // Projection GEMMs of the transduction layer on sm_100a: TMA + tcgen05 (TMEM).
 //
-//   C[M, N] = act(A[M, K] B[K, N] + bias[N]),  act = SiLU for f1, identity for f2
+//   C[M, N] = epi(A[M, K] B[K, N])
 //
 // ("DLRMv4 Brings Sequence-Based Recommendation Training to MLPerf", section
 // "Model Architecture": the projection that produces U, V, Q, K, and the output
-// projection after the gate.)  Persistent tiles of 128 x BN (BN = 256 or
-// 128): warp 0 streams A (K-major, 128 rows x 64 columns) and B (the weight,
-// row-major so N-contiguous: an MN-major operand, 64 K-rows x 64 columns per
-// box) through a 4-stage ring; warp 1 owns two TMEM accumulators and issues
-// tcgen05.mma from one thread; warps 2-9 read one accumulator row by row, add
-// the bias, apply SiLU and store bf16 while the next tile accumulates in the
-// other.  Bias and activation never make a separate pass over HBM.
+// projection after the gate; their gradients for the layer backward.)
+// Persistent tiles of 128 x BN (BN = 256 or 128): warp 0 streams A and B
+// through a 4-stage ring of 64-deep k-slices; warp 1 owns two TMEM
+// accumulators and issues tcgen05.mma from one thread; warps 2-9 read one
+// accumulator row by row while the next tile accumulates in the other.
+//
+// Operand layouts (all bf16, 128-byte swizzled k-slices):
+//   A K-major: A[m][k] row-major ([M, K]);  A MN-major: stored as X[k][m] ([K, M])
+//   B MN-major: B[k][n] row-major ([K, N]); B K-major: stored as W[n][k] ([N, K])
+// so that the layer backward's products dY W2^T, dZ W1^T (B K-major) and
+// G^T dY, X^T dZ (A MN-major, K = tokens) need no transposed copies.
+// Epilogues:
+//   EPI_ACT    bf16 out = acc + bias, optionally SiLU (forward projections);
+//   EPI_DSILU  bf16 out = aux * SiLU'(acc + bias) (the SiLU backward fused into
+//              the recompute of the pre-activation);
+//   EPI_RED    fp32 out += acc through a swizzled staging box and a TMA bulk
+//              reduce-add; the k range is split across CTAs (weight gradients,
+//              whose K is the token count).
 #include <algorithm>
 
 #include "internal.h"
@@ -24,41 +35,67 @@ constexpr int GBM = 128, GBK = 64, GSTAGES = 4;
 constexpr int kEpiWarpsG = 8;  // two per TMEM lane quarter, each half of the columns
 constexpr int kThreadsG = 64 + 32 * kEpiWarpsG;
 constexpr int kRegA = GBM * 128;  // 128 rows x 128 B
-constexpr int kRegB = GBK * 128;  // 64 K-rows x 128 B (64 N columns)
+constexpr int kReg64 = 64 * 128;  // a 64 x 64 bf16 box
 
-template <int BN>
+enum GemmEpi { EPI_ACT = 0, EPI_DSILU = 1, EPI_RED = 2 };
+
+template <int BN, int EPI>
 struct GL {
     static constexpr int A = 0;
     static constexpr int B = A + GSTAGES * kRegA;
-    static constexpr int BAR = B + GSTAGES * (BN / 64) * kRegB;
+    static constexpr int STG = B + GSTAGES * BN * 128;                   // EPI_RED: 2 x 4 KB per warp
+    static constexpr int BAR = STG + (EPI == EPI_RED ? kEpiWarpsG * 2 * 4096 : 0);
     static constexpr int NBAR = 2 * GSTAGES + 4;  // full, empty, acc_full[2], acc_empty[2]
     static constexpr int MISC = BAR + NBAR * 8;
     static constexpr int BYTES = MISC + 64;
 };
 
-// Persistent: CTA c computes output tiles c, c + gridDim.x, ... (row-block
-// major, so consecutive tiles reuse the same A rows from L2).  The TMA ring
-// runs across tile boundaries and the accumulator is double-buffered in
-// TMEM, so the epilogue of one tile overlaps the MMAs of the next.
-template <int BN>
+struct GemmArgs {
+    const __nv_bfloat16 *bias;  // [N] or null
+    const __nv_bfloat16 *aux;   // EPI_DSILU: [M, N] with row stride ldaux
+    int64_t ldaux;
+    void *C;                    // bf16 (EPI_ACT, EPI_DSILU) or unused (EPI_RED: through tmC)
+    int64_t ldc;
+    int64_t M;
+    int N, K, silu, splits;
+    WsHeader *hdr;
+};
+
+__device__ __forceinline__ float silu_grad_tanh(float z)
+{
+    // SiLU'(z) = sigma(z) (1 + z (1 - sigma(z))) with sigma(z) = (1 + tanh(z/2)) / 2
+    const float h = 0.5f * z, t = tanh_approx(h);
+    const float a = 1.f + t;
+    return 0.5f * fmaf(a, fmaf(-h, t, h), a);
+}
+
+// Persistent: CTA c takes work units c, c + gridDim.x, ...; unit = (tile, k split),
+// tiles row-block major so consecutive tiles reuse the same A rows from L2.
+template <int BN, bool A_MN, bool B_K, int EPI>
 __global__ void __launch_bounds__(kThreadsG, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ C, int64_t ldc, int64_t M,
-               int N, int K, int silu, WsHeader *hdr)
+               const __grid_constant__ CUtensorMap tmC, const GemmArgs g)
 {
-    using LY = GL<BN>;
+    using LY = GL<BN, EPI>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nk = K / GBK;
-    const int tiles_n = N / BN;
-    const int tiles = (int)((M + GBM - 1) / GBM) * tiles_n;
+    const int nk = (g.K + GBK - 1) / GBK;  // the TMA zero-fills past K
+    const int per = (nk + g.splits - 1) / g.splits;  // k-slices per split
+    const int tiles_n = g.N / BN;
+    const int tiles = (int)((g.M + GBM - 1) / GBM) * tiles_n;
+    const int units = tiles * g.splits;
     auto full_bar = [&](int s) { return base + LY::BAR + 8u * s; };
     auto empty_bar = [&](int s) { return base + LY::BAR + 8u * (GSTAGES + s); };
     auto accf_bar = [&](int b) { return base + LY::BAR + 8u * (2 * GSTAGES + b); };
     auto acce_bar = [&](int b) { return base + LY::BAR + 8u * (2 * GSTAGES + 2 + b); };
+    auto krange = [&](int u, int &k0, int &k1) {
+        const int sp = u % g.splits;
+        k0 = sp * per;
+        k1 = min(nk, k0 + per);
+    };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + LY::MISC + 8);
 
     if (threadIdx.x == 0) {
@@ -70,6 +107,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (warp == 0 && lane == 0) {
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
+        if (EPI == EPI_RED)
+            tma_prefetch(&tmC);
     }
     if (warp == 1)
         tmem_alloc(base + LY::MISC, 2 * BN);
@@ -80,43 +119,59 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     if (warp == 0) {
         if (lane == 0) {
-            int it = 0;  // k-tiles issued by this CTA, across its output tiles
+            int it = 0;  // k-slices issued by this CTA, across its units
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int tile = u / g.splits;
                 const int m0 = (tile / tiles_n) * GBM, n0 = (tile % tiles_n) * BN;
-                for (int kt = 0; kt < nk; kt++, it++) {
+                int k0, k1;
+                krange(u, k0, k1);
+                for (int kt = k0; kt < k1; kt++, it++) {
                     const int s = it % GSTAGES;
-                    if (it >= GSTAGES && !(ok = mbar_wait(empty_bar(s), ((it / GSTAGES) - 1) & 1, abort_flag, hdr)))
+                    if (it >= GSTAGES && !(ok = mbar_wait(empty_bar(s), ((it / GSTAGES) - 1) & 1, abort_flag, g.hdr)))
                         break;
-                    mbar_expect_tx(full_bar(s), kRegA + (BN / 64) * kRegB);
-                    tma_load_2d(base + LY::A + s * kRegA, &tmA, kt * GBK, m0, full_bar(s));
-                    for (int r = 0; r < BN / 64; r++)
-                        tma_load_2d(base + LY::B + (s * (BN / 64) + r) * kRegB, &tmB, n0 + 64 * r, kt * GBK,
-                                    full_bar(s));
+                    mbar_expect_tx(full_bar(s), kRegA + BN * 128);
+                    const uint32_t sa = base + LY::A + s * kRegA, sb = base + LY::B + s * BN * 128;
+                    if (A_MN) {
+                        for (int r = 0; r < 2; r++)
+                            tma_load_2d(sa + r * kReg64, &tmA, m0 + 64 * r, kt * GBK, full_bar(s));
+                    } else {
+                        tma_load_2d(sa, &tmA, kt * GBK, m0, full_bar(s));
+                    }
+                    if (B_K) {
+                        tma_load_2d(sb, &tmB, kt * GBK, n0, full_bar(s));
+                    } else {
+                        for (int r = 0; r < BN / 64; r++)
+                            tma_load_2d(sb + r * kReg64, &tmB, n0 + 64 * r, kt * GBK, full_bar(s));
+                    }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(GBM, BN, 0, 1);
+            constexpr uint32_t idesc = idesc_bf16(GBM, BN, A_MN ? 1 : 0, B_K ? 0 : 1);
             int it = 0, lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, lt++) {
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, lt++) {
                 const int ab = lt & 1;
-                // the epilogue must have drained this accumulator (tile lt - 2)
-                if (lt >= 2 && !(ok = mbar_wait(acce_bar(ab), ((lt >> 1) - 1) & 1, abort_flag, hdr)))
+                int k0, k1;
+                krange(u, k0, k1);
+                // the epilogue must have drained this accumulator (unit lt - 2)
+                if (lt >= 2 && !(ok = mbar_wait(acce_bar(ab), ((lt >> 1) - 1) & 1, abort_flag, g.hdr)))
                     break;
                 tc_fence_after();
-                for (int kt = 0; kt < nk; kt++, it++) {
+                for (int kt = k0; kt < k1; kt++, it++) {
                     const int s = it % GSTAGES;
-                    if (!(ok = mbar_wait(full_bar(s), (it / GSTAGES) & 1, abort_flag, hdr)))
+                    if (!(ok = mbar_wait(full_bar(s), (it / GSTAGES) & 1, abort_flag, g.hdr)))
                         break;
                     tc_fence_after();
                     for (int ks = 0; ks < GBK / 16; ks++) {
-                        const uint64_t a = smem_desc_sw128(base + LY::A + s * kRegA + ks * 32, 16, 1024);
-                        const uint64_t b =
-                            smem_desc_sw128(base + LY::B + s * (BN / 64) * kRegB + ks * 2048, kRegB, 1024);
-                        umma_bf16(tmem + ab * BN, a, b, idesc, (kt > 0 || ks > 0));
+                        const uint32_t sa = base + LY::A + s * kRegA, sb = base + LY::B + s * BN * 128;
+                        const uint64_t a = A_MN ? smem_desc_sw128(sa + ks * 2048, kReg64, 1024)
+                                                : smem_desc_sw128(sa + ks * 32, 16, 1024);
+                        const uint64_t b = B_K ? smem_desc_sw128(sb + ks * 32, 16, 1024)
+                                               : smem_desc_sw128(sb + ks * 2048, kReg64, 1024);
+                        umma_bf16(tmem + ab * BN, a, b, idesc, (kt > k0 || ks > 0));
                     }
                     umma_commit(empty_bar(s));
                 }
@@ -127,28 +182,67 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int ew = warp - 2, half = ew >> 2, quarter = warp & 3;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         constexpr int CW = BN / 2;  // columns per epilogue thread
-        int lt = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, lt++) {
+        int lt = 0, nstage = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, lt++) {
             const int ab = lt & 1;
-            if (!mbar_wait(accf_bar(ab), (lt >> 1) & 1, abort_flag, hdr))
+            const int tile = u / g.splits;
+            int k0, k1;
+            krange(u, k0, k1);
+            if (!mbar_wait(accf_bar(ab), (lt >> 1) & 1, abort_flag, g.hdr))
                 break;
             tc_fence_after();
-            const int64_t row = (int64_t)(tile / tiles_n) * GBM + quarter * 32 + lane;
+            const int64_t rowbase = (int64_t)(tile / tiles_n) * GBM + quarter * 32;
+            const int64_t row = rowbase + lane;
             const int n0 = (tile % tiles_n) * BN + half * CW;
-            __nv_bfloat16 *crow = C + row * ldc + n0;
 #pragma unroll 1
             for (int cc = 0; cc < CW; cc += 32) {
                 float v[32];
                 tmem_ld32(trow + ab * BN + half * CW + cc, v);
                 tmem_wait_ld();
-                if (row < M) {
+                if (EPI == EPI_RED) {
+                    // [32 rows x 32 columns] fp32 box, 128-byte swizzled, two buffers per warp
+                    if (k1 <= k0)
+                        continue;  // an empty split adds nothing
+                    const int bsel = nstage & 1;
+                    unsigned char *stg = sm + LY::STG + (ew * 2 + bsel) * 4096;
+                    if (lane == 0 && nstage >= 2)
+                        bulk_wait_read1();  // the box written two stages ago has been read
+                    __syncwarp();
 #pragma unroll
-                    for (int u = 0; u < 4; u++) {
+                    for (int c = 0; c < 8; c++)
+                        *reinterpret_cast<float4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_2d(&tmC, n0 + cc, (int)rowbase, smem_u32(stg));
+                        bulk_commit();
+                    }
+                    nstage++;
+                    continue;
+                }
+                if (row < g.M) {
+                    __nv_bfloat16 *crow = static_cast<__nv_bfloat16 *>(g.C) + row * g.ldc + n0;
+                    const __nv_bfloat16 *arow = EPI == EPI_DSILU ? g.aux + row * g.ldaux + n0 : nullptr;
+#pragma unroll
+                    for (int u4 = 0; u4 < 4; u4++) {
                         float x[8];
+                        float da[8];
+                        if (EPI == EPI_DSILU) {
+                            const uint4 w = *reinterpret_cast<const uint4 *>(arow + cc + 8 * u4);
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; e++) {
+                                da[2 * e] = __uint_as_float(ww[e] << 16);
+                                da[2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
+                            }
+                        }
 #pragma unroll
                         for (int e = 0; e < 8; e++) {
-                            x[e] = v[8 * u + e] + (bias ? __bfloat162float(bias[n0 + cc + 8 * u + e]) : 0.f);
-                            if (silu)
+                            x[e] = v[8 * u4 + e] + (g.bias ? __bfloat162float(g.bias[n0 + cc + 8 * u4 + e]) : 0.f);
+                            if (EPI == EPI_DSILU)
+                                x[e] = da[e] * silu_grad_tanh(x[e]);
+                            else if (g.silu)
                                 x[e] = silu_fast(x[e]);
                         }
                         uint4 w;
@@ -156,7 +250,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         w.y = pack_bf16(x[2], x[3]);
                         w.z = pack_bf16(x[4], x[5]);
                         w.w = pack_bf16(x[6], x[7]);
-                        *reinterpret_cast<uint4 *>(crow + cc + 8 * u) = w;
+                        *reinterpret_cast<uint4 *>(crow + cc + 8 * u4) = w;
                     }
                 }
             }
@@ -165,6 +259,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (lane == 0)
                 mbar_arrive(acce_bar(ab));
         }
+        if (EPI == EPI_RED && lane == 0)
+            bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
@@ -185,47 +281,125 @@ int num_sms()
     return n;
 }
 
-template <int BN>
-cudaError_t gemm_tc_launch(const void *A, int64_t lda, const void *Bm, const void *bias, void *C, int64_t ldc,
-                           int64_t M, int N, int K, bool silu, WsHeader *hdr, cudaStream_t stream)
+template <int BN, bool A_MN, bool B_K, int EPI>
+cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stream)
 {
-    CUtensorMap ma, mb;
-    cudaError_t e = make_tensor_map_2d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M, K, lda * 2, 64, GBM,
-                                       CU_TENSOR_MAP_SWIZZLE_128B);
-    if (e == cudaSuccess)
-        e = make_tensor_map_2d(&mb, Bm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, (int64_t)N * 2, 64, GBK,
+    CUtensorMap ma, mb, mc;
+    cudaError_t e;
+    if (A_MN)  // stored [K, M]: box 64 m x 64 k
+        e = make_tensor_map_2d(&ma, op.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.K, g.M, op.lda * 2, 64, 64,
                                CU_TENSOR_MAP_SWIZZLE_128B);
+    else       // [M, K]: box 64 k x 128 m
+        e = make_tensor_map_2d(&ma, op.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.M, g.K, op.lda * 2, 64, GBM,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess) {
+        if (B_K)  // stored [N, K]: box 64 k x BN n
+            e = make_tensor_map_2d(&mb, op.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.N, g.K, op.ldb * 2, 64, BN,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+        else      // [K, N]: box 64 n x 64 k
+            e = make_tensor_map_2d(&mb, op.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.K, g.N, op.ldb * 2, 64, GBK,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (e == cudaSuccess) {
+        if (EPI == EPI_RED)  // fp32 [M, N]: box 32 columns x 32 rows, 128-byte swizzle
+            e = make_tensor_map_2d(&mc, op.C32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.M, g.N, g.ldc * 4, 32, 32,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+        else
+            mc = mb;  // unused
+    }
     if (e != cudaSuccess)
         return e;
-    const size_t bytes = GL<BN>::BYTES + 1024;
-    e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    const size_t bytes = GL<BN, EPI>::BYTES + 1024;
+    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, A_MN, B_K, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bytes);
     if (e != cudaSuccess)
         return e;
-    const int64_t tiles = ((M + GBM - 1) / GBM) * (N / BN);
-    const unsigned grid = (unsigned)std::min<int64_t>(tiles, num_sms());
-    gemm_tc_kernel<BN><<<grid, kThreadsG, bytes, stream>>>(ma, mb, static_cast<const __nv_bfloat16 *>(bias),
-                                                          static_cast<__nv_bfloat16 *>(C), ldc, M, N, K, silu, hdr);
+    const int64_t units = ((g.M + GBM - 1) / GBM) * (g.N / BN) * g.splits;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, num_sms());
+    gemm_tc_kernel<BN, A_MN, B_K, EPI><<<grid, kThreadsG, bytes, stream>>>(ma, mb, mc, g);
     return cudaGetLastError();
+}
+
+template <int BN, int EPI>
+cudaError_t gemm_dispatch_layout(const GemmOperands &op, const GemmArgs &g, cudaStream_t stream)
+{
+    if (op.a_mn && op.b_k)
+        return gemm_tc_launch<BN, true, true, EPI>(op, g, stream);
+    if (op.a_mn)
+        return gemm_tc_launch<BN, true, false, EPI>(op, g, stream);
+    if (op.b_k)
+        return gemm_tc_launch<BN, false, true, EPI>(op, g, stream);
+    return gemm_tc_launch<BN, false, false, EPI>(op, g, stream);
 }
 
 }  // namespace
 
+bool gemm_tc_ok(const GemmOperands &op, int64_t M, int N, int K)
+{
+    const bool aligned = ((reinterpret_cast<uintptr_t>(op.A) | reinterpret_cast<uintptr_t>(op.B) |
+                           reinterpret_cast<uintptr_t>(op.C) | reinterpret_cast<uintptr_t>(op.C32) |
+                           reinterpret_cast<uintptr_t>(op.aux)) & 15u) == 0;
+    // K need not be a multiple of 64 (slices past K read zeros); a K-major operand
+    // needs K % 8 == 0 for its 16-byte rows, an MN-major A needs M % 64 == 0
+    const bool k_ok = K > 0 && K < ((int64_t)1 << 31) - GBK && ((op.a_mn && !op.b_k) || K % 8 == 0);
+    const bool mn_ok = !op.a_mn || M % 64 == 0;
+    return aligned && mn_ok && k_ok && M > 0 && M < ((int64_t)1 << 31) - GBM && N % 128 == 0 && op.lda % 8 == 0 &&
+           op.ldb % 8 == 0 && op.ldc % 8 == 0 && (!op.aux || op.ldaux % 8 == 0);
+}
+
+cudaError_t launch_gemm_tc_ex(const GemmOperands &op, int64_t M, int N, int K, GemmEpilogue epi, bool silu,
+                              int splits, WsHeader *hdr, cudaStream_t stream)
+{
+    if (M == 0)
+        return cudaSuccess;
+    GemmArgs g{};
+    g.bias = static_cast<const __nv_bfloat16 *>(op.bias);
+    g.aux = static_cast<const __nv_bfloat16 *>(op.aux);
+    g.ldaux = op.ldaux;
+    g.C = op.C;
+    g.ldc = op.ldc;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.silu = silu;
+    g.splits = std::max(1, std::min(splits, (K + GBK - 1) / GBK));
+    g.hdr = hdr;
+    switch (epi) {
+    case GEMM_RED_F32:
+        return gemm_dispatch_layout<128, EPI_RED>(op, g, stream);
+    case GEMM_DSILU:
+        return N % 256 == 0 ? gemm_dispatch_layout<256, EPI_DSILU>(op, g, stream)
+                            : gemm_dispatch_layout<128, EPI_DSILU>(op, g, stream);
+    default:
+        return N % 256 == 0 ? gemm_dispatch_layout<256, EPI_ACT>(op, g, stream)
+                            : gemm_dispatch_layout<128, EPI_ACT>(op, g, stream);
+    }
+}
+
 bool gemm_tc_supported(const void *A, int64_t lda, const void *Bm, void *C, int64_t ldc, int64_t M, int N, int K)
 {
-    const bool aligned = ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(Bm) |
-                           reinterpret_cast<uintptr_t>(C)) & 15u) == 0;
-    return aligned && M > 0 && M < ((int64_t)1 << 31) - GBM && K % GBK == 0 && K > 0 && N % 128 == 0 &&
-           lda % 8 == 0 && ldc % 8 == 0;
+    GemmOperands op{};
+    op.A = A;
+    op.lda = lda;
+    op.B = Bm;
+    op.ldb = N;
+    op.C = C;
+    op.ldc = ldc;
+    return gemm_tc_ok(op, M, N, K);
 }
 
 cudaError_t launch_gemm_tc(const void *A, int64_t lda, const void *Bm, const void *bias, void *C, int64_t ldc,
                            int64_t M, int N, int K, bool silu, WsHeader *hdr, cudaStream_t stream)
 {
-    if (M == 0)
-        return cudaSuccess;
-    if (N % 256 == 0)
-        return gemm_tc_launch<256>(A, lda, Bm, bias, C, ldc, M, N, K, silu, hdr, stream);
-    return gemm_tc_launch<128>(A, lda, Bm, bias, C, ldc, M, N, K, silu, hdr, stream);
+    GemmOperands op{};
+    op.A = A;
+    op.lda = lda;
+    op.B = Bm;
+    op.ldb = N;
+    op.bias = bias;
+    op.C = C;
+    op.ldc = ldc;
+    return launch_gemm_tc_ex(op, M, N, K, GEMM_ACT, silu, 1, hdr, stream);
 }
 
 }  // namespace hstu

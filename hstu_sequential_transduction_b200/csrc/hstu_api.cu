@@ -136,6 +136,64 @@ hstu_status attn_fwd_strided(const hstu_attn_desc *d, const void *q, int64_t sq,
     return cuda_status(launch_attn_fwd_f32(p, grid_items(d), stream));
 }
 
+// Attention backward with explicit row strides (elements) for every tensor; the
+// fp32 path needs dense dq, dk, dv (it zeroes them as whole buffers).
+hstu_status attn_bwd_strided(const hstu_attn_desc *desc, const void *q, int64_t sq, const void *k, int64_t sk,
+                             const void *v, int64_t sv, const int64_t *seq_offsets, const int64_t *timestamps,
+                             const int32_t *num_targets, const float *rab_pos, const float *rab_time,
+                             const void *dout, int64_t sdo, void *dq, int64_t sdq, void *dk, int64_t sdk, void *dv,
+                             int64_t sdv, float *d_rab_pos, float *d_rab_time, void *workspace, cudaStream_t st)
+{
+    const int npos = desc->pos_hi - desc->pos_lo + 1;
+    HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * npos, st));
+    HSTU_CUDA(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->num_time_buckets, st));
+    const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
+    const size_t tensor_bytes = (size_t)desc->total_tokens * row * elem_bytes(desc);
+    const bool bf16 = desc->dtype == HSTU_BF16;
+    AttnParams p = base_params(desc, seq_offsets, timestamps, num_targets, rab_pos, rab_time, workspace);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.sq = sq;
+    p.sk = sk;
+    p.sv = sv;
+    p.dout = dout;
+    p.sdo = sdo;
+    p.dq = dq;
+    p.dk = dk;
+    p.dvv = dv;
+    p.sdq = sdq;
+    p.sdk = sdk;
+    p.sdv = sdv;
+    p.d_rab_pos = d_rab_pos;
+    p.d_rab_time = d_rab_time;
+    if (bf16) {
+        p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + sizeof(WsHeader) +
+                                             items_bytes(desc));
+        HSTU_CUDA(cudaMemsetAsync(p.dq_acc, 0, sizeof(float) * (size_t)desc->total_tokens * row, st));
+        float dq_scale = 1.0f;
+        if (attn_bwd_tc_supported(p)) {
+            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st, kTcTile));
+            HSTU_CUDA(launch_attn_bwd_tc(p, grid_items(desc, kTcTile), st));
+            dq_scale = 0.5f * desc->inv_n;
+        } else {
+            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
+            HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
+        }
+        return cuda_status(launch_convert_dq(p.dq_acc, dq, desc->total_tokens, desc->num_heads,
+                                             desc->d_qk, sdq, dq_scale, st));
+    }
+    if (sdq != row || sdk != row || sdv != row)
+        return HSTU_ERR_UNSUPPORTED;
+    if (tensor_bytes) {
+        HSTU_CUDA(cudaMemsetAsync(dk, 0, tensor_bytes, st));
+        HSTU_CUDA(cudaMemsetAsync(dv, 0, tensor_bytes, st));
+        HSTU_CUDA(cudaMemsetAsync(dq, 0, tensor_bytes, st));
+    }
+    HSTU_TRY(schedule(desc, seq_offsets, num_targets, 0, workspace, st));
+    return cuda_status(launch_attn_bwd_f32(p, grid_items(desc), st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -198,49 +256,10 @@ hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void 
         !aligned16(dk) || !aligned16(dv))
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_ws(workspace, workspace_bytes, attn_ws(desc, 1)));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int npos = desc->pos_hi - desc->pos_lo + 1;
-    HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * npos, st));
-    HSTU_CUDA(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->num_time_buckets, st));
     const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
-    const size_t tensor_bytes = (size_t)desc->total_tokens * row * elem_bytes(desc);
-    const bool bf16 = desc->dtype == HSTU_BF16;
-    AttnParams p = base_params(desc, seq_offsets, timestamps, num_targets, rab_pos, rab_time, workspace);
-    p.q = q;
-    p.k = k;
-    p.v = v;
-    p.sq = p.sk = p.sv = row;
-    p.dout = dout;
-    p.sdo = row;
-    p.dq = dq;
-    p.dk = dk;
-    p.dvv = dv;
-    p.sdq = p.sdk = p.sdv = row;
-    p.d_rab_pos = d_rab_pos;
-    p.d_rab_time = d_rab_time;
-    if (bf16) {
-        p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + sizeof(WsHeader) +
-                                             items_bytes(desc));
-        HSTU_CUDA(cudaMemsetAsync(p.dq_acc, 0, sizeof(float) * (size_t)desc->total_tokens * row, st));
-        float dq_scale = 1.0f;
-        if (attn_bwd_tc_supported(p)) {
-            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st, kTcTile));
-            HSTU_CUDA(launch_attn_bwd_tc(p, grid_items(desc, kTcTile), st));
-            dq_scale = 0.5f * desc->inv_n;
-        } else {
-            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
-            HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
-        }
-        return cuda_status(launch_convert_dq(p.dq_acc, dq, desc->total_tokens, desc->num_heads,
-                                             desc->d_qk, row, dq_scale, st));
-    }
-    if (tensor_bytes) {
-        HSTU_CUDA(cudaMemsetAsync(dk, 0, tensor_bytes, st));
-        HSTU_CUDA(cudaMemsetAsync(dv, 0, tensor_bytes, st));
-        HSTU_CUDA(cudaMemsetAsync(dq, 0, tensor_bytes, st));
-    }
-    HSTU_TRY(schedule(desc, seq_offsets, num_targets, 0, workspace, st));
-    return cuda_status(launch_attn_bwd_f32(p, grid_items(desc), st));
+    return attn_bwd_strided(desc, q, row, k, row, v, row, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                            dout, row, dq, row, dk, row, dv, row, d_rab_pos, d_rab_time, workspace,
+                            static_cast<cudaStream_t>(stream));
 }
 
 static hstu_status check_layer_desc(const hstu_layer_desc *d)
@@ -340,6 +359,156 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
     return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(g), hv,
                                        static_cast<const float *>(w2), static_cast<const float *>(b2),
                                        static_cast<float *>(y), D, (int64_t)T, D, hv, false, st));
+}
+
+static size_t layer_bwd_ws(const hstu_layer_desc *d)
+{
+    const hstu_attn_desc *a = &d->attn;
+    const size_t T = (size_t)a->total_tokens, W = layer_width(a), hv = (size_t)a->num_heads * a->d_v;
+    // attention backward scratch, then G, dG, dO [T, H d_v] and dA, dZ [T, W] (bf16)
+    return attn_ws(a, 1) + 3 * align256(T * hv * 2) + 2 * align256(T * W * 2);
+}
+
+static bool layer_bwd_supported(const hstu_layer_desc *d)
+{
+    const hstu_attn_desc *a = &d->attn;
+    const int hv = a->num_heads * a->d_v, W = layer_width(a);
+    return a->dtype == HSTU_BF16 && d->d_model % 128 == 0 && hv % 128 == 0 && W % 128 == 0;
+}
+
+hstu_status hstu_layer_bwd_workspace_size(const hstu_layer_desc *desc, size_t *bytes)
+{
+    HSTU_TRY(check_layer_desc(desc));
+    if (!bytes)
+        return HSTU_ERR_INVALID_ARG;
+    *bytes = layer_bwd_ws(desc);
+    return HSTU_OK;
+}
+
+hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const void *w1, const void *b1,
+                           const void *w2, const float *ln_gamma, const float *ln_beta,
+                           const int64_t *seq_offsets, const int64_t *timestamps, const int32_t *num_targets,
+                           const float *rab_pos, const float *rab_time, const void *saved_uvqk,
+                           const void *saved_o, const void *dy, void *dx, float *dw1, float *db1, float *dw2,
+                           float *db2, float *d_ln_gamma, float *d_ln_beta, float *d_rab_pos,
+                           float *d_rab_time, void *workspace, size_t workspace_bytes, void *stream)
+{
+    HSTU_TRY(check_layer_desc(desc));
+    if (!layer_bwd_supported(desc))
+        return HSTU_ERR_UNSUPPORTED;
+    const hstu_attn_desc *a = &desc->attn;
+    if (!seq_offsets || !rab_pos || !rab_time || !w1 || !w2 || !ln_gamma || !ln_beta || !dw1 || !db1 || !dw2 ||
+        !db2 || !d_ln_gamma || !d_ln_beta || !d_rab_pos || !d_rab_time)
+        return HSTU_ERR_INVALID_ARG;
+    if (a->total_tokens > 0 && (!x || !dx || !dy || !saved_uvqk || !saved_o || !timestamps))
+        return HSTU_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, w1, b1, w2, saved_uvqk, saved_o, dy, dx, dw1, db1, dw2, db2};
+    for (const void *q : ptrs)
+        if (!aligned16(q))
+            return HSTU_ERR_INVALID_ARG;
+    HSTU_TRY(check_ws(workspace, workspace_bytes, layer_bwd_ws(desc)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t T = a->total_tokens;
+    const int W = layer_width(a), hv = a->num_heads * a->d_v, hq = a->num_heads * a->d_qk;
+    const int D = desc->d_model;
+    WsHeader *hdr = static_cast<WsHeader *>(workspace);
+
+    HSTU_CUDA(cudaMemsetAsync(dw1, 0, sizeof(float) * (size_t)D * W, st));
+    HSTU_CUDA(cudaMemsetAsync(db1, 0, sizeof(float) * W, st));
+    HSTU_CUDA(cudaMemsetAsync(dw2, 0, sizeof(float) * (size_t)hv * D, st));
+    HSTU_CUDA(cudaMemsetAsync(db2, 0, sizeof(float) * D, st));
+    HSTU_CUDA(cudaMemsetAsync(d_ln_gamma, 0, sizeof(float) * hv, st));
+    HSTU_CUDA(cudaMemsetAsync(d_ln_beta, 0, sizeof(float) * hv, st));
+    if (T == 0) {
+        HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (a->pos_hi - a->pos_lo + 1), st));
+        return cuda_status(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * a->num_time_buckets, st));
+    }
+    char *cur = static_cast<char *>(workspace) + attn_ws(a, 1);
+    auto take = [&](size_t bytes) {
+        char *p = cur;
+        cur += align256(bytes);
+        return p;
+    };
+    char *g = take((size_t)T * hv * 2), *dg = take((size_t)T * hv * 2), *dout = take((size_t)T * hv * 2);
+    char *da = take((size_t)T * W * 2), *dz = take((size_t)T * W * 2);
+    const char *uvqk = static_cast<const char *>(saved_uvqk);
+    const int sms = 148;
+    auto splits_for = [&](int64_t M, int N) {
+        const int64_t tiles = ((M + 127) / 128) * (N / 128);
+        return (int)std::max<int64_t>(1, std::min<int64_t>((2 * sms + tiles - 1) / tiles, (T + 63) / 64));
+    };
+
+    // G = LayerNorm(O) U, recomputed from the saved attention output
+    HSTU_CUDA(launch_norm_gate(true, saved_o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv, T, hv, st));
+    // output projection: dG = dy W2^T, dW2 = G^T dy, db2 = sum dy
+    GemmOperands op{};
+    op.A = dy;
+    op.lda = D;
+    op.B = w2;
+    op.ldb = D;
+    op.b_k = true;
+    op.C = dg;
+    op.ldc = hv;
+    if (!gemm_tc_ok(op, T, hv, D))
+        return HSTU_ERR_UNSUPPORTED;
+    HSTU_CUDA(launch_gemm_tc_ex(op, T, hv, D, GEMM_ACT, false, 1, hdr, st));
+    op = GemmOperands{};
+    op.A = g;
+    op.lda = hv;
+    op.a_mn = true;
+    op.B = dy;
+    op.ldb = D;
+    op.C32 = dw2;
+    op.ldc = D;
+    if (!gemm_tc_ok(op, hv, D, (int)T))
+        return HSTU_ERR_UNSUPPORTED;
+    HSTU_CUDA(launch_gemm_tc_ex(op, hv, D, (int)T, GEMM_RED_F32, false, splits_for(hv, D), hdr, st));
+    HSTU_CUDA(launch_colsum_bf16(dy, D, T, D, db2, st));
+    // gate: dO and dU (into the U block of dA), dgamma, dbeta
+    HSTU_CUDA(launch_norm_gate_bwd(dg, hv, saved_o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, dout, hv, da, W,
+                                   d_ln_gamma, d_ln_beta, T, hv, st));
+    // attention: dV, dQ, dK into their blocks of dA, bias-table gradients
+    HSTU_TRY(attn_bwd_strided(a, uvqk + (size_t)2 * hv * 2, W, uvqk + (size_t)(2 * hv + hq) * 2, W,
+                              uvqk + (size_t)hv * 2, W, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                              dout, hv, da + (size_t)2 * hv * 2, W, da + (size_t)(2 * hv + hq) * 2, W,
+                              da + (size_t)hv * 2, W, d_rab_pos, d_rab_time, workspace, st));
+    // projection: dZ = dA SiLU'(X W1 + b1) (recomputed in the GEMM), db1, dX = dZ W1^T, dW1 = X^T dZ
+    op = GemmOperands{};
+    op.A = x;
+    op.lda = D;
+    op.B = w1;
+    op.ldb = W;
+    op.bias = b1;
+    op.aux = da;
+    op.ldaux = W;
+    op.C = dz;
+    op.ldc = W;
+    if (!gemm_tc_ok(op, T, W, D))
+        return HSTU_ERR_UNSUPPORTED;
+    HSTU_CUDA(launch_gemm_tc_ex(op, T, W, D, GEMM_DSILU, false, 1, hdr, st));
+    HSTU_CUDA(launch_colsum_bf16(dz, W, T, W, db1, st));
+    op = GemmOperands{};
+    op.A = dz;
+    op.lda = W;
+    op.B = w1;
+    op.ldb = W;
+    op.b_k = true;
+    op.C = dx;
+    op.ldc = D;
+    if (!gemm_tc_ok(op, T, D, W))
+        return HSTU_ERR_UNSUPPORTED;
+    HSTU_CUDA(launch_gemm_tc_ex(op, T, D, W, GEMM_ACT, false, 1, hdr, st));
+    op = GemmOperands{};
+    op.A = x;
+    op.lda = D;
+    op.a_mn = true;
+    op.B = dz;
+    op.ldb = W;
+    op.C32 = dw1;
+    op.ldc = W;
+    if (!gemm_tc_ok(op, D, W, (int)T))
+        return HSTU_ERR_UNSUPPORTED;
+    return cuda_status(launch_gemm_tc_ex(op, D, W, (int)T, GEMM_RED_F32, false, splits_for(D, W), hdr, st));
 }
 
 hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream)

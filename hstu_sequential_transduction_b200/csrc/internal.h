@@ -62,9 +62,44 @@ cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const 
                             float *C, int64_t ldc, int64_t M, int N, int K, bool silu,
                             cudaStream_t stream);
 
+// General tcgen05 GEMM C[M, N] = epi(A B) (bf16 operands, fp32 accumulation).
+//   A: a_mn = false -> A[m][k] at A + m*lda + k;  a_mn = true -> at A + k*lda + m
+//   B: b_k = false  -> B[k][n] at B + k*ldb + n;  b_k = true  -> at B + n*ldb + k
+//   GEMM_ACT:    C bf16 = acc + bias (optionally SiLU)
+//   GEMM_DSILU:  C bf16 = aux * SiLU'(acc + bias), aux bf16 [M, N] (row stride ldaux)
+//   GEMM_RED_F32: C32 fp32 += acc, the k range split over `splits` CTAs (C32 must
+//                 hold its initial value, e.g. zeros); ldc in elements.
+enum GemmEpilogue { GEMM_ACT = 0, GEMM_DSILU = 1, GEMM_RED_F32 = 2 };
+struct GemmOperands {
+    const void *A;
+    int64_t lda;
+    bool a_mn;
+    const void *B;
+    int64_t ldb;
+    bool b_k;
+    const void *bias;
+    const void *aux;
+    int64_t ldaux;
+    void *C;
+    float *C32;
+    int64_t ldc;
+};
+bool gemm_tc_ok(const GemmOperands &op, int64_t M, int N, int K);
+cudaError_t launch_gemm_tc_ex(const GemmOperands &op, int64_t M, int N, int K, GemmEpilogue epi, bool silu,
+                              int splits, WsHeader *hdr, cudaStream_t stream);
+
 // G[t, :] = LayerNorm(O[t, :]) * U[t, :] over F features.
 cudaError_t launch_norm_gate(bool bf16, const void *O, int64_t ldo, const void *U, int64_t ldu,
                              const float *gamma, const float *beta, float eps, void *G,
                              int64_t ldg, int64_t T, int F, cudaStream_t stream);
+
+// Backward of G = LayerNorm(O) * U (bf16): writes dO and dU (row strides in
+// elements) and adds the parameter gradients to dgamma, dbeta (fp32 [F]).
+cudaError_t launch_norm_gate_bwd(const void *dG, int64_t ldd, const void *O, int64_t ldo, const void *U,
+                                 int64_t ldu, const float *gamma, const float *beta, float eps, void *dO,
+                                 int64_t lddo, void *dU, int64_t lddu, float *dgamma, float *dbeta, int64_t T,
+                                 int F, cudaStream_t stream);
+// out[n] += sum over T rows of A[row, n] (bf16 A, fp32 out).
+cudaError_t launch_colsum_bf16(const void *A, int64_t lda, int64_t T, int N, float *out, cudaStream_t stream);
 
 }  // namespace hstu

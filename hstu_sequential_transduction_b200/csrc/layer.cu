@@ -303,6 +303,136 @@ cudaError_t norm_gate_t(const T *O, int64_t ldo, const T *U, int64_t ldu, const 
     return cudaGetLastError();
 }
 
+// Backward of G = LayerNorm(O) * U, per token over F features (the gate of
+// the "HSTU Architecture" section): with xh = (x - mean) rstd, ln = xh g + b,
+// dy = dG U:  dU = dG ln,  dO = rstd (dy g - mean(dy g) - xh mean(dy g xh)),
+// dgamma += dy xh, dbeta += dy.  One warp per token (grid-stride over tokens);
+// each block folds its warps' parameter gradients in shared memory and adds
+// them to the outputs with one atomic per feature.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256)
+norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict__ O, int64_t ldo,
+                     const T *__restrict__ U, int64_t ldu, const float *__restrict__ gamma,
+                     const float *__restrict__ beta, float eps, T *__restrict__ dO, int64_t lddo,
+                     T *__restrict__ dU, int64_t lddu, float *__restrict__ dgamma, float *__restrict__ dbeta,
+                     int64_t Trows)
+{
+    constexpr int F = 32 * VPT;
+    __shared__ float sg[F], sb[F];
+    for (int f = threadIdx.x; f < F; f += blockDim.x) {
+        sg[f] = 0.f;
+        sb[f] = 0.f;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    float ga[VPT], be[VPT], pg[VPT], pb[VPT];
+    load_vec<float, VPT>(gamma + lane * VPT, ga);
+    load_vec<float, VPT>(beta + lane * VPT, be);
+#pragma unroll
+    for (int e = 0; e < VPT; e++) {
+        pg[e] = 0.f;
+        pb[e] = 0.f;
+    }
+    for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < Trows; row += warps) {
+        float x[VPT], u[VPT], dg[VPT];
+        load_vec<T, VPT>(O + row * ldo + lane * VPT, x);
+        load_vec<T, VPT>(U + row * ldu + lane * VPT, u);
+        load_vec<T, VPT>(dG + row * ldd + lane * VPT, dg);
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            sum += x[e];
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float mean = sum * (1.0f / F);
+        float var = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPT; e++) {
+            const float d = x[e] - mean;
+            var += d * d;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            var += __shfl_xor_sync(0xffffffffu, var, off);
+        const float rstd = rsqrtf(var * (1.0f / F) + eps);
+        float du[VPT], dxh[VPT], xh[VPT];
+        float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPT; e++) {
+            xh[e] = (x[e] - mean) * rstd;
+            du[e] = dg[e] * fmaf(xh[e], ga[e], be[e]);
+            const float dy = dg[e] * u[e];
+            pg[e] = fmaf(dy, xh[e], pg[e]);
+            pb[e] += dy;
+            dxh[e] = dy * ga[e];
+            s1 += dxh[e];
+            s2 = fmaf(dxh[e], xh[e], s2);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+        }
+        const float m1 = s1 * (1.0f / F), m2 = s2 * (1.0f / F);
+        float dx[VPT];
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            dx[e] = rstd * (dxh[e] - m1 - xh[e] * m2);
+        store_vec<T, VPT>(dO + row * lddo + lane * VPT, dx);
+        store_vec<T, VPT>(dU + row * lddu + lane * VPT, du);
+    }
+#pragma unroll
+    for (int e = 0; e < VPT; e++) {
+        atomicAdd(&sg[lane * VPT + e], pg[e]);
+        atomicAdd(&sb[lane * VPT + e], pb[e]);
+    }
+    __syncthreads();
+    for (int f = threadIdx.x; f < F; f += blockDim.x) {
+        atomicAdd(dgamma + f, sg[f]);
+        atomicAdd(dbeta + f, sb[f]);
+    }
+}
+
+template <typename T>
+cudaError_t norm_gate_bwd_t(const T *dG, int64_t ldd, const T *O, int64_t ldo, const T *U, int64_t ldu,
+                            const float *gamma, const float *beta, float eps, T *dO, int64_t lddo, T *dU,
+                            int64_t lddu, float *dgamma, float *dbeta, int64_t Trows, int F, cudaStream_t stream)
+{
+    const int64_t want = (Trows * 32 + 255) / 256;
+    const unsigned blocks = (unsigned)std::min<int64_t>(want, 148 * 8);
+#define HSTU_NGB(V)                                                                                              \
+    norm_gate_bwd_kernel<T, V><<<blocks, 256, 0, stream>>>(dG, ldd, O, ldo, U, ldu, gamma, beta, eps, dO, lddo, \
+                                                           dU, lddu, dgamma, dbeta, Trows)
+    switch (F) {
+    case 64: HSTU_NGB(2); break;
+    case 128: HSTU_NGB(4); break;
+    case 256: HSTU_NGB(8); break;
+    case 512: HSTU_NGB(16); break;
+    case 1024: HSTU_NGB(32); break;
+    default: return cudaErrorInvalidValue;
+    }
+#undef HSTU_NGB
+    return cudaGetLastError();
+}
+
+// out[n] += sum over rows of A[row, n] (bf16 rows of N columns, fp32 sums): each
+// block sums 256 columns over a chunk of rows, one atomic per column.
+__global__ void __launch_bounds__(256)
+colsum_bf16_kernel(const __nv_bfloat16 *__restrict__ A, int64_t lda, int64_t Trows, int N, int64_t chunk,
+                   float *__restrict__ out)
+{
+    const int n = blockIdx.x * 256 + threadIdx.x;
+    if (n >= N)
+        return;
+    const int64_t r0 = (int64_t)blockIdx.y * chunk, r1 = r0 + chunk < Trows ? r0 + chunk : Trows;
+    float acc = 0.f;
+    for (int64_t r = r0; r < r1; r++)
+        acc += __bfloat162float(A[r * lda + n]);
+    atomicAdd(out + n, acc);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
@@ -327,6 +457,30 @@ cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const 
         return cudaSuccess;
     dim3 grid((N + FT - 1) / FT, (unsigned)((M + FT - 1) / FT));
     gemm_f32_kernel<<<grid, 256, 0, stream>>>(A, lda, Bm, bias, C, ldc, M, N, K, silu);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_gate_bwd(const void *dG, int64_t ldd, const void *O, int64_t ldo, const void *U,
+                                 int64_t ldu, const float *gamma, const float *beta, float eps, void *dO,
+                                 int64_t lddo, void *dU, int64_t lddu, float *dgamma, float *dbeta, int64_t T,
+                                 int F, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    return norm_gate_bwd_t(static_cast<const __nv_bfloat16 *>(dG), ldd, static_cast<const __nv_bfloat16 *>(O), ldo,
+                           static_cast<const __nv_bfloat16 *>(U), ldu, gamma, beta, eps,
+                           static_cast<__nv_bfloat16 *>(dO), lddo, static_cast<__nv_bfloat16 *>(dU), lddu, dgamma,
+                           dbeta, T, F, stream);
+}
+
+cudaError_t launch_colsum_bf16(const void *A, int64_t lda, int64_t T, int N, float *out, cudaStream_t stream)
+{
+    if (T == 0 || N == 0)
+        return cudaSuccess;
+    const int64_t chunks = std::min<int64_t>((T + 127) / 128, 256);
+    const int64_t chunk = (T + chunks - 1) / chunks;
+    dim3 grid((N + 255) / 256, (unsigned)((T + chunk - 1) / chunk));
+    colsum_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(A), lda, T, N, chunk, out);
     return cudaGetLastError();
 }
 

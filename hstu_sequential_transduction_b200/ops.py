@@ -25,7 +25,7 @@ STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3:
 EXPORTED = ["hstu_status_string", "hstu_version", "hstu_attn_workspace_size",
             "hstu_layer_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd",
             "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule",
-            "hstu_attn_fwd_noalloc"]
+            "hstu_attn_fwd_noalloc", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"]
 
 
 class HstuError(RuntimeError):
@@ -232,6 +232,48 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
         _ptr(rab_time), _ptr(y), _ptr(saved_uvqk), _ptr(saved_o), _ptr(workspace),
         ctypes.c_size_t(workspace.numel()), _stream(stream)))
     return y
+
+
+def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("hstu_layer_bwd_workspace_size",
+           load_library().hstu_layer_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                   saved_uvqk, saved_o, dy, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
+                   inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, workspace=None, stream=None):
+    """Gradients of sum(Y * dy) for one layer (bf16): a dict with dx (bf16) and the
+    float32 parameter gradients dw1, db1, dw2, db2, d_ln_gamma, d_ln_beta,
+    d_rab_pos, d_rab_time."""
+    for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("saved_uvqk", saved_uvqk),
+                    ("saved_o", saved_o), ("dy", dy)):
+        _dev(t, name, x.dtype)
+    _dev(ln_gamma, "ln_gamma", torch.float32)
+    _dev(ln_beta, "ln_beta", torch.float32)
+    T, D = x.shape
+    W = w1.shape[1]
+    hv = num_heads * d_v
+    attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
+    desc = hstu_layer_desc(attn, int(D), float(ln_eps))
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty((T, D), dtype=x.dtype, device=dev), "dw1": torch.empty((D, W), **f32),
+           "db1": torch.empty(W, **f32), "dw2": torch.empty((hv, D), **f32), "db2": torch.empty(D, **f32),
+           "d_ln_gamma": torch.empty(hv, **f32), "d_ln_beta": torch.empty(hv, **f32),
+           "d_rab_pos": torch.empty(rab_pos.numel(), **f32), "d_rab_time": torch.empty(rab_time.numel(), **f32)}
+    if workspace is None:
+        workspace = alloc_workspace(hstu_layer_bwd_workspace_size(desc), dev)
+    _check("hstu_layer_bwd", load_library().hstu_layer_bwd(
+        ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(ln_gamma), _ptr(ln_beta),
+        _ptr(seq_offsets), _ptr(timestamps), _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time),
+        _ptr(saved_uvqk), _ptr(saved_o), _ptr(dy), _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["db1"]),
+        _ptr(out["dw2"]), _ptr(out["db2"]), _ptr(out["d_ln_gamma"]), _ptr(out["d_ln_beta"]),
+        _ptr(out["d_rab_pos"]), _ptr(out["d_rab_time"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+        _stream(stream)))
+    return out
 
 
 def hstu_check_device_flag(workspace: torch.Tensor, stream=None):

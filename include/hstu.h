@@ -141,6 +141,35 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Bytes of device workspace hstu_layer_bwd needs (256-byte aligned, scratch).
+ */
+hstu_status hstu_layer_bwd_workspace_size(const hstu_layer_desc *desc, size_t *bytes);
+
+/*
+ * One transduction layer backward for the loss sum(Y * dy) (the layer of
+ * hstu_layer_fwd; the DLRMv4 page's "Computation Cost Analysis" counts its
+ * GEMMs three times over the forward's).  bf16 only.
+ * Inputs: the forward's x, w1, b1, w2, ln_gamma, ln_beta, bias tables and
+ * sequence data; saved_uvqk = SiLU(X W1 + b1) and saved_o = the attention
+ * output, as hstu_layer_fwd keeps them; dy [T, D] (bf16).
+ * Outputs (all overwritten): dx [T, D] (bf16); dw1 [D, W], db1 [W], dw2 [H d_v, D],
+ * db2 [D], d_ln_gamma, d_ln_beta [H d_v], d_rab_pos [pos_hi - pos_lo + 1],
+ * d_rab_time [NB] (all float32; W = H(2 d_v + 2 d_qk)).
+ * The pre-activation X W1 + b1 is recomputed (its SiLU derivative is applied
+ * in that GEMM's epilogue), and G = LayerNorm(O) U from saved_o and U.
+ * Requires D, H d_v and W multiples of 128 (HSTU_ERR_UNSUPPORTED otherwise);
+ * every pointer 16-byte aligned (HSTU_ERR_INVALID_ARG).
+ */
+hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const void *w1, const void *b1,
+                           const void *w2, const float *ln_gamma, const float *ln_beta,
+                           const int64_t *seq_offsets, const int64_t *timestamps,
+                           const int32_t *num_targets, const float *rab_pos, const float *rab_time,
+                           const void *saved_uvqk, const void *saved_o, const void *dy, void *dx,
+                           float *dw1, float *db1, float *dw2, float *db2, float *d_ln_gamma,
+                           float *d_ln_beta, float *d_rab_pos, float *d_rab_time, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
  * Attention forward that allocates nothing (no counterpart on the HSTU
  * pages; it exists for callers, not for the method).  Same computation,
  * arguments and layouts as hstu_attn_fwd, without the workspace: some callers
