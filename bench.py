@@ -70,7 +70,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-stack", action="store_true",
                     help="skip the secondary eight-layer forward measurement")
-    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer"], default=None,
+    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer", "layer_bwd"], default=None,
                     help="run only a small case twice (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -223,7 +223,33 @@ def layer_stack_timing(dev, stream, reps: int = 3):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
+
+    # the first layer's backward (hstu_layer_bwd) for an upstream gradient dY ~ N(0, 1)
+    W = w.num_heads * (2 * w.d_v + 2 * w.d_qk)
+    uvqk = torch.empty((T, W), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((T, w.num_heads * w.d_v), dtype=torch.bfloat16, device=dev)
+    w1, b1, w2, b2, g, be = layers[0]
+    ops.hstu_layer_fwd(xs[0], w1, b1, w2, b2, g, be, off, ts, None, rp, rt, y=xs[1], saved_uvqk=uvqk,
+                       saved_o=o, workspace=ws, stream=stream, **kw)
+    gen = torch.Generator(device="cpu").manual_seed(2024)
+    dy = torch.randn((T, w.d_model), generator=gen).to(device=dev, dtype=torch.bfloat16)
+    wsb = ops.alloc_workspace(ops.hstu_layer_bwd_workspace_size(desc), dev)
+
+    def backward():
+        ops.hstu_layer_bwd(xs[0], w1, b1, w2, g, be, off, ts, None, rp, rt, uvqk, o, dy, workspace=wsb,
+                           stream=stream, **kw)
+
+    backward()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        backward()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bwd_ms = e0.elapsed_time(e1) / reps
     pairs = flops.attn_pairs(a.lengths)
+    bwd_fl = flops.layer_bwd_gemm_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
+        flops.attn_bwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
     attn_fl = flops.attn_fwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
     gemm_fl = flops.f1_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
         flops.f2_flops(T, w.d_model, w.num_heads, w.d_v)
@@ -231,7 +257,8 @@ def layer_stack_timing(dev, stream, reps: int = 3):
     return {"workload": "layer_stack_bf16", "layers": w.num_layers, "tokens": T,
             "ms_per_forward": ms, "tflops": total / (ms * 1e-3) / 1e12,
             "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
-            "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v)}
+            "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v),
+            "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12}}
 
 
 def run_reference(args):
@@ -471,7 +498,7 @@ def run_ours(args):
 def kernel_case(which: str):
     """A small case of one kernel, run twice, for ncu captures: 3 sequences of
     11k-13k tokens (long-history shapes, ~36k tokens, inputs > L2), or one
-    eight-layer stack forward."""
+    eight-layer stack forward followed by one layer backward (layer, layer_bwd)."""
     import numpy as np
     import torch
 
@@ -480,6 +507,28 @@ def kernel_case(which: str):
     dev = torch.device("cuda:0")
     if which == "layer":
         layer_stack_timing(dev, torch.cuda.current_stream(), reps=1)
+        torch.cuda.synchronize()
+        return
+    if which == "layer_bwd":
+        # one layer of the stack workload: a forward keeping U|V|Q|K and O, then two backwards
+        w = workloads.WORKLOADS["layer_stack_bf16"]
+        inp = workloads.generate(w)
+        a, lw = inp.attn, inp.layers[0]
+        T = a.total_tokens
+        kw = dict(num_heads=w.num_heads, d_qk=w.d_qk, d_v=w.d_v, max_seq_len=a.max_seq_len, inv_n=a.inv_n,
+                  pos_lo=a.pos_lo, pos_hi=a.pos_hi)
+        prm = [t.to(dev) for t in (lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta)]
+        seq = [a.seq_offsets.to(dev), a.timestamps.to(dev), None, a.rab_pos.to(dev), a.rab_time.to(dev)]
+        x = inp.x.to(dev)
+        W = w.num_heads * (2 * w.d_v + 2 * w.d_qk)
+        uvqk = torch.empty((T, W), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((T, w.num_heads * w.d_v), dtype=torch.bfloat16, device=dev)
+        ops.hstu_layer_fwd(x, *prm, *seq, saved_uvqk=uvqk, saved_o=o, **kw)
+        gen = torch.Generator(device="cpu").manual_seed(2024)
+        dy = torch.randn((T, w.d_model), generator=gen).to(device=dev, dtype=torch.bfloat16)
+        w1, b1, w2, _, g, be = prm
+        for _ in range(2):
+            ops.hstu_layer_bwd(x, w1, b1, w2, g, be, *seq, uvqk, o, dy, **kw)
         torch.cuda.synchronize()
         return
     rng = np.random.default_rng(7)

@@ -306,9 +306,11 @@ cudaError_t norm_gate_t(const T *O, int64_t ldo, const T *U, int64_t ldu, const 
 // Backward of G = LayerNorm(O) * U, per token over F features (the gate of
 // the "HSTU Architecture" section): with xh = (x - mean) rstd, ln = xh g + b,
 // dy = dG U:  dU = dG ln,  dO = rstd (dy g - mean(dy g) - xh mean(dy g xh)),
-// dgamma += dy xh, dbeta += dy.  One warp per token (grid-stride over tokens);
-// each block folds its warps' parameter gradients in shared memory and adds
-// them to the outputs with one atomic per feature.
+// dgamma += dy xh, dbeta += dy.  One warp per token (grid-stride over tokens),
+// two passes over the token's row (the second re-reads it from L1) so few
+// values stay live; each lane keeps its features' parameter gradients in
+// registers across tokens, each warp stores them once to its shared-memory
+// slot, and each block adds the sum of its slots to the outputs.
 template <typename T, int VPT>
 __global__ void __launch_bounds__(256)
 norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict__ O, int64_t ldo,
@@ -318,27 +320,20 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
                      int64_t Trows)
 {
     constexpr int F = 32 * VPT;
-    __shared__ float sg[F], sb[F];
-    for (int f = threadIdx.x; f < F; f += blockDim.x) {
-        sg[f] = 0.f;
-        sb[f] = 0.f;
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    float ga[VPT], be[VPT], pg[VPT], pb[VPT];
-    load_vec<float, VPT>(gamma + lane * VPT, ga);
-    load_vec<float, VPT>(beta + lane * VPT, be);
+    extern __shared__ float slots[];  // [warps][2][F]
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    float *sg = slots + wid * 2 * F, *sb = sg + F;
+    float pg[VPT], pb[VPT];
 #pragma unroll
     for (int e = 0; e < VPT; e++) {
         pg[e] = 0.f;
         pb[e] = 0.f;
     }
+    const int64_t warps = (int64_t)gridDim.x * nw;
     for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < Trows; row += warps) {
-        float x[VPT], u[VPT], dg[VPT];
-        load_vec<T, VPT>(O + row * ldo + lane * VPT, x);
-        load_vec<T, VPT>(U + row * ldu + lane * VPT, u);
-        load_vec<T, VPT>(dG + row * ldd + lane * VPT, dg);
+        const int64_t fo = lane * VPT;
+        float x[VPT];
+        load_vec<T, VPT>(O + row * ldo + fo, x);
         float sum = 0.f;
 #pragma unroll
         for (int e = 0; e < VPT; e++)
@@ -350,25 +345,28 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
         float var = 0.f;
 #pragma unroll
         for (int e = 0; e < VPT; e++) {
-            const float d = x[e] - mean;
-            var += d * d;
+            x[e] -= mean;
+            var += x[e] * x[e];
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1)
             var += __shfl_xor_sync(0xffffffffu, var, off);
         const float rstd = rsqrtf(var * (1.0f / F) + eps);
-        float du[VPT], dxh[VPT], xh[VPT];
+        // pass 1: the two row means of the LayerNorm backward, parameter gradients
         float s1 = 0.f, s2 = 0.f;
+        {
+            float u[VPT], dg[VPT], ga[VPT];
+            load_vec<T, VPT>(U + row * ldu + fo, u);
+            load_vec<T, VPT>(dG + row * ldd + fo, dg);
+            load_vec<float, VPT>(gamma + fo, ga);
 #pragma unroll
-        for (int e = 0; e < VPT; e++) {
-            xh[e] = (x[e] - mean) * rstd;
-            du[e] = dg[e] * fmaf(xh[e], ga[e], be[e]);
-            const float dy = dg[e] * u[e];
-            pg[e] = fmaf(dy, xh[e], pg[e]);
-            pb[e] += dy;
-            dxh[e] = dy * ga[e];
-            s1 += dxh[e];
-            s2 = fmaf(dxh[e], xh[e], s2);
+            for (int e = 0; e < VPT; e++) {
+                const float xh = x[e] * rstd, dy = dg[e] * u[e];
+                pg[e] = fmaf(dy, xh, pg[e]);
+                pb[e] += dy;
+                s1 = fmaf(dy, ga[e], s1);
+                s2 = fmaf(dy * ga[e], xh, s2);
+            }
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) {
@@ -376,22 +374,37 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
             s2 += __shfl_xor_sync(0xffffffffu, s2, off);
         }
         const float m1 = s1 * (1.0f / F), m2 = s2 * (1.0f / F);
-        float dx[VPT];
+        // pass 2: dO and dU
+        {
+            float u[VPT], dg[VPT], ga[VPT], be[VPT], dx[VPT], du[VPT];
+            load_vec<T, VPT>(U + row * ldu + fo, u);
+            load_vec<T, VPT>(dG + row * ldd + fo, dg);
+            load_vec<float, VPT>(gamma + fo, ga);
+            load_vec<float, VPT>(beta + fo, be);
 #pragma unroll
-        for (int e = 0; e < VPT; e++)
-            dx[e] = rstd * (dxh[e] - m1 - xh[e] * m2);
-        store_vec<T, VPT>(dO + row * lddo + lane * VPT, dx);
-        store_vec<T, VPT>(dU + row * lddu + lane * VPT, du);
+            for (int e = 0; e < VPT; e++) {
+                const float xh = x[e] * rstd;
+                du[e] = dg[e] * fmaf(xh, ga[e], be[e]);
+                dx[e] = rstd * (dg[e] * u[e] * ga[e] - m1 - xh * m2);
+            }
+            store_vec<T, VPT>(dO + row * lddo + fo, dx);
+            store_vec<T, VPT>(dU + row * lddu + fo, du);
+        }
     }
 #pragma unroll
     for (int e = 0; e < VPT; e++) {
-        atomicAdd(&sg[lane * VPT + e], pg[e]);
-        atomicAdd(&sb[lane * VPT + e], pb[e]);
+        sg[lane * VPT + e] = pg[e];
+        sb[lane * VPT + e] = pb[e];
     }
     __syncthreads();
     for (int f = threadIdx.x; f < F; f += blockDim.x) {
-        atomicAdd(dgamma + f, sg[f]);
-        atomicAdd(dbeta + f, sb[f]);
+        float a = 0.f, b = 0.f;
+        for (int w = 0; w < nw; w++) {
+            a += slots[w * 2 * F + f];
+            b += slots[w * 2 * F + F + f];
+        }
+        atomicAdd(dgamma + f, a);
+        atomicAdd(dbeta + f, b);
     }
 }
 
@@ -402,9 +415,20 @@ cudaError_t norm_gate_bwd_t(const T *dG, int64_t ldd, const T *O, int64_t ldo, c
 {
     const int64_t want = (Trows * 32 + 255) / 256;
     const unsigned blocks = (unsigned)std::min<int64_t>(want, 148 * 8);
-#define HSTU_NGB(V)                                                                                              \
-    norm_gate_bwd_kernel<T, V><<<blocks, 256, 0, stream>>>(dG, ldd, O, ldo, U, ldu, gamma, beta, eps, dO, lddo, \
-                                                           dU, lddu, dgamma, dbeta, Trows)
+    const size_t smem = (size_t)8 * 2 * F * sizeof(float);  // 8 warps x (dgamma, dbeta) slots
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaErrorInvalidValue;
+        switch (F) {
+        case 1024: e = cudaFuncSetAttribute(norm_gate_bwd_kernel<T, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)smem); break;
+        default: break;
+        }
+        if (e != cudaSuccess)
+            return e;
+    }
+#define HSTU_NGB(V)                                                                                                 \
+    norm_gate_bwd_kernel<T, V><<<blocks, 256, smem, stream>>>(dG, ldd, O, ldo, U, ldu, gamma, beta, eps, dO, lddo, \
+                                                              dU, lddu, dgamma, dbeta, Trows)
     switch (F) {
     case 64: HSTU_NGB(2); break;
     case 128: HSTU_NGB(4); break;

@@ -49,3 +49,14 @@ def f2_flops(tokens: int, d_model: int, num_heads: int, d_v: int, width_factor: 
 def gate_bytes(tokens: int, num_heads: int, d_v: int, elem_bytes: int = 2) -> float:
     """LayerNorm(O) * U: read O and U, write G (one pass each)."""
     return 3.0 * tokens * num_heads * d_v * elem_bytes
+
+
+def layer_bwd_gemm_flops(T: int, d_model: int, num_heads: int, d_qk: int, d_v: int) -> float:
+    """Algorithmic FLOPs of the layer backward's GEMMs, twice the forward's (the
+    DLRMv4 page's Table 7 counts forward + backward as three times the forward):
+    dG = dY W2^T, dW2 = G^T dY (2 T D H d_v each), dX = dZ W1^T, dW1 = X^T dZ
+    (2 T D W each).  A recompute of the pre-activation X W1 is not counted."""
+    hv = num_heads * d_v
+    width = num_heads * (2 * d_v + 2 * d_qk)
+    return 2.0 * T * (2 * d_model * hv + 2 * d_model * width)
+

@@ -410,6 +410,9 @@ def test_cost_table_reproduces_published_figures():
     assert round((attn + uvqk + outp) / 1e12, 2) == 323.26
     # backward is 2.5x forward: the "factor 3.5" for fwd+bwd
     assert flops.attn_bwd_flops(1, h, d, d) == 2.5 * flops.attn_fwd_flops(1, h, d, d)
+    # projections: the table's rows count forward + backward as 3x the forward GEMM
+    f1, f2 = flops.f1_flops(B * S, D, h, d, d), flops.f2_flops(B * S, D, h, d)
+    assert flops.layer_bwd_gemm_flops(B * S, D, h, d, d) == 2 * (f1 + f2)
 
 
 def test_pair_counter_by_brute_force():
