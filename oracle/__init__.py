@@ -55,6 +55,10 @@ def _load():
             lib.oracle_pos_index.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
             lib.oracle_visible.restype = ctypes.c_int
             lib.oracle_visible.argtypes = [ctypes.c_int64] * 4
+            lib.oracle_visible_sl.restype = ctypes.c_int
+            lib.oracle_visible_sl.argtypes = [ctypes.c_int64] * 6
+            lib.oracle_set_windows.restype = None
+            lib.oracle_set_windows.argtypes = [ctypes.c_int64] * 2
             _lib = lib
     return _lib
 
@@ -103,6 +107,25 @@ def visible(i: int, j: int, L: int, n_t: int) -> bool:
     return bool(_load().oracle_visible(int(i), int(j), int(L), int(n_t)))
 
 
+def visible_sl(i: int, j: int, L: int, n_t: int, local_window: int, global_window: int) -> bool:
+    """visible() restricted to the semi-local windows (local_window <= 0: no restriction)."""
+    return bool(_load().oracle_visible_sl(int(i), int(j), int(L), int(n_t), int(local_window),
+                                          int(global_window)))
+
+
+class _Windows:
+    """Semi-local windows applied by the oracle's attention for the duration of one call."""
+
+    def __init__(self, local_window=0, global_window=0):
+        self.w = (int(local_window), int(global_window))
+
+    def __enter__(self):
+        _load().oracle_set_windows(ctypes.c_int64(self.w[0]), ctypes.c_int64(self.w[1]))
+
+    def __exit__(self, *exc):
+        _load().oracle_set_windows(ctypes.c_int64(0), ctypes.c_int64(0))
+
+
 class _Attn:
     """Marshalled common attention arguments."""
 
@@ -132,27 +155,29 @@ class _Attn:
 
 
 def attn_fwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
-             inv_n, threads=None):
+             inv_n, threads=None, local_window=0, global_window=0):
     """O[T, H, dv] of the jagged SiLU attention (float64)."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     out = np.zeros((a.T, a.H, a.dv), dtype=np.float64)
-    _load().oracle_attn_fwd(*a.head(), _p(out, _f64p), ctypes.c_int(threads or default_threads()))
+    with _Windows(local_window, global_window):
+        _load().oracle_attn_fwd(*a.head(), _p(out, _f64p), ctypes.c_int(threads or default_threads()))
     return out
 
 
 def attn_fwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
-                  pos_hi, inv_n, rows, threads=None):
+                  pos_hi, inv_n, rows, threads=None, local_window=0, global_window=0):
     """O rows for the given global token indices: [n, H, dv]."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     rows = _i64(rows)
     out = np.zeros((len(rows), a.H, a.dv), dtype=np.float64)
-    _load().oracle_attn_fwd_rows(*a.head(), ctypes.c_int64(len(rows)), _p(rows, _i64p),
-                                 _p(out, _f64p), ctypes.c_int(threads or default_threads()))
+    with _Windows(local_window, global_window):
+        _load().oracle_attn_fwd_rows(*a.head(), ctypes.c_int64(len(rows)), _p(rows, _i64p),
+                                     _p(out, _f64p), ctypes.c_int(threads or default_threads()))
     return out
 
 
 def attn_bwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
-             inv_n, dout, threads=None):
+             inv_n, dout, threads=None, local_window=0, global_window=0):
     """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     do = _f64(dout)
@@ -161,13 +186,14 @@ def attn_bwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, p
     dv = np.zeros_like(a.v)
     drp = np.zeros_like(a.rp)
     drt = np.zeros_like(a.rt)
-    _load().oracle_attn_bwd(*a.head(), _p(do, _f64p), _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p),
-                            _p(drp, _f64p), _p(drt, _f64p), ctypes.c_int(threads or default_threads()))
+    with _Windows(local_window, global_window):
+        _load().oracle_attn_bwd(*a.head(), _p(do, _f64p), _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p),
+                                _p(drp, _f64p), _p(drt, _f64p), ctypes.c_int(threads or default_threads()))
     return dq, dk, dv, drp, drt
 
 
 def attn_bwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
-                  pos_hi, inv_n, dout, q_rows, k_rows, threads=None):
+                  pos_hi, inv_n, dout, q_rows, k_rows, threads=None, local_window=0, global_window=0):
     """dq for query rows `q_rows`; dk, dv for key rows `k_rows`."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     do = _f64(dout)
@@ -175,10 +201,11 @@ def attn_bwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_ti
     dq = np.zeros((len(qr), a.H, a.dqk))
     dk = np.zeros((len(kr), a.H, a.dqk))
     dv = np.zeros((len(kr), a.H, a.dv))
-    _load().oracle_attn_bwd_rows(*a.head(), _p(do, _f64p), ctypes.c_int64(len(qr)), _p(qr, _i64p),
-                                 _p(dq, _f64p), ctypes.c_int64(len(kr)), _p(kr, _i64p),
-                                 _p(dk, _f64p), _p(dv, _f64p),
-                                 ctypes.c_int(threads or default_threads()))
+    with _Windows(local_window, global_window):
+        _load().oracle_attn_bwd_rows(*a.head(), _p(do, _f64p), ctypes.c_int64(len(qr)), _p(qr, _i64p),
+                                     _p(dq, _f64p), ctypes.c_int64(len(kr)), _p(kr, _i64p),
+                                     _p(dk, _f64p), _p(dv, _f64p),
+                                     ctypes.c_int(threads or default_threads()))
     return dq, dk, dv
 
 

@@ -94,6 +94,31 @@ int oracle_visible(int64_t i, int64_t j, int64_t L, int64_t n_t)
     return j < hist || j == i;
 }
 
+/*
+ * Semi-local attention (the ULTRA-HSTU review in the pages: attention over a
+ * local and a global window instead of the full causal mask).  With
+ * local > 0, a pair the rule above keeps survives iff the query is less than
+ * `local` positions after the key, or the key is one of the first `global`
+ * tokens of the sequence.  local <= 0 keeps the full mask.
+ */
+int oracle_visible_sl(int64_t i, int64_t j, int64_t L, int64_t n_t, int64_t local, int64_t global)
+{
+    if (!oracle_visible(i, j, L, n_t))
+        return 0;
+    if (local <= 0)
+        return 1;
+    return token_pos(i, L, n_t) - token_pos(j, L, n_t) < local || j < global;
+}
+
+/* windows applied by the attention functions below (set per call by the caller) */
+static int64_t g_local_window = 0, g_global_window = 0;
+
+void oracle_set_windows(int64_t local, int64_t global)
+{
+    g_local_window = local;
+    g_global_window = global;
+}
+
 static double silu(double x) { return x / (1.0 + exp(-x)); }
 
 static double silu_grad(double x)
@@ -112,6 +137,7 @@ typedef struct {
     const double *rab_time;
     int num_buckets;
     double inv_n;
+    int64_t local_window, global_window;
 } attn_args;
 
 static int64_t seq_targets(const attn_args *a, int b)
@@ -140,7 +166,7 @@ static void fwd_row(const attn_args *a, const double *q, const double *k, const 
     for (int c = 0; c < a->d_v; c++)
         o_row[c] = 0.0;
     for (int64_t j = 0; j < L; j++) {
-        if (!oracle_visible(i, j, L, n_t))
+        if (!oracle_visible_sl(i, j, L, n_t, a->local_window, a->global_window))
             continue;
         double p = silu(score(a, q, k, s0, L, n_t, h, i, j)) * a->inv_n;
         const double *vj = v + ((s0 + j) * a->num_heads + h) * a->d_v;
@@ -167,6 +193,8 @@ static void fill_args(attn_args *a, int num_seqs, const int64_t *seq_offsets,
     a->rab_time = rab_time;
     a->num_buckets = num_buckets;
     a->inv_n = inv_n;
+    a->local_window = g_local_window;
+    a->global_window = g_global_window;
 }
 
 static void set_threads(int num_threads)
@@ -270,7 +298,7 @@ void oracle_attn_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *nu
             const double *doi = dout + ((s0 + i) * num_heads + h) * d_v;
             double *dqi = dq + ((s0 + i) * num_heads + h) * d_qk;
             for (int64_t j = 0; j < L; j++) {
-                if (!oracle_visible(i, j, L, n_t))
+                if (!oracle_visible_sl(i, j, L, n_t, a.local_window, a.global_window))
                     continue;
                 const double *kj = k + ((s0 + j) * num_heads + h) * d_qk;
                 const double *vj = v + ((s0 + j) * num_heads + h) * d_v;
@@ -338,7 +366,7 @@ void oracle_attn_bwd_rows(int num_seqs, const int64_t *seq_offsets, const int32_
             for (int c = 0; c < d_qk; c++)
                 out[c] = 0.0;
             for (int64_t j = 0; j < L; j++) {
-                if (!oracle_visible(i, j, L, n_t))
+                if (!oracle_visible_sl(i, j, L, n_t, a.local_window, a.global_window))
                     continue;
                 const double *kj = k + ((s0 + j) * num_heads + h) * d_qk;
                 const double *vj = v + ((s0 + j) * num_heads + h) * d_v;
@@ -364,7 +392,7 @@ void oracle_attn_bwd_rows(int num_seqs, const int64_t *seq_offsets, const int32_
             for (int c = 0; c < d_v; c++)
                 ovv[c] = 0.0;
             for (int64_t i = 0; i < L; i++) {
-                if (!oracle_visible(i, j, L, n_t))
+                if (!oracle_visible_sl(i, j, L, n_t, a.local_window, a.global_window))
                     continue;
                 const double *qi = q + ((s0 + i) * num_heads + h) * d_qk;
                 const double *doi = dout + ((s0 + i) * num_heads + h) * d_v;

@@ -567,3 +567,96 @@ def test_layer_bwd_central_finite_differences():
             plus[k], minus[k] = fp.reshape(prm[k].shape), fm.reshape(prm[k].shape)
             fd = (loss(plus) - loss(minus)) / (2 * h)
             assert abs(fd - ours[name].reshape(-1)[e]) < 1e-6 * max(1.0, abs(fd)), (name, e, fd)
+
+
+# ---- 9. semi-local windows ----------------------------------------------------
+
+def _window_mask(L, n_t, local, glob):
+    """Independent restatement: causal/candidate rule AND (p_i - p_j < local or j < glob)."""
+    hist = L - n_t
+    idx = np.arange(L)
+    p = np.where(idx < hist, idx, hist)
+    I, J = idx[:, None], idx[None, :]
+    base = np.where(I < hist, J <= I, (J < hist) | (J == I))
+    if local <= 0:
+        return base
+    return base & (((p[:, None] - p[None, :]) < local) | (J < glob))
+
+
+def _dense_sl(c, local, glob, dout=None):
+    """Dense torch float64 forward (and, with dout, autograd backward) under the windows."""
+    off, nt = c["seq_offsets"], c["num_targets"]
+    lo, hi = c["pos_lo"], c["pos_hi"]
+    t = {k: torch.tensor(c[k], requires_grad=True) for k in ("q", "k", "v", "rab_pos", "rab_time")}
+    outs = []
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        hist = L - n_t
+        idx = np.arange(L)
+        p = np.where(idx < hist, idx, hist)
+        rel = torch.tensor(np.clip(p[:, None] - p[None, :], lo, hi) - lo)
+        ts = c["timestamps"][s0:s1]
+        nbk = len(c["rab_time"])
+        bkt = torch.tensor([[min(nbk - 1, (int(max(ts[i] - ts[j], 0)) + 1).bit_length() - 1)
+                             for j in range(L)] for i in range(L)])
+        vis = torch.tensor(_window_mask(L, n_t, local, glob), dtype=torch.float64)
+        S = torch.einsum("ihc,jhc->hij", t["q"][s0:s1], t["k"][s0:s1]) + (t["rab_pos"][rel] + t["rab_time"][bkt])[None]
+        P = torch.nn.functional.silu(S) * c["inv_n"] * vis[None]
+        outs.append(torch.einsum("hij,jhc->ihc", P, t["v"][s0:s1]))
+    o = torch.cat(outs)
+    if dout is None:
+        return o.detach().numpy()
+    (o * torch.tensor(dout)).sum().backward()
+    return [t[k].grad.numpy() for k in ("q", "k", "v", "rab_pos", "rab_time")]
+
+
+def test_visible_sl_exhaustive():
+    for L in range(0, 9):
+        for n_t in range(0, L + 1):
+            for local in range(0, L + 2):
+                for glob in range(0, L + 1):
+                    m = _window_mask(L, n_t, local, glob)
+                    for i in range(L):
+                        for j in range(L):
+                            assert oracle.visible_sl(i, j, L, n_t, local, glob) == bool(m[i, j])
+
+
+@pytest.mark.parametrize("local,glob", [(3, 0), (2, 2), (5, 1), (1, 3)])
+def test_semi_local_matches_dense(local, glob):
+    rng = np.random.default_rng(500 + 7 * local + glob)
+    c = rand_case(rng, [7, 1, 0, 9], nt=[2, 0, 0, 3])
+    args = (c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"], c["rab_pos"],
+            c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+    o = oracle.attn_fwd(*args, local_window=local, global_window=glob)
+    np.testing.assert_allclose(o, _dense_sl(c, local, glob), rtol=0, atol=1e-12)
+    dout = rng.standard_normal(c["v"].shape)
+    ours = oracle.attn_bwd(*args, dout, local_window=local, global_window=glob)
+    for a, b in zip(ours, _dense_sl(c, local, glob, dout)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-11)
+
+
+def test_semi_local_limits():
+    rng = np.random.default_rng(520)
+    c = rand_case(rng, [6, 4], nt=[1, 0])
+    args = (c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"], c["rab_pos"],
+            c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+    full = oracle.attn_fwd(*args)
+    # a local window covering every distance, or a global window covering every key, is the full mask
+    np.testing.assert_array_equal(oracle.attn_fwd(*args, local_window=100, global_window=0), full)
+    np.testing.assert_array_equal(oracle.attn_fwd(*args, local_window=1, global_window=100), full)
+    # local 1, no global keys: only the diagonal, O_i = SiLU(s_ii) / N v_i
+    o = oracle.attn_fwd(*args, local_window=1, global_window=0)
+    off, nt = c["seq_offsets"], c["num_targets"]
+    for b in range(2):
+        s0, L = int(off[b]), int(off[b + 1] - off[b])
+        for i in range(L):
+            idx = int(np.clip(0, c["pos_lo"], c["pos_hi"]) - c["pos_lo"])
+            s = np.einsum("hc,hc->h", c["q"][s0 + i], c["k"][s0 + i]) + c["rab_pos"][idx] + c["rab_time"][0]
+            expect = (s / (1 + np.exp(-s)) * c["inv_n"])[:, None] * c["v"][s0 + i]
+            np.testing.assert_allclose(o[s0 + i], expect, rtol=0, atol=1e-12)
+    # the call leaves no windows behind
+    np.testing.assert_array_equal(oracle.attn_fwd(*args), full)
