@@ -40,6 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels of ours launched per step: fwd call (schedule, attention) and bwd call
 # (schedule, attention backward, dq conversion)
 LAUNCHES_PER_STEP = 5
+# semi-local windows of the secondary measurement (the pages give no sizes)
+SEMI_LOCAL = (1024, 256)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention-backward launch on
 # this workload, from a one-pass ncu capture of
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd_tc -c 1
@@ -298,7 +300,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from hstu_sequential_transduction_b200 import ops, parallel, workloads
+    from hstu_sequential_transduction_b200 import flops, ops, parallel, workloads
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -458,6 +460,38 @@ def run_ours(args):
 
     layer = None if args.no_layer_stack else layer_stack_timing(dev, stream)
 
+    # secondary: the same batch under semi-local windows (local 1024, global 256)
+    semi = None
+    if not args.no_layer_stack:
+        win = dict(local_window=SEMI_LOCAL[0], global_window=SEMI_LOCAL[1])
+        sl_pairs = flops.attn_pairs(inp.lengths, None, *SEMI_LOCAL)
+        sl_f = flops.attn_fwd_flops(sl_pairs, q.shape[1], q.shape[2], v.shape[2])
+        sl_b = flops.attn_bwd_flops(sl_pairs, q.shape[1], q.shape[2], v.shape[2])
+
+        def sl_step():
+            ops.hstu_attn_fwd(q, k, v, off, ts, None, rp, rt, out=out, workspace=ws_f, stream=stream, **kw, **win)
+            ev_mid.record(stream)
+            ops.hstu_attn_bwd(q, k, v, off, ts, None, rp, rt, dout, grads=grads, workspace=ws_b, stream=stream,
+                              **kw, **win)
+
+        ev_mid = torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            sl_step()
+        torch.cuda.synchronize()
+        f_ms = b_ms = 0.0
+        n_sl = 5
+        for _ in range(n_sl):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            sl_step()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            f_ms += a0.elapsed_time(ev_mid) / n_sl
+            b_ms += ev_mid.elapsed_time(a1) / n_sl
+        semi = {"local_window": SEMI_LOCAL[0], "global_window": SEMI_LOCAL[1], "visible_pairs_per_head": sl_pairs,
+                "fwd_ms": f_ms, "bwd_ms": b_ms, "tflops": (sl_f + sl_b) / ((f_ms + b_ms) * 1e-3) / 1e12,
+                "speedup_vs_full_mask": ms / (f_ms + b_ms)}
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
@@ -487,6 +521,8 @@ def run_ours(args):
         }
         if layer is not None:
             line["layer_stack"] = layer
+        if semi is not None:
+            line["semi_local"] = semi
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(line), flush=True)

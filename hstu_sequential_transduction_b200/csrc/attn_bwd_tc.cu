@@ -212,6 +212,8 @@ __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float 
     }
 }
 
+// SL: semi-local windows in use (otherwise every window test compiles away)
+template <bool SL>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
@@ -230,7 +232,16 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     const int L = (int)(p.seq_offsets[it.x + 1] - s0);
     const int hist = L - (p.num_targets ? p.num_targets[it.x] : 0);
     const int j0 = it.y * KB;
-    const int q_end = j0 < hist ? L : min(j0 + KB, L);
+    const int lw = SL ? p.lw : 0, gw = SL ? p.gw : 0;
+    int q_end = j0 < hist ? L : min(j0 + KB, L);
+    // Semi-local windows: without global keys in the tile, history queries past
+    // the local window of its last key see nothing, and candidates (position
+    // hist) see it only if hist is within the window of that key
+    if (lw > 0 && j0 >= gw && j0 < hist) {
+        const int last = min(j0 + KB, hist) - 1;
+        if (hist - last >= lw)
+            q_end = min(q_end, min(hist, last + lw));
+    }
     const int nq = (q_end - j0 + QB - 1) / QB;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -460,7 +471,10 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 prefetch(i + 1);
 
             const int q_last = min(iw0 + NC, L) - 1;  // last valid query of the block
-            const bool full_w = (iw0 >= jw0 + 31) && (jw0 + 32 <= hist) && (iw0 + NC <= L) && (iw0 + NC <= hist);
+            // every pair of the block inside the local window, or every key global
+            const bool band_w = lw <= 0 || iw0 + NC - 1 - jw0 < lw || jw0 + 32 <= gw;
+            const bool full_w = (iw0 >= jw0 + 31) && (jw0 + 32 <= hist) && (iw0 + NC <= L) && (iw0 + NC <= hist) &&
+                                band_w;
             const int dmin_w = dw - 31, dmax_w = dw + NC - 1;
             int cls = CLS_GENERAL;
             if (!rows_bad && !cols_bad) {
@@ -512,9 +526,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         o = mode == BK_ONE   ? bwd_row<false, true, BK_ONE>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
                             : mode == BK_TWO ? bwd_row<false, true, BK_TWO>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk)
                                              : bwd_row<false, true, BK_ANY>(sv, dv, TIw, tjf, Eb, wrow, 0.f, 0, NC, pk);
-                    else
+                    else {
+                        // this key row sees queries [j, L), cut at j + local_window
+                        // unless the key is global
+                        const int c_hi = (lw > 0 && j >= gw) ? min(NC, min(L, j + lw) - iw0) : min(NC, L - iw0);
                         o = bwd_row<true, true, BK_ANY>(sv, dv, TIw, tjf, Eb, wrow, 0.f, j - iw0,
-                                                       krow_ok ? min(NC, L - iw0) : 0, pk);
+                                                       krow_ok ? c_hi : 0, pk);
+                    }
                     float accP, accN;
                     warp_diagonals(dv, lane, accP, accN);
                     if (accP != 0.f)
@@ -548,7 +566,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         const int ii = iw0 + c + e;
                         pv[e] = 0.f;
                         dsv[e] = 0.f;
-                        if (krow_ok && ii < L && visible(ii, j, hist)) {
+                        if (krow_ok && ii < L && visible_w(ii, j, hist, lw, gw)) {
                             const int idx = pos_index(token_pos(ii, hist), pj, lo, hi);
                             const int b = time_bucket(p.timestamps[s0 + ii], tj, p.nb);
                             const float hh = 0.5f * (sv[c + e] + p.rab_pos[idx] + p.rab_time[b]);
@@ -666,10 +684,11 @@ cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t
     if (e != cudaSuccess)
         return e;
     const size_t bytes = BL::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    auto kern = p.lw > 0 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
-    attn_bwd_tc_kernel<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq);
+    kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq);
     return cudaGetLastError();
 }
 

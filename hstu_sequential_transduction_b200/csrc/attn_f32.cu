@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(TR) attn_fwd_f32_kernel(const AttnParams p)
         __syncthreads();
         for (int jj = 0; jj < TR; jj++) {
             const int j = j0 + jj;
-            if (!row_ok || j >= s.L || !visible(i, j, s.hist))
+            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw))
                 continue;
             float x = 0.f;
 #pragma unroll
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(TR) attn_bwd_f32_kernel(const AttnParams p)
         __syncthreads();
         for (int jj = 0; jj < TR; jj++) {
             const int j = j0 + jj;
-            if (!row_ok || j >= s.L || !visible(i, j, s.hist))
+            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw))
                 continue;
             float x = 0.f, dp = 0.f;
 #pragma unroll

@@ -77,14 +77,14 @@ __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float
 
 // P for the 64 key columns one thread owns (one query row), packed to bf16.
 // wr[-c]: positional bias / 2 of column c; tj[c]: rebased key stamp.
-// MASK: columns c >= c_lim are not visible.  TWO: the row's columns fall in
+// MASK: only columns c_lo <= c < c_lim are visible.  TWO: the row's columns fall in
 // at most two time buckets (hi for columns whose difference reaches `thr`).
 // MODE: 0 time bucket looked up per column, 1 one bucket for the whole row
 // (e_hi), 2 two buckets split at thr.  CONSTB: the positional index is clamped
 // for every column, so the positional bias is wr[0].
 template <bool MASK, int MODE, bool CONSTB>
 __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float *tj, float ti1,
-                                        const float *E, float e_hi, float e_lo, float thr, int c_lim,
+                                        const float *E, float e_hi, float e_lo, float thr, int c_lo, int c_lim,
                                         uint32_t *pk)
 {
     const float bconst = CONSTB ? wr[0] + (MODE == 1 ? e_hi : 0.f) : 0.f;
@@ -131,7 +131,7 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
                 const int cc = hb + c + e;
                 float v = fmaf(sv[cc], th[c + e], sv[cc]);
                 if (MASK)
-                    v = cc < c_lim ? v : 0.f;
+                    v = (cc >= c_lo && cc < c_lim) ? v : 0.f;
                 pv[e] = v;
             }
             pk[(hb + c) >> 1] = pack_bf16(pv[0], pv[1]);
@@ -139,7 +139,8 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
     }
 }
 
-template <int D>
+// SL: semi-local windows in use (otherwise every window test compiles away)
+template <int D, bool SL>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv)
@@ -159,9 +160,19 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
     const int L = (int)(p.seq_offsets[it.x + 1] - s0);
     const int hist = L - (p.num_targets ? p.num_targets[it.x] : 0);
     const int i0 = qt * TBM;
+    const int lw = SL ? p.lw : 0, gw = SL ? p.gw : 0;
     const int nh = (hist + TBN - 1) / TBN;
-    const int nfull = min(qt + 1, nh);
-    const int ntiles = nfull + (qt >= nh ? 1 : 0);
+    const int nfull = min(qt + 1, nh);  // history key tiles up to this query tile
+    // Semi-local windows: of those, the tiles holding global keys [0, gt) and the
+    // tiles reaching into the local window of the tile's first row [lt0, nfull).
+    int gt = nfull, lt0 = nfull;
+    if (lw > 0) {
+        gt = min(nfull, (gw + TBN - 1) / TBN);
+        lt0 = min(nfull, max(gt, max(0, token_pos(i0, hist) - lw + 1) / TBN));
+    }
+    const int nhist = gt + (nfull - lt0);
+    const int ntiles = nhist + (qt >= nh ? 1 : 0);  // + the candidates' own tile
+    auto tile_of = [&](int t) { return t >= nhist ? qt : (t < gt ? t : t - gt + lt0); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto bar = [&](int i) { return base + LY::BAR + 8u * i; };
@@ -203,7 +214,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 tma_load_2d(base + LY::Q + r * kRegion, &tq, h * D + 64 * r, (int)(s0 + i0), bar(Q_FULL));
             for (int t = 0; t < ntiles; t++) {
                 const int s = t & 1;
-                const int j0 = (t < nfull ? t : qt) * TBN;
+                const int j0 = tile_of(t) * TBN;
                 if (t >= 2 && !mbar_wait(bar(K_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, p.hdr))
                     break;
                 mbar_expect_tx(bar(K_FULL + s), LY::TILE);
@@ -299,7 +310,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         float w0 = 0.f, w1 = 0.f, w2 = 0.f;
         int64_t ta = tb, tc = tb;  // stamps of key columns 2 lane, 2 lane + 1
         auto prep = [&](int t) {
-            const int jw = (t < nfull ? t : qt) * TBN + 64 * g;
+            const int jw = tile_of(t) * TBN + 64 * g;
             const int dbase = pw - jw - 63;
             w0 = p.rab_pos[clamp_idx(dbase + lane)];
             w1 = p.rab_pos[clamp_idx(dbase + lane + 32)];
@@ -316,7 +327,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         bool ok = true;
         for (int t = 0; t < ntiles; t++) {
             const int s = t & 1;
-            const int j0 = (t < nfull ? t : qt) * TBN;
+            const int j0 = tile_of(t) * TBN;
             const int j = j0 + 64 * g + 2 * lane;
             const int64_t ta_next = __shfl_down_sync(full_mask, ta, 1);
             const bool kbad = (j < L && (ta - tb >= lim || ta - tb <= -lim)) ||
@@ -330,7 +341,11 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             Ww[lane + 32] = 0.5f * w1;
             Ww[lane + 64] = 0.5f * w2;
             __syncwarp();
-            const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0);
+            // every pair of the tile inside the local window (or every key global)?
+            const bool band_all = lw <= 0 || token_pos(min(i0 + TBM, L) - 1, hist) - j0 < lw ||
+                                  j0 + TBN <= gw;
+            const bool band_cut = !band_all;
+            const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0) && band_all;
             if (t + 1 < ntiles)
                 prep(t + 1);
 
@@ -345,7 +360,8 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             uint32_t pk[32];
             // diagonal / ragged tiles without candidate rows keep the fast math
             // with a per-column mask (positions equal indices there)
-            const bool masked_fast = !full && !slow_time && min(i0 + TBM, L) <= hist;
+            // one interval of visible columns per row: no band cut inside global keys
+            const bool masked_fast = !full && !slow_time && min(i0 + TBM, L) <= hist && (!band_cut || j0 >= gw);
             if ((full && !slow_time) || masked_fast) {
                 const float *wr = Ww + (pi - pw) + 63;  // wr[-c]: key column c of this row
                 const float *tj = TJw;
@@ -365,21 +381,23 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     const float thr = __uint_as_float(bh << 23);
                     if (one) {
                         if (cst)
-                            fwd_row<false, 1, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                            fwd_row<false, 1, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
                         else
-                            fwd_row<false, 1, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                            fwd_row<false, 1, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
                     } else if (two) {
                         if (cst)
-                            fwd_row<false, 2, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                            fwd_row<false, 2, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
                         else
-                            fwd_row<false, 2, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 64, pk);
+                            fwd_row<false, 2, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
                     } else {
-                        fwd_row<false, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 64, pk);
+                        fwd_row<false, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 0, 64, pk);
                     }
                 } else {
-                    // visible: key j <= i and j < L
+                    // visible: key j <= i, j < L and, when the tile crosses the local
+                    // window's edge (no global keys here), j > i - local_window
                     const int c_lim = min(i - j0 - 64 * g + 1, L - j0 - 64 * g);
-                    fwd_row<true, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lim, pk);
+                    const int c_lo = band_cut ? i - lw + 1 - (j0 + 64 * g) : 0;
+                    fwd_row<true, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lo, c_lim, pk);
                 }
             } else {
 #pragma unroll
@@ -389,7 +407,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     for (int e = 0; e < 2; e++) {
                         const int j = j0 + 64 * g + c + e;
                         pv[e] = 0.f;
-                        if (row_ok && j < L && visible(i, j, hist)) {
+                        if (row_ok && j < L && visible_w(i, j, hist, lw, gw)) {
                             const float bp = p.rab_pos[pos_index(pi, token_pos(j, hist), p.pos_lo, p.pos_hi)];
                             const float bt = p.rab_time[time_bucket(ti, p.timestamps[s0 + j], p.nb)];
                             const float hh = 0.5f * (sv[c + e] + bp + bt);
@@ -452,7 +470,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-template <int D>
+template <int D, bool SL>
 cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
     CUtensorMap maps[3];
@@ -466,10 +484,10 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     if (e != cudaSuccess)
         return e;
     const size_t bytes = FwdLayout<D>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
-    attn_fwd_tc_kernel<D><<<(unsigned)grid_items * p.H, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
+    attn_fwd_tc_kernel<D, SL><<<(unsigned)grid_items * p.H, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
     return cudaGetLastError();
 }
 
@@ -510,8 +528,10 @@ cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t
     if (grid_items <= 0)
         return cudaSuccess;
     switch (p.dqk) {
-    case 64: return fwd_tc_launch<64>(p, grid_items, stream);
-    case 128: return fwd_tc_launch<128>(p, grid_items, stream);
+    case 64: return p.lw > 0 ? fwd_tc_launch<64, true>(p, grid_items, stream)
+                             : fwd_tc_launch<64, false>(p, grid_items, stream);
+    case 128: return p.lw > 0 ? fwd_tc_launch<128, true>(p, grid_items, stream)
+                              : fwd_tc_launch<128, false>(p, grid_items, stream);
     default: return cudaErrorInvalidValue;
     }
 }

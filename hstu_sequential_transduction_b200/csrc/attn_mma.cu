@@ -203,7 +203,7 @@ attn_fwd_mma_kernel(const AttnParams p)
                 const int a = e >> 1;
                 const int c = n * 8 + 2 * t4 + (e & 1);
                 const int j = j0 + c;
-                const bool vis = ri[a] < s.L && j < s.L && visible(ri[a], j, s.hist);
+                const bool vis = ri[a] < s.L && j < s.L && visible_w(ri[a], j, s.hist, p.lw, p.gw);
                 float x = sacc[n][e] + tpos[pos_index(pi[a], token_pos(j, s.hist), p.pos_lo, p.pos_hi)] +
                           ttime[time_bucket(ti[a], cT[c], p.nb)];
                 sacc[n][e] = vis ? silu_fast(x) * p.inv_n : 0.f;
@@ -401,7 +401,7 @@ attn_bwd_mma_kernel(const AttnParams p)
                 const int a = e >> 1;
                 const int c = n * 8 + 2 * t4 + (e & 1);
                 const int i = i0 + c;
-                const bool vis = i < s.L && rj[a] < s.L && visible(i, rj[a], s.hist);
+                const bool vis = i < s.L && rj[a] < s.L && visible_w(i, rj[a], s.hist, p.lw, p.gw);
                 const int pidx = pos_index(token_pos(i, s.hist), pj[a], p.pos_lo, p.pos_hi);
                 const int bkt = time_bucket(cT[c], tj[a], p.nb);
                 float x = sacc[n][e] + tpos[pidx] + ttime[bkt];

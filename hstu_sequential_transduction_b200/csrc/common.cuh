@@ -44,6 +44,7 @@ struct AttnParams {
     int64_t T;
     float inv_n;
     int pos_lo, pos_hi, nb;
+    int lw, gw;  // semi-local windows (lw = 0: full mask)
     const int2 *items;
     WsHeader *hdr;
     // backward only
@@ -77,6 +78,14 @@ __device__ __forceinline__ int token_pos(int i, int hist) { return i < hist ? i 
 __device__ __forceinline__ bool visible(int i, int j, int hist)
 {
     return i < hist ? (j <= i) : (j < hist || j == i);
+}
+
+// visible() restricted to the semi-local windows: with lw > 0 the query must
+// be fewer than lw positions after the key, or the key among the first gw
+// tokens of the sequence.
+__device__ __forceinline__ bool visible_w(int i, int j, int hist, int lw, int gw)
+{
+    return visible(i, j, hist) && (lw <= 0 || token_pos(i, hist) - token_pos(j, hist) < lw || j < gw);
 }
 
 // SiLU on the fp32 score.  The fast form uses the hardware exponential.

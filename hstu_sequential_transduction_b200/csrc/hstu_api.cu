@@ -20,7 +20,8 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
     if (!d)
         return HSTU_ERR_INVALID_ARG;
     if (d->num_seqs < 0 || d->max_seq_len < 0 || d->total_tokens < 0 || d->num_heads < 1 ||
-        d->num_time_buckets < 1 || d->pos_hi < d->pos_lo || !std::isfinite(d->inv_n))
+        d->num_time_buckets < 1 || d->pos_hi < d->pos_lo || !std::isfinite(d->inv_n) ||
+        d->local_window < 0 || d->global_window < 0)
         return HSTU_ERR_INVALID_ARG;
     if (d->dtype != HSTU_F32 && d->dtype != HSTU_BF16)
         return HSTU_ERR_INVALID_ARG;
@@ -91,6 +92,8 @@ AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_
     p.pos_lo = d->pos_lo;
     p.pos_hi = d->pos_hi;
     p.nb = d->num_time_buckets;
+    p.lw = d->local_window;
+    p.gw = d->global_window;
     p.hdr = static_cast<WsHeader *>(ws);
     p.items = reinterpret_cast<const int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
     return p;

@@ -12,21 +12,31 @@ from __future__ import annotations
 import numpy as np
 
 
-def attn_pairs_per_seq(L: int, n_t: int = 0) -> int:
+def attn_pairs_per_seq(L: int, n_t: int = 0, local_window: int = 0, global_window: int = 0) -> int:
     """Visible (query, key) pairs of one sequence: history rows see j <= i,
-    each candidate row sees the whole history and itself."""
-    L, n_t = int(L), int(n_t)
+    each candidate row sees the whole history and itself.  With local_window
+    w > 0 (semi-local attention) a pair also needs p_i - p_j < w or j < g, the
+    global window: history row i keeps min(i + 1, w) local keys plus the global
+    keys before them, max(0, min(g, i + 1 - w)); a candidate (position hist)
+    keeps min(hist, w - 1) local history keys, the global ones before them,
+    and itself."""
+    L, n_t, w, g = int(L), int(n_t), int(local_window), int(global_window)
     hist = L - n_t
-    return hist * (hist + 1) // 2 + n_t * (hist + 1)
+    if w <= 0:
+        return hist * (hist + 1) // 2 + n_t * (hist + 1)
+    i = np.arange(hist, dtype=np.int64)
+    rows = np.minimum(i + 1, w) + np.maximum(0, np.minimum(g, i + 1 - w))
+    cand = min(hist, w - 1) + max(0, min(g, hist - w + 1)) + 1
+    return int(rows.sum()) + n_t * cand
 
 
-def attn_pairs(lengths, num_targets=None) -> int:
+def attn_pairs(lengths, num_targets=None, local_window: int = 0, global_window: int = 0) -> int:
     lengths = np.asarray(lengths, dtype=np.int64)
     if num_targets is None:
         nts = np.zeros_like(lengths)
     else:
         nts = np.asarray(num_targets, dtype=np.int64)
-    return int(sum(attn_pairs_per_seq(L, n) for L, n in zip(lengths, nts)))
+    return int(sum(attn_pairs_per_seq(L, n, local_window, global_window) for L, n in zip(lengths, nts)))
 
 
 def attn_fwd_flops(pairs: float, num_heads: int, d_qk: int, d_v: int) -> float:

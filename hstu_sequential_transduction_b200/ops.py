@@ -39,7 +39,8 @@ class hstu_attn_desc(ctypes.Structure):
                 ("total_tokens", ctypes.c_int64), ("num_heads", ctypes.c_int32),
                 ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("inv_n", ctypes.c_float), ("pos_lo", ctypes.c_int32), ("pos_hi", ctypes.c_int32),
-                ("num_time_buckets", ctypes.c_int32), ("debug_checks", ctypes.c_int32)]
+                ("num_time_buckets", ctypes.c_int32), ("debug_checks", ctypes.c_int32),
+                ("local_window", ctypes.c_int32), ("global_window", ctypes.c_int32)]
 
 
 class hstu_layer_desc(ctypes.Structure):
@@ -110,10 +111,10 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
 
 
 def make_attn_desc(num_seqs, max_seq_len, total_tokens, num_heads, d_qk, d_v, dtype, inv_n,
-                   pos_lo, pos_hi, num_time_buckets) -> hstu_attn_desc:
+                   pos_lo, pos_hi, num_time_buckets, local_window=0, global_window=0) -> hstu_attn_desc:
     return hstu_attn_desc(int(num_seqs), int(max_seq_len), int(total_tokens), int(num_heads),
                           int(d_qk), int(d_v), int(dtype), float(inv_n), int(pos_lo), int(pos_hi),
-                          int(num_time_buckets), 0)
+                          int(num_time_buckets), 0, int(local_window), int(global_window))
 
 
 def hstu_status_string(status: int) -> str:
@@ -143,15 +144,18 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time):
+def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window=0,
+                    global_window=0):
     return make_attn_desc(seq_offsets.numel() - 1, max_seq_len, q.shape[0], q.shape[1], q.shape[2],
-                          v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, rab_time.numel())
+                          v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window,
+                          global_window)
 
 
 def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, *,
                   max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, out=None,
-                  workspace=None, stream=None):
-    """O = jagged SiLU attention; q, k [T, H, d_qk], v [T, H, d_v] on CUDA."""
+                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0):
+    """O = jagged SiLU attention; q, k [T, H, d_qk], v [T, H, d_v] on CUDA.
+    local_window > 0 applies the semi-local mask (see hstu_attn_desc)."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         _dev(t, name, q.dtype)
     _dev(seq_offsets, "seq_offsets", torch.int64)
@@ -159,7 +163,8 @@ def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
     _dev(num_targets, "num_targets", torch.int32)
     _dev(rab_pos, "rab_pos", torch.float32)
     _dev(rab_time, "rab_time", torch.float32)
-    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window,
+                           global_window)
     if out is None:
         out = torch.empty_like(v)
     _dev(out, "out", q.dtype)
@@ -187,14 +192,15 @@ def hstu_attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, num_targets, rab_pos
 
 def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, dout, *,
                   max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, grads=None,
-                  workspace=None, stream=None):
+                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0):
     """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
     for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
         _dev(t, name, q.dtype)
     _dev(seq_offsets, "seq_offsets", torch.int64)
     _dev(timestamps, "timestamps", torch.int64)
     _dev(num_targets, "num_targets", torch.int32)
-    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window,
+                           global_window)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
                  torch.empty_like(rab_pos), torch.empty_like(rab_time))

@@ -75,6 +75,13 @@ typedef struct {
     int32_t pos_lo, pos_hi;   /* rab_pos covers distances pos_lo..pos_hi */
     int32_t num_time_buckets; /* NB >= 1 */
     int32_t debug_checks;     /* reserved; device input checks always run */
+    /* Semi-local attention (the ULTRA-HSTU review's local + global windows):
+     * local_window > 0 keeps, of the pairs the causal/candidate rule keeps,
+     * those whose query is fewer than local_window positions after the key or
+     * whose key is among the first global_window tokens of its sequence.
+     * local_window = 0 keeps the full mask; both must be >= 0. */
+    int32_t local_window;
+    int32_t global_window;
 } hstu_attn_desc;
 
 typedef struct {

@@ -57,18 +57,18 @@ def dev_attn(inp, dev):
                 dout=to_dev(inp.dout, dev) if inp.dout is not None else None)
 
 
-def gpu_fwd(inp, dev):
+def gpu_fwd(inp, dev, **windows):
     d = dev_attn(inp, dev)
     out = ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"],
-                            d["num_targets"], d["rab_pos"], d["rab_time"], **attn_kwargs(inp))
+                            d["num_targets"], d["rab_pos"], d["rab_time"], **attn_kwargs(inp), **windows)
     torch.cuda.synchronize()
     return out
 
 
-def gpu_bwd(inp, dev):
+def gpu_bwd(inp, dev, **windows):
     d = dev_attn(inp, dev)
     g = ops.hstu_attn_bwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], d["num_targets"],
-                          d["rab_pos"], d["rab_time"], d["dout"], **attn_kwargs(inp))
+                          d["rab_pos"], d["rab_time"], d["dout"], **attn_kwargs(inp), **windows)
     torch.cuda.synchronize()
     return g
 

@@ -660,3 +660,12 @@ def test_semi_local_limits():
             np.testing.assert_allclose(o[s0 + i], expect, rtol=0, atol=1e-12)
     # the call leaves no windows behind
     np.testing.assert_array_equal(oracle.attn_fwd(*args), full)
+
+
+def test_semi_local_pair_counter_by_brute_force():
+    for L in range(0, 12):
+        for n_t in range(0, L + 1):
+            for w in range(0, L + 2):
+                for g in range(0, L + 1):
+                    brute = sum(oracle.visible_sl(i, j, L, n_t, w, g) for i in range(L) for j in range(L))
+                    assert flops.attn_pairs_per_seq(L, n_t, w, g) == brute, (L, n_t, w, g)
