@@ -10,8 +10,9 @@ Inputs in bf16 are widened exactly to float64 before the call.
 
 Pins (tests/test_oracle_pins.py): a hand-worked three-token example, a dense
 brute-force formulation, torch float64 autograd, central finite differences,
-causality / independence / linearity invariants, the exhaustive bucket check
-and the cost formulas of the DLRMv4 page's Table 7.
+causality / independence / linearity invariants, the exhaustive bucket check,
+the cost formulas of the DLRMv4 page's Table 7, and for the truncation gather
+a hand-worked batch and its equivalence with a local attention window.
 """
 
 from __future__ import annotations
@@ -283,3 +284,26 @@ def attn_inputs_fwd(inp, threads=None):
     """Oracle forward over a `workloads.AttnInputs`-like object."""
     return attn_fwd(inp.seq_offsets, inp.timestamps, inp.num_targets, inp.q, inp.k, inp.v,
                     inp.rab_pos, inp.rab_time, inp.pos_lo, inp.pos_hi, inp.inv_n, threads)
+
+
+def jagged_truncate(seq_offsets, num_targets, keep, rows):
+    """Attention truncation (the ULTRA-HSTU review in the pages): after the
+    first layers over whole histories, later layers run only over a segment
+    of each history, its most recent events.  Reading: a sequence keeps its
+    last min(hist, keep) history tokens and all of its candidates, in order;
+    `rows` is any per-token array (layer activations, timestamps).  Returns
+    (new seq_offsets, kept rows).  Plain per-sequence slicing."""
+    off = np.asarray(seq_offsets, dtype=np.int64)
+    B = len(off) - 1
+    nt = np.zeros(B, np.int64) if num_targets is None else np.asarray(num_targets, np.int64)
+    rows = np.asarray(rows)
+    new_off = [0]
+    pieces = []
+    for b in range(B):
+        start, end = int(off[b]), int(off[b + 1])
+        hist = end - start - int(nt[b])
+        first = start + hist - min(hist, int(keep))   # first kept history token
+        pieces.append(rows[first:end])
+        new_off.append(new_off[-1] + (end - first))
+    kept = np.concatenate(pieces) if pieces else rows[:0]
+    return np.asarray(new_off, dtype=np.int64), kept

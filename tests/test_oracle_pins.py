@@ -669,3 +669,63 @@ def test_semi_local_pair_counter_by_brute_force():
                 for g in range(0, L + 1):
                     brute = sum(oracle.visible_sl(i, j, L, n_t, w, g) for i in range(L) for j in range(L))
                     assert flops.attn_pairs_per_seq(L, n_t, w, g) == brute, (L, n_t, w, g)
+
+
+# ---- attention truncation (segment gather) -----------------------------------
+
+def test_truncate_hand_worked():
+    g = _parse_golden("truncate_hand.txt")
+    off = np.asarray(g["seq_offsets"], np.int64)
+    nt = np.asarray(g["num_targets"], np.int32)
+    rows = np.arange(11, dtype=np.float64)
+    for keep in (0, 1, 2):
+        new_off, kept = oracle.jagged_truncate(off, nt, keep, rows)
+        np.testing.assert_array_equal(new_off, g[f"keep{keep}_offsets"])
+        np.testing.assert_array_equal(kept, g[f"keep{keep}_rows"])
+
+
+def test_truncate_limits():
+    rng = np.random.default_rng(700)
+    lengths = np.array([0, 1, 5, 9, 3])
+    nt = np.array([0, 1, 2, 0, 3], np.int32)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    rows = rng.standard_normal((int(off[-1]), 3))
+    # a segment at least as long as every history keeps everything
+    new_off, kept = oracle.jagged_truncate(off, nt, 9, rows)
+    np.testing.assert_array_equal(new_off, off)
+    np.testing.assert_array_equal(kept, rows)
+    # each sequence keeps min(hist, keep) + n_t tokens, and its last ones
+    for keep in range(0, 10):
+        new_off, kept = oracle.jagged_truncate(off, nt, keep, rows)
+        np.testing.assert_array_equal(np.diff(new_off), np.minimum(lengths - nt, keep) + nt)
+        for b in range(len(lengths)):
+            n = int(new_off[b + 1] - new_off[b])
+            np.testing.assert_array_equal(kept[new_off[b]:new_off[b + 1]], rows[off[b + 1] - n:off[b + 1]])
+    # no candidate information: every token is history
+    new_off, _ = oracle.jagged_truncate(off, None, 2, rows)
+    np.testing.assert_array_equal(np.diff(new_off), np.minimum(lengths, 2))
+    # empty batch
+    new_off, kept = oracle.jagged_truncate(np.zeros(1, np.int64), None, 4, rows[:0])
+    assert new_off.tolist() == [0] and len(kept) == 0
+
+
+def test_truncated_candidates_see_a_local_window():
+    # A candidate of the truncated sequence attends to the `keep` most recent
+    # history tokens and itself; relative positions and time gaps are unchanged
+    # by the cut, so its output equals the full sequence's with a local window
+    # of keep + 1 positions and no global window.
+    rng = np.random.default_rng(710)
+    c = rand_case(rng, [9, 4, 7], nt=[2, 1, 3])
+    for keep in (0, 2, 3, 6):
+        off, nt = c["seq_offsets"], c["num_targets"]
+        new_off, ts = oracle.jagged_truncate(off, nt, keep, c["timestamps"])
+        q, k, v = (oracle.jagged_truncate(off, nt, keep, c[n])[1] for n in ("q", "k", "v"))
+        cut = oracle.attn_fwd(new_off, ts, nt, q, k, v, c["rab_pos"], c["rab_time"], c["pos_lo"],
+                              c["pos_hi"], c["inv_n"])
+        win = oracle.attn_fwd(off, c["timestamps"], nt, c["q"], c["k"], c["v"], c["rab_pos"],
+                              c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], local_window=keep + 1,
+                              global_window=0)
+        for b in range(3):
+            n_t = int(nt[b])
+            np.testing.assert_allclose(cut[new_off[b + 1] - n_t:new_off[b + 1]], win[off[b + 1] - n_t:off[b + 1]],
+                                       rtol=0, atol=1e-13)
