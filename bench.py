@@ -72,7 +72,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-stack", action="store_true",
                     help="skip the secondary eight-layer forward measurement")
-    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer", "layer_bwd"], default=None,
+    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer", "layer_bwd", "truncate"], default=None,
                     help="run only a small case twice (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -261,6 +261,113 @@ def layer_stack_timing(dev, stream, reps: int = 3):
             "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
             "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v),
             "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12}}
+
+
+TRUNCATE = (3, 6, 512)   # layers over whole histories, layers over the segment, segment length
+
+
+def truncation_timing(dev, stream, reps: int = 3):
+    """Secondary measurement: attention truncation on the eight-layer stack's
+    batch (64 Zipf-length histories, D=512, 4 heads, d=128).  Three layers run
+    over whole histories, hstu_jagged_truncate keeps each history's last 512
+    tokens (activations and timestamps), six more layers run over the kept
+    batch; timed beside six layers over whole histories (forward, inference).
+    The gather itself is timed alone for its HBM roofline."""
+    import numpy as np
+    import torch
+
+    from hstu_sequential_transduction_b200 import flops, ops, workloads
+
+    n_full, n_cut, keep = TRUNCATE
+    w = workloads.WORKLOADS["layer_stack_bf16"]
+    inp = workloads.generate(w)
+    a = inp.attn
+    T, D = a.total_tokens, w.d_model
+    kept_len = np.minimum(a.lengths, keep)
+    Tk = int(kept_len.sum())
+    kw = dict(num_heads=w.num_heads, d_qk=w.d_qk, d_v=w.d_v, inv_n=a.inv_n, pos_lo=a.pos_lo, pos_hi=a.pos_hi)
+    off, ts = a.seq_offsets.to(dev), a.timestamps.to(dev)
+    rp, rt = a.rab_pos.to(dev), a.rab_time.to(dev)
+    layers = [tuple(t.to(dev) for t in (lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta))
+              for lw in inp.layers]
+    x0 = inp.x.to(dev)
+    xa, xb = torch.empty_like(x0), torch.empty_like(x0)
+    xk, tk = torch.empty_like(x0), torch.empty_like(ts)
+    koff, koff2 = (torch.empty_like(off) for _ in range(2))
+    desc = ops.hstu_layer_desc(ops.make_attn_desc(len(a.lengths), a.max_seq_len, T, w.num_heads, w.d_qk, w.d_v,
+                                                  ops.HSTU_BF16, a.inv_n, a.pos_lo, a.pos_hi, rt.numel()), D, 1e-5)
+    ws = ops.alloc_workspace(ops.hstu_layer_workspace_size(desc), dev)
+
+    def run_layers(x, n, first, o, t, T_, L_):
+        bufs = (xa[:T_], xb[:T_])
+        for i in range(n):
+            w1, b1, w2, b2, g, be = layers[(first + i) % len(layers)]
+            y = bufs[i % 2]
+            ops.hstu_layer_fwd(x, w1, b1, w2, b2, g, be, o, t, None, rp, rt, y=y, workspace=ws, stream=stream,
+                               max_seq_len=L_, **kw)
+            x = y
+        return x
+
+    def cut():
+        x = run_layers(x0, n_full, 0, off, ts, T, a.max_seq_len)
+        ops.hstu_jagged_truncate(off, None, keep, x, out=xk, out_offsets=koff, stream=stream)
+        ops.hstu_jagged_truncate(off, None, keep, ts, out=tk, out_offsets=koff2, stream=stream)
+        run_layers(xk[:Tk], n_cut, n_full, koff, tk[:Tk], Tk, int(kept_len.max()))
+
+    def full():
+        run_layers(x0, n_cut, 0, off, ts, T, a.max_seq_len)
+
+    def gather():
+        ops.hstu_jagged_truncate(off, None, keep, x0, out=xk, out_offsets=koff, stream=stream)
+
+    def timed(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    cut_ms, full_ms = timed(cut, reps), timed(full, reps)
+    # the gather alone: 20 launches replayed from a CUDA graph, so that the
+    # host's per-call cost does not hide a kernel of a few microseconds; its
+    # input is L2-resident, as right after the layer that wrote it
+    gather()
+    torch.cuda.synchronize()
+    graph, n_g = torch.cuda.CUDAGraph(), 20
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream()
+        for _ in range(n_g):
+            ops.hstu_jagged_truncate(off, None, keep, x0, out=xk, out_offsets=koff, stream=cs)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    g_ms = e0.elapsed_time(e1) / n_g
+    del graph
+
+    def stack_flops(lengths, n_layers):
+        toks = int(np.sum(lengths))
+        pairs = flops.attn_pairs(lengths)
+        return n_layers * (flops.attn_fwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
+                           + flops.f1_flops(toks, D, w.num_heads, w.d_qk, w.d_v)
+                           + flops.f2_flops(toks, D, w.num_heads, w.d_v))
+
+    cut_fl = stack_flops(a.lengths, n_full) + stack_flops(kept_len, n_cut)
+    full_fl = stack_flops(a.lengths, n_cut)
+    g_bytes = flops.truncate_bytes(Tk, D * 2, len(a.lengths))
+    return {"workload": "layer_stack_bf16", "layers_full": n_full, "layers_segment": n_cut, "segment_len": keep,
+            "tokens": T, "kept_tokens": Tk, "ms": cut_ms, "tflops": cut_fl / (cut_ms * 1e-3) / 1e12,
+            "gflop": cut_fl / 1e9, "baseline_full_layers": n_cut, "baseline_ms": full_ms,
+            "baseline_gflop": full_fl / 1e9, "flop_ratio": full_fl / cut_fl, "speedup": full_ms / cut_ms,
+            "gather": {"us": g_ms * 1e3, "bytes": g_bytes, "gbs": g_bytes / (g_ms * 1e-3) / 1e9,
+                       "timing": "20 launches in one CUDA graph; input L2-resident"}}
 
 
 def run_reference(args):
@@ -492,6 +599,8 @@ def run_ours(args):
                 "fwd_ms": f_ms, "bwd_ms": b_ms, "tflops": (sl_f + sl_b) / ((f_ms + b_ms) * 1e-3) / 1e12,
                 "speedup_vs_full_mask": ms / (f_ms + b_ms)}
 
+    trunc = None if args.no_layer_stack else truncation_timing(dev, stream)
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
@@ -523,6 +632,8 @@ def run_ours(args):
             line["layer_stack"] = layer
         if semi is not None:
             line["semi_local"] = semi
+        if trunc is not None:
+            line["truncation"] = trunc
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(line), flush=True)
@@ -543,6 +654,10 @@ def kernel_case(which: str):
     dev = torch.device("cuda:0")
     if which == "layer":
         layer_stack_timing(dev, torch.cuda.current_stream(), reps=1)
+        torch.cuda.synchronize()
+        return
+    if which == "truncate":
+        truncation_timing(dev, torch.cuda.current_stream(), reps=1)
         torch.cuda.synchronize()
         return
     if which == "layer_bwd":

@@ -514,6 +514,24 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
     return cuda_status(launch_gemm_tc_ex(op, D, W, (int)T, GEMM_RED_F32, false, splits_for(D, W), hdr, st));
 }
 
+hstu_status hstu_jagged_truncate(int32_t num_seqs, int64_t total_tokens, int32_t keep,
+                                 const int64_t *seq_offsets, const int32_t *num_targets, const void *in,
+                                 int64_t row_bytes, void *out, int64_t *out_offsets, void *stream)
+{
+    if (num_seqs < 0 || total_tokens < 0 || keep < 0 || row_bytes <= 0 || row_bytes % 4 != 0 ||
+        !seq_offsets || !out_offsets)
+        return HSTU_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!in || !out))
+        return HSTU_ERR_INVALID_ARG;
+    if (num_seqs > kTruncateMaxSeqs)
+        return HSTU_ERR_UNSUPPORTED;
+    const uintptr_t align = row_bytes % 16 == 0 ? 15u : 3u;
+    if ((reinterpret_cast<uintptr_t>(in) & align) || (reinterpret_cast<uintptr_t>(out) & align))
+        return HSTU_ERR_INVALID_ARG;
+    return cuda_status(launch_jagged_truncate(seq_offsets, num_targets, num_seqs, total_tokens, keep, row_bytes,
+                                              in, out, out_offsets, static_cast<cudaStream_t>(stream)));
+}
+
 hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream)
 {
     if (!workspace)

@@ -102,4 +102,13 @@ cudaError_t launch_norm_gate_bwd(const void *dG, int64_t ldd, const void *O, int
 // out[n] += sum over T rows of A[row, n] (bf16 A, fp32 out).
 cudaError_t launch_colsum_bf16(const void *A, int64_t lda, int64_t T, int N, float *out, cudaStream_t stream);
 
+// Attention truncation (at most kTruncateMaxSeqs sequences: the new offsets
+// live in shared memory): out_off [B+1] = offsets of every sequence's last
+// min(hist, keep) history tokens plus its candidates; out = those rows of in
+// (row_bytes a multiple of 4; 16-byte copies when it is a multiple of 16).
+constexpr int kTruncateMaxSeqs = 12288;
+cudaError_t launch_jagged_truncate(const int64_t *off, const int32_t *nt, int B, int64_t T, int keep,
+                                   int64_t row_bytes, const void *in, void *out, int64_t *out_off,
+                                   cudaStream_t stream);
+
 }  // namespace hstu

@@ -70,3 +70,9 @@ def layer_bwd_gemm_flops(T: int, d_model: int, num_heads: int, d_qk: int, d_v: i
     width = num_heads * (2 * d_v + 2 * d_qk)
     return 2.0 * T * (2 * d_model * hv + 2 * d_model * width)
 
+
+
+def truncate_bytes(kept_tokens: int, row_bytes: int, num_seqs: int) -> float:
+    """Attention-truncation gather: read and write each kept row once, plus the
+    two offset arrays."""
+    return 2.0 * kept_tokens * row_bytes + 2.0 * 8 * (num_seqs + 1)

@@ -10,6 +10,7 @@ cannot be loaded or built, every call raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 from typing import Optional
@@ -25,7 +26,8 @@ STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3:
 EXPORTED = ["hstu_status_string", "hstu_version", "hstu_attn_workspace_size",
             "hstu_layer_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd",
             "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule",
-            "hstu_attn_fwd_noalloc", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"]
+            "hstu_attn_fwd_noalloc", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
+            "hstu_jagged_truncate"]
 
 
 class HstuError(RuntimeError):
@@ -280,6 +282,29 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
         _ptr(out["d_rab_pos"]), _ptr(out["d_rab_time"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
         _stream(stream)))
     return out
+
+
+def hstu_jagged_truncate(seq_offsets, num_targets, keep: int, rows, *, out=None, out_offsets=None,
+                         stream=None):
+    """Attention truncation gather: each sequence's last min(hist, keep) history
+    rows and all its candidates.  `rows` is any contiguous per-token tensor
+    [T, ...] on the device.  Returns (out_offsets [B+1] int64, out) with `out`
+    shaped like `rows` (T rows of room; the kept batch is out[:out_offsets[-1]])."""
+    _dev(seq_offsets, "seq_offsets", torch.int64)
+    _dev(num_targets, "num_targets", torch.int32)
+    _dev(rows, "rows")
+    B, T = seq_offsets.numel() - 1, rows.shape[0]
+    row_bytes = rows.element_size() * math.prod(rows.shape[1:])
+    if out is None:
+        out = torch.empty_like(rows)
+    if out_offsets is None:
+        out_offsets = torch.empty(B + 1, dtype=torch.int64, device=rows.device)
+    _dev(out, "out", rows.dtype)
+    _dev(out_offsets, "out_offsets", torch.int64)
+    _check("hstu_jagged_truncate", load_library().hstu_jagged_truncate(
+        ctypes.c_int32(B), ctypes.c_int64(T), ctypes.c_int32(keep), _ptr(seq_offsets), _ptr(num_targets),
+        _ptr(rows), ctypes.c_int64(row_bytes), _ptr(out), _ptr(out_offsets), _stream(stream)))
+    return out_offsets, out
 
 
 def hstu_check_device_flag(workspace: torch.Tensor, stream=None):

@@ -177,6 +177,32 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
                            size_t workspace_bytes, void *stream);
 
 /*
+ * Attention truncation (the "ULTRA-HSTU (Meta)" review, "Attention
+ * Truncation"): the first layers run over whole histories, the remaining ones
+ * over each history's most recent segment only.  Sequence b (rows
+ * seq_offsets[b] .. seq_offsets[b+1]-1, n_t = num_targets[b] candidates at its
+ * end, 0 when num_targets is NULL, hist = L_b - n_t) keeps its last
+ * min(hist, keep) history tokens and all of its candidates, in order.
+ *   in          [total_tokens, row_bytes] bytes of any per-token tensor (layer
+ *               activations, timestamps); device.
+ *   out         room for total_tokens rows (the kept count is never larger);
+ *               receives the kept rows, packed; device.
+ *   out_offsets [num_seqs + 1] int64, device: the kept batch's seq_offsets.
+ * num_targets serves the kept batch unchanged.  Positions restart at 0 in the
+ * kept batch; the bias uses only differences of positions and timestamps, so
+ * every pair that survives the cut keeps its bias.  row_bytes must be a
+ * positive multiple of 4; in and out 16-byte aligned when row_bytes is a
+ * multiple of 16, else 4-byte aligned (HSTU_ERR_INVALID_ARG otherwise; also
+ * for keep < 0).  At most 12288 sequences per call (HSTU_ERR_UNSUPPORTED
+ * above).  Sequence data outside the jagged rules is clamped to
+ * [0, total_tokens]: the rows written are then unspecified, but nothing is
+ * read or written outside in and out.
+ */
+hstu_status hstu_jagged_truncate(int32_t num_seqs, int64_t total_tokens, int32_t keep,
+                                 const int64_t *seq_offsets, const int32_t *num_targets, const void *in,
+                                 int64_t row_bytes, void *out, int64_t *out_offsets, void *stream);
+
+/*
  * Attention forward that allocates nothing (no counterpart on the HSTU
  * pages; it exists for callers, not for the method).  Same computation,
  * arguments and layouts as hstu_attn_fwd, without the workspace: some callers
