@@ -233,13 +233,15 @@ def norm_gate(o, u, gamma, beta, eps=1e-5, threads=None):
 
 def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma, ln_beta,
               rab_pos, rab_time, pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, ln_eps=1e-5,
-              threads=None, want_intermediates=False):
-    """Y[T, D] of one transduction layer (and optionally uvqk, O)."""
+              threads=None, want_intermediates=False, out_cat=False):
+    """Y[T, D] of one transduction layer (and optionally uvqk, O).  out_cat: the
+    output projection reads [U | O | G] (W2 is [3 H d_v, D]) instead of G."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     x, w1, b1, w2, b2 = _f64(x), _f64(w1), _f64(b1), _f64(w2), _f64(b2)
     g, be, rp, rt = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time)
     T, D = x.shape
     W = num_heads * (2 * d_v + 2 * d_qk)
+    assert w2.shape == ((3 if out_cat else 1) * num_heads * d_v, D)
     y = np.zeros((T, D))
     uvqk = np.zeros((T, W)) if want_intermediates else None
     o = np.zeros((T, num_heads * d_v)) if want_intermediates else None
@@ -249,23 +251,26 @@ def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma,
         _p(b1, _f64p), _p(w2, _f64p), _p(b2, _f64p), _p(g, _f64p), _p(be, _f64p),
         ctypes.c_double(ln_eps), _p(ts, _i64p), _p(rp, _f64p), ctypes.c_int(int(pos_lo)),
         ctypes.c_int(int(pos_hi)), _p(rt, _f64p), ctypes.c_int(len(rt)), ctypes.c_double(inv_n),
-        _p(y, _f64p), _p(uvqk, _f64p), _p(o, _f64p), ctypes.c_int(threads or default_threads()))
+        _p(y, _f64p), _p(uvqk, _f64p), _p(o, _f64p), ctypes.c_int(int(out_cat)),
+        ctypes.c_int(threads or default_threads()))
     if want_intermediates:
         return y, uvqk, o
     return y
 
 
 def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_beta, rab_pos, rab_time,
-              pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None):
+              pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None, out_cat=False):
     """Gradients of sum(Y * dy) for one transduction layer: a dict with dx, dw1, db1,
-    dw2, db2, d_ln_gamma, d_ln_beta, d_rab_pos, d_rab_time."""
+    dw2, db2, d_ln_gamma, d_ln_beta, d_rab_pos, d_rab_time (out_cat as in layer_fwd)."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     x, w1, b1, w2 = _f64(x), _f64(w1), _f64(b1), _f64(w2)
     g, be, rp, rt, dyy = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time), _f64(dy)
     T, D = x.shape
     hv = num_heads * d_v
     W = num_heads * (2 * d_v + 2 * d_qk)
-    out = {"dx": np.zeros((T, D)), "dw1": np.zeros((D, W)), "db1": np.zeros(W), "dw2": np.zeros((hv, D)),
+    F = (3 if out_cat else 1) * hv
+    assert w2.shape == (F, D)
+    out = {"dx": np.zeros((T, D)), "dw1": np.zeros((D, W)), "db1": np.zeros(W), "dw2": np.zeros((F, D)),
            "db2": np.zeros(D), "d_ln_gamma": np.zeros(hv), "d_ln_beta": np.zeros(hv),
            "d_rab_pos": np.zeros(len(rp)), "d_rab_time": np.zeros(len(rt))}
     _load().oracle_layer_bwd(
@@ -276,7 +281,7 @@ def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_
         ctypes.c_int(len(rt)), ctypes.c_double(inv_n), _p(dyy, _f64p), _p(out["dx"], _f64p),
         _p(out["dw1"], _f64p), _p(out["db1"], _f64p), _p(out["dw2"], _f64p), _p(out["db2"], _f64p),
         _p(out["d_ln_gamma"], _f64p), _p(out["d_ln_beta"], _f64p), _p(out["d_rab_pos"], _f64p),
-        _p(out["d_rab_time"], _f64p), ctypes.c_int(threads or default_threads()))
+        _p(out["d_rab_time"], _f64p), ctypes.c_int(int(out_cat)), ctypes.c_int(threads or default_threads()))
     return out
 
 

@@ -464,6 +464,9 @@ void oracle_norm_gate(int64_t T, int F, const double *o, const double *u, const 
  *   [U | V | Q | K] = SiLU(X W1 + b1)   (column blocks in that order; each block
  *                                         is [T, H, d] with d fastest)
  *   O = attention(Q, K, V);  G = LayerNorm(O) * U;  Y = G W2 + b2.
+ * With out_cat set, the output projection reads the three H dv-wide blocks
+ * [U | O | G] (the 3 h d_v input width of the output-projection row of Table 7
+ * on the DLRMv4 page) and W2 is [3 H dv, D]: Y = [U | O | G] W2 + b2.
  * Optional outputs uvqk [T, H(2dv+2dqk)] and o [T, H dv] (may be NULL).
  */
 void oracle_layer_fwd(int num_seqs, const int64_t *seq_offsets, const int32_t *num_targets,
@@ -472,7 +475,7 @@ void oracle_layer_fwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
                       const double *ln_gamma, const double *ln_beta, double ln_eps,
                       const int64_t *timestamps, const double *rab_pos, int pos_lo, int pos_hi,
                       const double *rab_time, int num_buckets, double inv_n, double *y,
-                      double *uvqk_out, double *o_out, int num_threads)
+                      double *uvqk_out, double *o_out, int out_cat, int num_threads)
 {
     int64_t T = seq_offsets[num_seqs];
     int hv = num_heads * d_v, hq = num_heads * d_qk;
@@ -495,7 +498,19 @@ void oracle_layer_fwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
                     timestamps, rab_pos, pos_lo, pos_hi, rab_time, num_buckets, inv_n, o,
                     num_threads);
     oracle_norm_gate(T, hv, o, u, ln_gamma, ln_beta, ln_eps, g, num_threads);
-    oracle_linear(T, hv, d_model, g, w2, b2, 0, y, num_threads);
+    if (out_cat) {
+        /* the output projection reads [U | O | G], 3 h d_v wide */
+        double *cat = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * 3 * hv);
+        for (int64_t t = 0; t < T; t++) {
+            memcpy(cat + t * 3 * hv, u + t * hv, sizeof(double) * hv);
+            memcpy(cat + t * 3 * hv + hv, o + t * hv, sizeof(double) * hv);
+            memcpy(cat + t * 3 * hv + 2 * hv, g + t * hv, sizeof(double) * hv);
+        }
+        oracle_linear(T, 3 * hv, d_model, cat, w2, b2, 0, y, num_threads);
+        free(cat);
+    } else {
+        oracle_linear(T, hv, d_model, g, w2, b2, 0, y, num_threads);
+    }
     if (uvqk_out)
         memcpy(uvqk_out, uvqk, sizeof(double) * (size_t)T * W);
     if (o_out)
@@ -519,7 +534,9 @@ void oracle_layer_fwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
  *   dO = rstd (dL gamma - mean(dL gamma) - xh mean(dL gamma xh));
  *   (dQ, dK, dV, d_rab_pos, d_rab_time) = attention backward with dout = dO;
  *   dZ = [dU | dV | dQ | dK] * SiLU'(Z);  dW1 = X^T dZ, db1 = sum_t dZ, dX = dZ W1^T.
- * Every output is overwritten.
+ * With out_cat set (Y = [U | O | G] W2 + b2): dW2 = [U | O | G]^T dy, and of
+ * dcat = dy W2^T the G block is dG while the U and O blocks are added to dU and
+ * dO.  Every output is overwritten.
  */
 void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *num_targets,
                       int num_heads, int d_qk, int d_v, int d_model, const double *x,
@@ -529,11 +546,12 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
                       const double *rab_time, int num_buckets, double inv_n, const double *dy,
                       double *dx, double *dw1, double *db1, double *dw2, double *db2,
                       double *dgamma, double *dbeta, double *d_rab_pos, double *d_rab_time,
-                      int num_threads)
+                      int out_cat, int num_threads)
 {
     int64_t T = seq_offsets[num_seqs];
     int hv = num_heads * d_v, hq = num_heads * d_qk;
     int W = 2 * hv + 2 * hq, D = d_model;
+    int F = out_cat ? 3 * hv : hv; /* width of the output projection's input */
     size_t Tn = (size_t)(T > 0 ? T : 1);
     double *z = (double *)malloc(sizeof(double) * Tn * W);
     double *u = (double *)malloc(sizeof(double) * Tn * hv);
@@ -545,6 +563,8 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
     double *rstd = (double *)malloc(sizeof(double) * Tn);
     double *g = (double *)malloc(sizeof(double) * Tn * hv);
     double *dg = (double *)malloc(sizeof(double) * Tn * hv);
+    double *cat = (double *)malloc(sizeof(double) * Tn * F);
+    double *dcat = (double *)malloc(sizeof(double) * Tn * F);
     double *du = (double *)malloc(sizeof(double) * Tn * hv);
     double *dl = (double *)malloc(sizeof(double) * Tn * hv);
     double *dout = (double *)malloc(sizeof(double) * Tn * hv);
@@ -584,8 +604,19 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
         }
     }
 
-    /* output projection: dW2 = G^T dy, db2 = sum dy, dG = dy W2^T */
-    for (int j = 0; j < hv; j++)
+    /* the output projection's input: G, or [U | O | G] */
+    for (int64_t t = 0; t < T; t++) {
+        if (out_cat) {
+            memcpy(cat + t * F, u + t * hv, sizeof(double) * hv);
+            memcpy(cat + t * F + hv, o + t * hv, sizeof(double) * hv);
+            memcpy(cat + t * F + 2 * hv, g + t * hv, sizeof(double) * hv);
+        } else {
+            memcpy(cat + t * F, g + t * hv, sizeof(double) * hv);
+        }
+    }
+
+    /* output projection: dW2 = cat^T dy, db2 = sum dy, dcat = dy W2^T; dG is its G block */
+    for (int j = 0; j < F; j++)
         for (int c = 0; c < D; c++)
             dw2[(int64_t)j * D + c] = 0.0;
     for (int c = 0; c < D; c++)
@@ -593,14 +624,15 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
     for (int64_t t = 0; t < T; t++) {
         for (int c = 0; c < D; c++)
             db2[c] += dy[t * D + c];
-        for (int j = 0; j < hv; j++) {
-            double gj = g[t * hv + j], acc = 0.0;
+        for (int j = 0; j < F; j++) {
+            double cj = cat[t * F + j], acc = 0.0;
             for (int c = 0; c < D; c++) {
-                dw2[(int64_t)j * D + c] += gj * dy[t * D + c];
+                dw2[(int64_t)j * D + c] += cj * dy[t * D + c];
                 acc += dy[t * D + c] * w2[(int64_t)j * D + c];
             }
-            dg[t * hv + j] = acc;
+            dcat[t * F + j] = acc;
         }
+        memcpy(dg + t * hv, dcat + t * F + (F - hv), sizeof(double) * hv);
     }
 
     /* gate and LayerNorm */
@@ -625,6 +657,11 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
             int64_t e = t * hv + c;
             dout[e] = rstd[t] * (dl[e] * ln_gamma[c] - m1 - xh[e] * m2);
         }
+        if (out_cat) /* U and O also enter the projection directly */
+            for (int c = 0; c < hv; c++) {
+                du[t * hv + c] += dcat[t * F + c];
+                dout[t * hv + c] += dcat[t * F + hv + c];
+            }
     }
 
     /* attention */
@@ -670,6 +707,8 @@ void oracle_layer_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *n
     free(rstd);
     free(g);
     free(dg);
+    free(cat);
+    free(dcat);
     free(du);
     free(dl);
     free(dout);

@@ -467,17 +467,25 @@ def test_layer_matches_composition():
     g = torch.nn.functional.layer_norm(torch.tensor(o), (H * dv,), torch.tensor(gam),
                                        torch.tensor(bet), eps=1e-5).numpy() * u
     np.testing.assert_allclose(y, g @ w2 + b2, rtol=0, atol=1e-10)
+    # output projection over [U | O | G] (3 h d_v wide): each block meets its own rows of W2
+    w2c = rng.standard_normal((3 * H * dv, D))
+    yc = oracle.layer_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], x, w1, b1, w2c, b2,
+                          gam, bet, c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"],
+                          c["inv_n"], H, dqk, dv, out_cat=True)
+    hv = H * dv
+    np.testing.assert_allclose(yc, u @ w2c[:hv] + o @ w2c[hv:2 * hv] + g @ w2c[2 * hv:] + b2, rtol=0, atol=1e-10)
 
 
 # ---- 8. layer backward: torch float64 autograd and finite differences --------
 
-def _layer_case(seed, lengths=(4, 6, 1), nt=(0, 2, 0), H=2, dqk=3, dv=3, D=5):
+def _layer_case(seed, lengths=(4, 6, 1), nt=(0, 2, 0), H=2, dqk=3, dv=3, D=5, out_cat=False):
     rng = np.random.default_rng(seed)
     c = rand_case(rng, list(lengths), H=H, dqk=dqk, dv=dv, nt=list(nt))
     T = int(c["seq_offsets"][-1])
     W = H * (2 * dv + 2 * dqk)
+    F = (3 if out_cat else 1) * H * dv
     prm = {"x": rng.standard_normal((T, D)), "w1": rng.standard_normal((D, W)) * 0.5,
-           "b1": rng.standard_normal(W) * 0.1, "w2": rng.standard_normal((H * dv, D)),
+           "b1": rng.standard_normal(W) * 0.1, "w2": rng.standard_normal((F, D)),
            "b2": rng.standard_normal(D), "ln_gamma": 1 + 0.1 * rng.standard_normal(H * dv),
            "ln_beta": 0.1 * rng.standard_normal(H * dv), "rab_pos": c["rab_pos"], "rab_time": c["rab_time"]}
     dy = rng.standard_normal((T, D))
@@ -519,6 +527,8 @@ def _torch_layer_loss(c, prm, dy, dims):
         outs.append(torch.einsum("hij,jhc->ihc", P, vv[s0:s1]).reshape(L, hv))
     o = torch.cat(outs)
     g = torch.nn.functional.layer_norm(o, (hv,), t["ln_gamma"], t["ln_beta"], eps=1e-5) * u
+    if prm["w2"].shape[0] == 3 * hv:  # output projection over [U | O | G]
+        g = torch.cat([u, o, g], dim=1)
     y = g @ t["w2"] + t["b2"]
     (y * torch.tensor(dy)).sum().backward()
     return {k: v.grad.numpy() for k, v in t.items()}
@@ -528,31 +538,33 @@ def _olayer_bwd(c, prm, dy, dims):
     H, dqk, dv = dims
     return oracle.layer_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], prm["x"], prm["w1"],
                             prm["b1"], prm["w2"], prm["ln_gamma"], prm["ln_beta"], prm["rab_pos"],
-                            prm["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv, dy)
+                            prm["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv, dy,
+                            out_cat=prm["w2"].shape[0] == 3 * H * dv)
 
 
 _LAYER_GRAD_NAMES = {"x": "dx", "w1": "dw1", "b1": "db1", "w2": "dw2", "b2": "db2", "ln_gamma": "d_ln_gamma",
                      "ln_beta": "d_ln_beta", "rab_pos": "d_rab_pos", "rab_time": "d_rab_time"}
 
 
-@pytest.mark.parametrize("seed", [0, 1])
-def test_layer_bwd_matches_torch_autograd(seed):
-    c, prm, dy, dims = _layer_case(400 + seed)
+@pytest.mark.parametrize("seed,out_cat", [(0, False), (1, False), (2, True), (3, True)])
+def test_layer_bwd_matches_torch_autograd(seed, out_cat):
+    c, prm, dy, dims = _layer_case(400 + seed, out_cat=out_cat)
     ours = _olayer_bwd(c, prm, dy, dims)
     ref = _torch_layer_loss(c, prm, dy, dims)
     for k, name in _LAYER_GRAD_NAMES.items():
         np.testing.assert_allclose(ours[name], ref[k], rtol=1e-9, atol=1e-10, err_msg=name)
 
 
-def test_layer_bwd_central_finite_differences():
-    c, prm, dy, dims = _layer_case(410, lengths=(3, 2), nt=(1, 0), H=1, dqk=2, dv=2, D=3)
+@pytest.mark.parametrize("out_cat", [False, True])
+def test_layer_bwd_central_finite_differences(out_cat):
+    c, prm, dy, dims = _layer_case(410, lengths=(3, 2), nt=(1, 0), H=1, dqk=2, dv=2, D=3, out_cat=out_cat)
     H, dqk, dv = dims
     ours = _olayer_bwd(c, prm, dy, dims)
 
     def loss(p):
         y = oracle.layer_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], p["x"], p["w1"], p["b1"],
                              p["w2"], p["b2"], p["ln_gamma"], p["ln_beta"], p["rab_pos"], p["rab_time"],
-                             c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv)
+                             c["pos_lo"], c["pos_hi"], c["inv_n"], H, dqk, dv, out_cat=out_cat)
         return float(np.sum(y * dy))
 
     h = 1e-6
