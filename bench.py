@@ -249,9 +249,38 @@ def layer_stack_timing(dev, stream, reps: int = 3):
     e1.record(stream)
     torch.cuda.synchronize()
     bwd_ms = e0.elapsed_time(e1) / reps
+    # the first layer again with the output projection over [U | O | G] (3 H d_v wide)
+    hv = w.num_heads * w.d_v
+    gen_w = torch.Generator(device="cpu").manual_seed(2025)
+    w2c = (0.02 * torch.randn((3 * hv, w.d_model), generator=gen_w)).to(device=dev, dtype=torch.bfloat16)
+    desc_c = ops.hstu_layer_desc(attn0, w.d_model, 1e-5, 1)
+    ws_c = ops.alloc_workspace(max(ops.hstu_layer_workspace_size(desc_c),
+                                   ops.hstu_layer_bwd_workspace_size(desc_c)), dev)
+
+    def cat_forward():
+        ops.hstu_layer_fwd(xs[0], w1, b1, w2c, b2, g, be, off, ts, None, rp, rt, y=xs[1], saved_uvqk=uvqk,
+                           saved_o=o, workspace=ws_c, stream=stream, output_concat=True, **kw)
+
+    def cat_backward():
+        ops.hstu_layer_bwd(xs[0], w1, b1, w2c, g, be, off, ts, None, rp, rt, uvqk, o, dy, workspace=ws_c,
+                           stream=stream, output_concat=True, **kw)
+
+    cat_ms = {}
+    for name, fn in (("fwd", cat_forward), ("bwd", cat_backward)):
+        fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cat_ms[name] = e0.elapsed_time(e1) / reps
+
     pairs = flops.attn_pairs(a.lengths)
     bwd_fl = flops.layer_bwd_gemm_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
         flops.attn_bwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
+    f2_extra = flops.f2_flops(T, w.d_model, w.num_heads, w.d_v, width_factor=3) - \
+        flops.f2_flops(T, w.d_model, w.num_heads, w.d_v)
     attn_fl = flops.attn_fwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
     gemm_fl = flops.f1_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
         flops.f2_flops(T, w.d_model, w.num_heads, w.d_v)
@@ -260,7 +289,12 @@ def layer_stack_timing(dev, stream, reps: int = 3):
             "ms_per_forward": ms, "tflops": total / (ms * 1e-3) / 1e12,
             "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
             "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v),
-            "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12}}
+            "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12},
+            "output_concat": {
+                "what": "first layer with the output projection over [U | O | G] (3 H d_v = %d wide)" % (3 * hv),
+                "fwd_ms": cat_ms["fwd"], "bwd_ms": cat_ms["bwd"],
+                "fwd_tflops": (attn_fl + gemm_fl + f2_extra) / (cat_ms["fwd"] * 1e-3) / 1e12,
+                "bwd_tflops": (bwd_fl + 2 * f2_extra) / (cat_ms["bwd"] * 1e-3) / 1e12}}
 
 
 TRUNCATE = (3, 6, 512)   # layers over whole histories, layers over the segment, segment length

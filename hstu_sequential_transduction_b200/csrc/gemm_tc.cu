@@ -58,6 +58,7 @@ struct GemmArgs {
     int64_t ldc;
     int64_t M;
     int N, K, silu, splits;
+    int a_seg;                  // > 0: A is three stored matrices of a_seg columns each
     WsHeader *hdr;
 };
 
@@ -73,7 +74,8 @@ __device__ __forceinline__ float silu_grad_tanh(float z)
 // tiles row-block major so consecutive tiles reuse the same A rows from L2.
 template <int BN, bool A_MN, bool B_K, int EPI>
 __global__ void __launch_bounds__(kThreadsG, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA1,
+               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const GemmArgs g)
 {
     using LY = GL<BN, EPI>;
@@ -106,6 +108,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch(&tmA);
+        if (g.a_seg) {
+            tma_prefetch(&tmA1);
+            tma_prefetch(&tmA2);
+        }
         tma_prefetch(&tmB);
         if (EPI == EPI_RED)
             tma_prefetch(&tmC);
@@ -118,6 +124,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + LY::MISC);
 
     if (warp == 0) {
+        // the stored matrix holding stored column x of A, and x within it
+        auto a_map = [&](int x, int &xl) -> const CUtensorMap * {
+            if (!g.a_seg) {
+                xl = x;
+                return &tmA;
+            }
+            const int seg = min(x / g.a_seg, 2);  // past the end: the last matrix's zero fill
+            xl = x - seg * g.a_seg;
+            return seg == 0 ? &tmA : seg == 1 ? &tmA1 : &tmA2;
+        };
         if (lane == 0) {
             int it = 0;  // k-slices issued by this CTA, across its units
             bool ok = true;
@@ -133,10 +149,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     mbar_expect_tx(full_bar(s), kRegA + BN * 128);
                     const uint32_t sa = base + LY::A + s * kRegA, sb = base + LY::B + s * BN * 128;
                     if (A_MN) {
-                        for (int r = 0; r < 2; r++)
-                            tma_load_2d(sa + r * kReg64, &tmA, m0 + 64 * r, kt * GBK, full_bar(s));
+                        for (int r = 0; r < 2; r++) {
+                            int xl;
+                            const CUtensorMap *ma = a_map(m0 + 64 * r, xl);
+                            tma_load_2d(sa + r * kReg64, ma, xl, kt * GBK, full_bar(s));
+                        }
                     } else {
-                        tma_load_2d(sa, &tmA, kt * GBK, m0, full_bar(s));
+                        int xl;
+                        const CUtensorMap *ma = a_map(kt * GBK, xl);
+                        tma_load_2d(sa, ma, xl, m0, full_bar(s));
                     }
                     if (B_K) {
                         tma_load_2d(sb, &tmB, kt * GBK, n0, full_bar(s));
@@ -284,14 +305,21 @@ int num_sms()
 template <int BN, bool A_MN, bool B_K, int EPI>
 cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stream)
 {
-    CUtensorMap ma, mb, mc;
-    cudaError_t e;
-    if (A_MN)  // stored [K, M]: box 64 m x 64 k
-        e = make_tensor_map_2d(&ma, op.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.K, g.M, op.lda * 2, 64, 64,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-    else       // [M, K]: box 64 k x 128 m
-        e = make_tensor_map_2d(&ma, op.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.M, g.K, op.lda * 2, 64, GBM,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
+    CUtensorMap ma, ma1, ma2, mb, mc;
+    cudaError_t e = cudaSuccess;
+    const void *abase[3] = {op.A, op.A1, op.A2};
+    const int64_t ald[3] = {op.lda, op.lda1, op.lda2};
+    CUtensorMap *amap[3] = {&ma, &ma1, &ma2};
+    for (int i = 0; i < (g.a_seg ? 3 : 1) && e == cudaSuccess; i++) {
+        if (A_MN)  // stored [K, M]: box 64 m x 64 k
+            e = make_tensor_map_2d(amap[i], abase[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.K,
+                                   g.a_seg ? g.a_seg : g.M, ald[i] * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+        else       // [M, K]: box 64 k x 128 m
+            e = make_tensor_map_2d(amap[i], abase[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.M,
+                                   g.a_seg ? g.a_seg : g.K, ald[i] * 2, 64, GBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (!g.a_seg)
+        ma1 = ma2 = ma;  // unused
     if (e == cudaSuccess) {
         if (B_K)  // stored [N, K]: box 64 k x BN n
             e = make_tensor_map_2d(&mb, op.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.N, g.K, op.ldb * 2, 64, BN,
@@ -316,7 +344,7 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
         return e;
     const int64_t units = ((g.M + GBM - 1) / GBM) * (g.N / BN) * g.splits;
     const unsigned grid = (unsigned)std::min<int64_t>(units, num_sms());
-    gemm_tc_kernel<BN, A_MN, B_K, EPI><<<grid, kThreadsG, bytes, stream>>>(ma, mb, mc, g);
+    gemm_tc_kernel<BN, A_MN, B_K, EPI><<<grid, kThreadsG, bytes, stream>>>(ma, ma1, ma2, mb, mc, g);
     return cudaGetLastError();
 }
 
@@ -343,7 +371,13 @@ bool gemm_tc_ok(const GemmOperands &op, int64_t M, int N, int K)
     // needs K % 8 == 0 for its 16-byte rows, an MN-major A needs M % 64 == 0
     const bool k_ok = K > 0 && K < ((int64_t)1 << 31) - GBK && ((op.a_mn && !op.b_k) || K % 8 == 0);
     const bool mn_ok = !op.a_mn || M % 64 == 0;
-    return aligned && mn_ok && k_ok && M > 0 && M < ((int64_t)1 << 31) - GBM && N % 128 == 0 && op.lda % 8 == 0 &&
+    // a concatenated A: three bases, 64-column pieces, and exactly three of them
+    const bool seg_ok =
+        op.a_seg == 0 ||
+        (op.a_seg > 0 && op.a_seg % 64 == 0 && op.A1 && op.A2 && op.lda1 % 8 == 0 && op.lda2 % 8 == 0 &&
+         ((reinterpret_cast<uintptr_t>(op.A1) | reinterpret_cast<uintptr_t>(op.A2)) & 15u) == 0 &&
+         (op.a_mn ? M : (int64_t)K) == 3 * (int64_t)op.a_seg);
+    return aligned && mn_ok && k_ok && seg_ok && M > 0 && M < ((int64_t)1 << 31) - GBM && N % 128 == 0 && op.lda % 8 == 0 &&
            op.ldb % 8 == 0 && op.ldc % 8 == 0 && (!op.aux || op.ldaux % 8 == 0);
 }
 
@@ -363,6 +397,7 @@ cudaError_t launch_gemm_tc_ex(const GemmOperands &op, int64_t M, int N, int K, G
     g.K = K;
     g.silu = silu;
     g.splits = std::max(1, std::min(splits, (K + GBK - 1) / GBK));
+    g.a_seg = op.a_seg;
     g.hdr = hdr;
     switch (epi) {
     case GEMM_RED_F32:

@@ -270,7 +270,8 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
     if (!d)
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_attn_desc(&d->attn));
-    if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps))
+    if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps) ||
+        (d->output_concat != 0 && d->output_concat != 1))
         return HSTU_ERR_INVALID_ARG;
     const int F = d->attn.num_heads * d->attn.d_v;
     if (F != 64 && F != 128 && F != 256 && F != 512 && F != 1024)
@@ -282,6 +283,13 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
 
 static int layer_width(const hstu_attn_desc *a) { return a->num_heads * (2 * a->d_v + 2 * a->d_qk); }
 
+// the concatenated output projection reads [U | O | G] straight from its three
+// buffers on the tcgen05 GEMM (bf16, D % 128 == 0); other paths copy it first
+static bool layer_cat_copy(const hstu_layer_desc *d)
+{
+    return d->output_concat && (d->attn.dtype != HSTU_BF16 || d->d_model % 128 != 0);
+}
+
 static size_t layer_ws(const hstu_layer_desc *d, bool keep_uvqk, bool keep_o)
 {
     const hstu_attn_desc *a = &d->attn;
@@ -292,6 +300,8 @@ static size_t layer_ws(const hstu_layer_desc *d, bool keep_uvqk, bool keep_o)
     if (!keep_o)
         b += align256(T * a->num_heads * a->d_v * eb);
     b += align256(T * a->num_heads * a->d_v * eb);  // G
+    if (layer_cat_copy(d))
+        b += align256(T * 3 * a->num_heads * a->d_v * eb);  // [U | O | G]
     return b;
 }
 
@@ -355,6 +365,36 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
                               rab_pos, rab_time, o, hv, workspace, st));
     HSTU_CUDA(launch_norm_gate(bf16, o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv,
                                (int64_t)T, hv, st));
+    if (desc->output_concat) {
+        // Y = [U | O | G] W2 + b2
+        const int F = 3 * hv;
+        if (!layer_cat_copy(desc)) {
+            GemmOperands op{};
+            op.A = uvqk;
+            op.lda = W;
+            op.A1 = o;
+            op.lda1 = hv;
+            op.A2 = g;
+            op.lda2 = hv;
+            op.a_seg = hv;
+            op.B = w2;
+            op.ldb = D;
+            op.bias = b2;
+            op.C = y;
+            op.ldc = D;
+            if (!gemm_tc_ok(op, (int64_t)T, D, F))
+                return HSTU_ERR_UNSUPPORTED;
+            return cuda_status(launch_gemm_tc_ex(op, (int64_t)T, D, F, GEMM_ACT, false, 1, hdr, st));
+        }
+        char *cat = g + align256(T * hv * eb);
+        HSTU_CUDA(launch_concat3(uvqk, (int64_t)W * eb, o, (int64_t)hv * eb, g, (int64_t)hv * eb, cat,
+                                 (int64_t)T, (int64_t)hv * eb, st));
+        if (bf16)
+            return cuda_status(launch_gemm_bf16(cat, F, w2, b2, y, D, (int64_t)T, D, F, false, st));
+        return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(cat), F,
+                                           static_cast<const float *>(w2), static_cast<const float *>(b2),
+                                           static_cast<float *>(y), D, (int64_t)T, D, F, false, st));
+    }
     if (bf16 && gemm_tc_supported(g, hv, w2, y, D, (int64_t)T, D, hv))
         return cuda_status(launch_gemm_tc(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
     if (bf16)
@@ -368,8 +408,9 @@ static size_t layer_bwd_ws(const hstu_layer_desc *d)
 {
     const hstu_attn_desc *a = &d->attn;
     const size_t T = (size_t)a->total_tokens, W = layer_width(a), hv = (size_t)a->num_heads * a->d_v;
-    // attention backward scratch, then G, dG, dO [T, H d_v] and dA, dZ [T, W] (bf16)
-    return attn_ws(a, 1) + 3 * align256(T * hv * 2) + 2 * align256(T * W * 2);
+    const size_t F = (d->output_concat ? 3 : 1) * hv;
+    // attention backward scratch, then G [T, H d_v], dcat [T, F], dO [T, H d_v] and dA, dZ [T, W] (bf16)
+    return attn_ws(a, 1) + 2 * align256(T * hv * 2) + align256(T * F * 2) + 2 * align256(T * W * 2);
 }
 
 static bool layer_bwd_supported(const hstu_layer_desc *d)
@@ -414,11 +455,13 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
     const int64_t T = a->total_tokens;
     const int W = layer_width(a), hv = a->num_heads * a->d_v, hq = a->num_heads * a->d_qk;
     const int D = desc->d_model;
+    const bool cat = desc->output_concat != 0;
+    const int F = cat ? 3 * hv : hv;  // width of the output projection's input
     WsHeader *hdr = static_cast<WsHeader *>(workspace);
 
     HSTU_CUDA(cudaMemsetAsync(dw1, 0, sizeof(float) * (size_t)D * W, st));
     HSTU_CUDA(cudaMemsetAsync(db1, 0, sizeof(float) * W, st));
-    HSTU_CUDA(cudaMemsetAsync(dw2, 0, sizeof(float) * (size_t)hv * D, st));
+    HSTU_CUDA(cudaMemsetAsync(dw2, 0, sizeof(float) * (size_t)F * D, st));
     HSTU_CUDA(cudaMemsetAsync(db2, 0, sizeof(float) * D, st));
     HSTU_CUDA(cudaMemsetAsync(d_ln_gamma, 0, sizeof(float) * hv, st));
     HSTU_CUDA(cudaMemsetAsync(d_ln_beta, 0, sizeof(float) * hv, st));
@@ -432,7 +475,8 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
         cur += align256(bytes);
         return p;
     };
-    char *g = take((size_t)T * hv * 2), *dg = take((size_t)T * hv * 2), *dout = take((size_t)T * hv * 2);
+    char *g = take((size_t)T * hv * 2), *dcat = take((size_t)T * F * 2), *dout = take((size_t)T * hv * 2);
+    char *dg = dcat + (size_t)(F - hv) * 2;  // the G block of dcat
     char *da = take((size_t)T * W * 2), *dz = take((size_t)T * W * 2);
     const char *uvqk = static_cast<const char *>(saved_uvqk);
     const int sms = 148;
@@ -443,33 +487,42 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
 
     // G = LayerNorm(O) U, recomputed from the saved attention output
     HSTU_CUDA(launch_norm_gate(true, saved_o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv, T, hv, st));
-    // output projection: dG = dy W2^T, dW2 = G^T dy, db2 = sum dy
+    // output projection over cat = G or [U | O | G]: dcat = dy W2^T, dW2 = cat^T dy, db2 = sum dy
     GemmOperands op{};
     op.A = dy;
     op.lda = D;
     op.B = w2;
     op.ldb = D;
     op.b_k = true;
-    op.C = dg;
-    op.ldc = hv;
-    if (!gemm_tc_ok(op, T, hv, D))
+    op.C = dcat;
+    op.ldc = F;
+    if (!gemm_tc_ok(op, T, F, D))
         return HSTU_ERR_UNSUPPORTED;
-    HSTU_CUDA(launch_gemm_tc_ex(op, T, hv, D, GEMM_ACT, false, 1, hdr, st));
+    HSTU_CUDA(launch_gemm_tc_ex(op, T, F, D, GEMM_ACT, false, 1, hdr, st));
     op = GemmOperands{};
     op.A = g;
     op.lda = hv;
+    if (cat) {  // the rows of cat^T come from three buffers
+        op.A = uvqk;
+        op.lda = W;
+        op.A1 = saved_o;
+        op.lda1 = hv;
+        op.A2 = g;
+        op.lda2 = hv;
+        op.a_seg = hv;
+    }
     op.a_mn = true;
     op.B = dy;
     op.ldb = D;
     op.C32 = dw2;
     op.ldc = D;
-    if (!gemm_tc_ok(op, hv, D, (int)T))
+    if (!gemm_tc_ok(op, F, D, (int)T))
         return HSTU_ERR_UNSUPPORTED;
-    HSTU_CUDA(launch_gemm_tc_ex(op, hv, D, (int)T, GEMM_RED_F32, false, splits_for(hv, D), hdr, st));
+    HSTU_CUDA(launch_gemm_tc_ex(op, F, D, (int)T, GEMM_RED_F32, false, splits_for(F, D), hdr, st));
     HSTU_CUDA(launch_colsum_bf16(dy, D, T, D, db2, st));
-    // gate: dO and dU (into the U block of dA), dgamma, dbeta
-    HSTU_CUDA(launch_norm_gate_bwd(dg, hv, saved_o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, dout, hv, da, W,
-                                   d_ln_gamma, d_ln_beta, T, hv, st));
+    // gate: dO and dU (into the U block of dA; plus dcat's U and O blocks), dgamma, dbeta
+    HSTU_CUDA(launch_norm_gate_bwd(dg, F, saved_o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, dout, hv, da, W,
+                                   d_ln_gamma, d_ln_beta, T, hv, cat, st));
     // attention: dV, dQ, dK into their blocks of dA, bias-table gradients
     HSTU_TRY(attn_bwd_strided(a, uvqk + (size_t)2 * hv * 2, W, uvqk + (size_t)(2 * hv + hq) * 2, W,
                               uvqk + (size_t)hv * 2, W, seq_offsets, timestamps, num_targets, rab_pos, rab_time,

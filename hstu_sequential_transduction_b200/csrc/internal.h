@@ -69,10 +69,17 @@ cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const 
 //   GEMM_DSILU:  C bf16 = aux * SiLU'(acc + bias), aux bf16 [M, N] (row stride ldaux)
 //   GEMM_RED_F32: C32 fp32 += acc, the k range split over `splits` CTAs (C32 must
 //                 hold its initial value, e.g. zeros); ldc in elements.
+// A may be the column concatenation of three stored matrices with the same row
+// count: a_seg > 0 (a multiple of 64) is the width of each, A, A1, A2 their
+// bases and lda, lda1, lda2 their row strides.  The stored columns are K for a
+// K-major A and M for an MN-major A, so the concatenation runs along K or M.
 enum GemmEpilogue { GEMM_ACT = 0, GEMM_DSILU = 1, GEMM_RED_F32 = 2 };
 struct GemmOperands {
     const void *A;
     int64_t lda;
+    const void *A1, *A2;
+    int64_t lda1, lda2;
+    int a_seg;
     bool a_mn;
     const void *B;
     int64_t ldb;
@@ -98,7 +105,14 @@ cudaError_t launch_norm_gate(bool bf16, const void *O, int64_t ldo, const void *
 cudaError_t launch_norm_gate_bwd(const void *dG, int64_t ldd, const void *O, int64_t ldo, const void *U,
                                  int64_t ldu, const float *gamma, const float *beta, float eps, void *dO,
                                  int64_t lddo, void *dU, int64_t lddu, float *dgamma, float *dbeta, int64_t T,
-                                 int F, cudaStream_t stream);
+                                 int F, bool cat, cudaStream_t stream);
+// cat: dG is the last F-wide block of rows [dU' | dO' | dG] whose first two
+// blocks (direct gradients through an output projection over [U | O | G]) are
+// added to dU and dO.
+// out[t, :] = [a[t, :] | b[t, :] | c[t, :]], each block `bytes` wide (a multiple
+// of 4); row strides lda, ldb, ldc in bytes.
+cudaError_t launch_concat3(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c, int64_t ldc,
+                           void *out, int64_t T, int64_t bytes, cudaStream_t stream);
 // out[n] += sum over T rows of A[row, n] (bf16 A, fp32 out).
 cudaError_t launch_colsum_bf16(const void *A, int64_t lda, int64_t T, int N, float *out, cudaStream_t stream);
 

@@ -317,7 +317,7 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
                      const T *__restrict__ U, int64_t ldu, const float *__restrict__ gamma,
                      const float *__restrict__ beta, float eps, T *__restrict__ dO, int64_t lddo,
                      T *__restrict__ dU, int64_t lddu, float *__restrict__ dgamma, float *__restrict__ dbeta,
-                     int64_t Trows)
+                     int64_t Trows, int cat)
 {
     constexpr int F = 32 * VPT;
     extern __shared__ float slots[];  // [warps][2][F]
@@ -387,6 +387,18 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
                 du[e] = dg[e] * fmaf(xh, ga[e], be[e]);
                 dx[e] = rstd * (dg[e] * u[e] * ga[e] - m1 - xh * m2);
             }
+            if (cat) {
+                // output projection over [U | O | G]: dG is the last block of a
+                // row whose first two blocks are the direct gradients of U and O
+                float cu[VPT], co[VPT];
+                load_vec<T, VPT>(dG + row * ldd - 2 * F + fo, cu);
+                load_vec<T, VPT>(dG + row * ldd - F + fo, co);
+#pragma unroll
+                for (int e = 0; e < VPT; e++) {
+                    du[e] += cu[e];
+                    dx[e] += co[e];
+                }
+            }
             store_vec<T, VPT>(dO + row * lddo + fo, dx);
             store_vec<T, VPT>(dU + row * lddu + fo, du);
         }
@@ -411,7 +423,8 @@ norm_gate_bwd_kernel(const T *__restrict__ dG, int64_t ldd, const T *__restrict_
 template <typename T>
 cudaError_t norm_gate_bwd_t(const T *dG, int64_t ldd, const T *O, int64_t ldo, const T *U, int64_t ldu,
                             const float *gamma, const float *beta, float eps, T *dO, int64_t lddo, T *dU,
-                            int64_t lddu, float *dgamma, float *dbeta, int64_t Trows, int F, cudaStream_t stream)
+                            int64_t lddu, float *dgamma, float *dbeta, int64_t Trows, int F, int cat,
+                            cudaStream_t stream)
 {
     const int64_t want = (Trows * 32 + 255) / 256;
     const unsigned blocks = (unsigned)std::min<int64_t>(want, 148 * 8);
@@ -428,7 +441,7 @@ cudaError_t norm_gate_bwd_t(const T *dG, int64_t ldd, const T *O, int64_t ldo, c
     }
 #define HSTU_NGB(V)                                                                                                 \
     norm_gate_bwd_kernel<T, V><<<blocks, 256, smem, stream>>>(dG, ldd, O, ldo, U, ldu, gamma, beta, eps, dO, lddo, \
-                                                              dU, lddu, dgamma, dbeta, Trows)
+                                                              dU, lddu, dgamma, dbeta, Trows, cat)
     switch (F) {
     case 64: HSTU_NGB(2); break;
     case 128: HSTU_NGB(4); break;
@@ -487,14 +500,42 @@ cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const 
 cudaError_t launch_norm_gate_bwd(const void *dG, int64_t ldd, const void *O, int64_t ldo, const void *U,
                                  int64_t ldu, const float *gamma, const float *beta, float eps, void *dO,
                                  int64_t lddo, void *dU, int64_t lddu, float *dgamma, float *dbeta, int64_t T,
-                                 int F, cudaStream_t stream)
+                                 int F, bool cat, cudaStream_t stream)
 {
     if (T == 0)
         return cudaSuccess;
     return norm_gate_bwd_t(static_cast<const __nv_bfloat16 *>(dG), ldd, static_cast<const __nv_bfloat16 *>(O), ldo,
                            static_cast<const __nv_bfloat16 *>(U), ldu, gamma, beta, eps,
                            static_cast<__nv_bfloat16 *>(dO), lddo, static_cast<__nv_bfloat16 *>(dU), lddu, dgamma,
-                           dbeta, T, F, stream);
+                           dbeta, T, F, cat ? 1 : 0, stream);
+}
+
+// out[t] = [a[t] | b[t] | c[t]], each `bytes` wide (a multiple of 4), rows strided
+__global__ void __launch_bounds__(256)
+concat3_kernel(const unsigned char *__restrict__ a, int64_t lda, const unsigned char *__restrict__ b, int64_t ldb,
+               const unsigned char *__restrict__ c, int64_t ldc, unsigned char *__restrict__ out, int64_t Trows,
+               int64_t bytes)
+{
+    const int64_t words = bytes >> 2, total = Trows * 3 * words;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = e / (3 * words), r = e - row * 3 * words, blk = r / words, w = r - blk * words;
+        const unsigned char *src = blk == 0 ? a + row * lda : blk == 1 ? b + row * ldb : c + row * ldc;
+        reinterpret_cast<uint32_t *>(out + row * 3 * bytes)[blk * words + w] = reinterpret_cast<const uint32_t *>(src)[w];
+    }
+}
+
+cudaError_t launch_concat3(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c, int64_t ldc,
+                           void *out, int64_t T, int64_t bytes, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    const int64_t total = T * 3 * (bytes / 4);
+    const unsigned blocks = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 8);
+    concat3_kernel<<<blocks, 256, 0, stream>>>(static_cast<const unsigned char *>(a), lda,
+                                               static_cast<const unsigned char *>(b), ldb,
+                                               static_cast<const unsigned char *>(c), ldc,
+                                               static_cast<unsigned char *>(out), T, bytes);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_colsum_bf16(const void *A, int64_t lda, int64_t T, int N, float *out, cudaStream_t stream)

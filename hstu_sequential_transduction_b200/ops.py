@@ -46,7 +46,8 @@ class hstu_attn_desc(ctypes.Structure):
 
 
 class hstu_layer_desc(ctypes.Structure):
-    _fields_ = [("attn", hstu_attn_desc), ("d_model", ctypes.c_int32), ("ln_eps", ctypes.c_float)]
+    _fields_ = [("attn", hstu_attn_desc), ("d_model", ctypes.c_int32), ("ln_eps", ctypes.c_float),
+                ("output_concat", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -220,8 +221,9 @@ def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
 def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets,
                    rab_pos, rab_time, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, y=None,
-                   saved_uvqk=None, saved_o=None, workspace=None, stream=None):
-    """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer."""
+                   saved_uvqk=None, saved_o=None, workspace=None, stream=None, output_concat: bool = False):
+    """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer; with
+    output_concat, f2 reads [U | O | G] and w2 is [3 H d_v, D]."""
     for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("b2", b2)):
         _dev(t, name, x.dtype)
     _dev(ln_gamma, "ln_gamma", torch.float32)
@@ -229,7 +231,9 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
     T, D = x.shape
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
                           _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
-    desc = hstu_layer_desc(attn, int(D), float(ln_eps))
+    desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)))
+    if w2.shape[0] != (3 if output_concat else 1) * num_heads * d_v:
+        raise ValueError(f"w2 has {w2.shape[0]} rows for output_concat={output_concat}")
     if y is None:
         y = torch.empty((T, D), dtype=x.dtype, device=x.device)
     if workspace is None:
@@ -251,10 +255,11 @@ def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc) -> int:
 
 def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
                    saved_uvqk, saved_o, dy, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
-                   inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, workspace=None, stream=None):
+                   inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, workspace=None, stream=None,
+                   output_concat: bool = False):
     """Gradients of sum(Y * dy) for one layer (bf16): a dict with dx (bf16) and the
     float32 parameter gradients dw1, db1, dw2, db2, d_ln_gamma, d_ln_beta,
-    d_rab_pos, d_rab_time."""
+    d_rab_pos, d_rab_time (output_concat as in hstu_layer_fwd)."""
     for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("saved_uvqk", saved_uvqk),
                     ("saved_o", saved_o), ("dy", dy)):
         _dev(t, name, x.dtype)
@@ -265,11 +270,14 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
     hv = num_heads * d_v
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
                           _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
-    desc = hstu_layer_desc(attn, int(D), float(ln_eps))
+    desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)))
+    F = (3 if output_concat else 1) * hv
+    if w2.shape[0] != F:
+        raise ValueError(f"w2 has {w2.shape[0]} rows for output_concat={output_concat}")
     dev = x.device
     f32 = dict(dtype=torch.float32, device=dev)
     out = {"dx": torch.empty((T, D), dtype=x.dtype, device=dev), "dw1": torch.empty((D, W), **f32),
-           "db1": torch.empty(W, **f32), "dw2": torch.empty((hv, D), **f32), "db2": torch.empty(D, **f32),
+           "db1": torch.empty(W, **f32), "dw2": torch.empty((F, D), **f32), "db2": torch.empty(D, **f32),
            "d_ln_gamma": torch.empty(hv, **f32), "d_ln_beta": torch.empty(hv, **f32),
            "d_rab_pos": torch.empty(rab_pos.numel(), **f32), "d_rab_time": torch.empty(rab_time.numel(), **f32)}
     if workspace is None:

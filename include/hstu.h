@@ -88,6 +88,13 @@ typedef struct {
     hstu_attn_desc attn;      /* attention part; dtype also types x, w1, b1, w2, b2, y */
     int32_t d_model;          /* D: width of X and Y (a multiple of 32 for bf16) */
     float ln_eps;             /* LayerNorm epsilon (1e-5 in the workloads) */
+    /* Input of the output projection.  0: G = LayerNorm(O) U, H d_v wide, as in
+     * the layer equation.  1: the concatenation [U | O | G], 3 H d_v wide (the
+     * output-projection row of Table 7 on the DLRMv4 page counts that width; the
+     * pages do not name the blocks, these are the layer's three H d_v-wide
+     * tensors at that point), so that Y = U W2[0:F] + O W2[F:2F] + G W2[2F:3F]
+     * + b2 with F = H d_v.  w2 and dw2 are then [3 H d_v, D]. */
+    int32_t output_concat;
 } hstu_layer_desc;
 
 /* Human-readable name of a status code (static string). */
@@ -133,7 +140,8 @@ hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void 
 
 /*
  * One transduction layer forward.  x [T, D]; w1 [D, H(2 d_v + 2 d_qk)];
- * b1 [H(2 d_v + 2 d_qk)]; w2 [H d_v, D]; b2 [D] (dtype of the desc);
+ * b1 [H(2 d_v + 2 d_qk)]; w2 [H d_v, D] ([3 H d_v, D] with output_concat);
+ * b2 [D] (dtype of the desc);
  * ln_gamma, ln_beta float32 [H d_v]; y [T, D] (overwritten).
  * saved_uvqk [T, H(2 d_v + 2 d_qk)] and saved_o [T, H d_v] are optional
  * (NULL = not kept); when given they receive SiLU(X W1 + b1) and the
@@ -159,9 +167,10 @@ hstu_status hstu_layer_bwd_workspace_size(const hstu_layer_desc *desc, size_t *b
  * Inputs: the forward's x, w1, b1, w2, ln_gamma, ln_beta, bias tables and
  * sequence data; saved_uvqk = SiLU(X W1 + b1) and saved_o = the attention
  * output, as hstu_layer_fwd keeps them; dy [T, D] (bf16).
- * Outputs (all overwritten): dx [T, D] (bf16); dw1 [D, W], db1 [W], dw2 [H d_v, D],
- * db2 [D], d_ln_gamma, d_ln_beta [H d_v], d_rab_pos [pos_hi - pos_lo + 1],
- * d_rab_time [NB] (all float32; W = H(2 d_v + 2 d_qk)).
+ * Outputs (all overwritten): dx [T, D] (bf16); dw1 [D, W], db1 [W],
+ * dw2 [H d_v, D] ([3 H d_v, D] with output_concat), db2 [D], d_ln_gamma,
+ * d_ln_beta [H d_v], d_rab_pos [pos_hi - pos_lo + 1], d_rab_time [NB] (all
+ * float32; W = H(2 d_v + 2 d_qk)).
  * The pre-activation X W1 + b1 is recomputed (its SiLU derivative is applied
  * in that GEMM's epilogue), and G = LayerNorm(O) U from saved_o and U.
  * Requires D, H d_v and W multiples of 128 (HSTU_ERR_UNSUPPORTED otherwise);

@@ -42,13 +42,15 @@ def test_struct_layout_matches_header(tmp_path):
         ' offsetof(hstu_attn_desc,total_tokens), offsetof(hstu_attn_desc,inv_n),'
         ' offsetof(hstu_attn_desc,debug_checks), sizeof(hstu_layer_desc),'
         ' offsetof(hstu_layer_desc,ln_eps)); printf("%zu %zu\\n", offsetof(hstu_attn_desc,local_window),'
-        ' offsetof(hstu_attn_desc,global_window)); return 0;}\n')
+        ' offsetof(hstu_attn_desc,global_window)); printf("%zu\\n", offsetof(hstu_layer_desc,output_concat));'
+        ' return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
     D, L = ops.hstu_attn_desc, ops.hstu_layer_desc
     assert got == [ctypes.sizeof(D), D.total_tokens.offset, D.inv_n.offset, D.debug_checks.offset,
-                   ctypes.sizeof(L), L.ln_eps.offset, D.local_window.offset, D.global_window.offset]
+                   ctypes.sizeof(L), L.ln_eps.offset, D.local_window.offset, D.global_window.offset,
+                   L.output_concat.offset]
 
 
 def test_status_strings_and_version():
@@ -114,6 +116,11 @@ def test_layer_descriptor_checks():
     assert lib.hstu_layer_workspace_size(ctypes.byref(bad_d), ctypes.byref(n)) == 2
     bad_eps = ops.hstu_layer_desc(_desc(), 128, -1.0)
     assert lib.hstu_layer_workspace_size(ctypes.byref(bad_eps), ctypes.byref(n)) == 1
+    plain = n.value if lib.hstu_layer_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == 0 else None
+    cat = ops.hstu_layer_desc(_desc(num_heads=4, d_qk=128, d_v=128), 512, 1e-5, 1)
+    assert lib.hstu_layer_workspace_size(ctypes.byref(cat), ctypes.byref(n)) == 0 and n.value == plain
+    bad_cat = ops.hstu_layer_desc(_desc(num_heads=4, d_qk=128, d_v=128), 512, 1e-5, 2)
+    assert lib.hstu_layer_workspace_size(ctypes.byref(bad_cat), ctypes.byref(n)) == 1
 
 
 def test_library_has_no_oracle_dependency():
