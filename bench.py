@@ -276,6 +276,48 @@ def layer_stack_timing(dev, stream, reps: int = 3):
         torch.cuda.synchronize()
         cat_ms[name] = e0.elapsed_time(e1) / reps
 
+    # FP8 projections: the same stack with E4M3 f1 and f2 (weights quantised once,
+    # activations per row inside each layer call)
+    packs = [(ops.quantize_weight_e4m3(l[0]), ops.quantize_weight_e4m3(l[2])) for l in layers]
+    desc8 = ops.hstu_layer_desc(attn0, w.d_model, 1e-5, 0, 1)
+    ws8 = ops.alloc_workspace(ops.hstu_layer_workspace_size(desc8), dev)
+
+    def fp8_forward():
+        for li, (w1_, b1_, w2_, b2_, g_, be_) in enumerate(layers):
+            ops.hstu_layer_fwd(xs[li], packs[li][0], b1_, packs[li][1], b2_, g_, be_, off, ts, None, rp, rt,
+                               y=xs[li + 1], workspace=ws8, stream=stream, fp8_projections=True, **kw)
+
+    fp8_forward()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        fp8_forward()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    fp8_ms = e0.elapsed_time(e1) / reps
+    # the f1 GEMM alone in E4M3 ([T, D] x [D, W], bias + SiLU epilogue): 20 launches from a CUDA graph
+    W1n = w.num_heads * (2 * w.d_v + 2 * w.d_qk)
+    xq, sxq = ops.quantize_rows_e4m3(xs[0])
+    wsg = ops.alloc_workspace(256, dev)
+    graph, n_g = torch.cuda.CUDAGraph(), 20
+    ops.gemm_e4m3(xq, sxq, packs[0][0], W1n, bias=layers[0][1], apply_silu=True, y=uvqk, workspace=wsg,
+                  stream=stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream()
+        for _ in range(n_g):
+            ops.gemm_e4m3(xq, sxq, packs[0][0], W1n, bias=layers[0][1], apply_silu=True, y=uvqk, workspace=wsg,
+                          stream=cs)
+    graph.replay()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    graph.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    f1_fp8_ms = g0.elapsed_time(g1) / n_g
+    del graph
+
     pairs = flops.attn_pairs(a.lengths)
     bwd_fl = flops.layer_bwd_gemm_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
         flops.attn_bwd_flops(pairs, w.num_heads, w.d_qk, w.d_v)
@@ -290,6 +332,12 @@ def layer_stack_timing(dev, stream, reps: int = 3):
             "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
             "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v),
             "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12},
+            "fp8_projections": {
+                "what": "the stack forward with E4M3 f1 and f2 (per-row activation, per-column weight scales)",
+                "ms_per_forward": fp8_ms, "speedup_vs_bf16": ms / fp8_ms,
+                "f1_gemm": {"shape": [T, w.d_model, W1n], "us": f1_fp8_ms * 1e3,
+                            "tflops": flops.f1_flops(T, w.d_model, w.num_heads, w.d_qk, w.d_v) / (f1_fp8_ms * 1e-3) / 1e12,
+                            "timing": "20 launches in one CUDA graph"}},
             "output_concat": {
                 "what": "first layer with the output projection over [U | O | G] (3 H d_v = %d wide)" % (3 * hv),
                 "fwd_ms": cat_ms["fwd"], "bwd_ms": cat_ms["bwd"],

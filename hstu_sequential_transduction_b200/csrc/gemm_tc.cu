@@ -59,6 +59,7 @@ struct GemmArgs {
     int64_t M;
     int N, K, silu, splits;
     int a_seg;                  // > 0: A is three stored matrices of a_seg columns each
+    const float *sa, *sb;       // E4M3 operands: scale of each row of A and of each column of B
     WsHeader *hdr;
 };
 
@@ -72,7 +73,7 @@ __device__ __forceinline__ float silu_grad_tanh(float z)
 
 // Persistent: CTA c takes work units c, c + gridDim.x, ...; unit = (tile, k split),
 // tiles row-block major so consecutive tiles reuse the same A rows from L2.
-template <int BN, bool A_MN, bool B_K, int EPI>
+template <int BN, bool A_MN, bool B_K, int EPI, bool F8>
 __global__ void __launch_bounds__(kThreadsG, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
@@ -84,7 +85,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nk = (g.K + GBK - 1) / GBK;  // the TMA zero-fills past K
+    constexpr int KE = F8 ? 128 : GBK;     // K elements per 128-byte slice
+    const int nk = (g.K + KE - 1) / KE;    // the TMA zero-fills past K
     const int per = (nk + g.splits - 1) / g.splits;  // k-slices per split
     const int tiles_n = g.N / BN;
     const int tiles = (int)((g.M + GBM - 1) / GBM) * tiles_n;
@@ -152,25 +154,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         for (int r = 0; r < 2; r++) {
                             int xl;
                             const CUtensorMap *ma = a_map(m0 + 64 * r, xl);
-                            tma_load_2d(sa + r * kReg64, ma, xl, kt * GBK, full_bar(s));
+                            tma_load_2d(sa + r * kReg64, ma, xl, kt * KE, full_bar(s));
                         }
                     } else {
                         int xl;
-                        const CUtensorMap *ma = a_map(kt * GBK, xl);
+                        const CUtensorMap *ma = a_map(kt * KE, xl);
                         tma_load_2d(sa, ma, xl, m0, full_bar(s));
                     }
                     if (B_K) {
-                        tma_load_2d(sb, &tmB, kt * GBK, n0, full_bar(s));
+                        tma_load_2d(sb, &tmB, kt * KE, n0, full_bar(s));
                     } else {
                         for (int r = 0; r < BN / 64; r++)
-                            tma_load_2d(sb + r * kReg64, &tmB, n0 + 64 * r, kt * GBK, full_bar(s));
+                            tma_load_2d(sb + r * kReg64, &tmB, n0 + 64 * r, kt * KE, full_bar(s));
                     }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(GBM, BN, A_MN ? 1 : 0, B_K ? 0 : 1);
+            constexpr uint32_t idesc =
+                F8 ? idesc_e4m3(GBM, BN, A_MN ? 1 : 0, B_K ? 0 : 1) : idesc_bf16(GBM, BN, A_MN ? 1 : 0, B_K ? 0 : 1);
             int it = 0, lt = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, lt++) {
@@ -186,13 +189,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     if (!(ok = mbar_wait(full_bar(s), (it / GSTAGES) & 1, abort_flag, g.hdr)))
                         break;
                     tc_fence_after();
-                    for (int ks = 0; ks < GBK / 16; ks++) {
+                    // four 32-byte k-steps per slice: K = 16 bf16 or K = 32 E4M3 each
+                    for (int ks = 0; ks < 4; ks++) {
                         const uint32_t sa = base + LY::A + s * kRegA, sb = base + LY::B + s * BN * 128;
                         const uint64_t a = A_MN ? smem_desc_sw128(sa + ks * 2048, kReg64, 1024)
                                                 : smem_desc_sw128(sa + ks * 32, 16, 1024);
                         const uint64_t b = B_K ? smem_desc_sw128(sb + ks * 32, 16, 1024)
                                                : smem_desc_sw128(sb + ks * 2048, kReg64, 1024);
-                        umma_bf16(tmem + ab * BN, a, b, idesc, (kt > k0 || ks > 0));
+                        if (F8)
+                            umma_e4m3(tmem + ab * BN, a, b, idesc, (kt > k0 || ks > 0));
+                        else
+                            umma_bf16(tmem + ab * BN, a, b, idesc, (kt > k0 || ks > 0));
                     }
                     umma_commit(empty_bar(s));
                 }
@@ -219,8 +226,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int cc = 0; cc < CW; cc += 32) {
                 float v[32];
                 tmem_ld32(trow + ab * BN + half * CW + cc, v);
-                tmem_wait_ld();
                 if (EPI == EPI_RED) {
+                    tmem_wait_ld();
                     // [32 rows x 32 columns] fp32 box, 128-byte swizzled, two buffers per warp
                     if (k1 <= k0)
                         continue;  // an empty split adds nothing
@@ -242,29 +249,57 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     nstage++;
                     continue;
                 }
-                if (row < g.M) {
+                // the chunk's bias (and E4M3 column scales, and the dSiLU factor row)
+                // are fetched while the TMEM load is in flight
+                const bool live = row < g.M;
+                uint4 bw[4], aw[4];
+                float4 sc[8];
+                const bool bias_vec = (reinterpret_cast<uintptr_t>(g.bias) & 15u) == 0;
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    if (!g.bias) {
+                        bw[u] = make_uint4(0, 0, 0, 0);
+                    } else if (bias_vec) {
+                        bw[u] = reinterpret_cast<const uint4 *>(g.bias + n0 + cc)[u];
+                    } else {
+                        const unsigned short *b16 = reinterpret_cast<const unsigned short *>(g.bias + n0 + cc + 8 * u);
+                        bw[u] = make_uint4(b16[0] | ((uint32_t)b16[1] << 16), b16[2] | ((uint32_t)b16[3] << 16),
+                                           b16[4] | ((uint32_t)b16[5] << 16), b16[6] | ((uint32_t)b16[7] << 16));
+                    }
+                    if (EPI == EPI_DSILU)
+                        aw[u] = live ? reinterpret_cast<const uint4 *>(g.aux + row * g.ldaux + n0 + cc)[u]
+                                     : make_uint4(0, 0, 0, 0);
+                }
+                if (F8) {
+#pragma unroll
+                    for (int u = 0; u < 8; u++)
+                        sc[u] = reinterpret_cast<const float4 *>(g.sb + n0 + cc)[u];
+                }
+                const float rs = F8 && live ? g.sa[row] : 1.f;
+                tmem_wait_ld();
+                if (live) {
                     __nv_bfloat16 *crow = static_cast<__nv_bfloat16 *>(g.C) + row * g.ldc + n0;
-                    const __nv_bfloat16 *arow = EPI == EPI_DSILU ? g.aux + row * g.ldaux + n0 : nullptr;
 #pragma unroll
                     for (int u4 = 0; u4 < 4; u4++) {
+                        const uint32_t bb[4] = {bw[u4].x, bw[u4].y, bw[u4].z, bw[u4].w};
+                        const uint32_t ab4[4] = {aw[u4].x, aw[u4].y, aw[u4].z, aw[u4].w};
                         float x[8];
-                        float da[8];
-                        if (EPI == EPI_DSILU) {
-                            const uint4 w = *reinterpret_cast<const uint4 *>(arow + cc + 8 * u4);
-                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; e++) {
-                                da[2 * e] = __uint_as_float(ww[e] << 16);
-                                da[2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
-                            }
-                        }
 #pragma unroll
                         for (int e = 0; e < 8; e++) {
-                            x[e] = v[8 * u4 + e] + (g.bias ? __bfloat162float(g.bias[n0 + cc + 8 * u4 + e]) : 0.f);
-                            if (EPI == EPI_DSILU)
-                                x[e] = da[e] * silu_grad_tanh(x[e]);
-                            else if (g.silu)
+                            const float bias = __uint_as_float(e & 1 ? bb[e >> 1] & 0xffff0000u : bb[e >> 1] << 16);
+                            float acc = v[8 * u4 + e];
+                            if (F8) {
+                                const float4 s4 = sc[(8 * u4 + e) >> 2];
+                                const int q = e & 3;
+                                acc *= rs * (q == 0 ? s4.x : q == 1 ? s4.y : q == 2 ? s4.z : s4.w);
+                            }
+                            x[e] = acc + bias;
+                            if (EPI == EPI_DSILU) {
+                                const float da = __uint_as_float(e & 1 ? ab4[e >> 1] & 0xffff0000u : ab4[e >> 1] << 16);
+                                x[e] = da * silu_grad_tanh(x[e]);
+                            } else if (g.silu) {
                                 x[e] = silu_fast(x[e]);
+                            }
                         }
                         uint4 w;
                         w.x = pack_bf16(x[0], x[1]);
@@ -302,7 +337,7 @@ int num_sms()
     return n;
 }
 
-template <int BN, bool A_MN, bool B_K, int EPI>
+template <int BN, bool A_MN, bool B_K, int EPI, bool F8 = false>
 cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stream)
 {
     CUtensorMap ma, ma1, ma2, mb, mc;
@@ -311,7 +346,10 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
     const int64_t ald[3] = {op.lda, op.lda1, op.lda2};
     CUtensorMap *amap[3] = {&ma, &ma1, &ma2};
     for (int i = 0; i < (g.a_seg ? 3 : 1) && e == cudaSuccess; i++) {
-        if (A_MN)  // stored [K, M]: box 64 m x 64 k
+        if (F8)    // E4M3 [M, K]: box 128 k x 128 m
+            e = make_tensor_map_2d(amap[i], abase[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, g.M, g.K, ald[i], 128, GBM,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+        else if (A_MN)  // stored [K, M]: box 64 m x 64 k
             e = make_tensor_map_2d(amap[i], abase[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.K,
                                    g.a_seg ? g.a_seg : g.M, ald[i] * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
         else       // [M, K]: box 64 k x 128 m
@@ -321,7 +359,10 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
     if (!g.a_seg)
         ma1 = ma2 = ma;  // unused
     if (e == cudaSuccess) {
-        if (B_K)  // stored [N, K]: box 64 k x BN n
+        if (F8)   // E4M3 stored [N, K]: box 128 k x BN n
+            e = make_tensor_map_2d(&mb, op.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.N, g.K, op.ldb, 128, BN,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+        else if (B_K)  // stored [N, K]: box 64 k x BN n
             e = make_tensor_map_2d(&mb, op.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.N, g.K, op.ldb * 2, 64, BN,
                                    CU_TENSOR_MAP_SWIZZLE_128B);
         else      // [K, N]: box 64 n x 64 k
@@ -338,13 +379,13 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
     if (e != cudaSuccess)
         return e;
     const size_t bytes = GL<BN, EPI>::BYTES + 1024;
-    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, A_MN, B_K, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, A_MN, B_K, EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess)
         return e;
     const int64_t units = ((g.M + GBM - 1) / GBM) * (g.N / BN) * g.splits;
     const unsigned grid = (unsigned)std::min<int64_t>(units, num_sms());
-    gemm_tc_kernel<BN, A_MN, B_K, EPI><<<grid, kThreadsG, bytes, stream>>>(ma, ma1, ma2, mb, mc, g);
+    gemm_tc_kernel<BN, A_MN, B_K, EPI, F8><<<grid, kThreadsG, bytes, stream>>>(ma, ma1, ma2, mb, mc, g);
     return cudaGetLastError();
 }
 
@@ -409,6 +450,43 @@ cudaError_t launch_gemm_tc_ex(const GemmOperands &op, int64_t M, int N, int K, G
         return N % 256 == 0 ? gemm_dispatch_layout<256, EPI_ACT>(op, g, stream)
                             : gemm_dispatch_layout<128, EPI_ACT>(op, g, stream);
     }
+}
+
+bool gemm_e4m3_ok(const void *A, int64_t lda, const void *B, int64_t ldb, const void *C, int64_t ldc, int64_t M,
+                  int N, int K)
+{
+    const bool aligned = ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+                           reinterpret_cast<uintptr_t>(C)) & 15u) == 0;
+    return aligned && M > 0 && M < ((int64_t)1 << 31) - GBM && N > 0 && N % 128 == 0 && K > 0 && K % 16 == 0 &&
+           lda % 16 == 0 && ldb % 16 == 0 && ldc % 8 == 0;
+}
+
+cudaError_t launch_gemm_e4m3(const void *A, int64_t lda, const float *sa, const void *B, int64_t ldb,
+                             const float *sb, const void *bias, void *C, int64_t ldc, int64_t M, int N, int K,
+                             bool silu, WsHeader *hdr, cudaStream_t stream)
+{
+    if (M == 0)
+        return cudaSuccess;
+    GemmOperands op{};
+    op.A = A;
+    op.lda = lda;
+    op.B = B;
+    op.ldb = ldb;
+    op.b_k = true;
+    GemmArgs g{};
+    g.bias = static_cast<const __nv_bfloat16 *>(bias);
+    g.C = C;
+    g.ldc = ldc;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.silu = silu;
+    g.splits = 1;
+    g.sa = sa;
+    g.sb = sb;
+    g.hdr = hdr;
+    return N % 256 == 0 ? gemm_tc_launch<256, false, true, EPI_ACT, true>(op, g, stream)
+                        : gemm_tc_launch<128, false, true, EPI_ACT, true>(op, g, stream);
 }
 
 bool gemm_tc_supported(const void *A, int64_t lda, const void *Bm, void *C, int64_t ldc, int64_t M, int N, int K)

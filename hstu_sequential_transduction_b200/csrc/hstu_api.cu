@@ -271,8 +271,10 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_attn_desc(&d->attn));
     if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps) ||
-        (d->output_concat != 0 && d->output_concat != 1))
+        (d->output_concat != 0 && d->output_concat != 1) || (d->fp8_projections != 0 && d->fp8_projections != 1))
         return HSTU_ERR_INVALID_ARG;
+    if (d->fp8_projections && (d->attn.dtype != HSTU_BF16 || d->output_concat || d->d_model % 128))
+        return HSTU_ERR_UNSUPPORTED;
     const int F = d->attn.num_heads * d->attn.d_v;
     if (F != 64 && F != 128 && F != 256 && F != 512 && F != 1024)
         return HSTU_ERR_UNSUPPORTED;
@@ -302,6 +304,8 @@ static size_t layer_ws(const hstu_layer_desc *d, bool keep_uvqk, bool keep_o)
     b += align256(T * a->num_heads * a->d_v * eb);  // G
     if (layer_cat_copy(d))
         b += align256(T * 3 * a->num_heads * a->d_v * eb);  // [U | O | G]
+    if (d->fp8_projections)  // E4M3 codes and row scales of X and of G
+        b += align256(T * d->d_model) + align256(T * 4) + align256(T * a->num_heads * a->d_v) + align256(T * 4);
     return b;
 }
 
@@ -352,6 +356,26 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
     char *g = cur;
 
     WsHeader *hdr = static_cast<WsHeader *>(workspace);
+    if (desc->fp8_projections) {
+        // X and G quantised per row; W1, W2 are E4M3 packs [N][K] + scales
+        char *xq = g + align256(T * hv * eb);
+        float *sx = reinterpret_cast<float *>(xq + align256(T * D));
+        char *gq = reinterpret_cast<char *>(sx) + align256(T * 4);
+        float *sg = reinterpret_cast<float *>(gq + align256(T * hv));
+        const float *s1 = reinterpret_cast<const float *>(static_cast<const char *>(w1) + align256((size_t)W * D));
+        const float *s2 = reinterpret_cast<const float *>(static_cast<const char *>(w2) + align256((size_t)D * hv));
+        if (!gemm_e4m3_ok(xq, D, w1, D, uvqk, W, (int64_t)T, W, D) ||
+            !gemm_e4m3_ok(gq, hv, w2, hv, y, D, (int64_t)T, D, hv))
+            return HSTU_ERR_UNSUPPORTED;
+        HSTU_CUDA(launch_quantize_rows_e4m3(x, D, (int64_t)T, D, xq, D, sx, st));
+        HSTU_CUDA(launch_gemm_e4m3(xq, D, sx, w1, D, s1, b1, uvqk, W, (int64_t)T, W, D, true, hdr, st));
+        HSTU_TRY(attn_fwd_strided(a, uvqk + (size_t)2 * hv * eb, W, uvqk + (size_t)(2 * hv + hq) * eb, W,
+                                  uvqk + (size_t)hv * eb, W, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                                  o, hv, workspace, st));
+        HSTU_CUDA(launch_norm_gate(true, o, hv, uvqk, W, ln_gamma, ln_beta, desc->ln_eps, g, hv, (int64_t)T, hv, st));
+        HSTU_CUDA(launch_quantize_rows_e4m3(g, hv, (int64_t)T, hv, gq, hv, sg, st));
+        return cuda_status(launch_gemm_e4m3(gq, hv, sg, w2, hv, s2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
+    }
     if (bf16 && gemm_tc_supported(x, D, w1, uvqk, W, (int64_t)T, W, D))
         HSTU_CUDA(launch_gemm_tc(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, hdr, st));
     else if (bf16)
@@ -583,6 +607,51 @@ hstu_status hstu_jagged_truncate(int32_t num_seqs, int64_t total_tokens, int32_t
         return HSTU_ERR_INVALID_ARG;
     return cuda_status(launch_jagged_truncate(seq_offsets, num_targets, num_seqs, total_tokens, keep, row_bytes,
                                               in, out, out_offsets, static_cast<cudaStream_t>(stream)));
+}
+
+size_t hstu_e4m3_weight_bytes(int32_t K, int32_t N)
+{
+    if (K < 0 || N < 0)
+        return 0;
+    return align256((size_t)K * N) + (size_t)N * 4;
+}
+
+hstu_status hstu_quantize_weight_e4m3(const void *w, int32_t K, int32_t N, void *pack, void *stream)
+{
+    if (K <= 0 || N <= 0 || K % 16 || !w || !pack || !aligned16(w) || !aligned16(pack))
+        return HSTU_ERR_INVALID_ARG;
+    float *scales = reinterpret_cast<float *>(static_cast<char *>(pack) + align256((size_t)K * N));
+    return cuda_status(launch_quantize_cols_e4m3(w, K, N, pack, scales, static_cast<cudaStream_t>(stream)));
+}
+
+hstu_status hstu_quantize_rows_e4m3(const void *x, int64_t rows, int32_t K, void *codes, float *scales,
+                                    void *stream)
+{
+    if (rows < 0 || K <= 0 || K % 16)
+        return HSTU_ERR_INVALID_ARG;
+    if (rows > 0 && (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)))
+        return HSTU_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_rows_e4m3(x, K, rows, K, codes, K, scales, static_cast<cudaStream_t>(stream)));
+}
+
+hstu_status hstu_gemm_e4m3(const void *codes, const float *scales, int64_t M, int32_t K, const void *wpack,
+                           int32_t N, const void *bias, int32_t apply_silu, void *y, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    if (M < 0 || K <= 0 || N <= 0 || !wpack)
+        return HSTU_ERR_INVALID_ARG;
+    HSTU_TRY(check_ws(workspace, workspace_bytes, sizeof(WsHeader)));
+    if (M == 0)
+        return HSTU_OK;
+    if (!codes || !scales || !y)
+        return HSTU_ERR_INVALID_ARG;
+    if (!gemm_e4m3_ok(codes, K, wpack, K, y, N, M, N, K))
+        return (aligned16(codes) && aligned16(wpack) && aligned16(y)) ? HSTU_ERR_UNSUPPORTED : HSTU_ERR_INVALID_ARG;
+    const float *ws = reinterpret_cast<const float *>(static_cast<const char *>(wpack) + align256((size_t)K * N));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    HSTU_CUDA(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st));
+    return cuda_status(launch_gemm_e4m3(codes, K, scales, wpack, K, ws, bias, y, N, M, N, K, apply_silu != 0,
+                                        static_cast<WsHeader *>(workspace), st));
 }
 
 hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream)

@@ -95,6 +95,22 @@ bool gemm_tc_ok(const GemmOperands &op, int64_t M, int N, int K);
 cudaError_t launch_gemm_tc_ex(const GemmOperands &op, int64_t M, int N, int K, GemmEpilogue epi, bool silu,
                               int splits, WsHeader *hdr, cudaStream_t stream);
 
+// E4M3 GEMM on tcgen05 (kind::f8f6f4): C bf16 [M, N] = (A B^T) * sa[m] * sb[n]
+// + bias[n], optionally SiLU.  A codes [M, K] (row stride lda bytes), B codes
+// [N, K] (row stride ldb bytes), both K-major; sa [M], sb [N] float32.
+bool gemm_e4m3_ok(const void *A, int64_t lda, const void *B, int64_t ldb, const void *C, int64_t ldc, int64_t M,
+                  int N, int K);
+cudaError_t launch_gemm_e4m3(const void *A, int64_t lda, const float *sa, const void *B, int64_t ldb,
+                             const float *sb, const void *bias, void *C, int64_t ldc, int64_t M, int N, int K,
+                             bool silu, WsHeader *hdr, cudaStream_t stream);
+// Per-row E4M3 quantisation of a bf16 [R, K] matrix (row stride ldx elements):
+// codes [R, K] (row stride ldq bytes) and scales [R]; K a multiple of 8.
+cudaError_t launch_quantize_rows_e4m3(const void *x, int64_t ldx, int64_t R, int K, void *q, int64_t ldq,
+                                      float *scale, cudaStream_t stream);
+// Per-column E4M3 quantisation of a bf16 weight [K, N]: codes [N, K] (the
+// transpose) and scales [N].
+cudaError_t launch_quantize_cols_e4m3(const void *w, int64_t K, int N, void *q, float *scale, cudaStream_t stream);
+
 // G[t, :] = LayerNorm(O[t, :]) * U[t, :] over F features.
 cudaError_t launch_norm_gate(bool bf16, const void *O, int64_t ldo, const void *U, int64_t ldu,
                              const float *gamma, const float *beta, float eps, void *G,

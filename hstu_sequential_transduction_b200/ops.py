@@ -27,7 +27,8 @@ EXPORTED = ["hstu_status_string", "hstu_version", "hstu_attn_workspace_size",
             "hstu_layer_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd",
             "hstu_check_device_flag", "hstu_debug_bias_indices", "hstu_debug_schedule",
             "hstu_attn_fwd_noalloc", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
-            "hstu_jagged_truncate"]
+            "hstu_jagged_truncate", "hstu_quantize_weight_e4m3", "hstu_quantize_rows_e4m3", "hstu_gemm_e4m3",
+            "hstu_e4m3_weight_bytes"]
 
 
 class HstuError(RuntimeError):
@@ -47,7 +48,7 @@ class hstu_attn_desc(ctypes.Structure):
 
 class hstu_layer_desc(ctypes.Structure):
     _fields_ = [("attn", hstu_attn_desc), ("d_model", ctypes.c_int32), ("ln_eps", ctypes.c_float),
-                ("output_concat", ctypes.c_int32)]
+                ("output_concat", ctypes.c_int32), ("fp8_projections", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -74,6 +75,8 @@ def load_library(allow_build: bool = True) -> ctypes.CDLL:
             lib.hstu_version.restype = ctypes.c_int
             for name in EXPORTED[2:]:
                 getattr(lib, name).restype = ctypes.c_int
+            lib.hstu_e4m3_weight_bytes.restype = ctypes.c_size_t
+            lib.hstu_e4m3_weight_bytes.argtypes = [ctypes.c_int32, ctypes.c_int32]
             _lib = lib
     return _lib
 
@@ -221,18 +224,28 @@ def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
 def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets,
                    rab_pos, rab_time, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, y=None,
-                   saved_uvqk=None, saved_o=None, workspace=None, stream=None, output_concat: bool = False):
+                   saved_uvqk=None, saved_o=None, workspace=None, stream=None, output_concat: bool = False,
+                   fp8_projections: bool = False):
     """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer; with
-    output_concat, f2 reads [U | O | G] and w2 is [3 H d_v, D]."""
-    for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("b2", b2)):
+    output_concat, f2 reads [U | O | G] and w2 is [3 H d_v, D]; with
+    fp8_projections, w1 and w2 are E4M3 weight packs (quantize_weight_e4m3)."""
+    for name, t in (("x", x), ("b1", b1), ("b2", b2)) + (() if fp8_projections else (("w1", w1), ("w2", w2))):
         _dev(t, name, x.dtype)
+    if fp8_projections:
+        _dev(w1, "w1", torch.uint8)
+        _dev(w2, "w2", torch.uint8)
     _dev(ln_gamma, "ln_gamma", torch.float32)
     _dev(ln_beta, "ln_beta", torch.float32)
     T, D = x.shape
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
                           _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
-    desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)))
-    if w2.shape[0] != (3 if output_concat else 1) * num_heads * d_v:
+    desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)), int(bool(fp8_projections)))
+    if fp8_projections:
+        W = num_heads * (2 * d_v + 2 * d_qk)
+        for name, t, k, n in (("w1", w1, D, W), ("w2", w2, num_heads * d_v, D)):
+            if t.numel() < hstu_e4m3_weight_bytes(k, n):
+                raise ValueError(f"{name} is not an E4M3 pack of a [{k}, {n}] weight")
+    elif w2.shape[0] != (3 if output_concat else 1) * num_heads * d_v:
         raise ValueError(f"w2 has {w2.shape[0]} rows for output_concat={output_concat}")
     if y is None:
         y = torch.empty((T, D), dtype=x.dtype, device=x.device)
@@ -290,6 +303,57 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
         _ptr(out["d_rab_pos"]), _ptr(out["d_rab_time"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
         _stream(stream)))
     return out
+
+
+def hstu_e4m3_weight_bytes(K: int, N: int) -> int:
+    return int(load_library().hstu_e4m3_weight_bytes(int(K), int(N)))
+
+
+def quantize_weight_e4m3(w, stream=None):
+    """E4M3 weight pack of a bf16 weight w [K, N]: uint8 tensor holding the
+    codes [N, K] and, from byte align256(N K), the float32 scales [N]."""
+    _dev(w, "w", torch.bfloat16)
+    K, N = w.shape
+    pack = torch.empty(hstu_e4m3_weight_bytes(K, N), dtype=torch.uint8, device=w.device)
+    _check("hstu_quantize_weight_e4m3", load_library().hstu_quantize_weight_e4m3(
+        _ptr(w), ctypes.c_int32(K), ctypes.c_int32(N), _ptr(pack), _stream(stream)))
+    return pack
+
+
+def e4m3_pack_parts(pack, K: int, N: int):
+    """(codes [N, K] uint8, scales [N] float32) views of a weight pack."""
+    off = (N * K + 255) // 256 * 256
+    return pack[:N * K].view(N, K), pack[off:off + 4 * N].view(torch.float32)
+
+
+def quantize_rows_e4m3(x, stream=None):
+    """Per-row E4M3 codes [R, K] (uint8) and scales [R] (float32) of a bf16 x [R, K]."""
+    _dev(x, "x", torch.bfloat16)
+    R, K = x.shape
+    codes = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(R, dtype=torch.float32, device=x.device)
+    _check("hstu_quantize_rows_e4m3", load_library().hstu_quantize_rows_e4m3(
+        _ptr(x), ctypes.c_int64(R), ctypes.c_int32(K), _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def gemm_e4m3(codes, scales, wpack, N: int, bias=None, apply_silu: bool = False, y=None, workspace=None,
+              stream=None):
+    """bf16 y [M, N] = dequant(codes, scales) dequant(W)^T + bias (optionally SiLU)."""
+    _dev(codes, "codes", torch.uint8)
+    _dev(scales, "scales", torch.float32)
+    _dev(wpack, "wpack", torch.uint8)
+    _dev(bias, "bias", torch.bfloat16)
+    M, K = codes.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=codes.device)
+    if workspace is None:
+        workspace = alloc_workspace(256, codes.device)
+    _check("hstu_gemm_e4m3", load_library().hstu_gemm_e4m3(
+        _ptr(codes), _ptr(scales), ctypes.c_int64(M), ctypes.c_int32(K), _ptr(wpack), ctypes.c_int32(N),
+        _ptr(bias), ctypes.c_int32(int(apply_silu)), _ptr(y), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+        _stream(stream)))
+    return y
 
 
 def hstu_jagged_truncate(seq_offsets, num_targets, keep: int, rows, *, out=None, out_offsets=None,

@@ -95,6 +95,12 @@ typedef struct {
      * tensors at that point), so that Y = U W2[0:F] + O W2[F:2F] + G W2[2F:3F]
      * + b2 with F = H d_v.  w2 and dw2 are then [3 H d_v, D]. */
     int32_t output_concat;
+    /* 1: the projections f1 and f2 run in FP8 (the mixed-precision item of the
+     * ULTRA-HSTU review: matrix multiplications in FP8, the rest in bf16).  X and
+     * G are quantised per row to E4M3 inside the call; w1 and w2 are E4M3
+     * weight packs made by hstu_quantize_weight_e4m3 from the bf16 weights.
+     * Forward only, bf16 only, output_concat 0, D a multiple of 128. */
+    int32_t fp8_projections;
 } hstu_layer_desc;
 
 /* Human-readable name of a status code (static string). */
@@ -210,6 +216,39 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
 hstu_status hstu_jagged_truncate(int32_t num_seqs, int64_t total_tokens, int32_t keep,
                                  const int64_t *seq_offsets, const int32_t *num_targets, const void *in,
                                  int64_t row_bytes, void *out, int64_t *out_offsets, void *stream);
+
+/*
+ * FP8 (E4M3) projections.  Format and scaling (the pages name neither): E4M3
+ * (largest finite 448), round to nearest even with saturation; activations
+ * scaled per row and weights per output column so that the largest magnitude
+ * maps to 448: inv = 448 / amax, scale = amax / 448 (float32), code =
+ * E4M3(x * inv); an all-zero row or column has scale 1.
+ *
+ * Weight pack (device memory, hstu_e4m3_weight_bytes(K, N) bytes, 16-byte
+ * aligned): the codes of W^T, uint8 [N][K] (row n = output column n), then at
+ * byte offset align256(N K) the float32 scales [N].
+ */
+size_t hstu_e4m3_weight_bytes(int32_t K, int32_t N);
+
+/* Quantise a bf16 weight w [K, N] (row-major, device) into a weight pack.
+ * K a multiple of 16. */
+hstu_status hstu_quantize_weight_e4m3(const void *w, int32_t K, int32_t N, void *pack, void *stream);
+
+/* Quantise the rows of a bf16 matrix x [rows, K] (device, 16-byte aligned, K a
+ * multiple of 16): codes uint8 [rows, K] and scales float32 [rows] (device). */
+hstu_status hstu_quantize_rows_e4m3(const void *x, int64_t rows, int32_t K, void *codes, float *scales,
+                                    void *stream);
+
+/* y bf16 [M, N] = (dec(codes) scales) (dec(W) w_scales)^T + bias, optionally
+ * SiLU: the FP8 projection GEMM on the tensor cores (tcgen05 kind::f8f6f4,
+ * float32 accumulation).  codes [M, K] and scales [M] from
+ * hstu_quantize_rows_e4m3, wpack from hstu_quantize_weight_e4m3 (K x N),
+ * bias bf16 [N] or NULL.  N a multiple of 128, K of 16 (HSTU_ERR_UNSUPPORTED).
+ * workspace: at least 256 bytes of device memory (256-byte aligned); its flag
+ * reports a stalled pipeline through hstu_check_device_flag. */
+hstu_status hstu_gemm_e4m3(const void *codes, const float *scales, int64_t M, int32_t K, const void *wpack,
+                           int32_t N, const void *bias, int32_t apply_silu, void *y, void *workspace,
+                           size_t workspace_bytes, void *stream);
 
 /*
  * Attention forward that allocates nothing (no counterpart on the HSTU
