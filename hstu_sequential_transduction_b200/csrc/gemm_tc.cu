@@ -43,8 +43,10 @@ template <int BN, int EPI>
 struct GL {
     static constexpr int A = 0;
     static constexpr int B = A + GSTAGES * kRegA;
-    static constexpr int STG = B + GSTAGES * BN * 128;                   // EPI_RED: 2 x 4 KB per warp
-    static constexpr int BAR = STG + (EPI == EPI_RED ? kEpiWarpsG * 2 * 4096 : 0);
+    // output staging per epilogue warp: EPI_RED 2 x 4 KB fp32 boxes; otherwise one
+    // 2 KB bf16 box of 32 rows x 32 columns (64-byte swizzle) for a TMA store
+    static constexpr int STG = B + GSTAGES * BN * 128;
+    static constexpr int BAR = STG + kEpiWarpsG * (EPI == EPI_RED ? 2 * 4096 : 2048);
     static constexpr int NBAR = 2 * GSTAGES + 4;  // full, empty, acc_full[2], acc_empty[2]
     static constexpr int MISC = BAR + NBAR * 8;
     static constexpr int BYTES = MISC + 64;
@@ -62,6 +64,14 @@ struct GemmArgs {
     const float *sa, *sb;       // E4M3 operands: scale of each row of A and of each column of B
     WsHeader *hdr;
 };
+
+// SiLU(z) = h (1 + tanh h), h = z / 2: one MUFU op (tanh.approx, relative error
+// about 2^-11, below the bf16 output's rounding)
+__device__ __forceinline__ float silu_tanh(float z)
+{
+    const float h = 0.5f * z;
+    return fmaf(h, tanh_approx(h), h);
+}
 
 __device__ __forceinline__ float silu_grad_tanh(float z)
 {
@@ -277,8 +287,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 const float rs = F8 && live ? g.sa[row] : 1.f;
                 tmem_wait_ld();
-                if (live) {
-                    __nv_bfloat16 *crow = static_cast<__nv_bfloat16 *>(g.C) + row * g.ldc + n0;
+                uint4 packed[4];
+                {
 #pragma unroll
                     for (int u4 = 0; u4 < 4; u4++) {
                         const uint32_t bb[4] = {bw[u4].x, bw[u4].y, bw[u4].z, bw[u4].w};
@@ -298,16 +308,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                 const float da = __uint_as_float(e & 1 ? ab4[e >> 1] & 0xffff0000u : ab4[e >> 1] << 16);
                                 x[e] = da * silu_grad_tanh(x[e]);
                             } else if (g.silu) {
-                                x[e] = silu_fast(x[e]);
+                                x[e] = silu_tanh(x[e]);
                             }
                         }
-                        uint4 w;
-                        w.x = pack_bf16(x[0], x[1]);
-                        w.y = pack_bf16(x[2], x[3]);
-                        w.z = pack_bf16(x[4], x[5]);
-                        w.w = pack_bf16(x[6], x[7]);
-                        *reinterpret_cast<uint4 *>(crow + cc + 8 * u4) = w;
+                        packed[u4] = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                                pack_bf16(x[6], x[7]));
                     }
+                }
+                // this warp's 32 rows x 32 columns through shared memory and one TMA
+                // store (coalesced; rows past M are dropped by the tensor map)
+                unsigned char *stg = sm + LY::STG + ew * 2048;
+                if (lane == 0)
+                    bulk_wait_read0();  // the previous box has been read out
+                __syncwarp();
+#pragma unroll
+                for (int u4 = 0; u4 < 4; u4++)
+                    *reinterpret_cast<uint4 *>(stg + lane * 64 + ((u4 ^ ((lane >> 1) & 3)) << 4)) = packed[u4];
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, n0 + cc, (int)rowbase, smem_u32(stg));
+                    bulk_commit();
                 }
             }
             tc_fence_before();
@@ -315,7 +336,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (lane == 0)
                 mbar_arrive(acce_bar(ab));
         }
-        if (EPI == EPI_RED && lane == 0)
+        if (lane == 0)
             bulk_wait0();
     }
     tc_fence_before();
@@ -373,8 +394,9 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
         if (EPI == EPI_RED)  // fp32 [M, N]: box 32 columns x 32 rows, 128-byte swizzle
             e = make_tensor_map_2d(&mc, op.C32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.M, g.N, g.ldc * 4, 32, 32,
                                    CU_TENSOR_MAP_SWIZZLE_128B);
-        else
-            mc = mb;  // unused
+        else                 // bf16 [M, N]: box 32 columns x 32 rows, 64-byte swizzle
+            e = make_tensor_map_2d(&mc, g.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.M, g.N, g.ldc * 2, 32, 32,
+                                   CU_TENSOR_MAP_SWIZZLE_64B);
     }
     if (e != cudaSuccess)
         return e;

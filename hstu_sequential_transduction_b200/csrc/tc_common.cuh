@@ -284,6 +284,15 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x,
         : "memory");
 }
 
+// 2-D tiled store of a shared-memory box to global memory (rows past the tensor are dropped).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
 
 // Wait until the issuing thread's bulk groups have finished reading shared memory.
