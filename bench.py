@@ -345,6 +345,93 @@ def layer_stack_timing(dev, stream, reps: int = 3):
                 "bwd_tflops": (bwd_fl + 2 * f2_extra) / (cat_ms["bwd"] * 1e-3) / 1e12}}
 
 
+def config_timings(dev, stream, reps: int = 10):
+    """Secondary measurements on the other attention configurations: the short
+    bf16 batch (32 sequences, U[64,1024], 4 heads, d = 64) forward and backward,
+    and the ranking batch (16 users x (2048 history + 512 candidates), 2 heads,
+    d = 128) attention forward and layer forward.  CUDA events, warm."""
+    import numpy as np
+    import torch
+
+    from hstu_sequential_transduction_b200 import flops, ops, workloads
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    out = {}
+    inp = workloads.generate(workloads.WORKLOADS["attn_bf16_short"])
+    d = {k: getattr(inp, k).to(dev) for k in ("q", "k", "v", "seq_offsets", "timestamps", "rab_pos", "rab_time",
+                                              "dout")}
+    kw = dict(max_seq_len=inp.max_seq_len, inv_n=inp.inv_n, pos_lo=inp.pos_lo, pos_hi=inp.pos_hi)
+    ws_f = ops.alloc_workspace(ops.hstu_attn_workspace_size(
+        ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi,
+                            d["rab_time"]), False), dev)
+    ws_b = ops.alloc_workspace(ops.hstu_attn_workspace_size(
+        ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi,
+                            d["rab_time"]), True), dev)
+    o = torch.empty_like(d["v"])
+    f_ms = timed(lambda: ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None,
+                                           d["rab_pos"], d["rab_time"], out=o, workspace=ws_f, stream=stream, **kw))
+    b_ms = timed(lambda: ops.hstu_attn_bwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None,
+                                           d["rab_pos"], d["rab_time"], d["dout"], workspace=ws_b, stream=stream,
+                                           **kw))
+    pairs = flops.attn_pairs(inp.lengths)
+    H, dq_, dv_ = d["q"].shape[1], d["q"].shape[2], d["v"].shape[2]
+    ff, bf = flops.attn_fwd_flops(pairs, H, dq_, dv_), flops.attn_bwd_flops(pairs, H, dq_, dv_)
+    out["attn_bf16_short"] = {"tokens": inp.total_tokens, "visible_pairs_per_head": pairs,
+                              "fwd_ms": f_ms, "fwd_tflops": ff / (f_ms * 1e-3) / 1e12,
+                              "bwd_ms": b_ms, "bwd_tflops": bf / (b_ms * 1e-3) / 1e12,
+                              "fwd_input_gbs": 4 * inp.total_tokens * H * dq_ * 2 / (f_ms * 1e-3) / 1e9}
+
+    w = workloads.WORKLOADS["ranking_bf16"]
+    lay = workloads.generate(w)
+    a = lay.attn
+    rng = np.random.default_rng(7)
+    att = workloads.make_attn_inputs(rng, a.lengths, w.num_heads, w.d_qk, w.d_v, w.gap_mean_s, w.pos_lo, w.pos_hi,
+                                     w.num_time_buckets, w.n_scale, torch.bfloat16,
+                                     num_targets=a.num_targets.numpy())
+    r = {k: getattr(att, k).to(dev) for k in ("q", "k", "v", "seq_offsets", "timestamps", "num_targets", "rab_pos",
+                                              "rab_time")}
+    rkw = dict(max_seq_len=att.max_seq_len, inv_n=att.inv_n, pos_lo=att.pos_lo, pos_hi=att.pos_hi)
+    ro = torch.empty_like(r["v"])
+    rws = ops.alloc_workspace(ops.hstu_attn_workspace_size(
+        ops._attn_desc_from(r["q"], r["v"], r["seq_offsets"], att.max_seq_len, att.inv_n, att.pos_lo, att.pos_hi,
+                            r["rab_time"]), False), dev)
+    ra_ms = timed(lambda: ops.hstu_attn_fwd(r["q"], r["k"], r["v"], r["seq_offsets"], r["timestamps"],
+                                            r["num_targets"], r["rab_pos"], r["rab_time"], out=ro, workspace=rws,
+                                            stream=stream, **rkw))
+    rpairs = flops.attn_pairs(a.lengths, a.num_targets.numpy())
+    rf = flops.attn_fwd_flops(rpairs, w.num_heads, w.d_qk, w.d_v)
+    lw = lay.layers[0]
+    prm = [t.to(dev) for t in (lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta)]
+    seq = [a.seq_offsets.to(dev), a.timestamps.to(dev), a.num_targets.to(dev), a.rab_pos.to(dev),
+           a.rab_time.to(dev)]
+    x = lay.x.to(dev)
+    y = torch.empty_like(x)
+    lkw = dict(num_heads=w.num_heads, d_qk=w.d_qk, d_v=w.d_v, max_seq_len=a.max_seq_len, inv_n=a.inv_n,
+               pos_lo=a.pos_lo, pos_hi=a.pos_hi)
+    desc = ops.hstu_layer_desc(ops.make_attn_desc(len(a.lengths), a.max_seq_len, a.total_tokens, w.num_heads, w.d_qk,
+                                                  w.d_v, ops.HSTU_BF16, a.inv_n, a.pos_lo, a.pos_hi,
+                                                  a.rab_time.numel()), w.d_model, 1e-5)
+    lws = ops.alloc_workspace(ops.hstu_layer_workspace_size(desc), dev)
+    rl_ms = timed(lambda: ops.hstu_layer_fwd(x, *prm, *seq, y=y, workspace=lws, stream=stream, **lkw))
+    lf = rf + flops.f1_flops(a.total_tokens, w.d_model, w.num_heads, w.d_qk, w.d_v) + \
+        flops.f2_flops(a.total_tokens, w.d_model, w.num_heads, w.d_v)
+    out["ranking_bf16"] = {"tokens": a.total_tokens, "visible_pairs_per_head": rpairs,
+                           "attn_fwd_ms": ra_ms, "attn_fwd_tflops": rf / (ra_ms * 1e-3) / 1e12,
+                           "layer_fwd_ms": rl_ms, "layer_fwd_tflops": lf / (rl_ms * 1e-3) / 1e12}
+    return out
+
+
 TRUNCATE = (3, 6, 512)   # layers over whole histories, layers over the segment, segment length
 
 
@@ -682,6 +769,7 @@ def run_ours(args):
                 "speedup_vs_full_mask": ms / (f_ms + b_ms)}
 
     trunc = None if args.no_layer_stack else truncation_timing(dev, stream)
+    others = None if args.no_layer_stack else config_timings(dev, stream)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -716,6 +804,11 @@ def run_ours(args):
             line["semi_local"] = semi
         if trunc is not None:
             line["truncation"] = trunc
+        if others is not None:
+            for k, v in others.items():
+                v["pct_of_bf16_peak"] = {kk.replace("_tflops", ""): 100 * vv / burst
+                                         for kk, vv in v.items() if kk.endswith("_tflops")}
+            line["other_configs"] = others
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(line), flush=True)

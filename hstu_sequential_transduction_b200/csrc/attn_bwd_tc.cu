@@ -39,7 +39,6 @@ namespace {
 
 constexpr int KB = 128;  // key rows per CTA
 constexpr int QB = 64;   // query rows per step
-constexpr int DH = 128;  // head dim
 constexpr int kEpiWarpsB = 8;                   // 2 per TMEM lane quarter
 constexpr int kEpiThreadsB = kEpiWarpsB * 32;
 constexpr int kThreadsB = kEpiThreadsB + 64;
@@ -53,14 +52,19 @@ constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384,
 enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 3, S_FULL = 5, S_FREE = 6, P_FULL = 7, P_FREE = 8,
              DQ_FULL = 9, DQ_FREE = 10, ACC_FULL = 11, NBARS_B = 12 };
 
+// Shared-memory layout for head dim DH (64 or 128): NR = DH / 64 swizzled
+// 128-byte-wide regions per tile.  V directly follows K, so that for DH = 64 the
+// dQ^T MMA can run with M = 128: its second 64 rows read V^T and are discarded.
+template <int DH>
 struct BL {
+    static constexpr int NR = DH / 64;
     static constexpr int K = 0;
-    static constexpr int V = K + 2 * kRegK;
-    static constexpr int Q0 = V + 2 * kRegK;       // 2 stages x 2 regions
-    static constexpr int O0 = Q0 + 4 * kRegQ;      // dO, 2 stages x 2 regions
-    static constexpr int DST = O0 + 4 * kRegQ;     // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
+    static constexpr int V = K + NR * kRegK;
+    static constexpr int Q0 = V + NR * kRegK;      // 2 stages x NR regions
+    static constexpr int O0 = Q0 + 2 * NR * kRegQ;  // dO, 2 stages x NR regions
+    static constexpr int DST = O0 + 2 * NR * kRegQ;  // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
     static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, per warp [NC x 32]
-    static constexpr int E = DQS + QB * DH * 4;    // time bias by exponent (512)
+    static constexpr int E = DQS + QB * 128 * 4;   // time bias by exponent (512)
     static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
     static constexpr int PW = EG + 512 * 4;        // per warp: NC query stamps + 64 bias window
     static constexpr int PW_FLOATS = NC + 64;
@@ -212,13 +216,16 @@ __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float 
     }
 }
 
-// SL: semi-local windows in use (otherwise every window test compiles away)
-template <bool SL>
+// DH: head dim (64 or 128); SL: semi-local windows in use (otherwise every
+// window test compiles away)
+template <int DH, bool SL>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ)
 {
+    using BL = hstu::BL<DH>;
+    constexpr int NR = BL::NR;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -282,8 +289,8 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            mbar_expect_tx(bar(KV_FULL), 4 * kRegK);
-            for (int r = 0; r < 2; r++) {
+            mbar_expect_tx(bar(KV_FULL), 2 * NR * kRegK);
+            for (int r = 0; r < NR; r++) {
                 tma_load_2d(base + BL::K + r * kRegK, &tmK, h * DH + 64 * r, (int)(s0 + j0), bar(KV_FULL));
                 tma_load_2d(base + BL::V + r * kRegK, &tmV, h * DH + 64 * r, (int)(s0 + j0), bar(KV_FULL));
             }
@@ -292,10 +299,10 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 const int y = (int)(s0 + j0 + i * QB);
                 if (i >= 2 && !mbar_wait(bar(Q_EMPTY + s), ((i - 2) >> 1) & 1, abort_flag, p.hdr))
                     break;
-                mbar_expect_tx(bar(Q_FULL + s), 4 * kRegQ);
-                for (int r = 0; r < 2; r++) {
-                    tma_load_2d(base + BL::Q0 + s * 2 * kRegQ + r * kRegQ, &tmQ, h * DH + 64 * r, y, bar(Q_FULL + s));
-                    tma_load_2d(base + BL::O0 + s * 2 * kRegQ + r * kRegQ, &tmO, h * DH + 64 * r, y, bar(Q_FULL + s));
+                mbar_expect_tx(bar(Q_FULL + s), 2 * NR * kRegQ);
+                for (int r = 0; r < NR; r++) {
+                    tma_load_2d(base + BL::Q0 + s * NR * kRegQ + r * kRegQ, &tmQ, h * DH + 64 * r, y, bar(Q_FULL + s));
+                    tma_load_2d(base + BL::O0 + s * NR * kRegQ + r * kRegQ, &tmO, h * DH + 64 * r, y, bar(Q_FULL + s));
                 }
             }
         }
@@ -304,12 +311,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         if (lane == 0) {
             constexpr uint32_t idSdP = idesc_bf16(KB, QB, 0, 0);
             constexpr uint32_t idGrad = idesc_bf16(KB, DH, 0, 1);
-            constexpr uint32_t idDQ = idesc_bf16(DH, QB, 1, 1);
+            constexpr uint32_t idDQ = idesc_bf16(128, QB, 1, 1);  // DH = 64: rows 64-127 are discarded
             auto issue_SdP = [&](int i) {
                 const int s = i & 1;
                 for (int ks = 0; ks < DH / 16; ks++) {
                     const uint32_t ok_ = (ks >> 2) * kRegK + (ks & 3) * 32;
-                    const uint32_t oq = s * 2 * kRegQ + (ks >> 2) * kRegQ + (ks & 3) * 32;
+                    const uint32_t oq = s * NR * kRegQ + (ks >> 2) * kRegQ + (ks & 3) * 32;
                     umma_bf16(tmem + COL_S, smem_desc_sw128(base + BL::K + ok_, 16, 1024),
                               smem_desc_sw128(base + BL::Q0 + oq, 16, 1024), idSdP, ks > 0);
                     umma_bf16(tmem + COL_DP, smem_desc_sw128(base + BL::V + ok_, 16, 1024),
@@ -323,9 +330,9 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 for (int ks = 0; ks < QB / 16; ks++) {
                     const uint32_t acc = (i > 0 || ks > 0);
                     umma_bf16_ts(tmem + COL_DV, tmem + COL_PT + 8 * ks,
-                                 smem_desc_sw128(base + BL::O0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                                 smem_desc_sw128(base + BL::O0 + s * NR * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
                     umma_bf16_ts(tmem + COL_DK, tmem + COL_DST + 8 * ks,
-                                 smem_desc_sw128(base + BL::Q0 + s * 2 * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
+                                 smem_desc_sw128(base + BL::Q0 + s * NR * kRegQ + ks * 2048, kRegQ, 1024), idGrad, acc);
                 }
             };
             auto issue_dq = [&]() {
@@ -418,6 +425,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             if (!mbar_wait(bar(DQ_FULL), k & 1, abort_flag, p.hdr))
                 return false;
             tc_fence_after();
+            if (32 * quarter >= DH) {  // rows past the head dim (DH = 64): nothing to add
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(DQ_FREE));
+                return true;
+            }
             float qv[NC];
             tmem_ld_nc(trow + COL_DQ + NC * g, qv);
             tmem_wait_ld();
@@ -660,13 +674,14 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
 
 bool attn_bwd_tc_supported(const AttnParams &p)
 {
-    return p.dqk == DH && p.dv == DH && attn_tc_supported(p);
+    return p.dqk == p.dv && (p.dqk == 64 || p.dqk == 128) && attn_tc_supported(p);
 }
 
-cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
+namespace {
+
+template <int DH>
+cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
-    if (grid_items <= 0)
-        return cudaSuccess;
     CUtensorMap mk, mv, mq, mo, mdq;
     const int cols = p.H * DH;
     cudaError_t e = make_row_tensor_map(&mk, p.k, p.T, cols, p.sk);
@@ -683,13 +698,22 @@ cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t
                                32, NC, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess)
         return e;
-    const size_t bytes = BL::BYTES + 1024;
-    auto kern = p.lw > 0 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+    const size_t bytes = BL<DH>::BYTES + 1024;
+    auto kern = p.lw > 0 ? attn_bwd_tc_kernel<DH, true> : attn_bwd_tc_kernel<DH, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
     kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
+{
+    if (grid_items <= 0)
+        return cudaSuccess;
+    return p.dqk == 64 ? bwd_tc_launch<64>(p, grid_items, stream) : bwd_tc_launch<128>(p, grid_items, stream);
 }
 
 }  // namespace hstu
