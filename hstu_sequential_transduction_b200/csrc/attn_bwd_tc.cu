@@ -274,13 +274,6 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     }
     if (warp == 1)
         tmem_alloc(base + BL::MISC, kTmemColsB);
-    if (warp >= 2) {
-        const int etid = threadIdx.x - 64;
-        for (int e = etid; e < 512; e += kEpiThreadsB) {
-            E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
-            EG[e] = 0.f;
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -373,6 +366,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         }
     } else {
         // ---------------- epilogue ----------------
+        // time tables, filled while the first tiles load; only the epilogue warps use them
+        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreadsB) {
+            E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
+            EG[e] = 0.f;
+        }
+        named_bar(1, kEpiThreadsB);
         // Every warp handles a 32-key x NC-query block of each step on its own:
         // stamps, bias window, class and bias-table gradients are per warp, so
         // the loop has no CTA-wide barrier.

@@ -194,13 +194,6 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
     }
     if (warp == 1)
         tmem_alloc(base + LY::MISC, kTmemCols);
-    if (warp >= 2) {
-        // expanded time table: index = sign:exponent of the fp32 (1 + dt)
-        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreads) {
-            const int bkt = (e >= 256 || e < 127) ? 0 : min(e - 127, p.nb - 1);
-            E[e] = 0.5f * p.rab_time[bkt];
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -284,6 +277,13 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         }
     } else {
         // ---------------- epilogue ----------------
+        // expanded time table (index = sign:exponent of the fp32 (1 + dt)), filled
+        // while the first tiles load; only the epilogue warps read it
+        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreads) {
+            const int bkt = (e >= 256 || e < 127) ? 0 : min(e - 127, p.nb - 1);
+            E[e] = 0.5f * p.rab_time[bkt];
+        }
+        named_bar(1, kEpiThreads);
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const int i = i0 + r;
