@@ -2,13 +2,17 @@
 //
 // Computes, per (sequence, 128-row query tile, head) work item,
 //   O = inv_n * sum_j SiLU(Q K_j^T + rab_pos + rab_time) V_j
+// Persistent: one CTA per SM walks a share of the work items, so the next
+// item's query and first key tiles load and its first S MMAs run while the
+// epilogue still writes out the previous item's O.
 // over the visible 128-row key tiles j (the pointwise attention of the
 // "HSTU Architecture" section; causal block with appended candidates of the
 // DLRMv4 page's "Model Architecture" section).  No score matrix reaches HBM.
 //
 // Warp roles (320 threads):
-//   warp 0     TMA producer: Q once, then K_j and V_j into two-stage rings
-//              (separate K and V rings, so K_{j+2} loads as soon as S_j is done);
+//   warp 0     TMA producer: Q of each item into one of two buffers, then K_j
+//              and V_j into two-stage rings (separate K and V rings, so K_{j+2}
+//              loads as soon as S_j is done);
 //   warp 1     owns TMEM (512 columns) and issues every tcgen05.mma from one
 //              thread: S_j = Q K_j^T into one of two S buffers, O += P_j V_j;
 //   warps 2-9  epilogue: two warpgroups, each takes 64 of the 128 key columns
@@ -32,6 +36,8 @@
 // 2^24 s, take the general path (per-pair visibility, exact int64 bucket).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -46,18 +52,21 @@ constexpr int kThreadsTc = kEpiThreads + 64;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRegion = 16384;  // one 128-row x 128-byte swizzled region
 
-// P_FULL + b: P of the tile in S buffer b is in TMEM (one barrier per buffer, so
-// the epilogue can never be two phases ahead of the MMA thread on one of them);
-// P_FREE: P_j V_j has completed (its A operand, P_j in TMEM, is consumed)
-enum Bars { Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, P_FULL = 11,
-            P_FREE = 13, O_FULL = 14, NBARS = 15 };
+// Every barrier that can be waited on more than once per work item comes in
+// pairs, one per buffer, so that no wait ever sees its barrier two phases on.
+// Q_FULL / Q_EMPTY + b: query buffer b loaded / read by its last S MMA;
+// K_*, V_*, S_FULL, P_FULL + b: the tile in stage / S buffer b;
+// P_FREE + b: P V of the tile in S buffer b has completed (buffer b is free);
+// O_FULL: a work item's O is complete in TMEM; O_FREE: the epilogue has read it.
+enum Bars { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10, S_FULL = 12,
+            P_FULL = 14, P_FREE = 16, O_FULL = 18, O_FREE = 19, NBARS = 20 };
 
 template <int D>
 struct FwdLayout {
     static constexpr int NREG = D / 64;
     static constexpr int TILE = NREG * kRegion;
-    static constexpr int Q = 0;
-    static constexpr int K0 = Q + TILE;
+    static constexpr int Q = 0;                 // two query buffers
+    static constexpr int K0 = Q + 2 * TILE;
     static constexpr int V0 = K0 + 2 * TILE;
     static constexpr int E = V0 + 2 * TILE;
     // per epilogue warp: 64 key stamps + 96-entry positional-bias window of a tile
@@ -151,28 +160,45 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
 
-    const int item = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    if (item >= p.hdr->n_items)
-        return;
-    const int2 it = p.items[item];
-    const int qt = it.y;
-    const int64_t s0 = p.seq_offsets[it.x];
-    const int L = (int)(p.seq_offsets[it.x + 1] - s0);
-    const int hist = L - (p.num_targets ? p.num_targets[it.x] : 0);
-    const int i0 = qt * TBM;
+    // Persistent: each CTA takes one unit per round of gridDim.x units of the
+    // scheduler's (cost-ordered) list, unit w = (item w / H, head w % H).  Every
+    // role walks the same units; `g` below counts K/V/S tiles across them.
+    const int n_units = p.hdr->n_items * p.H;
+    // the u-th unit of this CTA: rounds of gridDim.x units, alternating direction,
+    // so that over the cost-ordered list every CTA gets a similar total
+    auto unit_index = [&](int u) {
+        const int G = (int)gridDim.x, b = (int)blockIdx.x;
+        return u * G + ((u & 1) ? G - 1 - b : b);
+    };
     const int lw = SL ? p.lw : 0, gw = SL ? p.gw : 0;
-    const int nh = (hist + TBN - 1) / TBN;
-    const int nfull = min(qt + 1, nh);  // history key tiles up to this query tile
-    // Semi-local windows: of those, the tiles holding global keys [0, gt) and the
-    // tiles reaching into the local window of the tile's first row [lt0, nfull).
-    int gt = nfull, lt0 = nfull;
-    if (lw > 0) {
-        gt = min(nfull, (gw + TBN - 1) / TBN);
-        lt0 = min(nfull, max(gt, max(0, token_pos(i0, hist) - lw + 1) / TBN));
-    }
-    const int nhist = gt + (nfull - lt0);
-    const int ntiles = nhist + (qt >= nh ? 1 : 0);  // + the candidates' own tile
-    auto tile_of = [&](int t) { return t >= nhist ? qt : (t < gt ? t : t - gt + lt0); };
+    struct Unit {
+        int64_t s0;
+        int L, hist, qt, i0, h, gt, lt0, nhist, ntiles;
+        __device__ int tile_of(int t) const { return t >= nhist ? qt : (t < gt ? t : t - gt + lt0); }
+    };
+    auto unit = [&](int w) {
+        Unit U;
+        const int2 it = p.items[w / p.H];
+        U.h = w % p.H;
+        U.qt = it.y;
+        U.s0 = p.seq_offsets[it.x];
+        U.L = (int)(p.seq_offsets[it.x + 1] - U.s0);
+        U.hist = U.L - (p.num_targets ? p.num_targets[it.x] : 0);
+        U.i0 = U.qt * TBM;
+        const int nh = (U.hist + TBN - 1) / TBN;
+        const int nfull = min(U.qt + 1, nh);  // history key tiles up to this query tile
+        // Semi-local windows: of those, the tiles holding global keys [0, gt) and the
+        // tiles reaching into the local window of the tile's first row [lt0, nfull).
+        U.gt = nfull;
+        U.lt0 = nfull;
+        if (lw > 0) {
+            U.gt = min(nfull, (gw + TBN - 1) / TBN);
+            U.lt0 = min(nfull, max(U.gt, max(0, token_pos(U.i0, U.hist) - lw + 1) / TBN));
+        }
+        U.nhist = U.gt + (nfull - U.lt0);
+        U.ntiles = U.nhist + (U.qt >= nh ? 1 : 0);  // + the candidates' own tile
+        return U;
+    };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto bar = [&](int i) { return base + LY::BAR + 8u * i; };
@@ -181,7 +207,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS; i++) {
-            const bool epi = (i == P_FULL || i == P_FULL + 1);
+            const bool epi = (i == P_FULL || i == P_FULL + 1 || i == O_FREE);
             mbar_init(bar(i), epi ? kEpiWarps : 1);
         }
         *abort_flag = 0;
@@ -202,24 +228,33 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            mbar_expect_tx(bar(Q_FULL), LY::TILE);
-            for (int r = 0; r < LY::NREG; r++)
-                tma_load_2d(base + LY::Q + r * kRegion, &tq, h * D + 64 * r, (int)(s0 + i0), bar(Q_FULL));
-            for (int t = 0; t < ntiles; t++) {
-                const int s = t & 1;
-                const int j0 = tile_of(t) * TBN;
-                if (t >= 2 && !mbar_wait(bar(K_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, p.hdr))
+            bool ok = true;
+            int g = 0;
+            for (int u = 0, w = unit_index(0); ok && w < n_units; u++, w = unit_index(u)) {
+                const Unit U = unit(w);
+                const int qs = u & 1;
+                if (u >= 2 && !(ok = mbar_wait(bar(Q_EMPTY + qs), ((u >> 1) - 1) & 1, abort_flag, p.hdr)))
                     break;
-                mbar_expect_tx(bar(K_FULL + s), LY::TILE);
+                mbar_expect_tx(bar(Q_FULL + qs), LY::TILE);
                 for (int r = 0; r < LY::NREG; r++)
-                    tma_load_2d(base + LY::K0 + s * LY::TILE + r * kRegion, &tk, h * D + 64 * r,
-                                (int)(s0 + j0), bar(K_FULL + s));
-                if (t >= 2 && !mbar_wait(bar(V_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, p.hdr))
-                    break;
-                mbar_expect_tx(bar(V_FULL + s), LY::TILE);
-                for (int r = 0; r < LY::NREG; r++)
-                    tma_load_2d(base + LY::V0 + s * LY::TILE + r * kRegion, &tv, h * D + 64 * r,
-                                (int)(s0 + j0), bar(V_FULL + s));
+                    tma_load_2d(base + LY::Q + qs * LY::TILE + r * kRegion, &tq, U.h * D + 64 * r,
+                                (int)(U.s0 + U.i0), bar(Q_FULL + qs));
+                for (int t = 0; t < U.ntiles; t++, g++) {
+                    const int s = g & 1;
+                    const int j0 = U.tile_of(t) * TBN;
+                    if (g >= 2 && !(ok = mbar_wait(bar(K_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
+                        break;
+                    mbar_expect_tx(bar(K_FULL + s), LY::TILE);
+                    for (int r = 0; r < LY::NREG; r++)
+                        tma_load_2d(base + LY::K0 + s * LY::TILE + r * kRegion, &tk, U.h * D + 64 * r,
+                                    (int)(U.s0 + j0), bar(K_FULL + s));
+                    if (g >= 2 && !(ok = mbar_wait(bar(V_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
+                        break;
+                    mbar_expect_tx(bar(V_FULL + s), LY::TILE);
+                    for (int r = 0; r < LY::NREG; r++)
+                        tma_load_2d(base + LY::V0 + s * LY::TILE + r * kRegion, &tv, U.h * D + 64 * r,
+                                    (int)(U.s0 + j0), bar(V_FULL + s));
+                }
             }
         }
     } else if (warp == 1) {
@@ -227,53 +262,77 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(TBM, TBN, 0, 0);
             constexpr uint32_t idO = idesc_bf16(TBM, D, 0, 1);
-            auto issue_S = [&](int t) {
-                const int s = t & 1;
+            // S of tile g (query buffer qs) into S buffer g % 2
+            auto issue_S = [&](int g, int qs) {
+                const int s = g & 1;
                 for (int ks = 0; ks < D / 16; ks++) {
                     const uint32_t off = (ks >> 2) * kRegion + (ks & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(base + LY::Q + off, 16, 1024);
+                    const uint64_t a = smem_desc_sw128(base + LY::Q + qs * LY::TILE + off, 16, 1024);
                     const uint64_t b = smem_desc_sw128(base + LY::K0 + s * LY::TILE + off, 16, 1024);
                     umma_bf16(tmem + s * TBN, a, b, idS, ks > 0);
                 }
                 umma_commit(bar(K_EMPTY + s));
                 umma_commit(bar(S_FULL + s));
             };
-            auto issue_PV = [&](int t) {
-                const int s = t & 1;
-                // A = P_t from TMEM: keys 16 ks .. sit in S buffer columns 64 (ks / 4) + 8 (ks % 4)
+            // O (+)= P_g V_g; `first` starts a work item's accumulator
+            auto issue_PV = [&](int g, bool first) {
+                const int s = g & 1;
+                // A = P_g from TMEM: keys 16 ks .. sit in S buffer columns 64 (ks / 4) + 8 (ks % 4)
                 for (int ks = 0; ks < TBN / 16; ks++) {
                     const uint64_t b = smem_desc_sw128(base + LY::V0 + s * LY::TILE + ks * 2048, kRegion, 1024);
                     umma_bf16_ts(tmem + 2 * TBN, tmem + s * TBN + 64 * (ks >> 2) + 8 * (ks & 3), b, idO,
-                                 (t > 0 || ks > 0));
+                                 (!first || ks > 0));
                 }
                 umma_commit(bar(V_EMPTY + s));
-                umma_commit(bar(P_FREE));
+                umma_commit(bar(P_FREE + s));
             };
-            bool ok = mbar_wait(bar(Q_FULL), 0, abort_flag, p.hdr);
-            for (int t = 0; ok && t < min(2, ntiles); t++) {
-                ok = mbar_wait(bar(K_FULL + t), 0, abort_flag, p.hdr);
-                if (ok) {
-                    tc_fence_after();
-                    issue_S(t);
-                }
-            }
-            for (int j = 0; ok && j < ntiles; j++) {
-                ok = mbar_wait(bar(P_FULL + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr) &&
-                     mbar_wait(bar(V_FULL + (j & 1)), (j >> 1) & 1, abort_flag, p.hdr);
-                if (!ok)
+            // S buffer g % 2 is free once P V of tile g - 2 has completed
+            auto s_free = [&](int g) {
+                return g < 2 || mbar_wait(bar(P_FREE + (g & 1)), ((g >> 1) - 1) & 1, abort_flag, p.hdr);
+            };
+            bool ok = true;
+            int gb = 0;  // first tile of the current unit
+            for (int u = 0, w = unit_index(0); ok && w < n_units; u++, w = unit_index(u)) {
+                const Unit U = unit(w);
+                const int qs = u & 1, nt = U.ntiles;
+                if (!(ok = mbar_wait(bar(Q_FULL + qs), (u >> 1) & 1, abort_flag, p.hdr)))
                     break;
-                tc_fence_after();
-                issue_PV(j);
-                if (j + 2 < ntiles) {
-                    ok = mbar_wait(bar(P_FREE), j & 1, abort_flag, p.hdr) &&
-                         mbar_wait(bar(K_FULL + (j & 1)), ((j + 2) >> 1) & 1, abort_flag, p.hdr);
+                for (int t = 0; ok && t < min(2, nt); t++) {
+                    const int g = gb + t;
+                    ok = s_free(g) && mbar_wait(bar(K_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr);
+                    if (ok) {
+                        tc_fence_after();
+                        issue_S(g, qs);
+                    }
+                }
+                if (ok && nt <= 2)
+                    umma_commit(bar(Q_EMPTY + qs));
+                // the previous unit's O has been read out of TMEM
+                if (ok && u >= 1)
+                    ok = mbar_wait(bar(O_FREE), (u - 1) & 1, abort_flag, p.hdr);
+                for (int j = 0; ok && j < nt; j++) {
+                    const int g = gb + j;
+                    ok = mbar_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr) &&
+                         mbar_wait(bar(V_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr);
                     if (!ok)
                         break;
                     tc_fence_after();
-                    issue_S(j + 2);
+                    issue_PV(g, j == 0);
+                    if (j + 2 < nt) {
+                        ok = s_free(g + 2) &&
+                             mbar_wait(bar(K_FULL + (g & 1)), ((g + 2) >> 1) & 1, abort_flag, p.hdr);
+                        if (!ok)
+                            break;
+                        tc_fence_after();
+                        issue_S(g + 2, qs);
+                        if (j + 3 == nt)
+                            umma_commit(bar(Q_EMPTY + qs));  // the unit's last S has been issued
+                    }
                 }
+                if (ok)
+                    umma_commit(bar(O_FULL));
+                gb += nt;
             }
-            umma_commit(bar(O_FULL));
         }
     } else {
         // ---------------- epilogue ----------------
@@ -286,6 +345,13 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         named_bar(1, kEpiThreads);
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;
+        bool ok = true;
+        int gtile = 0;  // tiles of this CTA so far (S buffer gtile % 2)
+        for (int u = 0, w = unit_index(0); ok && w < n_units; u++, w = unit_index(u)) {
+        const Unit U = unit(w);
+        const int64_t s0 = U.s0;
+        const int L = U.L, hist = U.hist, i0 = U.i0, h = U.h, ntiles = U.ntiles;
+        auto tile_of = [&](int t) { return U.tile_of(t); };
         const int i = i0 + r;
         const bool row_ok = i < L;
         const int64_t tb = p.timestamps[s0 + i0];
@@ -324,9 +390,8 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 tc = p.timestamps[s0 + j + 1];
         };
         prep(0);
-        bool ok = true;
-        for (int t = 0; t < ntiles; t++) {
-            const int s = t & 1;
+        for (int t = 0; t < ntiles; t++, gtile++) {
+            const int s = gtile & 1;
             const int j0 = tile_of(t) * TBN;
             const int j = j0 + 64 * g + 2 * lane;
             const int64_t ta_next = __shfl_down_sync(full_mask, ta, 1);
@@ -349,7 +414,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             if (t + 1 < ntiles)
                 prep(t + 1);
 
-            if (!(ok = mbar_wait(bar(S_FULL + s), (t >> 1) & 1, abort_flag, p.hdr)))
+            if (!(ok = mbar_wait(bar(S_FULL + s), (gtile >> 1) & 1, abort_flag, p.hdr)))
                 break;
             tc_fence_after();
             float sv[64];
@@ -426,7 +491,9 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             if (lane == 0)
                 mbar_arrive(bar(P_FULL + s));
         }
-        if (ok && mbar_wait(bar(O_FULL), 0, abort_flag, p.hdr)) {
+        if (!(ok = ok && mbar_wait(bar(O_FULL), u & 1, abort_flag, p.hdr)))
+            break;
+        {
             tc_fence_after();
             __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (s0 + i) * p.so + (int64_t)h * D + g * (D / 2);
 #pragma unroll
@@ -436,16 +503,22 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
-                    for (int u = 0; u < 4; u++) {
+                    for (int q4 = 0; q4 < 4; q4++) {
                         uint4 v;
-                        v.x = pack_bf16(ov[8 * u] * p.inv_n, ov[8 * u + 1] * p.inv_n);
-                        v.y = pack_bf16(ov[8 * u + 2] * p.inv_n, ov[8 * u + 3] * p.inv_n);
-                        v.z = pack_bf16(ov[8 * u + 4] * p.inv_n, ov[8 * u + 5] * p.inv_n);
-                        v.w = pack_bf16(ov[8 * u + 6] * p.inv_n, ov[8 * u + 7] * p.inv_n);
-                        *reinterpret_cast<uint4 *>(orow + cc + 8 * u) = v;
+                        v.x = pack_bf16(ov[8 * q4] * p.inv_n, ov[8 * q4 + 1] * p.inv_n);
+                        v.y = pack_bf16(ov[8 * q4 + 2] * p.inv_n, ov[8 * q4 + 3] * p.inv_n);
+                        v.z = pack_bf16(ov[8 * q4 + 4] * p.inv_n, ov[8 * q4 + 5] * p.inv_n);
+                        v.w = pack_bf16(ov[8 * q4 + 6] * p.inv_n, ov[8 * q4 + 7] * p.inv_n);
+                        *reinterpret_cast<uint4 *>(orow + cc + 8 * q4) = v;
                     }
                 }
             }
+        }
+        // O has been read out of TMEM: the next unit's first P V may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar(O_FREE));
         }
     }
     tc_fence_before();
@@ -487,7 +560,17 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
-    attn_fwd_tc_kernel<D, SL><<<(unsigned)grid_items * p.H, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
+    // persistent: at most one CTA per SM, each walking its share of the work units
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    const int64_t units = (int64_t)grid_items * p.H;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, sms);
+    attn_fwd_tc_kernel<D, SL><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
     return cudaGetLastError();
 }
 
