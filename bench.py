@@ -47,8 +47,8 @@ SEMI_LOCAL = (1024, 256)
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd_tc -c 1
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
 # valid only for the kernel source it was taken on (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "1b8a55b0641219d7f4310bb032c88334daeb67a4aacc93c11d8f04258198d067",
-               "bytes": 4.66e9 + 2.54e9}
+BWD_TRAFFIC = {"source_sha256": "10055fa6583963d0f73501c9346155d0623e8ffa5f2d9665a2a2102053624655",
+               "bytes": 4.61e9 + 2.47e9}
 
 
 def bwd_traffic():
