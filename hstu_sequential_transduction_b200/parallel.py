@@ -83,3 +83,24 @@ def allreduce_bias_grads(d_rab_pos: torch.Tensor, d_rab_time: torch.Tensor, grou
     dist.all_reduce(flat, group=group)
     d_rab_pos.copy_(flat[:npos].view_as(d_rab_pos))
     d_rab_time.copy_(flat[npos:].view_as(d_rab_time))
+
+
+# parameter gradients of one transduction layer (per-token dx stays on its rank)
+LAYER_PARAM_GRADS = ("dw1", "db1", "dw2", "db2", "d_ln_gamma", "d_ln_beta", "d_rab_pos", "d_rab_time")
+
+
+def allreduce_layer_grads(grads: dict, group=None) -> None:
+    """Sum a layer's parameter gradients (the dict of `ops.hstu_layer_bwd`) over
+    all ranks in place, packed into one buffer and one all-reduce."""
+    import torch.distributed as dist
+
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return
+    parts = [grads[k] for k in LAYER_PARAM_GRADS]
+    flat = torch.cat([t.reshape(-1) for t in parts])
+    dist.all_reduce(flat, group=group)
+    o = 0
+    for t in parts:
+        n = t.numel()
+        t.copy_(flat[o:o + n].view_as(t))
+        o += n

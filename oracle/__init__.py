@@ -233,9 +233,10 @@ def norm_gate(o, u, gamma, beta, eps=1e-5, threads=None):
 
 def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma, ln_beta,
               rab_pos, rab_time, pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, ln_eps=1e-5,
-              threads=None, want_intermediates=False, out_cat=False):
+              threads=None, want_intermediates=False, out_cat=False, local_window=0, global_window=0):
     """Y[T, D] of one transduction layer (and optionally uvqk, O).  out_cat: the
-    output projection reads [U | O | G] (W2 is [3 H d_v, D]) instead of G."""
+    output projection reads [U | O | G] (W2 is [3 H d_v, D]) instead of G;
+    local_window / global_window: semi-local attention (see visible_sl)."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     x, w1, b1, w2, b2 = _f64(x), _f64(w1), _f64(b1), _f64(w2), _f64(b2)
     g, be, rp, rt = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time)
@@ -245,6 +246,16 @@ def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma,
     y = np.zeros((T, D))
     uvqk = np.zeros((T, W)) if want_intermediates else None
     o = np.zeros((T, num_heads * d_v)) if want_intermediates else None
+    with _Windows(local_window, global_window):
+        _layer_fwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, b2, g, be, ln_eps, ts, rp, pos_lo,
+                        pos_hi, rt, inv_n, y, uvqk, o, out_cat, threads)
+    if want_intermediates:
+        return y, uvqk, o
+    return y
+
+
+def _layer_fwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, b2, g, be, ln_eps, ts, rp, pos_lo, pos_hi,
+                    rt, inv_n, y, uvqk, o, out_cat, threads):
     _load().oracle_layer_fwd(
         ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
         ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
@@ -253,13 +264,11 @@ def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma,
         ctypes.c_int(int(pos_hi)), _p(rt, _f64p), ctypes.c_int(len(rt)), ctypes.c_double(inv_n),
         _p(y, _f64p), _p(uvqk, _f64p), _p(o, _f64p), ctypes.c_int(int(out_cat)),
         ctypes.c_int(threads or default_threads()))
-    if want_intermediates:
-        return y, uvqk, o
-    return y
 
 
 def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_beta, rab_pos, rab_time,
-              pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None, out_cat=False):
+              pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None, out_cat=False,
+              local_window=0, global_window=0):
     """Gradients of sum(Y * dy) for one transduction layer: a dict with dx, dw1, db1,
     dw2, db2, d_ln_gamma, d_ln_beta, d_rab_pos, d_rab_time (out_cat as in layer_fwd)."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
@@ -273,6 +282,14 @@ def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_
     out = {"dx": np.zeros((T, D)), "dw1": np.zeros((D, W)), "db1": np.zeros(W), "dw2": np.zeros((F, D)),
            "db2": np.zeros(D), "d_ln_gamma": np.zeros(hv), "d_ln_beta": np.zeros(hv),
            "d_rab_pos": np.zeros(len(rp)), "d_rab_time": np.zeros(len(rt))}
+    with _Windows(local_window, global_window):
+        _layer_bwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, g, be, ln_eps, ts, rp, pos_lo, pos_hi,
+                        rt, inv_n, dyy, out, out_cat, threads)
+    return out
+
+
+def _layer_bwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, g, be, ln_eps, ts, rp, pos_lo, pos_hi, rt,
+                    inv_n, dyy, out, out_cat, threads):
     _load().oracle_layer_bwd(
         ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
         ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
@@ -282,7 +299,6 @@ def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_
         _p(out["dw1"], _f64p), _p(out["db1"], _f64p), _p(out["dw2"], _f64p), _p(out["db2"], _f64p),
         _p(out["d_ln_gamma"], _f64p), _p(out["d_ln_beta"], _f64p), _p(out["d_rab_pos"], _f64p),
         _p(out["d_rab_time"], _f64p), ctypes.c_int(int(out_cat)), ctypes.c_int(threads or default_threads()))
-    return out
 
 
 def attn_inputs_fwd(inp, threads=None):

@@ -94,3 +94,65 @@ def test_dp_shards_reproduce_full_batch_gradients(tmp_path):
             np.testing.assert_allclose(z["dv"], full[2][rows], rtol=0, atol=1e-12)
         covered += list(z["seqs"])
     assert sorted(covered) == list(range(len(off) - 1))
+
+
+def _layer_batch():
+    rng = np.random.default_rng(41)
+    attn = workloads.make_attn_inputs(rng, [8, 2, 11, 0, 6, 13], 2, 4, 4, 30.0, -6, 6, 5, 16, torch.float32,
+                                      num_targets=[1, 0, 2, 0, 0, 3], with_values=False)
+    T, D, W, hv = attn.total_tokens, 6, 2 * 4 * 4, 8
+    prm = {"x": rng.standard_normal((T, D)), "w1": rng.standard_normal((D, W)) * 0.4,
+           "b1": rng.standard_normal(W) * 0.1, "w2": rng.standard_normal((hv, D)),
+           "g": 1 + 0.1 * rng.standard_normal(hv), "be": 0.1 * rng.standard_normal(hv),
+           "dy": rng.standard_normal((T, D))}
+    return attn, prm
+
+
+def _layer_grads(attn, prm, rows=None, off=None, nt=None):
+    import oracle
+    x, dy, ts = prm["x"], prm["dy"], attn.timestamps.numpy()
+    if rows is not None:
+        x, dy, ts = x[rows], dy[rows], ts[rows]
+    return oracle.layer_bwd(attn.seq_offsets if off is None else off, ts,
+                            attn.num_targets if nt is None else nt, x, prm["w1"], prm["b1"], prm["w2"],
+                            prm["g"], prm["be"], attn.rab_pos, attn.rab_time, attn.pos_lo, attn.pos_hi,
+                            attn.inv_n, 2, 4, 4, dy, threads=1)
+
+
+def _layer_worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        attn, prm = _layer_batch()
+        costs = parallel.sequence_costs(attn.lengths, attn.num_targets.numpy())
+        mine = parallel.lpt_partition(costs, world)[rank]
+        off = attn.seq_offsets.numpy()
+        rows = np.concatenate([np.arange(off[b], off[b + 1]) for b in mine]).astype(np.int64)
+        sub_off = np.concatenate([[0], np.cumsum([off[b + 1] - off[b] for b in mine])]).astype(np.int64)
+        g = _layer_grads(attn, prm, rows, sub_off, attn.num_targets[list(mine)])
+        grads = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in g.items()}
+        parallel.allreduce_layer_grads(grads)
+        np.savez(os.path.join(out_dir, f"layer{rank}.npz"), rows=rows, **{k: v.numpy() for k, v in grads.items()})
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dp_layer_backward_sums_parameter_gradients(tmp_path):
+    import oracle
+    oracle.build()
+    world = 2
+    port = _free_port()
+    mp.start_processes(_layer_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    attn, prm = _layer_batch()
+    full = _layer_grads(attn, prm)
+    seen = []
+    for rank in range(world):
+        z = np.load(tmp_path / f"layer{rank}.npz")
+        for k in parallel.LAYER_PARAM_GRADS:
+            np.testing.assert_allclose(z[k], full[k], rtol=1e-12, atol=1e-12, err_msg=k)
+        np.testing.assert_allclose(z["dx"], full["dx"][z["rows"]], rtol=1e-12, atol=1e-12)
+        seen += list(z["rows"])
+    assert sorted(seen) == list(range(attn.total_tokens))

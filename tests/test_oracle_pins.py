@@ -741,3 +741,27 @@ def test_truncated_candidates_see_a_local_window():
             n_t = int(nt[b])
             np.testing.assert_allclose(cut[new_off[b + 1] - n_t:new_off[b + 1]], win[off[b + 1] - n_t:off[b + 1]],
                                        rtol=0, atol=1e-13)
+
+
+def test_windowed_layer_is_the_composition_with_windowed_attention():
+    # the layer's attention takes the same windows as the attention alone (pinned above)
+    rng = np.random.default_rng(730)
+    H, dqk, dv, D = 2, 3, 2, 5
+    c = rand_case(rng, [9, 4, 12], H=H, dqk=dqk, dv=dv, nt=[2, 0, 3])
+    T = int(c["seq_offsets"][-1])
+    W = H * (2 * dv + 2 * dqk)
+    x = rng.standard_normal((T, D))
+    w1, b1 = rng.standard_normal((D, W)) * 0.5, rng.standard_normal(W) * 0.1
+    w2, b2 = rng.standard_normal((H * dv, D)), rng.standard_normal(D)
+    gam, bet = 1 + 0.1 * rng.standard_normal(H * dv), 0.1 * rng.standard_normal(H * dv)
+    args = (c["seq_offsets"], c["timestamps"], c["num_targets"])
+    tables = (c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+    y = oracle.layer_fwd(*args, x, w1, b1, w2, b2, gam, bet, *tables, H, dqk, dv, local_window=3, global_window=2)
+    a = oracle.linear(x, w1, b1, apply_silu=True)
+    hv, hq = H * dv, H * dqk
+    o = oracle.attn_fwd(*args, a[:, 2 * hv:2 * hv + hq].reshape(T, H, dqk), a[:, 2 * hv + hq:].reshape(T, H, dqk),
+                        a[:, hv:2 * hv].reshape(T, H, dv), *tables, local_window=3, global_window=2)
+    g = oracle.norm_gate(o.reshape(T, hv), a[:, :hv], gam, bet)
+    np.testing.assert_allclose(y, oracle.linear(g, w2, b2), rtol=0, atol=1e-12)
+    # and differs from the full-mask layer
+    assert np.abs(y - oracle.layer_fwd(*args, x, w1, b1, w2, b2, gam, bet, *tables, H, dqk, dv)).max() > 1e-6
