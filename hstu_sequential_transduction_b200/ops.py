@@ -225,7 +225,7 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
                    rab_pos, rab_time, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, y=None,
                    saved_uvqk=None, saved_o=None, workspace=None, stream=None, output_concat: bool = False,
-                   fp8_projections: bool = False):
+                   fp8_projections: bool = False, local_window: int = 0, global_window: int = 0):
     """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer; with
     output_concat, f2 reads [U | O | G] and w2 is [3 H d_v, D]; with
     fp8_projections, w1 and w2 are E4M3 weight packs (quantize_weight_e4m3)."""
@@ -238,7 +238,7 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
     _dev(ln_beta, "ln_beta", torch.float32)
     T, D = x.shape
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
-                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window, global_window)
     desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)), int(bool(fp8_projections)))
     if fp8_projections:
         W = num_heads * (2 * d_v + 2 * d_qk)
@@ -269,7 +269,7 @@ def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc) -> int:
 def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
                    saved_uvqk, saved_o, dy, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, workspace=None, stream=None,
-                   output_concat: bool = False):
+                   output_concat: bool = False, local_window: int = 0, global_window: int = 0):
     """Gradients of sum(Y * dy) for one layer (bf16): a dict with dx (bf16) and the
     float32 parameter gradients dw1, db1, dw2, db2, d_ln_gamma, d_ln_beta,
     d_rab_pos, d_rab_time (output_concat as in hstu_layer_fwd)."""
@@ -282,7 +282,7 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
     W = w1.shape[1]
     hv = num_heads * d_v
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
-                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel())
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window, global_window)
     desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)))
     F = (3 if output_concat else 1) * hv
     if w2.shape[0] != F:

@@ -84,3 +84,38 @@ def test_semi_local_long_history_sampled(cuda_device):
     assert_bf16_close(dv[idx], rv, what="semi-local long dv rows")
     tp, tt = float(drp.double().sum()), float(drt.double().sum())
     assert abs(tp - tt) <= 1e-3 * max(abs(tp), float(drp.abs().sum())), (tp, tt)
+
+
+def test_semi_local_layer_fwd_bwd(cuda_device):
+    """One bf16 layer (D = 128, 2 heads of 64) forward and backward with the
+    windows, against the oracle's windowed layer."""
+    import oracle as _oracle
+    from hstu_sequential_transduction_b200 import ops as _ops
+    from parity_utils import assert_bf16_close, to_dev
+    rng = np.random.default_rng(760)
+    attn = workloads.make_attn_inputs(rng, [300, 1, 90, 0, 257], 2, 64, 64, 300.0, -400, 400, 32, 300,
+                                      torch.bfloat16, num_targets=[20, 0, 0, 0, 7], with_values=False)
+    lw = workloads.make_layer_weights(rng, 128, 2, 64, 64, torch.bfloat16, weight_std=0.1, random_affine=True)
+    T = attn.total_tokens
+    x = torch.from_numpy(rng.standard_normal((T, 128)).astype(np.float32)).to(torch.bfloat16)
+    dy = torch.from_numpy(rng.standard_normal((T, 128)).astype(np.float32)).to(torch.bfloat16)
+    dev = cuda_device
+    win = dict(local_window=64, global_window=16)
+    kw = dict(num_heads=2, d_qk=64, d_v=64, max_seq_len=attn.max_seq_len, inv_n=attn.inv_n, pos_lo=attn.pos_lo,
+              pos_hi=attn.pos_hi, **win)
+    prm = [to_dev(t, dev) for t in (lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta)]
+    seq = [to_dev(t, dev) for t in (attn.seq_offsets, attn.timestamps, attn.num_targets, attn.rab_pos, attn.rab_time)]
+    uvqk = torch.empty((T, 512), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((T, 128), dtype=torch.bfloat16, device=dev)
+    y = _ops.hstu_layer_fwd(to_dev(x, dev), *prm, *seq, saved_uvqk=uvqk, saved_o=o, **kw)
+    w1, b1, w2, _, g, be = prm
+    grads = _ops.hstu_layer_bwd(to_dev(x, dev), w1, b1, w2, g, be, *seq, uvqk, o, to_dev(dy, dev), **kw)
+    torch.cuda.synchronize()
+    oargs = (attn.seq_offsets, attn.timestamps, attn.num_targets)
+    ref = _oracle.layer_fwd(*oargs, x, lw.w1, lw.b1, lw.w2, lw.b2, lw.ln_gamma, lw.ln_beta, attn.rab_pos,
+                            attn.rab_time, attn.pos_lo, attn.pos_hi, attn.inv_n, 2, 64, 64, **win)
+    assert_bf16_close(y, ref, what="windowed layer output")
+    refg = _oracle.layer_bwd(*oargs, x, lw.w1, lw.b1, lw.w2, lw.ln_gamma, lw.ln_beta, attn.rab_pos, attn.rab_time,
+                             attn.pos_lo, attn.pos_hi, attn.inv_n, 2, 64, 64, dy, **win)
+    for n in ("dx", "dw1", "db1", "dw2", "db2", "d_ln_gamma", "d_ln_beta", "d_rab_pos", "d_rab_time"):
+        assert_bf16_close(grads[n], refg[n], what=n)
