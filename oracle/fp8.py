@@ -1,4 +1,4 @@
-"""FP8 (E4M3) projections for the oracle.  TEST INFRASTRUCTURE ONLY, like the
+"""FP8 (E4M3) projections and scores for the oracle.  TEST INFRASTRUCTURE ONLY, like the
 rest of `oracle/`: only the tests, the smoke check and the bench's CPU leg use it.
 
 The ULTRA-HSTU review in the pages (its mixed-precision item) keeps most of the
@@ -14,8 +14,11 @@ the FP8 format nor the scaling; the readings taken here are:
     a code stands for is decode(code) * scale; an all-zero row has scale 1;
   * the product of two quantised operands is exact and accumulated in float64
     here, then scaled: y[m, n] = sum_k dec(xq[m, k]) dec(wq[n, k]) sx[m] sw[n].
-Only the projections f1 and f2 are quantised; the attention and the gate stay
-as in the bf16 layer.
+In the FP8 layer only the projections f1 and f2 are quantised; the attention
+and the gate stay as in the bf16 layer.  The FP8-score attention (attn_fwd_qk)
+quantises q and k per (token, head) row the same way and keeps P V in bf16:
+the pages name the product QK^T and AV together, and the reading taken keeps P
+and V out of FP8, since a row's P has no scale known before all its key tiles.
 """
 
 from __future__ import annotations
@@ -117,3 +120,27 @@ def layer_fwd(seq_offsets, timestamps, num_targets, x, w1q, s1, b1, w2q, s2, b2,
     if want_intermediates:
         return y, a, o
     return y
+
+
+def quantize_heads(x):
+    """Per-(token, head) row E4M3 quantisation of q or k [T, H, d]: (codes uint8
+    [T, H, d], scales float32 [T, H])."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().float().numpy()
+    x = np.asarray(x, dtype=np.float32)
+    T, H, d = x.shape
+    codes, scales = quantize_rows(x.reshape(T * H, d))
+    return codes.reshape(T, H, d), scales.reshape(T, H)
+
+
+def attn_fwd_qk(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n,
+                **windows):
+    """Attention forward with the score product in FP8: q and k quantised per
+    (token, head) row, s = dec(q) . dec(k) exactly, the rest (bias, SiLU, P V
+    with bf16-valued P and V in the kernels) as in the bf16 attention."""
+    qq, sq = quantize_heads(q)
+    kq, sk = quantize_heads(k)
+    qd = e4m3_decode(qq) * sq[..., None].astype(np.float64)
+    kd = e4m3_decode(kq) * sk[..., None].astype(np.float64)
+    return attn_fwd(seq_offsets, timestamps, num_targets, qd, kd, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n,
+                    **windows)

@@ -118,3 +118,34 @@ def test_fp8_layer_is_close_to_the_bf16_layer():
     # 3-bit mantissas: a few percent of the output's range, not more
     err = np.abs(y - ref).max() / np.abs(ref).max()
     assert 1e-4 < err < 0.1, err
+
+
+def test_fp8_scores_are_exact_when_q_and_k_are_representable():
+    # rows whose values are E4M3 codes times a power of two, with the row's largest
+    # magnitude at 448 times that power: the quantisation is exact, so the FP8-score
+    # attention equals the plain one
+    rng = np.random.default_rng(905)
+    lengths = [7, 1, 12]
+    T, H, d = sum(lengths), 2, 8
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    ts = np.concatenate([np.cumsum(rng.integers(0, 50, L)) for L in lengths]).astype(np.int64)
+    finite = np.array([c for c in range(256) if c & 0x7F != 0x7F and c & 0x7F <= 0x7E], np.uint8)
+
+    def exact(shape):
+        codes = rng.choice(finite, size=shape)
+        codes[..., 0] = 0x7E  # the row's amax maps to 448 exactly
+        pw = np.exp2(rng.integers(-12, -6, shape[:-1]))[..., None]
+        return fp8.e4m3_decode(codes) * pw
+
+    q, k = exact((T, H, d)), exact((T, H, d))
+    v = rng.standard_normal((T, H, d))
+    rp, rt = rng.standard_normal(21) * 0.1, rng.standard_normal(6) * 0.1
+    args = (off, ts, None)
+    ref = oracle.attn_fwd(*args, q, k, v, rp, rt, -10, 10, 0.1)
+    np.testing.assert_allclose(fp8.attn_fwd_qk(*args, q, k, v, rp, rt, -10, 10, 0.1), ref, rtol=0, atol=1e-12)
+    # general values: within the 3-bit mantissa's error of the plain attention
+    q2, k2 = rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d))
+    a = fp8.attn_fwd_qk(*args, q2, k2, v, rp, rt, -10, 10, 0.1)
+    b = oracle.attn_fwd(*args, q2, k2, v, rp, rt, -10, 10, 0.1)
+    err = np.abs(a - b).max() / np.abs(b).max()
+    assert 1e-4 < err < 0.1, err
