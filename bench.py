@@ -768,6 +768,30 @@ def run_ours(args):
                 "fwd_ms": f_ms, "bwd_ms": b_ms, "tflops": (sl_f + sl_b) / ((f_ms + b_ms) * 1e-3) / 1e12,
                 "speedup_vs_full_mask": ms / (f_ms + b_ms)}
 
+    # secondary: the same forward with Q K^T on E4M3 codes (q, k quantised inside the call)
+    fp8s = None
+    if not args.no_layer_stack:
+        desc8 = ops._attn_desc_from(q, v, off, inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi, rt, fp8_qk=True)
+        ws8 = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc8, False), dev)
+
+        def f8():
+            ops.hstu_attn_fwd(q, k, v, off, ts, None, rp, rt, out=out, workspace=ws8, stream=stream, fp8_qk=True,
+                              **kw)
+
+        for _ in range(2):
+            f8()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(5):
+            f8()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        f8_ms = a0.elapsed_time(a1) / 5
+        fp8s = {"what": "forward with Q K^T on E4M3 codes of q and k (per (token, head) row scales, "
+                        "quantisation inside the call); P V in bf16",
+                "fwd_ms": f8_ms, "tflops": fwd_fl / (f8_ms * 1e-3) / 1e12, "speedup_vs_bf16": fwd_ms / f8_ms}
+
     trunc = None if args.no_layer_stack else truncation_timing(dev, stream)
     others = None if args.no_layer_stack else config_timings(dev, stream)
 
@@ -802,6 +826,8 @@ def run_ours(args):
             line["layer_stack"] = layer
         if semi is not None:
             line["semi_local"] = semi
+        if fp8s is not None:
+            line["fp8_scores"] = fp8s
         if trunc is not None:
             line["truncation"] = trunc
         if others is not None:

@@ -68,6 +68,8 @@ extern "C" hstu_status hstu_attn_fwd_noalloc(const hstu_attn_desc *desc, const v
     hstu_status st = hstu_attn_workspace_size(desc, 0, &need);
     if (st != HSTU_OK)
         return st;
+    if (desc->fp8_qk)  // the FP8 codes need a caller's workspace
+        return HSTU_ERR_UNSUPPORTED;
     if (need > kNoAllocScratchBytes)
         return HSTU_ERR_UNSUPPORTED;  // problem larger than the static scratch
     void *scratch = nullptr;

@@ -61,17 +61,20 @@ constexpr int kRegion = 16384;  // one 128-row x 128-byte swizzled region
 enum Bars { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10, S_FULL = 12,
             P_FULL = 14, P_FREE = 16, O_FULL = 18, O_FREE = 19, NBARS = 20 };
 
-template <int D>
+// F8: Q and K tiles are E4M3 codes (one 128-byte region for D = 128)
+template <int D, bool F8 = false>
 struct FwdLayout {
     static constexpr int NREG = D / 64;
-    static constexpr int TILE = NREG * kRegion;
+    static constexpr int TILE = NREG * kRegion;       // a bf16 tile (V; Q and K unless F8)
+    static constexpr int QKT = F8 ? kRegion : TILE;   // a Q or K tile
     static constexpr int Q = 0;                 // two query buffers
-    static constexpr int K0 = Q + 2 * TILE;
-    static constexpr int V0 = K0 + 2 * TILE;
+    static constexpr int K0 = Q + 2 * QKT;
+    static constexpr int V0 = K0 + 2 * QKT;
     static constexpr int E = V0 + 2 * TILE;
     // per epilogue warp: 64 key stamps + 96-entry positional-bias window of a tile
+    // (+ 64 key scales / 2 with F8)
     static constexpr int PW = E + 512 * 4;
-    static constexpr int PW_FLOATS = 64 + 96;
+    static constexpr int PW_FLOATS = 64 + 96 + (F8 ? 64 : 0);
     static constexpr int BAR = PW + kEpiWarps * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS * 8;
     static constexpr int BYTES = MISC + 64;
@@ -91,10 +94,12 @@ __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float
 // MODE: 0 time bucket looked up per column, 1 one bucket for the whole row
 // (e_hi), 2 two buckets split at thr.  CONSTB: the positional index is clamped
 // for every column, so the positional bias is wr[0].
-template <bool MASK, int MODE, bool CONSTB>
+// F8: the raw score is dec(q) . dec(k) without the row scales; column c's half
+// scale is ks[c] and the row's scale rsq, so h = s rsq ks[c] + bias / 2.
+template <bool MASK, int MODE, bool CONSTB, bool F8 = false>
 __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float *tj, float ti1,
                                         const float *E, float e_hi, float e_lo, float thr, int c_lo, int c_lim,
-                                        uint32_t *pk)
+                                        uint32_t *pk, const float *ks = nullptr, float rsq = 0.f)
 {
     const float bconst = CONSTB ? wr[0] + (MODE == 1 ? e_hi : 0.f) : 0.f;
     // three passes per 32 columns (biased half-scores, tanh, products) so the
@@ -103,7 +108,14 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
     for (int hb = 0; hb < 64; hb += 32) {
 #pragma unroll
         for (int u = 0; u < 8; u++) {
-            float tv[4];
+            float tv[4], kf[4];
+            if (F8) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(ks + hb + 4 * u);  // shared by the warp
+                kf[0] = rsq * k4.x;
+                kf[1] = rsq * k4.y;
+                kf[2] = rsq * k4.z;
+                kf[3] = rsq * k4.w;
+            }
             if (MODE != 1) {
                 const float4 t4 = *reinterpret_cast<const float4 *>(tj + hb + 4 * u);  // shared by the warp
                 tv[0] = t4.x;
@@ -114,8 +126,9 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const int cc = hb + 4 * u + e;
+                const float sc = F8 ? kf[e] : 0.5f;
                 if (CONSTB && MODE == 1) {
-                    sv[cc] = fmaf(sv[cc], 0.5f, bconst);
+                    sv[cc] = fmaf(sv[cc], sc, bconst);
                     continue;
                 }
                 float bt;
@@ -125,7 +138,7 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
                     bt = __fsub_rz(ti1, tv[e]) >= thr ? e_hi : e_lo;
                 else
                     bt = time_bias_fast(ti1, tv[e], E);
-                sv[cc] = fmaf(sv[cc], 0.5f, CONSTB ? wr[0] : wr[-cc]) + bt;
+                sv[cc] = fmaf(sv[cc], sc, CONSTB ? wr[0] : wr[-cc]) + bt;
             }
         }
         float th[32];
@@ -148,13 +161,14 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
     }
 }
 
-// SL: semi-local windows in use (otherwise every window test compiles away)
-template <int D, bool SL>
+// SL: semi-local windows in use (otherwise every window test compiles away);
+// F8: S = Q K^T on E4M3 codes (tq, tk map the codes), rescaled in the epilogue
+template <int D, bool SL, bool F8 = false>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv)
 {
-    using LY = FwdLayout<D>;
+    using LY = FwdLayout<D, F8>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -235,18 +249,18 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 const int qs = u & 1;
                 if (u >= 2 && !(ok = mbar_wait(bar(Q_EMPTY + qs), ((u >> 1) - 1) & 1, abort_flag, p.hdr)))
                     break;
-                mbar_expect_tx(bar(Q_FULL + qs), LY::TILE);
-                for (int r = 0; r < LY::NREG; r++)
-                    tma_load_2d(base + LY::Q + qs * LY::TILE + r * kRegion, &tq, U.h * D + 64 * r,
+                mbar_expect_tx(bar(Q_FULL + qs), LY::QKT);
+                for (int r = 0; r < LY::QKT / kRegion; r++)
+                    tma_load_2d(base + LY::Q + qs * LY::QKT + r * kRegion, &tq, U.h * D + 64 * r,
                                 (int)(U.s0 + U.i0), bar(Q_FULL + qs));
                 for (int t = 0; t < U.ntiles; t++, g++) {
                     const int s = g & 1;
                     const int j0 = U.tile_of(t) * TBN;
                     if (g >= 2 && !(ok = mbar_wait(bar(K_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
                         break;
-                    mbar_expect_tx(bar(K_FULL + s), LY::TILE);
-                    for (int r = 0; r < LY::NREG; r++)
-                        tma_load_2d(base + LY::K0 + s * LY::TILE + r * kRegion, &tk, U.h * D + 64 * r,
+                    mbar_expect_tx(bar(K_FULL + s), LY::QKT);
+                    for (int r = 0; r < LY::QKT / kRegion; r++)
+                        tma_load_2d(base + LY::K0 + s * LY::QKT + r * kRegion, &tk, U.h * D + 64 * r,
                                     (int)(U.s0 + j0), bar(K_FULL + s));
                     if (g >= 2 && !(ok = mbar_wait(bar(V_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
                         break;
@@ -265,11 +279,20 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             // S of tile g (query buffer qs) into S buffer g % 2
             auto issue_S = [&](int g, int qs) {
                 const int s = g & 1;
-                for (int ks = 0; ks < D / 16; ks++) {
-                    const uint32_t off = (ks >> 2) * kRegion + (ks & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(base + LY::Q + qs * LY::TILE + off, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(base + LY::K0 + s * LY::TILE + off, 16, 1024);
-                    umma_bf16(tmem + s * TBN, a, b, idS, ks > 0);
+                if (F8) {  // E4M3: 32 codes (32 bytes) of K per MMA, one 128-byte region
+                    constexpr uint32_t idS8 = idesc_e4m3(TBM, TBN, 0, 0);
+                    for (int ks = 0; ks < D / 32; ks++) {
+                        const uint64_t a = smem_desc_sw128(base + LY::Q + qs * LY::QKT + ks * 32, 16, 1024);
+                        const uint64_t b = smem_desc_sw128(base + LY::K0 + s * LY::QKT + ks * 32, 16, 1024);
+                        umma_e4m3(tmem + s * TBN, a, b, idS8, ks > 0);
+                    }
+                } else {
+                    for (int ks = 0; ks < D / 16; ks++) {
+                        const uint32_t off = (ks >> 2) * kRegion + (ks & 3) * 32;
+                        const uint64_t a = smem_desc_sw128(base + LY::Q + qs * LY::TILE + off, 16, 1024);
+                        const uint64_t b = smem_desc_sw128(base + LY::K0 + s * LY::TILE + off, 16, 1024);
+                        umma_bf16(tmem + s * TBN, a, b, idS, ks > 0);
+                    }
                 }
                 umma_commit(bar(K_EMPTY + s));
                 umma_commit(bar(S_FULL + s));
@@ -367,6 +390,9 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         // Ww[m]: positional bias / 2 at offset pw - jw - 63 + m, pw = the warp's first row position
         // (positions grow with the row, candidates share one, so a row's pi - pw is in [0, 31])
         float *Ww = TJw + 64;
+        float *KSw = Ww + 96;  // F8: half scales of the key columns
+        // F8: this row's q scale
+        const float rsq = F8 && row_ok ? p.sq8[(s0 + i) * p.H + h] : 0.f;
         const int pw = token_pos(i0 + 32 * quarter, hist);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         auto clamp_idx = [&](int d) { return (d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d)) - p.pos_lo; };
@@ -375,6 +401,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         // so the loads stay in flight while this tile is processed
         float w0 = 0.f, w1 = 0.f, w2 = 0.f;
         int64_t ta = tb, tc = tb;  // stamps of key columns 2 lane, 2 lane + 1
+        float ka = 0.f, kc = 0.f;  // F8: scales of key columns 2 lane, 2 lane + 1
         auto prep = [&](int t) {
             const int jw = tile_of(t) * TBN + 64 * g;
             const int dbase = pw - jw - 63;
@@ -388,6 +415,10 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 ta = p.timestamps[s0 + j];
             if (j + 1 < L)
                 tc = p.timestamps[s0 + j + 1];
+            if (F8) {
+                ka = j < L ? p.sk8[(s0 + j) * p.H + h] : 0.f;
+                kc = j + 1 < L ? p.sk8[(s0 + j + 1) * p.H + h] : 0.f;
+            }
         };
         prep(0);
         for (int t = 0; t < ntiles; t++, gtile++) {
@@ -405,6 +436,8 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             Ww[lane] = 0.5f * w0;
             Ww[lane + 32] = 0.5f * w1;
             Ww[lane + 64] = 0.5f * w2;
+            if (F8)
+                *reinterpret_cast<float2 *>(KSw + 2 * lane) = make_float2(0.5f * ka, 0.5f * kc);
             __syncwarp();
             // every pair of the tile inside the local window (or every key global)?
             const bool band_all = lw <= 0 || token_pos(min(i0 + TBM, L) - 1, hist) - j0 < lw ||
@@ -446,23 +479,23 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     const float thr = __uint_as_float(bh << 23);
                     if (one) {
                         if (cst)
-                            fwd_row<false, 1, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
+                            fwd_row<false, 1, true, F8>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk, KSw, rsq);
                         else
-                            fwd_row<false, 1, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
+                            fwd_row<false, 1, false, F8>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk, KSw, rsq);
                     } else if (two) {
                         if (cst)
-                            fwd_row<false, 2, true>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
+                            fwd_row<false, 2, true, F8>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk, KSw, rsq);
                         else
-                            fwd_row<false, 2, false>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk);
+                            fwd_row<false, 2, false, F8>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk, KSw, rsq);
                     } else {
-                        fwd_row<false, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 0, 64, pk);
+                        fwd_row<false, 0, false, F8>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, 0, 64, pk, KSw, rsq);
                     }
                 } else {
                     // visible: key j <= i, j < L and, when the tile crosses the local
                     // window's edge (no global keys here), j > i - local_window
                     const int c_lim = min(i - j0 - 64 * g + 1, L - j0 - 64 * g);
                     const int c_lo = band_cut ? i - lw + 1 - (j0 + 64 * g) : 0;
-                    fwd_row<true, 0, false>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lo, c_lim, pk);
+                    fwd_row<true, 0, false, F8>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lo, c_lim, pk, KSw, rsq);
                 }
             } else {
 #pragma unroll
@@ -475,7 +508,8 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                         if (row_ok && j < L && visible_w(i, j, hist, lw, gw)) {
                             const float bp = p.rab_pos[pos_index(pi, token_pos(j, hist), p.pos_lo, p.pos_hi)];
                             const float bt = p.rab_time[time_bucket(ti, p.timestamps[s0 + j], p.nb)];
-                            const float hh = 0.5f * (sv[c + e] + bp + bt);
+                            const float sr = F8 ? sv[c + e] * (2.f * rsq * KSw[c + e]) : sv[c + e];
+                            const float hh = 0.5f * (sr + bp + bt);
                             pv[e] = fmaf(hh, tanh_approx(hh), hh);
                         }
                     }
@@ -543,21 +577,30 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-template <int D, bool SL>
+template <int D, bool SL, bool F8 = false>
 cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
     CUtensorMap maps[3];
     const void *ptrs[3] = {p.q, p.k, p.v};
     const int64_t strides[3] = {p.sq, p.sk, p.sv};
-    cudaError_t e = make_row_tensor_map(&maps[0], ptrs[0], p.T, p.H * D, strides[0]);
-    if (e == cudaSuccess)
-        e = make_row_tensor_map(&maps[1], ptrs[1], p.T, p.H * D, strides[1]);
+    cudaError_t e;
+    if (F8) {  // E4M3 codes [T, H D] bytes: boxes of 128 codes x 128 rows
+        e = make_tensor_map_2d(&maps[0], p.q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.T, p.H * D, (int64_t)p.H * D, 128,
+                               128, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e == cudaSuccess)
+            e = make_tensor_map_2d(&maps[1], p.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.T, p.H * D, (int64_t)p.H * D,
+                                   128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        e = make_row_tensor_map(&maps[0], ptrs[0], p.T, p.H * D, strides[0]);
+        if (e == cudaSuccess)
+            e = make_row_tensor_map(&maps[1], ptrs[1], p.T, p.H * D, strides[1]);
+    }
     if (e == cudaSuccess)
         e = make_row_tensor_map(&maps[2], ptrs[2], p.T, p.H * D, strides[2]);
     if (e != cudaSuccess)
         return e;
-    const size_t bytes = FwdLayout<D>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    const size_t bytes = FwdLayout<D, F8>::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
     // persistent: at most one CTA per SM, each walking its share of the work units
@@ -570,7 +613,7 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     }
     const int64_t units = (int64_t)grid_items * p.H;
     const unsigned grid = (unsigned)std::min<int64_t>(units, sms);
-    attn_fwd_tc_kernel<D, SL><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
+    attn_fwd_tc_kernel<D, SL, F8><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
     return cudaGetLastError();
 }
 
@@ -613,8 +656,12 @@ cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t
     switch (p.dqk) {
     case 64: return p.lw > 0 ? fwd_tc_launch<64, true>(p, grid_items, stream)
                              : fwd_tc_launch<64, false>(p, grid_items, stream);
-    case 128: return p.lw > 0 ? fwd_tc_launch<128, true>(p, grid_items, stream)
-                              : fwd_tc_launch<128, false>(p, grid_items, stream);
+    case 128:
+        if (p.q8)  // FP8 scores
+            return p.lw > 0 ? fwd_tc_launch<128, true, true>(p, grid_items, stream)
+                            : fwd_tc_launch<128, false, true>(p, grid_items, stream);
+        return p.lw > 0 ? fwd_tc_launch<128, true>(p, grid_items, stream)
+                        : fwd_tc_launch<128, false>(p, grid_items, stream);
     default: return cudaErrorInvalidValue;
     }
 }

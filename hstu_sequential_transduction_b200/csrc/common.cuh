@@ -45,6 +45,10 @@ struct AttnParams {
     float inv_n;
     int pos_lo, pos_hi, nb;
     int lw, gw;  // semi-local windows (lw = 0: full mask)
+    // FP8 scores (forward): E4M3 codes of q and k, [T, H, d] bytes, and their
+    // per-(token, head) scales [T, H]; null for bf16 scores
+    const void *q8, *k8;
+    const float *sq8, *sk8;
     const int2 *items;
     WsHeader *hdr;
     // backward only

@@ -33,6 +33,10 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
         return HSTU_ERR_UNSUPPORTED;
     if (d->dtype == HSTU_F32 && d->d_qk != 32 && d->d_qk != 64)
         return HSTU_ERR_UNSUPPORTED;
+    if (d->fp8_qk != 0 && d->fp8_qk != 1)
+        return HSTU_ERR_INVALID_ARG;
+    if (d->fp8_qk && (d->dtype != HSTU_BF16 || d->d_qk != 128))
+        return HSTU_ERR_UNSUPPORTED;
     if (max_items(d->total_tokens, d->num_seqs, kMmaTile) > INT_MAX / 4 ||
         d->total_tokens * d->num_heads > ((int64_t)1 << 40))
         return HSTU_ERR_UNSUPPORTED;
@@ -51,6 +55,9 @@ size_t attn_ws(const hstu_attn_desc *d, int is_bwd)
     size_t b = sizeof(WsHeader) + items_bytes(d);
     if (is_bwd && d->dtype == HSTU_BF16)
         b += align256(sizeof(float) * (size_t)d->total_tokens * d->num_heads * d->d_qk);
+    if (!is_bwd && d->fp8_qk)  // E4M3 codes of q and k, then their row scales
+        b += 2 * align256((size_t)d->total_tokens * d->num_heads * d->d_qk) +
+             2 * align256(sizeof(float) * (size_t)d->total_tokens * d->num_heads);
     return b;
 }
 
@@ -239,6 +246,32 @@ hstu_status hstu_attn_fwd(const hstu_attn_desc *desc, const void *q, const void 
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_ws(workspace, workspace_bytes, attn_ws(desc, 0)));
     const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
+    if (desc->fp8_qk) {
+        // q and k to E4M3 per (token, head) row, then the FP8-score kernel
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const int64_t T = desc->total_tokens, R = T * desc->num_heads;
+        char *cur = static_cast<char *>(workspace) + sizeof(WsHeader) + items_bytes(desc);
+        char *q8 = cur;
+        char *k8 = q8 + align256((size_t)R * 128);
+        float *sq = reinterpret_cast<float *>(k8 + align256((size_t)R * 128));
+        float *sk = reinterpret_cast<float *>(reinterpret_cast<char *>(sq) + align256(sizeof(float) * R));
+        HSTU_CUDA(launch_quantize_rows_e4m3(q, 128, R, 128, q8, 128, sq, st));
+        HSTU_CUDA(launch_quantize_rows_e4m3(k, 128, R, 128, k8, 128, sk, st));
+        AttnParams p = base_params(desc, seq_offsets, timestamps, num_targets, rab_pos, rab_time, workspace);
+        p.q = q;
+        p.k = k;
+        p.v = v;
+        p.o = out;
+        p.sq = p.sk = p.sv = p.so = row;
+        p.q8 = q8;
+        p.k8 = k8;
+        p.sq8 = sq;
+        p.sk8 = sk;
+        if (!attn_tc_supported(p))
+            return HSTU_ERR_UNSUPPORTED;
+        HSTU_TRY(schedule(desc, seq_offsets, num_targets, 0, workspace, st, kTcTile));
+        return cuda_status(launch_attn_fwd_tc(p, grid_items(desc, kTcTile), st));
+    }
     return attn_fwd_strided(desc, q, row, k, row, v, row, seq_offsets, timestamps, num_targets,
                             rab_pos, rab_time, out, row, workspace, static_cast<cudaStream_t>(stream));
 }
@@ -250,6 +283,8 @@ hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void 
                           float *d_rab_time, void *workspace, size_t workspace_bytes, void *stream)
 {
     HSTU_TRY(check_attn_desc(desc));
+    if (desc->fp8_qk)  // FP8 scores are a forward-only option
+        return HSTU_ERR_UNSUPPORTED;
     if (!seq_offsets || !rab_pos || !rab_time || !d_rab_pos || !d_rab_time)
         return HSTU_ERR_INVALID_ARG;
     if (desc->total_tokens > 0 &&
@@ -270,6 +305,8 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
     if (!d)
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_attn_desc(&d->attn));
+    if (d->attn.fp8_qk)  // FP8 scores: standalone attention forward only
+        return HSTU_ERR_UNSUPPORTED;
     if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps) ||
         (d->output_concat != 0 && d->output_concat != 1) || (d->fp8_projections != 0 && d->fp8_projections != 1))
         return HSTU_ERR_INVALID_ARG;

@@ -43,7 +43,7 @@ class hstu_attn_desc(ctypes.Structure):
                 ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("inv_n", ctypes.c_float), ("pos_lo", ctypes.c_int32), ("pos_hi", ctypes.c_int32),
                 ("num_time_buckets", ctypes.c_int32), ("debug_checks", ctypes.c_int32),
-                ("local_window", ctypes.c_int32), ("global_window", ctypes.c_int32)]
+                ("local_window", ctypes.c_int32), ("global_window", ctypes.c_int32), ("fp8_qk", ctypes.c_int32)]
 
 
 class hstu_layer_desc(ctypes.Structure):
@@ -117,10 +117,11 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
 
 
 def make_attn_desc(num_seqs, max_seq_len, total_tokens, num_heads, d_qk, d_v, dtype, inv_n,
-                   pos_lo, pos_hi, num_time_buckets, local_window=0, global_window=0) -> hstu_attn_desc:
+                   pos_lo, pos_hi, num_time_buckets, local_window=0, global_window=0,
+                   fp8_qk=False) -> hstu_attn_desc:
     return hstu_attn_desc(int(num_seqs), int(max_seq_len), int(total_tokens), int(num_heads),
                           int(d_qk), int(d_v), int(dtype), float(inv_n), int(pos_lo), int(pos_hi),
-                          int(num_time_buckets), 0, int(local_window), int(global_window))
+                          int(num_time_buckets), 0, int(local_window), int(global_window), int(bool(fp8_qk)))
 
 
 def hstu_status_string(status: int) -> str:
@@ -151,17 +152,19 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window=0,
-                    global_window=0):
+                    global_window=0, fp8_qk=False):
     return make_attn_desc(seq_offsets.numel() - 1, max_seq_len, q.shape[0], q.shape[1], q.shape[2],
                           v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window,
-                          global_window)
+                          global_window, fp8_qk)
 
 
 def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, *,
                   max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, out=None,
-                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0):
+                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0,
+                  fp8_qk: bool = False):
     """O = jagged SiLU attention; q, k [T, H, d_qk], v [T, H, d_v] on CUDA.
-    local_window > 0 applies the semi-local mask (see hstu_attn_desc)."""
+    local_window > 0 applies the semi-local mask; fp8_qk computes Q K^T on E4M3
+    codes of q and k (see hstu_attn_desc)."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         _dev(t, name, q.dtype)
     _dev(seq_offsets, "seq_offsets", torch.int64)
@@ -170,7 +173,7 @@ def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
     _dev(rab_pos, "rab_pos", torch.float32)
     _dev(rab_time, "rab_time", torch.float32)
     desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window,
-                           global_window)
+                           global_window, fp8_qk)
     if out is None:
         out = torch.empty_like(v)
     _dev(out, "out", q.dtype)

@@ -82,6 +82,14 @@ typedef struct {
      * local_window = 0 keeps the full mask; both must be >= 0. */
     int32_t local_window;
     int32_t global_window;
+    /* 1: the attention forward computes Q K^T on the tensor cores in FP8 (the
+     * mixed-precision item of the ULTRA-HSTU review): q and k are quantised per
+     * (token, head) row to E4M3 inside hstu_attn_fwd (the scaling of
+     * hstu_quantize_rows_e4m3) and the scores are rescaled by the two row scales;
+     * P V stays bf16.  bf16 with d_qk = d_v = 128 only (HSTU_ERR_UNSUPPORTED
+     * otherwise); the backward, the layer calls and hstu_attn_fwd_noalloc reject
+     * it.  0: bf16 scores. */
+    int32_t fp8_qk;
 } hstu_attn_desc;
 
 typedef struct {

@@ -43,14 +43,14 @@ def test_struct_layout_matches_header(tmp_path):
         ' offsetof(hstu_attn_desc,debug_checks), sizeof(hstu_layer_desc),'
         ' offsetof(hstu_layer_desc,ln_eps)); printf("%zu %zu\\n", offsetof(hstu_attn_desc,local_window),'
         ' offsetof(hstu_attn_desc,global_window)); printf("%zu\\n", offsetof(hstu_layer_desc,output_concat));'
-        ' return 0;}\n')
+        ' printf("%zu\\n", offsetof(hstu_attn_desc,fp8_qk)); return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
     D, L = ops.hstu_attn_desc, ops.hstu_layer_desc
     assert got == [ctypes.sizeof(D), D.total_tokens.offset, D.inv_n.offset, D.debug_checks.offset,
                    ctypes.sizeof(L), L.ln_eps.offset, D.local_window.offset, D.global_window.offset,
-                   L.output_concat.offset]
+                   L.output_concat.offset, D.fp8_qk.offset]
 
 
 def test_status_strings_and_version():

@@ -3,6 +3,8 @@ bit for bit (codes and float32 scales, the sign of a zero code aside), the
 tcgen05 kind::f8f6f4 GEMM against the oracle's float64 product of its own
 codes, and the layer with FP8 projections against the oracle's FP8 layer."""
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -150,3 +152,51 @@ def test_fp8_rejects_unsupported(cuda_device):
     pack = torch.zeros(ops.hstu_e4m3_weight_bytes(32, 100), dtype=torch.uint8, device=cuda_device)
     with pytest.raises(ops.HstuError):  # N not a multiple of 128
         ops.gemm_e4m3(codes, scales, pack, 100)
+
+
+def _fp8_attn_case(seed, lengths, nt, H=2, pos=300, nb=32):
+    rng = np.random.default_rng(seed)
+    return workloads.make_attn_inputs(rng, lengths, H, 128, 128, 300.0, -pos, pos, nb, max(lengths), torch.bfloat16,
+                                      num_targets=nt)
+
+
+@pytest.mark.parametrize("windows", [{}, {"local_window": 100, "global_window": 20}])
+def test_fp8_score_attention_matches_oracle(cuda_device, windows):
+    """Q K^T on E4M3 codes (q, k quantised per (token, head) row inside the
+    call): ragged batch with candidates, an empty and a one-token sequence."""
+    inp = _fp8_attn_case(1020, [300, 1, 0, 257, 129], [20, 0, 0, 0, 9])
+    dev = cuda_device
+    d = {k: (None if getattr(inp, k) is None else getattr(inp, k).to(dev))
+         for k in ("q", "k", "v", "seq_offsets", "timestamps", "num_targets", "rab_pos", "rab_time")}
+    out = ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], d["num_targets"],
+                            d["rab_pos"], d["rab_time"], max_seq_len=inp.max_seq_len, inv_n=inp.inv_n,
+                            pos_lo=inp.pos_lo, pos_hi=inp.pos_hi, fp8_qk=True, **windows)
+    torch.cuda.synchronize()
+    ref = ofp8.attn_fwd_qk(inp.seq_offsets, inp.timestamps, inp.num_targets, inp.q, inp.k, inp.v, inp.rab_pos,
+                           inp.rab_time, inp.pos_lo, inp.pos_hi, inp.inv_n, **windows)
+    assert_bf16_close(out, ref, what="FP8-score attention")
+
+
+def test_fp8_score_attention_rejections(cuda_device):
+    inp = _fp8_attn_case(1021, [64, 30], None)
+    dev = cuda_device
+    d = {k: (None if getattr(inp, k) is None else getattr(inp, k).to(dev))
+         for k in ("q", "k", "v", "seq_offsets", "timestamps", "rab_pos", "rab_time")}
+    kw = dict(max_seq_len=inp.max_seq_len, inv_n=inp.inv_n, pos_lo=inp.pos_lo, pos_hi=inp.pos_hi)
+    # d = 64: not supported with FP8 scores
+    q64 = d["q"][..., :64].contiguous()
+    with pytest.raises(ops.HstuError):
+        ops.hstu_attn_fwd(q64, q64, q64, d["seq_offsets"], d["timestamps"], None, d["rab_pos"], d["rab_time"],
+                          fp8_qk=True, **kw)
+    # the backward rejects the option
+    desc = ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo,
+                               inp.pos_hi, d["rab_time"], fp8_qk=True)
+    n = ctypes.c_size_t(0)
+    assert ops.load_library().hstu_attn_workspace_size(ctypes.byref(desc), 1, ctypes.byref(n)) == 0
+    ws = ops.alloc_workspace(n.value, dev)
+    g = [torch.empty_like(d["q"]) for _ in range(3)] + [torch.empty_like(d["rab_pos"]), torch.empty_like(d["rab_time"])]
+    st = ops.load_library().hstu_attn_bwd(
+        ctypes.byref(desc), ops._ptr(d["q"]), ops._ptr(d["k"]), ops._ptr(d["v"]), ops._ptr(d["seq_offsets"]),
+        ops._ptr(d["timestamps"]), None, ops._ptr(d["rab_pos"]), ops._ptr(d["rab_time"]), ops._ptr(d["q"]),
+        *[ops._ptr(t) for t in g], ops._ptr(ws), ctypes.c_size_t(ws.numel()), None)
+    assert st == 2  # HSTU_ERR_UNSUPPORTED
