@@ -86,14 +86,17 @@ quantize_cols_kernel(const __nv_bfloat16 *__restrict__ w, int64_t K, int N, unsi
         amax = fmaxf(amax, fabsf(__bfloat162float(w[k * N + n])));
     const float inv = amax > 0.f ? __fdiv_rn(kE4M3Max, amax) : 1.f;
     scale[n] = amax > 0.f ? __fdiv_rn(amax, kE4M3Max) : 1.f;
+    // sixteen codes per 16-byte store (K is a multiple of 16); the loads of each
+    // k are coalesced across the block's columns
     unsigned char *qr = q + (int64_t)n * K;
-    for (int64_t k = 0; k < K; k += 2) {
-        const float a = __fmul_rn(__bfloat162float(w[k * N + n]), inv);
-        const float b = k + 1 < K ? __fmul_rn(__bfloat162float(w[(k + 1) * N + n]), inv) : 0.f;
-        const uint32_t c = e4m3x2(a, b);
-        qr[k] = (unsigned char)(c & 0xff);
-        if (k + 1 < K)
-            qr[k + 1] = (unsigned char)(c >> 8);
+    for (int64_t k = 0; k < K; k += 16) {
+        uint32_t c[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++)
+            c[e] = e4m3x2(__fmul_rn(__bfloat162float(w[(k + 2 * e) * N + n]), inv),
+                          __fmul_rn(__bfloat162float(w[(k + 2 * e + 1) * N + n]), inv));
+        *reinterpret_cast<uint4 *>(qr + k) = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16),
+                                                        c[4] | (c[5] << 16), c[6] | (c[7] << 16));
     }
 }
 
