@@ -610,18 +610,27 @@ def run_ours(args):
     ev_f1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_b1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
+    nvtx = torch.cuda.nvtx
+
     def step(i=None, q=q, k=k, v=v, off=off, ts=ts, rp=rp, rt=rt, dout=dout, out=out, grads=grads):
+        # NVTX ranges name the phases for a timeline profiler (host-side markers only)
         if i is not None:
             ev_f0[i].record(stream)
+        nvtx.range_push("hstu_attn_fwd")
         ops.hstu_attn_fwd(q, k, v, off, ts, None, rp, rt, out=out, workspace=ws_f, stream=stream, **kw)
+        nvtx.range_pop()
         if i is not None:
             ev_f1[i].record(stream)
+        nvtx.range_push("hstu_attn_bwd")
         ops.hstu_attn_bwd(q, k, v, off, ts, None, rp, rt, dout, grads=grads, workspace=ws_b,
                           stream=stream, **kw)
+        nvtx.range_pop()
         if i is not None:
             ev_b1[i].record(stream)
         if world > 1:
+            nvtx.range_push("allreduce_bias_grads")
             parallel.allreduce_bias_grads(grads[3], grads[4])
+            nvtx.range_pop()
 
     def barrier():
         if world > 1:
