@@ -72,7 +72,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-stack", action="store_true",
                     help="skip the secondary eight-layer forward measurement")
-    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer", "layer_bwd", "truncate"], default=None,
+    ap.add_argument("--kernel-case", choices=["fwd", "bwd", "layer", "layer_bwd", "truncate", "others"], default=None,
                     help="run only a small case twice (for ncu captures) and exit")
     return ap.parse_args()
 
@@ -868,6 +868,12 @@ def kernel_case(which: str):
         return
     if which == "truncate":
         truncation_timing(dev, torch.cuda.current_stream(), reps=1)
+        torch.cuda.synchronize()
+        return
+    if which == "others":
+        # the short and ranking configurations (their attention forwards are
+        # launches 4-16 and 30-42 of this case)
+        config_timings(dev, torch.cuda.current_stream(), reps=10)
         torch.cuda.synchronize()
         return
     if which == "layer_bwd":
