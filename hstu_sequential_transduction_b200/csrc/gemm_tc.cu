@@ -10,13 +10,19 @@
 // accumulators and issues tcgen05.mma from one thread; warps 2-9 read one
 // accumulator row by row while the next tile accumulates in the other.
 //
-// Operand layouts (all bf16, 128-byte swizzled k-slices):
+// Operand layouts (bf16, 128-byte swizzled k-slices of 64 elements):
 //   A K-major: A[m][k] row-major ([M, K]);  A MN-major: stored as X[k][m] ([K, M])
 //   B MN-major: B[k][n] row-major ([K, N]); B K-major: stored as W[n][k] ([N, K])
 // so that the layer backward's products dY W2^T, dZ W1^T (B K-major) and
-// G^T dY, X^T dZ (A MN-major, K = tokens) need no transposed copies.
-// Epilogues:
-//   EPI_ACT    bf16 out = acc + bias, optionally SiLU (forward projections);
+// G^T dY, X^T dZ (A MN-major, K = tokens) need no transposed copies.  A may be
+// three stored matrices concatenated along their columns (the output
+// projection over [U | O | G]).  The E4M3 instantiation (F8) takes K-major A
+// and B codes in slices of 128 and kind::f8f6f4 MMAs of K = 32.
+// Epilogues (the chunk's bias, scales and dSiLU factors are fetched while its
+// TMEM load is in flight; bf16 outputs leave through a per-warp 32 x 32
+// swizzled box and a TMA store):
+//   EPI_ACT    bf16 out = acc (x row scale x column scale for F8) + bias,
+//              optionally SiLU as h (1 + tanh h), h = x / 2 (forward projections);
 //   EPI_DSILU  bf16 out = aux * SiLU'(acc + bias) (the SiLU backward fused into
 //              the recompute of the pre-activation);
 //   EPI_RED    fp32 out += acc through a swizzled staging box and a TMA bulk
