@@ -65,12 +65,13 @@ struct BL {
     static constexpr int DST = O0 + 2 * NR * kRegQ;  // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
     static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, per warp [NC x 32]
     static constexpr int E = DQS + QB * 128 * 4;   // time bias by exponent (512)
-    static constexpr int EG = E + 512 * 4;         // time grads by exponent (512)
-    static constexpr int PW = EG + 512 * 4;        // per warp: NC query stamps + 64 bias window
+    static constexpr int TG = E + 512 * 4;         // per warp: 32 lanes x 32 time-bucket partial sums
+    static constexpr int PW = TG + kEpiWarpsB * 32 * 32 * 4;  // per warp: NC query stamps + 64 bias window
     static constexpr int PW_FLOATS = NC + 64;
     static constexpr int BAR = PW + kEpiWarpsB * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS_B * 8;
     static constexpr int BYTES = MISC + 64;
+    static_assert(BYTES + 1024 <= 227 * 1024, "backward tile does not fit in shared memory");
 };
 
 __device__ __forceinline__ uint32_t exp_offset(float ti1, float tj)
@@ -255,7 +256,6 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     auto bar = [&](int i) { return base + BL::BAR + 8u * i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + BL::MISC + 8);
     float *E = reinterpret_cast<float *>(sm + BL::E);
-    float *EG = reinterpret_cast<float *>(sm + BL::EG);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS_B; i++) {
@@ -367,16 +367,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     } else {
         // ---------------- epilogue ----------------
         // time tables, filled while the first tiles load; only the epilogue warps use them
-        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreadsB) {
+        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreadsB)
             E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
-            EG[e] = 0.f;
-        }
         named_bar(1, kEpiThreadsB);
         // Every warp handles a 32-key x NC-query block of each step on its own:
         // stamps, bias window, class and bias-table gradients are per warp, so
         // the loop has no CTA-wide barrier.
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
-        const int etid = threadIdx.x - 64;
         const uint32_t full = 0xffffffffu;
         const int r = quarter * 32 + lane;  // key row of the tile (TMEM lane); d index for dQ^T
         const int j = j0 + r;
@@ -403,19 +400,51 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         auto clamp_idx = [&](int d) { return (d < lo ? lo : (d > hi ? hi : d)) - lo; };
 
-        // time-bucket run carried across steps (buckets only grow along a key row
-        // of sorted stamps, so a thread changes bins a few dozen times per CTA)
-        uint32_t tcur = 0xFFFFFFFFu;
-        float tacc = 0.f;
-        auto time_add = [&](uint32_t off, float v) {
-            if (off == tcur) {
-                tacc += v;
-                return;
+        // Time-bias gradient.  Outside the exact path every stamp difference lies
+        // in (-2^25, 2^25), so its exponent bucket k = e - 127 (e the biased
+        // exponent of the float difference; k = 0 for e < 127 or a negative
+        // difference, which the bucketisation also sends to bucket 0) is below 26:
+        // lane k of the warp holds the warp's running sum for k in hacc, and
+        // the global table gets one reduction per lane when the CTA ends.
+        // Blocks whose pairs span at most two adjacent buckets (klo, klo + 1 for
+        // the whole warp) add to per-thread carries c0 / c1, summed across the
+        // warp only when klo moves, which it does a few dozen times per CTA
+        // since buckets only grow along a key row of sorted stamps.  Other blocks
+        // go through TGw: each thread writes the sums of its row's bucket runs
+        // to its own 32-float row (groups of four XOR-swizzled by the lane, so
+        // the zeroing and the column reads are conflict free) and lane k then
+        // adds up column k.
+        float hacc = 0.f, c0 = 0.f, c1 = 0.f;
+        int kc = -1;
+        float *TGw = reinterpret_cast<float *>(sm + BL::TG) + ew * 32 * 32;
+        float *tgr = TGw + lane * 32;
+        auto tg_slot = [&](uint32_t k, int row) { return (((k >> 2) ^ (uint32_t)(row & 7)) << 2) | (k & 3); };
+        auto k_of = [](uint32_t off) {  // exp_offset -> bucket k
+            const uint32_t k = (off >> 2) - 127u;
+            return k < 32u ? k : 0u;
+        };
+        auto warp_sum = [&](float v) {
+#pragma unroll
+            for (int o = 16; o; o >>= 1)
+                v += __shfl_xor_sync(full, v, o);
+            return v;
+        };
+        auto carry_flush = [&](int klo) {  // warp-uniform
+            if (kc >= 0) {
+                const float r0 = warp_sum(c0);
+                if (lane == kc)
+                    hacc += r0;
+                if (klo == kc + 1) {
+                    c0 = c1;
+                } else {
+                    const float r1 = warp_sum(c1);
+                    if (lane == kc + 1)
+                        hacc += r1;
+                    c0 = 0.f;
+                }
             }
-            if (tcur != 0xFFFFFFFFu && tacc != 0.f)
-                atomicAdd(EG + (tcur >> 2), tacc);
-            tcur = off;
-            tacc = v;
+            c1 = 0.f;
+            kc = klo;
         };
 
         // dQ'^T of step k for this warp: TMEM -> [NC queries x 32 d] staging ->
@@ -497,12 +526,14 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     cls = full_w ? CLS_WINDOW : CLS_WINDOW_MASKED;
             }
             int mode = BK_ANY;
+            int klo = 0;  // bucket of the block's smallest stamp difference (BK_ONE, BK_TWO)
             if (cls != CLS_GENERAL && q_last >= iw0 && jw_n > 0) {
                 const float dlo = __fsub_rz(TIw[0], tjf_last);
                 const float dhi = __fsub_rz(TIw[q_last - iw0], tjf_first);
                 const uint32_t de = (__float_as_uint(dhi) >> 23) - (__float_as_uint(dlo) >> 23);
                 if (dlo >= 1.f)
                     mode = de == 0 ? BK_ONE : (de == 1 ? BK_TWO : BK_ANY);
+                klo = (int)(__float_as_uint(dlo) >> 23) - 127;
             }
 
             if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
@@ -553,18 +584,52 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     if (accN != 0.f)
                         red_add_global(p.d_rab_pos + clamp_idx(dw + lane - 32), accN * gscale);
                 }
-                if (!o.mid) {
-                    if (o.b1 != o.b0) {
-                        time_add(o.b0, o.all - o.hi);
-                        time_add(o.b1, o.hi);
-                    } else {
-                        time_add(o.b0, o.all);
-                    }
+                const bool two = o.b1 != o.b0;
+                const float v0 = two ? o.all - o.hi : o.all, v1 = two ? o.hi : 0.f;
+                if (mode != BK_ANY) {
+                    // every visible pair of the block is in bucket klo or klo + 1
+                    if (klo != kc)
+                        carry_flush(klo);
+                    const bool up0 = (int)k_of(o.b0) != kc, up1 = (int)k_of(o.b1) != kc;
+                    c0 += (up0 ? 0.f : v0) + (up1 ? 0.f : v1);
+                    c1 += (up0 ? v0 : 0.f) + (up1 ? v1 : 0.f);
                 } else {
+                    __syncwarp();  // lanes finished reading the rows of the previous block
 #pragma unroll
-                    for (int c = 0; c < NC; c++)
-                        if (dv[c] != 0.f)
-                            time_add(exp_offset(TIw[c], tjf), dv[c]);
+                    for (int u = 0; u < 8; u++)
+                        *reinterpret_cast<float4 *>(tgr + ((u ^ (lane & 7)) << 2)) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (!o.mid) {
+                        // at most two runs, b0 then b1 (distinct offsets below 2 share bucket 0)
+                        const uint32_t k0 = k_of(o.b0), k1 = k_of(o.b1);
+                        tgr[tg_slot(k0, lane)] = k1 == k0 ? v0 + v1 : v0;
+                        if (k1 != k0)
+                            tgr[tg_slot(k1, lane)] = v1;
+                    } else {
+                        // buckets never decrease along the row, so each run is one store
+                        uint32_t kcur = 32u;
+                        float racc = 0.f;
+#pragma unroll
+                        for (int c = 0; c < NC; c++) {
+                            if (dv[c] != 0.f) {
+                                const uint32_t k = k_of(exp_offset(TIw[c], tjf));
+                                if (k != kcur) {
+                                    if (kcur < 32u)
+                                        tgr[tg_slot(kcur, lane)] = racc;
+                                    kcur = k;
+                                    racc = 0.f;
+                                }
+                                racc += dv[c];
+                            }
+                        }
+                        if (kcur < 32u)
+                            tgr[tg_slot(kcur, lane)] = racc;
+                    }
+                    __syncwarp();
+                    float sum = 0.f;
+#pragma unroll
+                    for (int l = 0; l < 32; l++)
+                        sum += TGw[l * 32 + tg_slot((uint32_t)lane, l)];
+                    hacc += sum;
                 }
 #pragma unroll
                 for (int c = 0; c < NC; c += 2)
@@ -622,14 +687,9 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         }
         if (ok)
             ok = handle_dq(nq - 1);
-        if (tcur != 0xFFFFFFFFu && tacc != 0.f)
-            atomicAdd(EG + (tcur >> 2), tacc);
-        named_bar(1, kEpiThreadsB);
-        for (int e = etid; e < 512; e += kEpiThreadsB) {
-            const float v = EG[e];
-            if (v != 0.f)
-                red_add_global(p.d_rab_time + exp_bucket(e, p.nb), v * gscale);
-        }
+        carry_flush(-1);
+        if (hacc != 0.f)
+            red_add_global(p.d_rab_time + min(lane, p.nb - 1), hacc * gscale);
         if (ok && mbar_wait(bar(ACC_FULL), 0, abort_flag, p.hdr)) {
             tc_fence_after();
             constexpr int DC = DH / kGroupsB;  // dK / dV columns per thread
