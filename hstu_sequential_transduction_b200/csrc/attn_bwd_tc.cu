@@ -49,8 +49,9 @@ constexpr int kRegK = 16384;  // 128 rows x 128 B
 constexpr int kRegQ = 8192;   // 64 rows x 128 B
 constexpr int COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384, COL_PT = 448, COL_DST = 480;
 
-enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = 3, S_FULL = 5, S_FREE = 6, P_FULL = 7, P_FREE = 8,
-             DQ_FULL = 9, DQ_FREE = 10, ACC_FULL = 11, NBARS_B = 12 };
+constexpr int QS = 3;  // Q / dO ring stages
+enum BBars { KV_FULL = 0, Q_FULL = 1, Q_EMPTY = Q_FULL + QS, S_FULL = Q_EMPTY + QS, S_FREE, P_FULL, P_FREE,
+             DQ_FULL, DQ_FREE, ACC_FULL, NBARS_B };
 
 // Shared-memory layout for head dim DH (64 or 128): NR = DH / 64 swizzled
 // 128-byte-wide regions per tile.  V directly follows K, so that for DH = 64 the
@@ -60,13 +61,14 @@ struct BL {
     static constexpr int NR = DH / 64;
     static constexpr int K = 0;
     static constexpr int V = K + NR * kRegK;
-    static constexpr int Q0 = V + NR * kRegK;      // 2 stages x NR regions
-    static constexpr int O0 = Q0 + 2 * NR * kRegQ;  // dO, 2 stages x NR regions
-    static constexpr int DST = O0 + 2 * NR * kRegQ;  // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
-    static constexpr int DQS = DST + kRegK;        // dQ staging, fp32, per warp [NC x 32]
+    static constexpr int Q0 = V + NR * kRegK;       // QS stages x NR regions
+    static constexpr int O0 = Q0 + QS * NR * kRegQ;  // dO, QS stages x NR regions
+    static constexpr int DST = O0 + QS * NR * kRegQ;  // dS'^T [128 keys x 64 queries] (B operand of dQ^T)
+    // per warp, 4 KB used in turn: dQ staging, fp32 [NC x 32], and 32 lanes x 32
+    // time-bucket partial sums
+    static constexpr int DQS = DST + kRegK;
     static constexpr int E = DQS + QB * 128 * 4;   // time bias by exponent (512)
-    static constexpr int TG = E + 512 * 4;         // per warp: 32 lanes x 32 time-bucket partial sums
-    static constexpr int PW = TG + kEpiWarpsB * 32 * 32 * 4;  // per warp: NC query stamps + 64 bias window
+    static constexpr int PW = E + 512 * 4;         // per warp: NC query stamps + 64 bias window
     static constexpr int PW_FLOATS = NC + 64;
     static constexpr int BAR = PW + kEpiWarpsB * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS_B * 8;
@@ -288,9 +290,9 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 tma_load_2d(base + BL::V + r * kRegK, &tmV, h * DH + 64 * r, (int)(s0 + j0), bar(KV_FULL));
             }
             for (int i = 0; i < nq; i++) {
-                const int s = i & 1;
+                const int s = i % QS;
                 const int y = (int)(s0 + j0 + i * QB);
-                if (i >= 2 && !mbar_wait(bar(Q_EMPTY + s), ((i - 2) >> 1) & 1, abort_flag, p.hdr))
+                if (i >= QS && !mbar_wait(bar(Q_EMPTY + s), ((i - QS) / QS) & 1, abort_flag, p.hdr))
                     break;
                 mbar_expect_tx(bar(Q_FULL + s), 2 * NR * kRegQ);
                 for (int r = 0; r < NR; r++) {
@@ -306,7 +308,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             constexpr uint32_t idGrad = idesc_bf16(KB, DH, 0, 1);
             constexpr uint32_t idDQ = idesc_bf16(128, QB, 1, 1);  // DH = 64: rows 64-127 are discarded
             auto issue_SdP = [&](int i) {
-                const int s = i & 1;
+                const int s = i % QS;
                 for (int ks = 0; ks < DH / 16; ks++) {
                     const uint32_t ok_ = (ks >> 2) * kRegK + (ks & 3) * 32;
                     const uint32_t oq = s * NR * kRegQ + (ks >> 2) * kRegQ + (ks & 3) * 32;
@@ -318,7 +320,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                 umma_commit(bar(S_FULL));
             };
             auto issue_grads = [&](int i) {
-                const int s = i & 1;
+                const int s = i % QS;
                 // A = P^T / dS'^T from TMEM (lane = key, column = query pair)
                 for (int ks = 0; ks < QB / 16; ks++) {
                     const uint32_t acc = (i > 0 || ks > 0);
@@ -342,7 +344,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             for (int i = 0; ok && i < nq; i++) {
                 if (i + 1 < nq) {
                     ok = mbar_wait(bar(S_FREE), i & 1, abort_flag, p.hdr) &&
-                         mbar_wait(bar(Q_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1, abort_flag, p.hdr);
+                         mbar_wait(bar(Q_FULL + (i + 1) % QS), ((i + 1) / QS) & 1, abort_flag, p.hdr);
                     if (!ok)
                         break;
                     tc_fence_after();
@@ -358,7 +360,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     tc_fence_after();
                 }
                 issue_dq();
-                umma_commit(bar(Q_EMPTY + (i & 1)));
+                umma_commit(bar(Q_EMPTY + i % QS));
                 umma_commit(bar(P_FREE));
                 umma_commit(bar(DQ_FULL));
             }
@@ -416,7 +418,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         // adds up column k.
         float hacc = 0.f, c0 = 0.f, c1 = 0.f;
         int kc = -1;
-        float *TGw = reinterpret_cast<float *>(sm + BL::TG) + ew * 32 * 32;
+        float *TGw = reinterpret_cast<float *>(sm + BL::DQS) + ew * 32 * 32;  // shares the dQ staging
         float *tgr = TGw + lane * 32;
         auto tg_slot = [&](uint32_t k, int row) { return (((k >> 2) ^ (uint32_t)(row & 7)) << 2) | (k & 3); };
         auto k_of = [](uint32_t off) {  // exp_offset -> bucket k
@@ -594,7 +596,11 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     c0 += (up0 ? 0.f : v0) + (up1 ? 0.f : v1);
                     c1 += (up0 ? v0 : 0.f) + (up1 ? v1 : 0.f);
                 } else {
-                    __syncwarp();  // lanes finished reading the rows of the previous block
+                    // the bulk reduction of the previous dQ has read the staging, and
+                    // the lanes have read the rows of the previous block
+                    if (lane == 0)
+                        bulk_wait_read0();
+                    __syncwarp();
 #pragma unroll
                     for (int u = 0; u < 8; u++)
                         *reinterpret_cast<float4 *>(tgr + ((u ^ (lane & 7)) << 2)) = make_float4(0.f, 0.f, 0.f, 0.f);
