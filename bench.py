@@ -44,11 +44,12 @@ LAUNCHES_PER_STEP = 5
 SEMI_LOCAL = (1024, 256)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention-backward launch on
 # this workload, from a one-pass ncu capture of
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd_tc -c 1
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_ -c 2
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
-# valid only for the kernel source it was taken on (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "10055fa6583963d0f73501c9346155d0623e8ffa5f2d9665a2a2102053624655",
-               "bytes": 4.61e9 + 2.47e9}
+# (the second captured launch is the backward); valid only for the kernel source it was taken on
+# (else the line reports null)
+BWD_TRAFFIC = {"source_sha256": "1329ff684da7e81228fdfd0d00936f0190cbd1b6f29a0f611f0b0417005f346b",
+               "bytes": 611.22e6 + 350.18e6}
 
 
 def bwd_traffic():

@@ -234,7 +234,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
 
-    const int item = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    // head-major: every tile of head 0 (in the schedule's longest-first order),
+    // then head 1, ...  The tiles running at one time then share one head's Q,
+    // dO and dQ accumulator rows (T x 1 KB for d = 128), which stay in L2 for
+    // batches of up to ~100k tokens, instead of all heads' at once.
+    const int grid_items = gridDim.x / p.H;
+    const int h = blockIdx.x / grid_items, item = blockIdx.x % grid_items;
     if (item >= p.hdr->n_items)
         return;
     const int2 it = p.items[item];
