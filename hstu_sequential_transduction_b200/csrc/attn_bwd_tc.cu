@@ -225,7 +225,7 @@ template <int DH, bool SL>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
-                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ)
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ, int head_major)
 {
     using BL = hstu::BL<DH>;
     constexpr int NR = BL::NR;
@@ -234,12 +234,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
 
-    // head-major: every tile of head 0 (in the schedule's longest-first order),
-    // then head 1, ...  The tiles running at one time then share one head's Q,
-    // dO and dQ accumulator rows (T x 1 KB for d = 128), which stay in L2 for
-    // batches of up to ~100k tokens, instead of all heads' at once.
+    // Block order over the schedule's longest-first tile list: the heads of a
+    // tile side by side, or head-major (every tile for head 0, then head 1, ...)
+    // when the launch asks for it, so that the tiles in flight share one head's
+    // Q, dO and dQ accumulator rows in L2
     const int grid_items = gridDim.x / p.H;
-    const int h = blockIdx.x / grid_items, item = blockIdx.x % grid_items;
+    const int item = head_major ? blockIdx.x % grid_items : blockIdx.x / p.H;
+    const int h = head_major ? blockIdx.x / grid_items : blockIdx.x % p.H;
     if (item >= p.hdr->n_items)
         return;
     const int2 it = p.items[item];
@@ -773,7 +774,28 @@ cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;
-    kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq);
+    // Head-major order pays where a key tile's Q / dO / dQ rows leave L2 before
+    // the sequence's next tile reads them: one sequence's tiles over all heads
+    // do not fit one wave of CTAs, and the batch's rows (8 d bytes per token
+    // and head) exceed twice the L2.  Windowed masks keep each tile's rows near
+    // its keys, and short or few rows stay in L2 in tile order, where the heads
+    // side by side balance better (same-process timings: head-major 10-34 %
+    // faster on long-history batches, 3-19 % slower on short, Zipf and
+    // windowed ones).
+    static const int2 dev_info = [] {
+        int dev = 0, sms = 0, l2 = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+        if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
+            l2 = 126 << 20;
+        return make_int2(sms, l2);
+    }();
+    const int sms = dev_info.x;
+    const int64_t l2 = dev_info.y;
+    const int64_t max_tiles = ((int64_t)p.max_seq_len + KB - 1) / KB;
+    const int head_major = p.lw == 0 && max_tiles * p.H > sms && p.T * p.H * 8 * DH > 2 * l2;
+    kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq, head_major);
     return cudaGetLastError();
 }
 
