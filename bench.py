@@ -48,8 +48,8 @@ SEMI_LOCAL = (1024, 256)
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
 # (the second captured launch is the backward); valid only for the kernel source it was taken on
 # (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "1329ff684da7e81228fdfd0d00936f0190cbd1b6f29a0f611f0b0417005f346b",
-               "bytes": 611.22e6 + 350.18e6}
+BWD_TRAFFIC = {"source_sha256": "5d4f19369838ce28cccee2a2625c3d96593ec104c8664fa113f79f77dd63c254",
+               "bytes": 602.77e6 + 346.32e6}
 
 
 def bwd_traffic():
