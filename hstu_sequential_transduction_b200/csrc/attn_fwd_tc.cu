@@ -62,7 +62,7 @@ enum Bars { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPT
             P_FULL = 14, P_FREE = 16, O_FULL = 18, O_FREE = 19, NBARS = 20 };
 
 // F8: Q and K tiles are E4M3 codes (one 128-byte region for D = 128)
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool CAND = false>
 struct FwdLayout {
     static constexpr int NREG = D / 64;
     static constexpr int TILE = NREG * kRegion;       // a bf16 tile (V; Q and K unless F8)
@@ -70,7 +70,10 @@ struct FwdLayout {
     static constexpr int Q = 0;                 // two query buffers
     static constexpr int K0 = Q + 2 * QKT;
     static constexpr int V0 = K0 + 2 * QKT;
-    static constexpr int E = V0 + 2 * TILE;
+    // CAND: per epilogue warp, a [32 rows x 32 columns] bf16 box of O (64-byte
+    // swizzle) on its way to a TMA store
+    static constexpr int OST = V0 + 2 * TILE;
+    static constexpr int E = OST + (CAND ? kEpiWarps * 2048 : 0);
     // per epilogue warp: 64 key stamps + 96-entry positional-bias window of a tile
     // (+ 64 key scales / 2 with F8)
     static constexpr int PW = E + 512 * 4;
@@ -78,6 +81,7 @@ struct FwdLayout {
     static constexpr int BAR = PW + kEpiWarps * PW_FLOATS * 4;
     static constexpr int MISC = BAR + NBARS * 8;
     static constexpr int BYTES = MISC + 64;
+    static_assert(BYTES + 1024 <= 227 * 1024, "forward tile does not fit in shared memory");
 };
 
 __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float *E)
@@ -161,14 +165,85 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
     }
 }
 
+// The two rare tile kinds, kept out of line so that the common tile loop stays
+// small.  Both read this thread's 64 S columns from TMEM at taddr and write P
+// (bf16) back over the first 32 of them.
+//
+// Exact per-pair rule: candidate rows, unsorted or far-apart stamps.  ts points
+// at the sequence's stamps; jc0 is the key index of the thread's first column.
+template <bool F8>
+__device__ __noinline__ void p_tile_exact(uint32_t taddr, int i, bool row_ok, int jc0, int L, int hist, int lw,
+                                          int gw, int pi, int64_t ti, const int64_t *ts, const float *rab_pos,
+                                          const float *rab_time, int pos_lo, int pos_hi, int nb, float rsq,
+                                          const float *KSw)
+{
+    float sv[64];
+    tmem_ld32(taddr, sv);
+    tmem_ld32(taddr + 32, sv + 32);
+    tmem_wait_ld();
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        float pv[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int j = jc0 + c + e;
+            pv[e] = 0.f;
+            if (row_ok && j < L && visible_w(i, j, hist, lw, gw)) {
+                const float bp = rab_pos[pos_index(pi, token_pos(j, hist), pos_lo, pos_hi)];
+                const float bt = rab_time[time_bucket(ti, ts[j], nb)];
+                const float sr = F8 ? sv[c + e] * (2.f * rsq * KSw[c + e]) : sv[c + e];
+                const float hh = 0.5f * (sr + bp + bt);
+                pv[e] = fmaf(hh, tanh_approx(hh), hh);
+            }
+        }
+        pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+    }
+    tmem_st16(taddr, pk);
+    tmem_st16(taddr + 16, pk + 16);
+}
+
+// The candidates' own tile: a candidate sees only itself, at position and time
+// difference 0, so every row has the same bias bself; cd is the row's own column
+// among the thread's 64 (outside [0, 64): none).
+template <bool F8>
+__device__ __noinline__ void p_tile_own(uint32_t taddr, int cd, bool row_ok, float bself, float rsq,
+                                        const float *KSw)
+{
+    float sv[64];
+    tmem_ld32(taddr, sv);
+    tmem_ld32(taddr + 32, sv + 32);
+    tmem_wait_ld();
+    float sd = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; c++)
+        sd = c == cd ? sv[c] : sd;
+    float pd = 0.f;
+    if (row_ok && cd >= 0 && cd < 64) {
+        const float sr = F8 ? sd * (2.f * rsq * KSw[cd]) : sd;
+        const float hh = 0.5f * (sr + bself);
+        pd = fmaf(hh, tanh_approx(hh), hh);
+    }
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 64; c += 2)
+        pk[c >> 1] = pack_bf16(c == cd ? pd : 0.f, c + 1 == cd ? pd : 0.f);
+    tmem_st16(taddr, pk);
+    tmem_st16(taddr + 16, pk + 16);
+}
+
 // SL: semi-local windows in use (otherwise every window test compiles away);
-// F8: S = Q K^T on E4M3 codes (tq, tk map the codes), rescaled in the epilogue
-template <int D, bool SL, bool F8 = false>
+// F8: S = Q K^T on E4M3 codes (tq, tk map the codes), rescaled in the epilogue;
+// CAND: the batch has candidate rows (the candidates' own tiles take their own
+// path, O leaves through TMA stores); the instantiation without them keeps the
+// leaner tile loop
+template <int D, bool SL, bool F8 = false, bool CAND = false>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
-                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv)
+                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ CUtensorMap to, int o_tma)
 {
-    using LY = FwdLayout<D, F8>;
+    using LY = FwdLayout<D, F8, CAND>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -456,6 +531,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             tmem_wait_ld();
 
             uint32_t pk[32];
+            bool stored = false;  // P already in TMEM (the out-of-line tile kinds)
             // diagonal / ragged tiles without candidate rows keep the fast math
             // with a per-column mask (positions equal indices there)
             // one interval of visible columns per row: no band cut inside global keys
@@ -497,6 +573,14 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     const int c_lo = band_cut ? i - lw + 1 - (j0 + 64 * g) : 0;
                     fwd_row<true, 0, false, F8>(sv, wr, tj, ti1f, E, 0.f, 0.f, 0.f, c_lo, c_lim, pk, KSw, rsq);
                 }
+            } else if (CAND && i0 >= hist && j0 == i0) {
+                p_tile_own<F8>(trow + s * TBN + 64 * g, i - j0 - 64 * g, row_ok,
+                               p.rab_pos[pos_index(hist, hist, p.pos_lo, p.pos_hi)] + p.rab_time[0], rsq, KSw);
+                stored = true;
+            } else if (CAND) {
+                p_tile_exact<F8>(trow + s * TBN + 64 * g, i, row_ok, j0 + 64 * g, L, hist, lw, gw, pi, ti,
+                                 p.timestamps + s0, p.rab_pos, p.rab_time, p.pos_lo, p.pos_hi, p.nb, rsq, KSw);
+                stored = true;
             } else {
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
@@ -517,8 +601,10 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 }
             }
             // P over the first 32 of this thread's S columns (already read)
-            tmem_st16(trow + s * TBN + 64 * g, pk);
-            tmem_st16(trow + s * TBN + 64 * g + 16, pk + 16);
+            if (!stored) {
+                tmem_st16(trow + s * TBN + 64 * g, pk);
+                tmem_st16(trow + s * TBN + 64 * g + 16, pk + 16);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -527,7 +613,37 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         }
         if (!(ok = ok && mbar_wait(bar(O_FULL), u & 1, abort_flag, p.hdr)))
             break;
-        {
+        if (CAND && o_tma && i0 + 32 * quarter + 32 <= L) {
+            // every row of this warp in the sequence: [32 x 32] boxes through shared
+            // memory and one TMA store each (coalesced, one instruction per box)
+            tc_fence_after();
+            unsigned char *stg = sm + LY::OST + ew * 2048;
+#pragma unroll
+            for (int cc = 0; cc < D / 2; cc += 32) {
+                float ov[32];
+                tmem_ld32(trow + 2 * TBN + g * (D / 2) + cc, ov);
+                tmem_wait_ld();
+                uint4 packed[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++)
+                    packed[q4] = make_uint4(pack_bf16(ov[8 * q4] * p.inv_n, ov[8 * q4 + 1] * p.inv_n),
+                                            pack_bf16(ov[8 * q4 + 2] * p.inv_n, ov[8 * q4 + 3] * p.inv_n),
+                                            pack_bf16(ov[8 * q4 + 4] * p.inv_n, ov[8 * q4 + 5] * p.inv_n),
+                                            pack_bf16(ov[8 * q4 + 6] * p.inv_n, ov[8 * q4 + 7] * p.inv_n));
+                if (lane == 0)
+                    bulk_wait_read0();  // the previous box has been read out
+                __syncwarp();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++)
+                    *reinterpret_cast<uint4 *>(stg + lane * 64 + ((q4 ^ ((lane >> 1) & 3)) << 4)) = packed[q4];
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&to, h * D + g * (D / 2) + cc, (int)(s0 + i0 + 32 * quarter), smem_u32(stg));
+                    bulk_commit();
+                }
+            }
+        } else {
             tc_fence_after();
             __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (s0 + i) * p.so + (int64_t)h * D + g * (D / 2);
 #pragma unroll
@@ -554,6 +670,8 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         if (lane == 0)
             mbar_arrive(bar(O_FREE));
         }
+        if (lane == 0)
+            bulk_wait0();  // the O boxes have left shared memory
     }
     tc_fence_before();
     __syncthreads();
@@ -577,7 +695,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-template <int D, bool SL, bool F8 = false>
+template <int D, bool SL, bool F8 = false, bool CAND = false>
 cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
     CUtensorMap maps[3];
@@ -599,8 +717,17 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
         e = make_row_tensor_map(&maps[2], ptrs[2], p.T, p.H * D, strides[2]);
     if (e != cudaSuccess)
         return e;
-    const size_t bytes = FwdLayout<D, F8>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    // O by TMA stores of [32 x 32] boxes where its rows are 16-byte aligned;
+    // otherwise (and for warps whose rows run past the sequence) plain stores
+    CUtensorMap mo;
+    memset(&mo, 0, sizeof(mo));
+    int o_tma = CAND && (reinterpret_cast<uintptr_t>(p.o) % 16 == 0) && (p.so * 2) % 16 == 0;
+    if (o_tma && make_tensor_map_2d(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.T, p.H * D, p.so * 2, 32, 32,
+                                    CU_TENSOR_MAP_SWIZZLE_64B) != cudaSuccess)
+        o_tma = 0;
+    const size_t bytes = FwdLayout<D, F8, CAND>::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL, F8, CAND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bytes);
     if (e != cudaSuccess)
         return e;
     // persistent: at most one CTA per SM, each walking its share of the work units
@@ -613,7 +740,7 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     }
     const int64_t units = (int64_t)grid_items * p.H;
     const unsigned grid = (unsigned)std::min<int64_t>(units, sms);
-    attn_fwd_tc_kernel<D, SL, F8><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2]);
+    attn_fwd_tc_kernel<D, SL, F8, CAND><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2], mo, o_tma);
     return cudaGetLastError();
 }
 
@@ -653,13 +780,21 @@ cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t
 {
     if (grid_items <= 0)
         return cudaSuccess;
+    const bool cand = p.num_targets != nullptr;  // FP8 scores keep the one instantiation
     switch (p.dqk) {
-    case 64: return p.lw > 0 ? fwd_tc_launch<64, true>(p, grid_items, stream)
-                             : fwd_tc_launch<64, false>(p, grid_items, stream);
+    case 64:
+        if (cand)
+            return p.lw > 0 ? fwd_tc_launch<64, true, false, true>(p, grid_items, stream)
+                            : fwd_tc_launch<64, false, false, true>(p, grid_items, stream);
+        return p.lw > 0 ? fwd_tc_launch<64, true>(p, grid_items, stream)
+                        : fwd_tc_launch<64, false>(p, grid_items, stream);
     case 128:
         if (p.q8)  // FP8 scores
             return p.lw > 0 ? fwd_tc_launch<128, true, true>(p, grid_items, stream)
                             : fwd_tc_launch<128, false, true>(p, grid_items, stream);
+        if (cand)
+            return p.lw > 0 ? fwd_tc_launch<128, true, false, true>(p, grid_items, stream)
+                            : fwd_tc_launch<128, false, false, true>(p, grid_items, stream);
         return p.lw > 0 ? fwd_tc_launch<128, true>(p, grid_items, stream)
                         : fwd_tc_launch<128, false>(p, grid_items, stream);
     default: return cudaErrorInvalidValue;

@@ -221,6 +221,33 @@ def test_bwd_f32(cuda_device):
     _check_bwd(gpu_bwd(inp, cuda_device), _oracle_bwd(inp), assert_f32_close, "bwd f32")
 
 
+def _blockwise_stamps(lengths, seed, spread):
+    """Stamps sorted inside every aligned 32-token block but descending from
+    block to block, so that visible pairs across blocks have negative
+    differences while every warp's keys and queries are each sorted; `spread`
+    makes the gaps inside a block grow geometrically (rows over many buckets)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for L in lengths:
+        for b in range(0, L, 32):
+            n = min(32, L - b)
+            gaps = rng.exponential(300.0, n) * (spread ** np.arange(n))
+            out.append(10**7 - 200_000 * (b // 32) + np.cumsum(gaps).astype(np.int64))
+    return torch.from_numpy(np.concatenate(out).astype(np.int64))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("spread", [1.0, 1.3])
+def test_blockwise_sorted_stamps(cuda_device, d, spread):
+    # fast-path classes with negative cross-block differences (bucket 0) and
+    # rows spanning many buckets; forward and backward with the bias grads
+    lengths = [200, 96, 130]
+    inp = _small(lengths, H=2, d=d, seed=40 + d, nb=32)
+    inp = dataclasses.replace(inp, timestamps=_blockwise_stamps(lengths, 41 + d, spread))
+    assert_bf16_close(gpu_fwd(inp, cuda_device), _oracle_fwd(inp), what=f"fwd d={d} spread={spread}")
+    _check_bwd(gpu_bwd(inp, cuda_device), _oracle_bwd(inp), assert_bf16_close, f"bwd d={d} spread={spread}")
+
+
 def test_bwd_long_history_full_size_sampled(cuda_device):
     w = workloads.WORKLOADS["long_history_bf16"]
     inp = workloads.generate(w)
