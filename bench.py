@@ -44,12 +44,11 @@ LAUNCHES_PER_STEP = 5
 SEMI_LOCAL = (1024, 256)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention-backward launch on
 # this workload, from a one-pass ncu capture of
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_ -c 2
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd -c 1
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
-# (the second captured launch is the backward); valid only for the kernel source it was taken on
-# (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "5d4f19369838ce28cccee2a2625c3d96593ec104c8664fa113f79f77dd63c254",
-               "bytes": 602.77e6 + 346.32e6}
+# valid only for the kernel source it was taken on (else the line reports null)
+BWD_TRAFFIC = {"source_sha256": "f95cf640f241b868eba53bffc8f6f06bc29fcc154eff7e74d5dfb27f10f64d95",
+               "bytes": 616.24e6 + 355.64e6}
 
 
 def bwd_traffic():

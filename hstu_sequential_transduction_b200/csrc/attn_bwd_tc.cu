@@ -225,7 +225,8 @@ template <int DH, bool SL>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
-                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ, int head_major)
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ, int head_major,
+                   const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV, int kv_tma)
 {
     using BL = hstu::BL<DH>;
     constexpr int NR = BL::NR;
@@ -707,6 +708,44 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             constexpr int DC = DH / kGroupsB;  // dK / dV columns per thread
             __nv_bfloat16 *gdk = static_cast<__nv_bfloat16 *>(p.dk) + (s0 + j) * p.sdk + (int64_t)h * DH + DC * g;
             __nv_bfloat16 *gdv = static_cast<__nv_bfloat16 *>(p.dvv) + (s0 + j) * p.sdv + (int64_t)h * DH + DC * g;
+            if (kv_tma && j0 + 32 * quarter + 32 <= L) {
+                // every key row of this warp in the sequence: [32 x 32] boxes staged
+                // in the (now idle) Q / dO ring and written by TMA stores, instead
+                // of 16-byte stores from every row
+                unsigned char *stg = sm + BL::Q0 + ew * (2 * DC / 32) * 2048;
+#pragma unroll
+                for (int which = 0; which < 2; which++) {
+                    const uint32_t col = (which ? COL_DV : COL_DK) + DC * g;
+                    const float scale = which ? p.inv_n : gscale;
+#pragma unroll
+                    for (int cc = 0; cc < DC; cc += 32) {
+                        float v[32];
+                        tmem_ld32(trow + col + cc, v);
+                        tmem_wait_ld();
+                        unsigned char *box = stg + (which * (DC / 32) + cc / 32) * 2048;
+#pragma unroll
+                        for (int u = 0; u < 4; u++) {
+                            uint4 w;
+                            w.x = pack_bf16(v[8 * u] * scale, v[8 * u + 1] * scale);
+                            w.y = pack_bf16(v[8 * u + 2] * scale, v[8 * u + 3] * scale);
+                            w.z = pack_bf16(v[8 * u + 4] * scale, v[8 * u + 5] * scale);
+                            w.w = pack_bf16(v[8 * u + 6] * scale, v[8 * u + 7] * scale);
+                            *reinterpret_cast<uint4 *>(box + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) = w;
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int which = 0; which < 2; which++)
+#pragma unroll
+                        for (int cc = 0; cc < DC; cc += 32)
+                            tma_store_2d(which ? &tmDV : &tmDK, h * DH + DC * g + cc, (int)(s0 + j0 + 32 * quarter),
+                                         smem_u32(stg + (which * (DC / 32) + cc / 32) * 2048));
+                    bulk_commit();
+                }
+            } else {
 #pragma unroll
             for (int which = 0; which < 2; which++) {
                 const uint32_t col = (which ? COL_DV : COL_DK) + DC * g;
@@ -729,6 +768,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         }
                     }
                 }
+            }
             }
         }
         if (lane == 0)
@@ -795,7 +835,19 @@ cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     const int64_t l2 = dev_info.y;
     const int64_t max_tiles = ((int64_t)p.max_seq_len + KB - 1) / KB;
     const int head_major = p.lw == 0 && max_tiles * p.H > sms && p.T * p.H * 8 * DH > 2 * l2;
-    kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq, head_major);
+    // dK and dV by TMA stores of [32 x 32] boxes where their rows are 16-byte aligned
+    CUtensorMap mdk, mdv;
+    memset(&mdk, 0, sizeof(mdk));
+    memset(&mdv, 0, sizeof(mdv));
+    int kv_tma = reinterpret_cast<uintptr_t>(p.dk) % 16 == 0 && reinterpret_cast<uintptr_t>(p.dvv) % 16 == 0 &&
+                 (p.sdk * 2) % 16 == 0 && (p.sdv * 2) % 16 == 0;
+    if (kv_tma && (make_tensor_map_2d(&mdk, p.dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.T, cols, p.sdk * 2, 32, 32,
+                                      CU_TENSOR_MAP_SWIZZLE_64B) != cudaSuccess ||
+                   make_tensor_map_2d(&mdv, p.dvv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.T, cols, p.sdv * 2, 32, 32,
+                                      CU_TENSOR_MAP_SWIZZLE_64B) != cudaSuccess))
+        kv_tma = 0;
+    kern<<<(unsigned)grid_items * p.H, kThreadsB, bytes, stream>>>(p, mk, mv, mq, mo, mdq, head_major, mdk, mdv,
+                                                                     kv_tma);
     return cudaGetLastError();
 }
 
