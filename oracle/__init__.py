@@ -114,6 +114,22 @@ def visible_sl(i: int, j: int, L: int, n_t: int, local_window: int, global_windo
                                           int(global_window)))
 
 
+def bias_pair_counts(seq_offsets, timestamps, num_targets, pos_lo, pos_hi, num_buckets,
+                     local_window=0, global_window=0, threads=None):
+    """Visible pairs per rab_pos entry and per rab_time bucket, one head (int64
+    arrays [pos_hi - pos_lo + 1] and [num_buckets]), with the attention's own
+    visibility rule, windows and index functions."""
+    off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
+    pc = np.zeros(int(pos_hi) - int(pos_lo) + 1, dtype=np.int64)
+    tc = np.zeros(int(num_buckets), dtype=np.int64)
+    _load().oracle_bias_pair_counts(ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), _p(ts, _i64p),
+                                    ctypes.c_int(int(pos_lo)), ctypes.c_int(int(pos_hi)),
+                                    ctypes.c_int(int(num_buckets)), ctypes.c_int64(int(local_window)),
+                                    ctypes.c_int64(int(global_window)), _p(pc, _i64p), _p(tc, _i64p),
+                                    ctypes.c_int(threads or default_threads()))
+    return pc, tc
+
+
 class _Windows:
     """Semi-local windows applied by the oracle's attention for the duration of one call."""
 

@@ -260,6 +260,54 @@ void oracle_attn_fwd_rows(int num_seqs, const int64_t *seq_offsets, const int32_
     }
 }
 
+/* ---- visible pairs per bias entry --------------------------------------- */
+
+/*
+ * How many visible pairs of the batch land on each relative-bias entry (one
+ * head): pos_counts [pos_hi - pos_lo + 1] and time_counts [num_buckets],
+ * int64, overwritten.  Every pair goes through the same visibility rule (with
+ * the semi-local windows local, global) and index functions as the attention.
+ * When every visible pair carries the same score gradient g, the gradient of
+ * rab_pos[e] is H g pos_counts[e] and that of rab_time[k] is H g time_counts[k]
+ * (the tables are shared by the heads).  Sequences run in parallel, each into
+ * its own count arrays, added up in sequence order.
+ */
+void oracle_bias_pair_counts(int num_seqs, const int64_t *seq_offsets, const int32_t *num_targets,
+                             const int64_t *timestamps, int pos_lo, int pos_hi, int num_buckets,
+                             int64_t local, int64_t global, int64_t *pos_counts, int64_t *time_counts,
+                             int num_threads)
+{
+    const int npos = pos_hi - pos_lo + 1;
+    int64_t *per_pos = (int64_t *)calloc((size_t)(num_seqs > 0 ? num_seqs : 1) * npos, sizeof(int64_t));
+    int64_t *per_time = (int64_t *)calloc((size_t)(num_seqs > 0 ? num_seqs : 1) * num_buckets, sizeof(int64_t));
+    set_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < num_seqs; b++) {
+        const int64_t s0 = seq_offsets[b], L = seq_offsets[b + 1] - s0;
+        const int64_t n_t = num_targets ? (int64_t)num_targets[b] : 0;
+        int64_t *pc = per_pos + (size_t)b * npos, *tc = per_time + (size_t)b * num_buckets;
+        for (int64_t i = 0; i < L; i++)
+            for (int64_t j = 0; j < L; j++) {
+                if (!oracle_visible_sl(i, j, L, n_t, local, global))
+                    continue;
+                pc[oracle_pos_index(token_pos(i, L, n_t), token_pos(j, L, n_t), pos_lo, pos_hi)]++;
+                tc[oracle_time_bucket(timestamps[s0 + i], timestamps[s0 + j], num_buckets)]++;
+            }
+    }
+    for (int e = 0; e < npos; e++)
+        pos_counts[e] = 0;
+    for (int k = 0; k < num_buckets; k++)
+        time_counts[k] = 0;
+    for (int b = 0; b < num_seqs; b++) {
+        for (int e = 0; e < npos; e++)
+            pos_counts[e] += per_pos[(size_t)b * npos + e];
+        for (int k = 0; k < num_buckets; k++)
+            time_counts[k] += per_time[(size_t)b * num_buckets + k];
+    }
+    free(per_pos);
+    free(per_time);
+}
+
 /* ---- attention backward ------------------------------------------------- */
 /*
  * Exact derivatives of the forward above for the loss sum(O * dO):

@@ -765,3 +765,101 @@ def test_windowed_layer_is_the_composition_with_windowed_attention():
     np.testing.assert_allclose(y, oracle.linear(g, w2, b2), rtol=0, atol=1e-12)
     # and differs from the full-mask layer
     assert np.abs(y - oracle.layer_fwd(*args, x, w1, b1, w2, b2, gam, bet, *tables, H, dqk, dv)).max() > 1e-6
+
+
+# ---- visible pairs per bias entry --------------------------------------------
+
+def _counts(lengths, ts, nts=None, lo=0, hi=10**6, nb=64, local=0, glob=0):
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    return oracle.bias_pair_counts(off, np.asarray(ts, dtype=np.int64), nts, lo, hi, nb, local, glob)
+
+
+def test_bias_pair_counts_causal_unit_gaps_closed_form():
+    # one causal sequence with stamps t_j = j: distance k = i - j occurs L - k times,
+    # and bucket b holds the distances 2^b - 1 .. 2^(b+1) - 2 (the last bucket the rest)
+    L, nb = 300, 6
+    pc, tc = _counts([L], np.arange(L), lo=0, hi=L - 1, nb=nb)
+    assert list(pc) == [L - k for k in range(L)]
+    exp = []
+    for b in range(nb):
+        lo_d = 2 ** b - 1
+        hi_d = 2 ** (b + 1) - 2 if b < nb - 1 else L - 1
+        exp.append(sum(L - d for d in range(lo_d, min(hi_d, L - 1) + 1)))
+    assert list(tc) == exp
+    assert tc.sum() == pc.sum() == L * (L + 1) // 2
+
+
+def test_bias_pair_counts_clamps_closed_form():
+    L, lo, hi = 120, 2, 40
+    pc, _ = _counts([L], np.zeros(L), lo=lo, hi=hi, nb=4)
+    assert pc[0] == sum(L - d for d in range(0, lo + 1))          # distances 0..2 clamp to 2
+    assert pc[-1] == (L - hi) * (L - hi + 1) // 2                 # distances >= 40 clamp to 40
+    assert list(pc[1:-1]) == [L - d for d in range(lo + 1, hi)]
+
+
+def test_bias_pair_counts_candidates_closed_form():
+    # 43 history tokens + 7 candidates at position 43 with the last history stamp:
+    # history pairs as before, each candidate adds one pair at distances 1..43 and its own at 0
+    hist, nt = 43, 7
+    L = hist + nt
+    ts = np.concatenate([np.arange(hist) * 5, np.full(nt, (hist - 1) * 5)])
+    pc, tc = _counts([L], ts, nts=np.array([nt], dtype=np.int32), lo=0, hi=100, nb=40)
+    exp = np.zeros(101, dtype=np.int64)
+    for k in range(hist):
+        exp[k] += hist - k
+    exp[1:hist + 1] += nt
+    exp[0] += nt
+    assert np.array_equal(pc, exp)
+    assert tc.sum() == hist * (hist + 1) // 2 + nt * (hist + 1)
+    # a candidate and its own pair: dt = 0 -> bucket 0, as for every diagonal pair
+    assert tc[0] >= hist + nt
+
+
+def test_bias_pair_counts_local_window_closed_form():
+    # causal, local window 10, first 3 keys global: distance k < 10 keeps all L - k pairs,
+    # a larger distance only the pairs whose key is global
+    L, w, g = 100, 10, 3
+    pc, _ = _counts([L], np.arange(L), lo=0, hi=L - 1, nb=8, local=w, glob=g)
+    exp = [L - k if k < w else min(g, L - k) for k in range(L)]
+    assert list(pc) == exp
+
+
+def test_bias_pair_counts_by_brute_force():
+    # random tiny batch with candidates, windows, unsorted stamps and an empty sequence,
+    # against loops over the scalar visibility and index functions
+    rng = np.random.default_rng(3)
+    lengths, nts = [9, 0, 14, 5], np.array([2, 0, 4, 0], dtype=np.int32)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    ts = rng.integers(0, 3000, size=off[-1]).astype(np.int64)
+    lo, hi, nb, w, g = -2, 6, 7, 4, 2
+    pc, tc = oracle.bias_pair_counts(off, ts, nts, lo, hi, nb, w, g)
+    epc, etc = np.zeros_like(pc), np.zeros_like(tc)
+    for b, L in enumerate(lengths):
+        n = int(nts[b])
+        hist = L - n
+        for i in range(L):
+            for j in range(L):
+                if not oracle.visible_sl(i, j, L, n, w, g):
+                    continue
+                epc[oracle.pos_index(min(i, hist), min(j, hist), lo, hi)] += 1
+                etc[oracle.time_bucket(ts[off[b] + i], ts[off[b] + j], nb)] += 1
+    assert np.array_equal(pc, epc) and np.array_equal(tc, etc)
+
+
+def test_bias_pair_counts_are_the_uniform_score_gradient():
+    # q = k = 0 and zero tables give s = 0 on every visible pair; with v = dout = 1 every
+    # pair's dS is d_v SiLU'(0) / N = d_v / (2N), so the backward's table gradients are
+    # H d_v / (2N) times the pair counts (the backward is pinned by finite differences)
+    rng = np.random.default_rng(8)
+    lengths, nts = [12, 7, 0, 20], np.array([3, 0, 0, 5], dtype=np.int32)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T, H, d, lo, hi, nb, inv_n = int(off[-1]), 2, 4, -3, 9, 6, 1 / 16
+    ts = np.cumsum(rng.integers(0, 40, size=T)).astype(np.int64)
+    z = np.zeros((T, H, d))
+    one = np.ones((T, H, d))
+    for w, g in [(0, 0), (5, 2)]:
+        _, _, _, drp, drt = oracle.attn_bwd(off, ts, nts, z, z, one, np.zeros(hi - lo + 1), np.zeros(nb),
+                                            lo, hi, inv_n, one, local_window=w, global_window=g)
+        pc, tc = oracle.bias_pair_counts(off, ts, nts, lo, hi, nb, w, g)
+        assert np.array_equal(drp, pc * (H * d * 0.5 * inv_n))
+        assert np.array_equal(drt, tc * (H * d * 0.5 * inv_n))
