@@ -781,14 +781,27 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         tmem_dealloc(tmem, kTmemColsB);
 }
 
-}  // namespace
-
-bool attn_bwd_tc_supported(const AttnParams &p)
+// dQ (bf16, row stride sdq) = scale * the fp32 accumulator [T, H d]: eight
+// elements per thread and iteration (two 16-byte loads, one 16-byte store);
+// H d is a multiple of 64, so a group of eight never crosses a row.
+__global__ void __launch_bounds__(256)
+convert_dq_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *__restrict__ dq, int64_t T, int hd, int64_t sdq,
+                  float scale)
 {
-    return p.dqk == p.dv && (p.dqk == 64 || p.dqk == 128) && attn_tc_supported(p);
+    const int64_t groups = T * (hd / 8);
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < groups;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = e / (hd / 8);
+        const int c = (int)(e - t * (hd / 8)) * 8;
+        const float4 a = acc[2 * e], b = acc[2 * e + 1];
+        uint4 w;
+        w.x = pack_bf16(a.x * scale, a.y * scale);
+        w.y = pack_bf16(a.z * scale, a.w * scale);
+        w.z = pack_bf16(b.x * scale, b.y * scale);
+        w.w = pack_bf16(b.z * scale, b.w * scale);
+        *reinterpret_cast<uint4 *>(dq + t * sdq + c) = w;
+    }
 }
-
-namespace {
 
 template <int DH>
 cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
@@ -822,17 +835,9 @@ cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     // side by side balance better (same-process timings: head-major 10-34 %
     // faster on long-history batches, 3-19 % slower on short, Zipf and
     // windowed ones).
-    static const int2 dev_info = [] {
-        int dev = 0, sms = 0, l2 = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-        if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0)
-            l2 = 126 << 20;
-        return make_int2(sms, l2);
-    }();
-    const int sms = dev_info.x;
-    const int64_t l2 = dev_info.y;
+    const DeviceInfo info = device_info();
+    const int sms = info.sms;
+    const int64_t l2 = info.l2_bytes;
     const int64_t max_tiles = ((int64_t)p.max_seq_len + KB - 1) / KB;
     const int head_major = p.lw == 0 && max_tiles * p.H > sms && p.T * p.H * 8 * DH > 2 * l2;
     // dK and dV by TMA stores of [32 x 32] boxes where their rows are 16-byte aligned
@@ -855,9 +860,24 @@ cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
 
 cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
-    if (grid_items <= 0)
+    if (grid_items <= 0 || p.T == 0)
         return cudaSuccess;
     return p.dqk == 64 ? bwd_tc_launch<64>(p, grid_items, stream) : bwd_tc_launch<128>(p, grid_items, stream);
+}
+
+cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int d, int64_t sdq,
+                              float scale, cudaStream_t stream)
+{
+    if (T == 0)
+        return cudaSuccess;
+    // 16-byte stores: the caller's dq rows start on 16-byte boundaries
+    if ((H * d) % 8 || sdq % 8 || (reinterpret_cast<uintptr_t>(dq) & 15u))
+        return cudaErrorInvalidValue;
+    const int64_t groups = T * (H * d / 8);
+    const int blocks = (int)std::min<int64_t>((groups + 255) / 256, (int64_t)device_info().sms * 8);
+    convert_dq_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(acc),
+                                                  static_cast<__nv_bfloat16 *>(dq), T, H * d, sdq, scale);
+    return cudaGetLastError();
 }
 
 }  // namespace hstu

@@ -322,7 +322,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             for (int u = 0, w = unit_index(0); ok && w < n_units; u++, w = unit_index(u)) {
                 const Unit U = unit(w);
                 const int qs = u & 1;
-                if (u >= 2 && !(ok = mbar_wait(bar(Q_EMPTY + qs), ((u >> 1) - 1) & 1, abort_flag, p.hdr)))
+                if (u >= 2 && !(ok = mbar_wait(bar(Q_EMPTY + qs), ((u >> 1) - 1) & 1, abort_flag, p.hdr, p.wait_limit)))
                     break;
                 mbar_expect_tx(bar(Q_FULL + qs), LY::QKT);
                 for (int r = 0; r < LY::QKT / kRegion; r++)
@@ -331,13 +331,17 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 for (int t = 0; t < U.ntiles; t++, g++) {
                     const int s = g & 1;
                     const int j0 = U.tile_of(t) * TBN;
-                    if (g >= 2 && !(ok = mbar_wait(bar(K_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
+                    if (g >= 2 && !(ok = mbar_wait(bar(K_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr, p.wait_limit)))
                         break;
+                    // test hook: CTA 0 never loads its first key tile, so the waits on
+                    // it run out (every load that is issued still completes)
+                    if (g == 0 && p.withhold_first_k && blockIdx.x == 0)
+                        continue;
                     mbar_expect_tx(bar(K_FULL + s), LY::QKT);
                     for (int r = 0; r < LY::QKT / kRegion; r++)
                         tma_load_2d(base + LY::K0 + s * LY::QKT + r * kRegion, &tk, U.h * D + 64 * r,
                                     (int)(U.s0 + j0), bar(K_FULL + s));
-                    if (g >= 2 && !(ok = mbar_wait(bar(V_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr)))
+                    if (g >= 2 && !(ok = mbar_wait(bar(V_EMPTY + s), ((g >> 1) - 1) & 1, abort_flag, p.hdr, p.wait_limit)))
                         break;
                     mbar_expect_tx(bar(V_FULL + s), LY::TILE);
                     for (int r = 0; r < LY::NREG; r++)
@@ -386,18 +390,18 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             };
             // S buffer g % 2 is free once P V of tile g - 2 has completed
             auto s_free = [&](int g) {
-                return g < 2 || mbar_wait(bar(P_FREE + (g & 1)), ((g >> 1) - 1) & 1, abort_flag, p.hdr);
+                return g < 2 || mbar_wait(bar(P_FREE + (g & 1)), ((g >> 1) - 1) & 1, abort_flag, p.hdr, p.wait_limit);
             };
             bool ok = true;
             int gb = 0;  // first tile of the current unit
             for (int u = 0, w = unit_index(0); ok && w < n_units; u++, w = unit_index(u)) {
                 const Unit U = unit(w);
                 const int qs = u & 1, nt = U.ntiles;
-                if (!(ok = mbar_wait(bar(Q_FULL + qs), (u >> 1) & 1, abort_flag, p.hdr)))
+                if (!(ok = mbar_wait(bar(Q_FULL + qs), (u >> 1) & 1, abort_flag, p.hdr, p.wait_limit)))
                     break;
                 for (int t = 0; ok && t < min(2, nt); t++) {
                     const int g = gb + t;
-                    ok = s_free(g) && mbar_wait(bar(K_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr);
+                    ok = s_free(g) && mbar_wait(bar(K_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr, p.wait_limit);
                     if (ok) {
                         tc_fence_after();
                         issue_S(g, qs);
@@ -407,18 +411,18 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     umma_commit(bar(Q_EMPTY + qs));
                 // the previous unit's O has been read out of TMEM
                 if (ok && u >= 1)
-                    ok = mbar_wait(bar(O_FREE), (u - 1) & 1, abort_flag, p.hdr);
+                    ok = mbar_wait(bar(O_FREE), (u - 1) & 1, abort_flag, p.hdr, p.wait_limit);
                 for (int j = 0; ok && j < nt; j++) {
                     const int g = gb + j;
-                    ok = mbar_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr) &&
-                         mbar_wait(bar(V_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr);
+                    ok = mbar_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr, p.wait_limit) &&
+                         mbar_wait(bar(V_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.hdr, p.wait_limit);
                     if (!ok)
                         break;
                     tc_fence_after();
                     issue_PV(g, j == 0);
                     if (j + 2 < nt) {
                         ok = s_free(g + 2) &&
-                             mbar_wait(bar(K_FULL + (g & 1)), ((g + 2) >> 1) & 1, abort_flag, p.hdr);
+                             mbar_wait(bar(K_FULL + (g & 1)), ((g + 2) >> 1) & 1, abort_flag, p.hdr, p.wait_limit);
                         if (!ok)
                             break;
                         tc_fence_after();
@@ -522,7 +526,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             if (t + 1 < ntiles)
                 prep(t + 1);
 
-            if (!(ok = mbar_wait(bar(S_FULL + s), (gtile >> 1) & 1, abort_flag, p.hdr)))
+            if (!(ok = mbar_wait(bar(S_FULL + s), (gtile >> 1) & 1, abort_flag, p.hdr, p.wait_limit)))
                 break;
             tc_fence_after();
             float sv[64];
@@ -611,7 +615,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
             if (lane == 0)
                 mbar_arrive(bar(P_FULL + s));
         }
-        if (!(ok = ok && mbar_wait(bar(O_FULL), u & 1, abort_flag, p.hdr)))
+        if (!(ok = ok && mbar_wait(bar(O_FULL), u & 1, abort_flag, p.hdr, p.wait_limit)))
             break;
         if (CAND && o_tma && i0 + 32 * quarter + 32 <= L) {
             // every row of this warp in the sequence: [32 x 32] boxes through shared
@@ -682,16 +686,15 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // looked up once per process (a function-local static: thread-safe)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    }();
     return fn;
 }
 
@@ -731,13 +734,7 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     if (e != cudaSuccess)
         return e;
     // persistent: at most one CTA per SM, each walking its share of the work units
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
+    const int sms = device_info().sms;
     const int64_t units = (int64_t)grid_items * p.H;
     const unsigned grid = (unsigned)std::min<int64_t>(units, sms);
     attn_fwd_tc_kernel<D, SL, F8, CAND><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2], mo, o_tma);
@@ -770,15 +767,16 @@ cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows
                               64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+bool tensor_maps_available() { return tensor_map_encoder() != nullptr; }
+
 bool attn_tc_supported(const AttnParams &p)
 {
-    return (p.dqk == 64 || p.dqk == 128) && p.dv == p.dqk && p.T > 0 && p.T < ((int64_t)1 << 31) - 256 &&
-           tensor_map_encoder() != nullptr;
+    return (p.dqk == 64 || p.dqk == 128) && p.dv == p.dqk && p.T >= 0 && p.T < ((int64_t)1 << 31) - 256;
 }
 
 cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
-    if (grid_items <= 0)
+    if (grid_items <= 0 || p.T == 0)
         return cudaSuccess;
     const bool cand = p.num_targets != nullptr;  // FP8 scores keep the one instantiation
     switch (p.dqk) {

@@ -31,6 +31,13 @@ enum : int {
     FLAG_TOTAL = 16,
 };
 
+// A pipeline wait that runs out records FLAG_TIMEOUT in the header's flag.
+enum : int { FLAG_TIMEOUT = 32 };
+constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
+// the limit under the bounded-wait test hook (HSTU_DEBUG_WAIT_TEST): ~1 ms, far
+// above any wait of a working pipeline (a few tile times), short for a test
+constexpr long long kTestWaitLimitCycles = 2000000LL;
+
 // Everything an attention kernel reads; strides are in elements between rows.
 struct AttnParams {
     const void *q, *k, *v;
@@ -51,6 +58,11 @@ struct AttnParams {
     const float *sq8, *sk8;
     const int2 *items;
     WsHeader *hdr;
+    // clock cycles after which a pipeline wait gives up (FLAG_TIMEOUT), and the
+    // test hook of the bounded waits: the forward's first CTA withholds the load
+    // of its first key tile
+    long long wait_limit;
+    int withhold_first_k;
     // backward only
     const void *dout;
     int64_t sdo;
@@ -92,12 +104,7 @@ __device__ __forceinline__ bool visible_w(int i, int j, int hist, int lw, int gw
     return visible(i, j, hist) && (lw <= 0 || token_pos(i, hist) - token_pos(j, hist) < lw || j < gw);
 }
 
-// SiLU on the fp32 score.  The fast form uses the hardware exponential.
-__device__ __forceinline__ float silu_fast(float x)
-{
-    return x * __frcp_rn(1.0f + __expf(-x));
-}
-
+// SiLU and its derivative on the fp32 path (IEEE division, expf).
 __device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
 
 __device__ __forceinline__ float silu_grad_precise(float x)
@@ -106,52 +113,11 @@ __device__ __forceinline__ float silu_grad_precise(float x)
     return s * (1.0f + x * (1.0f - s));
 }
 
-// ---- bf16 / async-copy / tensor-core helpers (legacy mma.sync path) -------
+// ---- shared-memory addresses and bf16 packing -------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// 16-byte async copy; src_bytes < 16 zero-fills the rest.
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
-                 "l"(gmem), "r"(src_bytes));
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
-                                            const void *p)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(smem_u32(p)));
-}
-
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2,
-                                                  uint32_t &r3, const void *p)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(smem_u32(p)));
-}
-
-// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_16816(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)

@@ -107,7 +107,7 @@ cudaError_t launch_quantize_rows_e4m3(const void *x, int64_t ldx, int64_t R, int
 {
     if (R == 0)
         return cudaSuccess;
-    const unsigned blocks = (unsigned)std::min<int64_t>((R + 7) / 8, 148 * 8);
+    const unsigned blocks = (unsigned)std::min<int64_t>((R + 7) / 8, (int64_t)device_info().sms * 8);
     quantize_rows_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), ldx, R, K,
                                                      static_cast<unsigned char *>(q), ldq, scale);
     return cudaGetLastError();

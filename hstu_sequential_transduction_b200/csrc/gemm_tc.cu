@@ -5,7 +5,8 @@
 // ("DLRMv4 Brings Sequence-Based Recommendation Training to MLPerf", section
 // "Model Architecture": the projection that produces U, V, Q, K, and the output
 // projection after the gate; their gradients for the layer backward.)
-// Persistent tiles of 128 x BN (BN = 256 or 128): warp 0 streams A and B
+// Persistent tiles of 128 x BN (BN = 256 when it divides N, else 128 with a
+// partial last column tile; N a multiple of 32): warp 0 streams A and B
 // through a 4-stage ring of 64-deep k-slices; warp 1 owns two TMEM
 // accumulators and issues tcgen05.mma from one thread; warps 2-9 read one
 // accumulator row by row while the next tile accumulates in the other.
@@ -104,7 +105,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     constexpr int KE = F8 ? 128 : GBK;     // K elements per 128-byte slice
     const int nk = (g.K + KE - 1) / KE;    // the TMA zero-fills past K
     const int per = (nk + g.splits - 1) / g.splits;  // k-slices per split
-    const int tiles_n = g.N / BN;
+    // N a multiple of 32: the last column tile may be partial (its B columns past
+    // N load as zeros, its output chunks past N are skipped)
+    const int tiles_n = (g.N + BN - 1) / BN;
     const int tiles = (int)((g.M + GBM - 1) / GBM) * tiles_n;
     const int units = tiles * g.splits;
     auto full_bar = [&](int s) { return base + LY::BAR + 8u * s; };
@@ -239,7 +242,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int64_t row = rowbase + lane;
             const int n0 = (tile % tiles_n) * BN + half * CW;
 #pragma unroll 1
-            for (int cc = 0; cc < CW; cc += 32) {
+            for (int cc = 0; cc < CW && n0 + cc < g.N; cc += 32) {
                 float v[32];
                 tmem_ld32(trow + ab * BN + half * CW + cc, v);
                 if (EPI == EPI_RED) {
@@ -352,18 +355,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tmem_dealloc(tmem, 2 * BN);
 }
 
-int num_sms()
-{
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 template <int BN, bool A_MN, bool B_K, int EPI, bool F8 = false>
 cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stream)
 {
@@ -411,8 +402,8 @@ cudaError_t gemm_tc_launch(const GemmOperands &op, GemmArgs g, cudaStream_t stre
                              (int)bytes);
     if (e != cudaSuccess)
         return e;
-    const int64_t units = ((g.M + GBM - 1) / GBM) * (g.N / BN) * g.splits;
-    const unsigned grid = (unsigned)std::min<int64_t>(units, num_sms());
+    const int64_t units = ((g.M + GBM - 1) / GBM) * ((g.N + BN - 1) / BN) * g.splits;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, device_info().sms);
     gemm_tc_kernel<BN, A_MN, B_K, EPI, F8><<<grid, kThreadsG, bytes, stream>>>(ma, ma1, ma2, mb, mc, g);
     return cudaGetLastError();
 }
@@ -446,7 +437,8 @@ bool gemm_tc_ok(const GemmOperands &op, int64_t M, int N, int K)
         (op.a_seg > 0 && op.a_seg % 64 == 0 && op.A1 && op.A2 && op.lda1 % 8 == 0 && op.lda2 % 8 == 0 &&
          ((reinterpret_cast<uintptr_t>(op.A1) | reinterpret_cast<uintptr_t>(op.A2)) & 15u) == 0 &&
          (op.a_mn ? M : (int64_t)K) == 3 * (int64_t)op.a_seg);
-    return aligned && mn_ok && k_ok && seg_ok && M > 0 && M < ((int64_t)1 << 31) - GBM && N % 128 == 0 && op.lda % 8 == 0 &&
+    return aligned && mn_ok && k_ok && seg_ok && M > 0 && M < ((int64_t)1 << 31) - GBM && N > 0 && N % 32 == 0 &&
+           op.lda % 8 == 0 &&
            op.ldb % 8 == 0 && op.ldc % 8 == 0 && (!op.aux || op.ldaux % 8 == 0);
 }
 

@@ -29,11 +29,14 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
         return HSTU_ERR_UNSUPPORTED;
     if (d->d_qk != d->d_v)
         return HSTU_ERR_UNSUPPORTED;
-    if (d->dtype == HSTU_BF16 && d->d_qk != 32 && d->d_qk != 64 && d->d_qk != 128)
+    // bf16 runs on the tcgen05 kernels only, which take head dims 64 and 128
+    if (d->dtype == HSTU_BF16 && d->d_qk != 64 && d->d_qk != 128)
         return HSTU_ERR_UNSUPPORTED;
     if (d->dtype == HSTU_F32 && d->d_qk != 32 && d->d_qk != 64)
         return HSTU_ERR_UNSUPPORTED;
     if (d->fp8_qk != 0 && d->fp8_qk != 1)
+        return HSTU_ERR_INVALID_ARG;
+    if (d->debug_checks != 0 && d->debug_checks != HSTU_DEBUG_WAIT_TEST)
         return HSTU_ERR_INVALID_ARG;
     if (d->fp8_qk && (d->dtype != HSTU_BF16 || d->d_qk != 128))
         return HSTU_ERR_UNSUPPORTED;
@@ -79,6 +82,16 @@ hstu_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HST
 
 #define HSTU_CUDA(x) HSTU_TRY(cuda_status(x))
 
+// The bf16 attention runs on the tcgen05 kernels and nowhere else: a driver
+// without the tensor-map encoder is a CUDA error, a shape those kernels do not
+// take is unsupported.
+hstu_status tc_status(const AttnParams &p)
+{
+    if (!tensor_maps_available())
+        return HSTU_ERR_CUDA;
+    return attn_tc_supported(p) ? HSTU_OK : HSTU_ERR_UNSUPPORTED;
+}
+
 AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_t *ts,
                        const int32_t *nt, const float *rp, const float *rt, void *ws)
 {
@@ -102,6 +115,9 @@ AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_
     p.lw = d->local_window;
     p.gw = d->global_window;
     p.hdr = static_cast<WsHeader *>(ws);
+    const bool wait_test = d->debug_checks == HSTU_DEBUG_WAIT_TEST;
+    p.wait_limit = wait_test ? kTestWaitLimitCycles : kWaitLimitCycles;
+    p.withhold_first_k = wait_test ? 1 : 0;
     p.items = reinterpret_cast<const int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
     return p;
 }
@@ -136,13 +152,12 @@ hstu_status attn_fwd_strided(const hstu_attn_desc *d, const void *q, int64_t sq,
     p.sk = sk;
     p.sv = sv;
     p.so = so;
-    if (d->dtype == HSTU_BF16 && attn_tc_supported(p)) {
+    if (d->dtype == HSTU_BF16) {
+        HSTU_TRY(tc_status(p));
         HSTU_TRY(schedule(d, off, nt, 0, ws, stream, kTcTile));
         return cuda_status(launch_attn_fwd_tc(p, grid_items(d, kTcTile), stream));
     }
     HSTU_TRY(schedule(d, off, nt, 0, ws, stream));
-    if (d->dtype == HSTU_BF16)
-        return cuda_status(launch_attn_fwd_mma(p, grid_items(d), stream));
     return cuda_status(launch_attn_fwd_f32(p, grid_items(d), stream));
 }
 
@@ -181,17 +196,11 @@ hstu_status attn_bwd_strided(const hstu_attn_desc *desc, const void *q, int64_t 
         p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + sizeof(WsHeader) +
                                              items_bytes(desc));
         HSTU_CUDA(cudaMemsetAsync(p.dq_acc, 0, sizeof(float) * (size_t)desc->total_tokens * row, st));
-        float dq_scale = 1.0f;
-        if (attn_bwd_tc_supported(p)) {
-            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st, kTcTile));
-            HSTU_CUDA(launch_attn_bwd_tc(p, grid_items(desc, kTcTile), st));
-            dq_scale = 0.5f * desc->inv_n;
-        } else {
-            HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st));
-            HSTU_CUDA(launch_attn_bwd_mma(p, grid_items(desc), st));
-        }
+        HSTU_TRY(tc_status(p));
+        HSTU_TRY(schedule(desc, seq_offsets, num_targets, 1, workspace, st, kTcTile));
+        HSTU_CUDA(launch_attn_bwd_tc(p, grid_items(desc, kTcTile), st));
         return cuda_status(launch_convert_dq(p.dq_acc, dq, desc->total_tokens, desc->num_heads,
-                                             desc->d_qk, sdq, dq_scale, st));
+                                             desc->d_qk, sdq, 0.5f * desc->inv_n, st));
     }
     if (sdq != row || sdk != row || sdv != row)
         return HSTU_ERR_UNSUPPORTED;
@@ -267,8 +276,7 @@ hstu_status hstu_attn_fwd(const hstu_attn_desc *desc, const void *q, const void 
         p.k8 = k8;
         p.sq8 = sq;
         p.sk8 = sk;
-        if (!attn_tc_supported(p))
-            return HSTU_ERR_UNSUPPORTED;
+        HSTU_TRY(tc_status(p));
         HSTU_TRY(schedule(desc, seq_offsets, num_targets, 0, workspace, st, kTcTile));
         return cuda_status(launch_attn_fwd_tc(p, grid_items(desc, kTcTile), st));
     }
@@ -283,7 +291,7 @@ hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void 
                           float *d_rab_time, void *workspace, size_t workspace_bytes, void *stream)
 {
     HSTU_TRY(check_attn_desc(desc));
-    if (desc->fp8_qk)  // FP8 scores are a forward-only option
+    if (desc->fp8_qk || desc->debug_checks)  // forward-only options
         return HSTU_ERR_UNSUPPORTED;
     if (!seq_offsets || !rab_pos || !rab_time || !d_rab_pos || !d_rab_time)
         return HSTU_ERR_INVALID_ARG;
@@ -305,7 +313,7 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
     if (!d)
         return HSTU_ERR_INVALID_ARG;
     HSTU_TRY(check_attn_desc(&d->attn));
-    if (d->attn.fp8_qk)  // FP8 scores: standalone attention forward only
+    if (d->attn.fp8_qk || d->attn.debug_checks)  // standalone attention forward only
         return HSTU_ERR_UNSUPPORTED;
     if (d->d_model < 1 || !(d->ln_eps >= 0.f) || !std::isfinite(d->ln_eps) ||
         (d->output_concat != 0 && d->output_concat != 1) || (d->fp8_projections != 0 && d->fp8_projections != 1))
@@ -323,10 +331,10 @@ static hstu_status check_layer_desc(const hstu_layer_desc *d)
 static int layer_width(const hstu_attn_desc *a) { return a->num_heads * (2 * a->d_v + 2 * a->d_qk); }
 
 // the concatenated output projection reads [U | O | G] straight from its three
-// buffers on the tcgen05 GEMM (bf16, D % 128 == 0); other paths copy it first
+// buffers on the tcgen05 GEMM (bf16); the fp32 path copies it first
 static bool layer_cat_copy(const hstu_layer_desc *d)
 {
-    return d->output_concat && (d->attn.dtype != HSTU_BF16 || d->d_model % 128 != 0);
+    return d->output_concat && d->attn.dtype != HSTU_BF16;
 }
 
 static size_t layer_ws(const hstu_layer_desc *d, bool keep_uvqk, bool keep_o)
@@ -413,10 +421,29 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
         HSTU_CUDA(launch_quantize_rows_e4m3(g, hv, (int64_t)T, hv, gq, hv, sg, st));
         return cuda_status(launch_gemm_e4m3(gq, hv, sg, w2, hv, s2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
     }
-    if (bf16 && gemm_tc_supported(x, D, w1, uvqk, W, (int64_t)T, W, D))
+    // bf16 projections run on the tcgen05 GEMM only: every shape is checked
+    // before the first launch.  Y = [U | O | G] W2 + b2 reads its three blocks
+    // from their buffers.
+    GemmOperands cat_op{};
+    cat_op.A = uvqk;
+    cat_op.lda = W;
+    cat_op.A1 = o;
+    cat_op.lda1 = hv;
+    cat_op.A2 = g;
+    cat_op.lda2 = hv;
+    cat_op.a_seg = hv;
+    cat_op.B = w2;
+    cat_op.ldb = D;
+    cat_op.bias = b2;
+    cat_op.C = y;
+    cat_op.ldc = D;
+    if (bf16 && T > 0 &&
+        (!gemm_tc_supported(x, D, w1, uvqk, W, (int64_t)T, W, D) ||
+         (desc->output_concat ? !gemm_tc_ok(cat_op, (int64_t)T, D, 3 * hv)
+                              : !gemm_tc_supported(g, hv, w2, y, D, (int64_t)T, D, hv))))
+        return HSTU_ERR_UNSUPPORTED;
+    if (bf16)
         HSTU_CUDA(launch_gemm_tc(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, hdr, st));
-    else if (bf16)
-        HSTU_CUDA(launch_gemm_bf16(x, D, w1, b1, uvqk, W, (int64_t)T, W, D, true, st));
     else
         HSTU_CUDA(launch_gemm_f32(static_cast<const float *>(x), D, static_cast<const float *>(w1),
                                   static_cast<const float *>(b1), reinterpret_cast<float *>(uvqk), W,
@@ -429,37 +456,17 @@ hstu_status hstu_layer_fwd(const hstu_layer_desc *desc, const void *x, const voi
     if (desc->output_concat) {
         // Y = [U | O | G] W2 + b2
         const int F = 3 * hv;
-        if (!layer_cat_copy(desc)) {
-            GemmOperands op{};
-            op.A = uvqk;
-            op.lda = W;
-            op.A1 = o;
-            op.lda1 = hv;
-            op.A2 = g;
-            op.lda2 = hv;
-            op.a_seg = hv;
-            op.B = w2;
-            op.ldb = D;
-            op.bias = b2;
-            op.C = y;
-            op.ldc = D;
-            if (!gemm_tc_ok(op, (int64_t)T, D, F))
-                return HSTU_ERR_UNSUPPORTED;
-            return cuda_status(launch_gemm_tc_ex(op, (int64_t)T, D, F, GEMM_ACT, false, 1, hdr, st));
-        }
+        if (!layer_cat_copy(desc))
+            return cuda_status(launch_gemm_tc_ex(cat_op, (int64_t)T, D, F, GEMM_ACT, false, 1, hdr, st));
         char *cat = g + align256(T * hv * eb);
         HSTU_CUDA(launch_concat3(uvqk, (int64_t)W * eb, o, (int64_t)hv * eb, g, (int64_t)hv * eb, cat,
                                  (int64_t)T, (int64_t)hv * eb, st));
-        if (bf16)
-            return cuda_status(launch_gemm_bf16(cat, F, w2, b2, y, D, (int64_t)T, D, F, false, st));
         return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(cat), F,
                                            static_cast<const float *>(w2), static_cast<const float *>(b2),
                                            static_cast<float *>(y), D, (int64_t)T, D, F, false, st));
     }
-    if (bf16 && gemm_tc_supported(g, hv, w2, y, D, (int64_t)T, D, hv))
-        return cuda_status(launch_gemm_tc(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
     if (bf16)
-        return cuda_status(launch_gemm_bf16(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, st));
+        return cuda_status(launch_gemm_tc(g, hv, w2, b2, y, D, (int64_t)T, D, hv, false, hdr, st));
     return cuda_status(launch_gemm_f32(reinterpret_cast<const float *>(g), hv,
                                        static_cast<const float *>(w2), static_cast<const float *>(b2),
                                        static_cast<float *>(y), D, (int64_t)T, D, hv, false, st));
@@ -540,7 +547,7 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
     char *dg = dcat + (size_t)(F - hv) * 2;  // the G block of dcat
     char *da = take((size_t)T * W * 2), *dz = take((size_t)T * W * 2);
     const char *uvqk = static_cast<const char *>(saved_uvqk);
-    const int sms = 148;
+    const int sms = device_info().sms;
     auto splits_for = [&](int64_t M, int N) {
         const int64_t tiles = ((M + 127) / 128) * (N / 128);
         return (int)std::max<int64_t>(1, std::min<int64_t>((2 * sms + tiles - 1) / tiles, (T + 63) / 64));

@@ -10,6 +10,13 @@ namespace hstu {
 struct WsHeader;
 struct AttnParams;
 
+// SM count and L2 size of the current device (cached per device).
+struct DeviceInfo {
+    int sms = 148;
+    int64_t l2_bytes = 126 << 20;
+};
+DeviceInfo device_info();
+
 // Tile rows of the work items each attention implementation consumes.
 constexpr int kMmaTile = 64;
 constexpr int kTcTile = 128;
@@ -22,11 +29,10 @@ cudaError_t launch_debug_indices(const int64_t *off, const int64_t *ts, const in
                                  int lo, int hi, int nb, const int64_t *rows, int64_t n,
                                  int32_t *pos_out, int32_t *bkt_out, cudaStream_t stream);
 
-// bf16 attention on the legacy tensor-core path (mma.sync), 64-row tiles.
-cudaError_t launch_attn_fwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
-cudaError_t launch_attn_bwd_mma(const AttnParams &p, int grid_items, cudaStream_t stream);
-
 // bf16 attention on tcgen05 / TMA (sm_100a), 128-row tiles, head dims 64 and 128.
+// tensor_maps_available: the driver exposes cuTensorMapEncodeTiled (without it no
+// tcgen05 kernel can run).  attn_tc_supported: the shape is one the kernels take.
+bool tensor_maps_available();
 bool attn_tc_supported(const AttnParams &p);
 cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream);
 // 2-D bf16 tensor map over [rows, cols] with a row stride, 64 x 128 boxes, 128B swizzle.
@@ -36,25 +42,22 @@ cudaError_t make_row_tensor_map(CUtensorMap *map, const void *base, int64_t rows
 cudaError_t make_tensor_map_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
                                int64_t rows, int64_t cols, int64_t row_stride_bytes, int box_cols,
                                int box_rows, CUtensorMapSwizzle swizzle);
-// bf16 backward on tcgen05 (head dim 128), key tiles of 128 rows; dq_acc receives
-// dQ / (0.5 * inv_n) (apply that scale when converting).
-bool attn_bwd_tc_supported(const AttnParams &p);
+// bf16 backward on tcgen05 (head dims 64, 128), key tiles of 128 rows; dq_acc
+// receives dQ / (0.5 * inv_n) (apply that scale when converting).
 cudaError_t launch_attn_bwd_tc(const AttnParams &p, int grid_items, cudaStream_t stream);
 
 // fp32 attention on CUDA cores, 64-row tiles.
 cudaError_t launch_attn_fwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
 cudaError_t launch_attn_bwd_f32(const AttnParams &p, int grid_items, cudaStream_t stream);
 
-// dq (bf16) <- scale * dq_acc (fp32), n elements of rows with stride.
+// dq (bf16, rows of stride sdq, 16-byte aligned) <- scale * dq_acc (fp32 [T, H d]).
 cudaError_t launch_convert_dq(const float *acc, void *dq, int64_t T, int H, int d, int64_t sdq,
                               float scale, cudaStream_t stream);
 
-// C[M, N] = act(A[M, K] B[K, N] + bias[N]); act = SiLU if silu.  Row strides
-// lda, ldc in elements; B is dense [K, N].
-cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
-                             int64_t ldc, int64_t M, int N, int K, bool silu, cudaStream_t stream);
-// The same on tcgen05 / TMA (sm_100a): K a multiple of 64, N of 128; hdr receives
-// a timeout flag if a pipeline wait ever gives up.
+// C[M, N] = act(A[M, K] B[K, N] + bias[N]) on tcgen05 / TMA (sm_100a); act =
+// SiLU if silu.  Row strides lda, ldc in elements; B is dense [K, N]; K a
+// multiple of 8, N of 32.  hdr receives a timeout flag if a pipeline wait ever
+// gives up.  launch_gemm_f32 is the same in fp32 on CUDA cores.
 bool gemm_tc_supported(const void *A, int64_t lda, const void *Bm, void *C, int64_t ldc, int64_t M, int N, int K);
 cudaError_t launch_gemm_tc(const void *A, int64_t lda, const void *Bm, const void *bias, void *C, int64_t ldc,
                            int64_t M, int N, int K, bool silu, WsHeader *hdr, cudaStream_t stream);

@@ -152,7 +152,7 @@ cudaError_t launch_jagged_truncate(const int64_t *off, const int32_t *nt, int B,
     }
     const int64_t chunks = std::max<int64_t>(1, T * (vec ? row_bytes / 16 : row_bytes / 4));
     // about four chunks per thread; at most 4 blocks of 256 threads per SM
-    const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>((chunks + 1023) / 1024, 148 * 4));
+    const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>((chunks + 1023) / 1024, (int64_t)device_info().sms * 4));
     kern<<<blocks, 256, smem, stream>>>(off, nt, B, T, keep, static_cast<const unsigned char *>(in),
                                         static_cast<unsigned char *>(out), row_bytes, out_off);
     return cudaGetLastError();

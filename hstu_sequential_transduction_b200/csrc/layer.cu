@@ -17,104 +17,6 @@ namespace hstu {
 
 namespace {
 
-// ---- bf16 GEMM on the legacy tensor-core path (mma.sync) -------------------
-constexpr int GM = 128, GN = 128, GK = 32, kGemmThreads = 256;
-constexpr int LDA = GK + 8, LDB = GN + 8;
-
-__global__ void __launch_bounds__(kGemmThreads)
-gemm_bf16_kernel(const __nv_bfloat16 *__restrict__ A, int64_t lda, const __nv_bfloat16 *__restrict__ Bm,
-                 const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ C, int64_t ldc,
-                 int64_t M, int N, int K, int silu)
-{
-    __shared__ __align__(16) __nv_bfloat16 sA[2][GM * LDA];
-    __shared__ __align__(16) __nv_bfloat16 sB[2][GK * LDB];
-    const int64_t m0 = (int64_t)blockIdx.y * GM;
-    const int n0 = blockIdx.x * GN;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wm = warp >> 2, wn = warp & 3, g = lane >> 2, t4 = lane & 3, m = lane >> 3;
-
-    auto load = [&](int buf, int k0) {
-        for (int c = threadIdx.x; c < GM * (GK / 8); c += kGemmThreads) {
-            int r = c / (GK / 8), ch = c % (GK / 8);
-            bool ok = m0 + r < M;
-            const __nv_bfloat16 *src = ok ? A + (m0 + r) * lda + k0 + ch * 8 : A;
-            cp_async16(&sA[buf][r * LDA + ch * 8], src, ok ? 16 : 0);
-        }
-        for (int c = threadIdx.x; c < GK * (GN / 8); c += kGemmThreads) {
-            int r = c / (GN / 8), ch = c % (GN / 8);
-            bool ok = n0 + ch * 8 < N;
-            const __nv_bfloat16 *src = ok ? Bm + (int64_t)(k0 + r) * N + n0 + ch * 8 : Bm;
-            cp_async16(&sB[buf][r * LDB + ch * 8], src, ok ? 16 : 0);
-        }
-        cp_async_commit();
-    };
-
-    float acc[4][4][4];
-#pragma unroll
-    for (int a = 0; a < 4; a++)
-#pragma unroll
-        for (int b = 0; b < 4; b++)
-#pragma unroll
-            for (int e = 0; e < 4; e++)
-                acc[a][b][e] = 0.f;
-
-    const int nk = K / GK;
-    load(0, 0);
-    for (int kt = 0; kt < nk; kt++) {
-        const int buf = kt & 1;
-        if (kt + 1 < nk) {
-            load(buf ^ 1, (kt + 1) * GK);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < GK / 16; kk++) {
-            uint32_t af[4][4];
-#pragma unroll
-            for (int mi = 0; mi < 4; mi++)
-                ldmatrix_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3],
-                            &sA[buf][(wm * 64 + mi * 16 + (lane & 7) + 8 * (m & 1)) * LDA + kk * 16 + 8 * (m >> 1)]);
-#pragma unroll
-            for (int np = 0; np < 2; np++) {
-                uint32_t r0, r1, r2, r3;
-                ldmatrix_x4_trans(r0, r1, r2, r3,
-                                  &sB[buf][(kk * 16 + (lane & 7) + 8 * (m & 1)) * LDB + wn * 32 + np * 16 + 8 * (m >> 1)]);
-#pragma unroll
-                for (int mi = 0; mi < 4; mi++) {
-                    mma_bf16_16816(acc[mi][2 * np], af[mi], r0, r1);
-                    mma_bf16_16816(acc[mi][2 * np + 1], af[mi], r2, r3);
-                }
-            }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int mi = 0; mi < 4; mi++) {
-#pragma unroll
-        for (int ni = 0; ni < 4; ni++) {
-            const int col = n0 + wn * 32 + ni * 8 + 2 * t4;
-            if (col >= N)
-                continue;
-            const float b0 = bias ? __bfloat162float(bias[col]) : 0.f;
-            const float b1 = bias ? __bfloat162float(bias[col + 1]) : 0.f;
-#pragma unroll
-            for (int a = 0; a < 2; a++) {
-                const int64_t row = m0 + wm * 64 + mi * 16 + g + 8 * a;
-                if (row >= M)
-                    continue;
-                float x0 = acc[mi][ni][2 * a] + b0, x1 = acc[mi][ni][2 * a + 1] + b1;
-                if (silu) {
-                    x0 = silu_fast(x0);
-                    x1 = silu_fast(x1);
-                }
-                *reinterpret_cast<uint32_t *>(C + row * ldc + col) = pack_bf16(x0, x1);
-            }
-        }
-    }
-}
-
 // ---- fp32 GEMM on CUDA cores ---------------------------------------------------
 constexpr int FT = 64, FK = 16;
 
@@ -427,7 +329,7 @@ cudaError_t norm_gate_bwd_t(const T *dG, int64_t ldd, const T *O, int64_t ldo, c
                             cudaStream_t stream)
 {
     const int64_t want = (Trows * 32 + 255) / 256;
-    const unsigned blocks = (unsigned)std::min<int64_t>(want, 148 * 8);
+    const unsigned blocks = (unsigned)std::min<int64_t>(want, (int64_t)device_info().sms * 8);
     const size_t smem = (size_t)8 * 2 * F * sizeof(float);  // 8 warps x (dgamma, dbeta) slots
     if (smem > 48 * 1024) {
         cudaError_t e = cudaErrorInvalidValue;
@@ -471,20 +373,6 @@ colsum_bf16_kernel(const __nv_bfloat16 *__restrict__ A, int64_t lda, int64_t Tro
 }
 
 }  // namespace
-
-cudaError_t launch_gemm_bf16(const void *A, int64_t lda, const void *Bm, const void *bias, void *C,
-                             int64_t ldc, int64_t M, int N, int K, bool silu, cudaStream_t stream)
-{
-    if (M == 0)
-        return cudaSuccess;
-    if (K % GK || N % 8)
-        return cudaErrorInvalidValue;
-    dim3 grid((N + GN - 1) / GN, (unsigned)((M + GM - 1) / GM));
-    gemm_bf16_kernel<<<grid, kGemmThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(A), lda, static_cast<const __nv_bfloat16 *>(Bm),
-        static_cast<const __nv_bfloat16 *>(bias), static_cast<__nv_bfloat16 *>(C), ldc, M, N, K, silu);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_gemm_f32(const float *A, int64_t lda, const float *Bm, const float *bias,
                             float *C, int64_t ldc, int64_t M, int N, int K, bool silu,
@@ -530,7 +418,7 @@ cudaError_t launch_concat3(const void *a, int64_t lda, const void *b, int64_t ld
     if (T == 0)
         return cudaSuccess;
     const int64_t total = T * 3 * (bytes / 4);
-    const unsigned blocks = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 8);
+    const unsigned blocks = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)device_info().sms * 8);
     concat3_kernel<<<blocks, 256, 0, stream>>>(static_cast<const unsigned char *>(a), lda,
                                                static_cast<const unsigned char *>(b), ldb,
                                                static_cast<const unsigned char *>(c), ldc,

@@ -13,9 +13,6 @@
 
 namespace hstu {
 
-enum : int { FLAG_TIMEOUT = 32 };
-
-constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 // ---- mbarrier ---------------------------------------------------------------
 
@@ -67,9 +64,10 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (after
-// recording the timeout) if it did not complete in time or the CTA aborted.
+// recording the timeout) if it did not complete within `limit` clock cycles or
+// the CTA aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          WsHeader *hdr)
+                                          WsHeader *hdr, long long limit = kWaitLimitCycles)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -79,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return true;
         if (*abort_flag)
             return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(&hdr->flag, FLAG_TIMEOUT);
             return false;

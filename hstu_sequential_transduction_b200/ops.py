@@ -20,6 +20,8 @@ import torch
 from . import build as _build
 
 HSTU_F32, HSTU_BF16 = 0, 1
+# hstu_attn_desc.debug_checks: the bounded-wait test hook (see include/hstu.h)
+HSTU_DEBUG_WAIT_TEST = 2
 STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3: "HSTU_ERR_WORKSPACE",
           4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_DEVICE_CHECK"}
 

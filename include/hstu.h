@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     HSTU_OK = 0,
     HSTU_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad range */
-    HSTU_ERR_UNSUPPORTED = 2,  /* head dims other than 32/64/128, d_qk != d_v, ... */
+    HSTU_ERR_UNSUPPORTED = 2,  /* a head dim the dtype's kernels do not take, d_qk != d_v, ... */
     HSTU_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
     HSTU_ERR_CUDA = 4,         /* a CUDA runtime call failed */
     HSTU_ERR_DEVICE_CHECK = 5  /* the device-side input check flagged the last call */
@@ -63,18 +63,31 @@ typedef enum {
 
 typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype;
 
+/* Test hook of the bounded pipeline waits (hstu_attn_desc.debug_checks; bf16
+ * hstu_attn_fwd and hstu_attn_fwd_noalloc only, HSTU_ERR_UNSUPPORTED elsewhere).
+ * Every wait of the attention forward's pipeline gives up after about a
+ * millisecond instead of about two seconds, and the first CTA withholds the
+ * load of its first key tile, so its waits run out: the call still returns
+ * HSTU_OK, its kernel ends without a fault, leaves that CTA's share of the
+ * output unwritten, and sets bit 32 (timeout) of the workspace flag, which
+ * hstu_check_device_flag reports.  The next ordinary call on the same
+ * workspace clears the flag.  For tests of the timeout path only. */
+#define HSTU_DEBUG_WAIT_TEST 2
+
 typedef struct {
     int32_t num_seqs;         /* B >= 0 */
     int32_t max_seq_len;      /* >= every L_b; sizes the schedule */
     int64_t total_tokens;     /* T = seq_offsets[B] */
     int32_t num_heads;        /* H >= 1 */
-    int32_t d_qk;             /* per-head query/key width: 32, 64 or 128 */
+    int32_t d_qk;             /* per-head query/key width: 64 or 128 (bf16, tcgen05 kernels), 32 or 64 (fp32) */
     int32_t d_v;              /* per-head value width: equal to d_qk */
     int32_t dtype;            /* hstu_dtype of q, k, v, out and their gradients */
     float inv_n;              /* the 1/N scale applied after SiLU */
     int32_t pos_lo, pos_hi;   /* rab_pos covers distances pos_lo..pos_hi */
     int32_t num_time_buckets; /* NB >= 1 */
-    int32_t debug_checks;     /* reserved; device input checks always run */
+    /* 0, or HSTU_DEBUG_WAIT_TEST (hstu_attn_fwd only; see below).  The device
+     * input checks of seq_offsets and num_targets always run. */
+    int32_t debug_checks;
     /* Semi-local attention (the ULTRA-HSTU review's local + global windows):
      * local_window > 0 keeps, of the pairs the causal/candidate rule keeps,
      * those whose query is fewer than local_window positions after the key or
@@ -286,7 +299,9 @@ hstu_status hstu_attn_fwd_noalloc(const hstu_attn_desc *desc, const void *q, con
  * recent call that used `workspace`: HSTU_OK or HSTU_ERR_DEVICE_CHECK.  The
  * flag's bits (1 = seq_offsets[0] != 0, 2 = a sequence decreasing or past T,
  * 4 = a sequence longer than max_seq_len, 8 = num_targets outside [0, L_b],
- * 16 = seq_offsets[B] != T) are stored in *bits when bits is not NULL.
+ * 16 = seq_offsets[B] != T, 32 = a pipeline wait of a tcgen05 kernel ran
+ * out: the kernel gave up instead of hanging, and its output is incomplete)
+ * are stored in *bits when bits is not NULL.
  */
 hstu_status hstu_check_device_flag(const void *workspace, int32_t *bits, void *stream);
 

@@ -71,12 +71,30 @@ def _desc(**kw):
     (dict(num_time_buckets=0), 1), (dict(dtype=7), 1), (dict(d_qk=48, d_v=48), 2),
     (dict(d_v=32), 2), (dict(dtype=ops.HSTU_F32, d_qk=128, d_v=128), 2),
     (dict(inv_n=float("inf")), 1),
+    # bf16 runs on the tcgen05 kernels only (head dims 64, 128); fp32 takes 32 and 64
+    (dict(d_qk=32, d_v=32), 2), (dict(dtype=ops.HSTU_F32, d_qk=32, d_v=32), 0),
+    (dict(d_qk=128, d_v=128), 0),
 ])
 def test_bad_descriptors_rejected(kw, status):
     lib = ops.load_library()
     n = ctypes.c_size_t(0)
     d = _desc(**kw)
     assert lib.hstu_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == status
+
+
+def test_wait_test_hook_is_forward_only():
+    lib = ops.load_library()
+    n = ctypes.c_size_t(0)
+    d = _desc()
+    d.debug_checks = ops.HSTU_DEBUG_WAIT_TEST
+    assert lib.hstu_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 0
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    assert lib.hstu_attn_bwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake, fake, fake,
+                             fake, fake, fake, fake, fake, fake, ctypes.c_size_t(1 << 20), None) == 2
+    layer = ops.hstu_layer_desc(d, 128, 1e-5)
+    assert lib.hstu_layer_workspace_size(ctypes.byref(layer), ctypes.byref(n)) == 2
+    d.debug_checks = 1  # any other value is an argument error
+    assert lib.hstu_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 1
 
 
 def test_workspace_and_pointer_checks_before_launch():

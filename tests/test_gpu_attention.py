@@ -137,9 +137,37 @@ def test_device_flag_reports_bad_offsets_without_fault(cuda_device):
     assert ops.hstu_check_device_flag(ws) == (0, 0)
 
 
+def test_bounded_wait_runs_out_without_fault(cuda_device):
+    # The timeout path of the pipeline waits, made to run on purpose with the
+    # host-chosen test hook: the first CTA never loads its first key tile, its
+    # waits give up after ~1 ms, the kernel ends, and the workspace flag
+    # reports bit 32.  The next ordinary call on the same workspace is correct
+    # and clears the flag.
+    import ctypes
+    inp = _small([700, 300, 513], H=2, d=64, seed=77)
+    d = dev_attn(inp, cuda_device)
+    desc = ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo,
+                               inp.pos_hi, d["rab_time"])
+    desc.debug_checks = ops.HSTU_DEBUG_WAIT_TEST
+    ws = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc, False), cuda_device)
+    out = torch.zeros_like(d["v"])
+    lib = ops.load_library()
+    p = lambda t: ctypes.c_void_p(0 if t is None else t.data_ptr())
+    st = lib.hstu_attn_fwd(ctypes.byref(desc), p(d["q"]), p(d["k"]), p(d["v"]), p(d["seq_offsets"]),
+                           p(d["timestamps"]), None, p(d["rab_pos"]), p(d["rab_time"]), p(out), p(ws),
+                           ctypes.c_size_t(ws.numel()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    st, bits = ops.hstu_check_device_flag(ws)
+    assert st == 5 and bits == 32
+    ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None, d["rab_pos"],
+                      d["rab_time"], out=out, workspace=ws, **attn_kwargs(inp))
+    assert ops.hstu_check_device_flag(ws) == (0, 0)
+    assert_bf16_close(out, _oracle_fwd(inp), what="ordinary call after the timeout")
+
+
 # ---- forward parity ------------------------------------------------------------
 
-@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("d", [64, 128])
 def test_fwd_small_ragged(cuda_device, d):
     # several tiles, ragged tails, an empty sequence, a single token, candidates
     inp = _small([1, 0, 63, 64, 65, 200, 129], H=2, d=d, nt=[0, 0, 5, 0, 64, 17, 1], seed=d)
@@ -204,7 +232,7 @@ def _check_bwd(gpu, ref, tol_fn, what):
         tol_fn(g, r, what=f"{what} {n}")
 
 
-@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("d", [64, 128])
 def test_bwd_small_ragged(cuda_device, d):
     inp = _small([1, 0, 63, 64, 65, 200, 129], H=2, d=d, nt=[0, 0, 5, 0, 64, 17, 1], seed=10 + d)
     _check_bwd(gpu_bwd(inp, cuda_device), _oracle_bwd(inp), assert_bf16_close, f"bwd d={d}")

@@ -70,8 +70,9 @@ def test_concat_fwd_bf16_tcgen05(cuda_device):
     assert_bf16_close(y, _oracle_fwd(attn, lw, w2, x, 2, 64), what="layer output")
 
 
-def test_concat_fwd_bf16_copy_path(cuda_device):
-    # D = 96 is not a multiple of 128: the concatenation is copied, then the bf16 GEMM
+def test_concat_fwd_bf16_partial_column_tile(cuda_device):
+    # D = 96 is not a multiple of the GEMM's 128-column tile: the tcgen05 GEMM reads
+    # [U | O | G] from the three buffers and its one column tile is partial
     attn, lw, w2, x, _ = _case(92, [70, 3, 129], [5, 0, 9], 2, 64, 96, 100, 16, 0.1)
     y, _, _, _ = _fwd(attn, lw, w2, x, 2, 64, cuda_device)
     assert_bf16_close(y, _oracle_fwd(attn, lw, w2, x, 2, 64), what="layer output")

@@ -1,7 +1,7 @@
 """GPU parity of semi-local attention (local + global windows) against the CPU oracle.
 
-Every kernel path sees the windows: tcgen05 (d = 64, 128 forward, d = 128
-backward), mma.sync (d = 32 forward and backward, d = 64 backward) and fp32."""
+Every kernel path sees the windows: tcgen05 (d = 64, 128, forward and
+backward) and fp32."""
 
 import numpy as np
 import pytest
@@ -32,7 +32,7 @@ def _args(inp):
 WINDOWS = [(70, 0), (200, 130), (1000, 64)]
 
 
-@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("lw,gw", WINDOWS)
 def test_semi_local_fwd_bwd_ragged(cuda_device, d, lw, gw):
     inp = _inp([1, 0, 300, 77, 513, 129], [0, 0, 10, 0, 40, 1], d, seed=600 + d + lw)
