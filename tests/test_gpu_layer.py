@@ -112,6 +112,40 @@ def test_layer_stack_bf16_per_layer(cuda_device):
     assert compared >= 2
 
 
+def test_layer_stack_bf16_every_layer_representable(cuda_device):
+    """The eight-layer stack of the Zipf-length batch (64 histories up to 4096
+    tokens, D = 512, 4 heads of 128) at full batch on the GPU, with weights
+    N(0, 0.06) and inputs N(0, 1) so that no layer underflows (the layer
+    outputs stay between ~1 and ~100 in magnitude).  Every layer is compared:
+    the oracle runs each layer on the rows of three sequences (32, ~300 and
+    4096 tokens, the longest length of the batch) taking as input the same bf16
+    values the GPU layer consumed, and its attention output O and layer output
+    Y are held to the bf16 tolerance."""
+    w = workloads.WORKLOADS["layer_stack_bf16"]
+    inp = workloads.generate(w)
+    attn = inp.attn
+    lengths = attn.lengths
+    seqs = sorted(set(_pick(lengths, 32, 32, 1) + _pick(lengths, 250, 400, 1) + _pick(lengths, 4096, 4096, 1)))
+    assert len(seqs) == 3 and lengths[seqs].max() == 4096
+    rows = rows_of(attn, seqs)
+    sub_off = np.concatenate([[0], np.cumsum(lengths[seqs])]).astype(np.int64)
+    sub_ts = attn.timestamps[torch.from_numpy(rows)]
+    rng = np.random.default_rng(2024)
+    layers = [workloads.make_layer_weights(rng, w.d_model, w.num_heads, w.d_qk, w.d_v, torch.bfloat16,
+                                           weight_std=0.06) for _ in range(w.num_layers)]
+    x = (torch.from_numpy(rng.standard_normal((attn.total_tokens, w.d_model)).astype(np.float32))
+         .to(torch.bfloat16).to(cuda_device))
+    rows_dev = torch.from_numpy(rows).to(cuda_device)
+    for layer, lw in enumerate(layers):
+        x_in = x[rows_dev].cpu()
+        y, _, o = _gpu_layer(x, lw, attn, w, cuda_device, saved=True)
+        ry, _, ro = _oracle_layer(x_in, lw, attn, w, off=sub_off, ts=sub_ts, nt=None, inter=True)
+        assert np.abs(ry).max() > 1e-1, f"layer {layer} degenerated"
+        assert_bf16_close(o[rows_dev], ro, what=f"layer {layer} attention output")
+        assert_bf16_close(y[rows_dev], ry, what=f"layer {layer} output")
+        x = y
+
+
 def test_ranking_layer_one_user(cuda_device):
     """Ranking layer (2048 history + 512 candidates per user) at full batch on the
     GPU; the oracle recomputes one user."""
