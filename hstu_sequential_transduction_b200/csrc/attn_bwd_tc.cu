@@ -117,7 +117,8 @@ enum BucketMode { BK_ANY = 0, BK_ONE = 1, BK_TWO = 2 };
 // Elementwise backward of the NC query columns one thread owns (one key row):
 // P = SiLU, dS' = dP (1+t)(1+h(1-t)); dS' replaces dP in dv[], P is packed.
 // Columns outside [c_lo, c_hi) are masked when MASK.  The time bucket of a
-// column: BK_ONE, the whole block is in one bucket; BK_TWO, every row spans
+// column: BK_ONE, the whole block is in one bucket, whose bias the caller has
+// already added to the positional term (wrow / bconst); BK_TWO, every row spans
 // at most two buckets, so the bucket is one compare of the exact
 // round-toward-zero difference against the upper bucket's power of two;
 // BK_ANY, looked up per column.  No atomics, no data-dependent branches.
@@ -132,8 +133,8 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
     const int f = MASK ? min(max(c_lo, 0), NC - 1) : 0, l = MASK ? min(max(c_hi - 1, 0), NC - 1) : NC - 1;
     o.b0 = exp_offset(ti[f], tjf);
     o.b1 = MODE == BK_ONE ? o.b0 : exp_offset(ti[l], tjf);
-    const float E0 = *reinterpret_cast<const float *>(Eb + o.b0);
-    const float E1 = *reinterpret_cast<const float *>(Eb + o.b1);
+    const float E0 = MODE == BK_ONE ? 0.f : *reinterpret_cast<const float *>(Eb + o.b0);
+    const float E1 = MODE == BK_ONE ? 0.f : *reinterpret_cast<const float *>(Eb + o.b1);
     const float thr = __uint_as_float(o.b1 << 21);  // 2^(bucket of b1), exact
     o.mid = false;
     float upf[NC];  // 1 where the column is in bucket b1
@@ -152,7 +153,7 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
             const int c = 4 * u + e;
             float bt;
             if (MODE == BK_ONE) {
-                bt = E0;
+                bt = 0.f;  // the block's one time bias is folded into bp by the caller
                 upf[c] = 0.f;
             } else if (MODE == BK_TWO) {
                 const bool up = __fsub_rz(tv[e], tjf) >= thr;
@@ -165,14 +166,15 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
                 o.mid |= (!MASK || (c >= c_lo && c < c_hi)) && (off != o.b0) && (off != o.b1);
             }
             const float bp = WINDOW ? wrow[c] : bconst;
-            sv[c] = fmaf(sv[c], 0.5f, bp) + bt;
+            sv[c] = MODE == BK_ONE ? fmaf(sv[c], 0.5f, bp) : fmaf(sv[c], 0.5f, bp) + bt;
         }
     }
     float th[NC];
 #pragma unroll
     for (int c = 0; c < NC; c++)
         th[c] = tanh_approx(sv[c]);
-    float all = 0.f, hi = 0.f;
+    // four partial sums each, so that the additions do not form one serial chain
+    float all[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < NC; c += 2) {
         float pv[2];
@@ -190,14 +192,14 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
             }
             dv[cc] = ds;
             pv[e] = pval;
-            all += ds;
+            all[cc & 3] += ds;
             if (MODE != BK_ONE)
-                hi = fmaf(upf[cc], ds, hi);
+                hi[cc & 3] = fmaf(upf[cc], ds, hi[cc & 3]);
         }
         pk[c >> 1] = pack_bf16(pv[0], pv[1]);
     }
-    o.all = all;
-    o.hi = hi;
+    o.all = (all[0] + all[1]) + (all[2] + all[3]);
+    o.hi = (hi[0] + hi[1]) + (hi[2] + hi[3]);
     return o;
 }
 
@@ -206,17 +208,18 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
 // l >= NC) and diagonal l - 32 in accN, with one shuffle per column.
 __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float &accP, float &accN)
 {
-    accP = 0.f;
-    accN = 0.f;
+    float p2[2] = {0.f, 0.f}, n2[2] = {0.f, 0.f};  // two chains each
 #pragma unroll
     for (int k = 0; k < NC; k++) {
         // the source lane is taken modulo 32: k - lane wraps to the row on diagonal lane or lane - 32
         const float y = __shfl_sync(0xffffffffu, ds[k], k - lane);
         if (k >= lane)
-            accP += y;
+            p2[k & 1] += y;
         else
-            accN += y;
+            n2[k & 1] += y;
     }
+    accP = p2[0] + p2[1];
+    accN = n2[0] + n2[1];
 }
 
 // DH: head dim (64 or 128); SL: semi-local windows in use (otherwise every
@@ -425,6 +428,11 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         // adds up column k.
         float hacc = 0.f, c0 = 0.f, c1 = 0.f;
         int kc = -1;
+        // Gradient of the two clamped positional entries (distance >= pos_hi and
+        // <= pos_lo), summed per thread over the whole CTA and reduced once at the
+        // end: every far block lands on them, and adding each step's small partial
+        // sums straight into their large global totals would round most of them away.
+        float cl_hi = 0.f, cl_lo = 0.f;
         float *TGw = reinterpret_cast<float *>(sm + BL::DQS) + ew * 32 * 32;  // shares the dQ staging
         float *tgr = TGw + lane * 32;
         auto tg_slot = [&](uint32_t k, int row) { return (((k >> 2) ^ (uint32_t)(row & 7)) << 2) | (k & 3); };
@@ -512,14 +520,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             const bool q_ok = lane < NC && iw0 + lane < L;
             const bool cols_bad = __any_sync(full, q_ok && ((tq - tb + 1 >= lim) || (tq - tb + 1 <= -lim) ||
                                                             (lane > 0 && tq_up > tq)));
-            __syncwarp();
-            if (lane < NC)
-                TIw[lane] = (float)(tq - tb + 1);
-            Ww[lane] = wlo;
-            Ww[lane + 32] = whi;
-            __syncwarp();
-            if (i + 1 < nq)
-                prefetch(i + 1);
+            const float tqf = (float)(tq - tb + 1);
 
             const int q_last = min(iw0 + NC, L) - 1;  // last valid query of the block
             // every pair of the block inside the local window, or every key global
@@ -536,14 +537,26 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             }
             int mode = BK_ANY;
             int klo = 0;  // bucket of the block's smallest stamp difference (BK_ONE, BK_TWO)
+            const float dlo = __fsub_rz(__shfl_sync(full, tqf, 0), tjf_last);
+            const float dhi = __fsub_rz(__shfl_sync(full, tqf, max(0, q_last - iw0)), tjf_first);
+            float e_one = 0.f;  // BK_ONE: the block's time bias / 2, folded into the window
             if (cls != CLS_GENERAL && q_last >= iw0 && jw_n > 0) {
-                const float dlo = __fsub_rz(TIw[0], tjf_last);
-                const float dhi = __fsub_rz(TIw[q_last - iw0], tjf_first);
                 const uint32_t de = (__float_as_uint(dhi) >> 23) - (__float_as_uint(dlo) >> 23);
                 if (dlo >= 1.f)
                     mode = de == 0 ? BK_ONE : (de == 1 ? BK_TWO : BK_ANY);
                 klo = (int)(__float_as_uint(dlo) >> 23) - 127;
+                // (a masked block runs the per-column variant, which adds the bias itself)
+                if (mode == BK_ONE && cls != CLS_WINDOW_MASKED)
+                    e_one = *reinterpret_cast<const float *>(Eb + ((__float_as_uint(dlo) >> 21) & 0x7FCu));
             }
+            __syncwarp();
+            if (lane < NC)
+                TIw[lane] = tqf;
+            Ww[lane] = wlo + e_one;
+            Ww[lane + 32] = whi + e_one;
+            __syncwarp();
+            if (i + 1 < nq)
+                prefetch(i + 1);
 
             if (!(ok = mbar_wait(bar(S_FULL), i & 1, abort_flag, p.hdr)))
                 break;
@@ -567,12 +580,10 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         o = bwd_row<false, false, BK_TWO>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
                     else
                         o = bwd_row<false, false, BK_ANY>(sv, dv, TIw, tjf, Eb, nullptr, Ww[0], 0, NC, pk);
-                    float sum = o.all;
-#pragma unroll
-                    for (int s = 16; s; s >>= 1)
-                        sum += __shfl_xor_sync(full, sum, s);
-                    if (lane == 0 && sum != 0.f)
-                        red_add_global(p.d_rab_pos + clamp_idx(dmin_w), sum * gscale);
+                    if (dmin_w >= hi)
+                        cl_hi += o.all;
+                    else
+                        cl_lo += o.all;
                 } else {
                     const float *wrow = Ww + 31 - lane;  // wrow[c]: diagonal c - lane
                     if (cls == CLS_WINDOW)
@@ -588,10 +599,18 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     }
                     float accP, accN;
                     warp_diagonals(dv, lane, accP, accN);
-                    if (accP != 0.f)
-                        red_add_global(p.d_rab_pos + clamp_idx(dw + lane), accP * gscale);
-                    if (accN != 0.f)
-                        red_add_global(p.d_rab_pos + clamp_idx(dw + lane - 32), accN * gscale);
+                    // diagonal sums: past either clamp into the CTA's accumulators,
+                    // otherwise straight to the table
+                    auto diag_add = [&](int dd, float v) {
+                        if (dd >= hi)
+                            cl_hi += v;
+                        else if (dd <= lo)
+                            cl_lo += v;
+                        else if (v != 0.f)
+                            red_add_global(p.d_rab_pos + (dd - lo), v * gscale);
+                    };
+                    diag_add(dw + lane, accP);
+                    diag_add(dw + lane - 32, accN);
                 }
                 const bool two = o.b1 != o.b0;
                 const float v0 = two ? o.all - o.hi : o.all, v1 = two ? o.hi : 0.f;
@@ -703,6 +722,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         carry_flush(-1);
         if (hacc != 0.f)
             red_add_global(p.d_rab_time + min(lane, p.nb - 1), hacc * gscale);
+        {
+            const float sh = warp_sum(cl_hi), sl = warp_sum(cl_lo);
+            if (lane == 0 && sh != 0.f)
+                red_add_global(p.d_rab_pos + (hi - lo), sh * gscale);
+            if (lane == 0 && sl != 0.f)
+                red_add_global(p.d_rab_pos, sl * gscale);
+        }
         if (ok && mbar_wait(bar(ACC_FULL), 0, abort_flag, p.hdr)) {
             tc_fence_after();
             constexpr int DC = DH / kGroupsB;  // dK / dV columns per thread
