@@ -144,47 +144,162 @@ __device__ __forceinline__ void store_vec(T *p, const float *y)
     }
 }
 
-// One warp per token; lane l holds features l*VPT .. l*VPT + VPT - 1, moved
-// with 16-byte vector loads and stores (memory-bound: read O and U, write G).
+// One warp per token at a time; lane l holds features l*VPT .. l*VPT + VPT - 1,
+// moved with 16-byte vector loads and stores (memory-bound: read O and U, write
+// G).  Each warp walks the tokens warp, warp + W, ... (W = warps of the grid):
+// gamma and beta stay in registers, and the O and U rows of the next two tokens
+// are kept in flight as raw 16-byte words while this token is normalised.
+template <typename T, int VPT>
+struct RawRow {
+    static constexpr int WORDS = VPT * (int)sizeof(T) / 16;  // 16-byte words per lane
+    uint4 w[WORDS];
+};
+
+template <typename T, int VPT>
+__device__ __forceinline__ void raw_load(const T *p, RawRow<T, VPT> &r)
+{
+#pragma unroll
+    for (int b = 0; b < RawRow<T, VPT>::WORDS; b++)
+        r.w[b] = __ldg(reinterpret_cast<const uint4 *>(p) + b);
+}
+
+template <typename T, int VPT>
+__device__ __forceinline__ void raw_unpack(const RawRow<T, VPT> &r, float *x)
+{
+#pragma unroll
+    for (int b = 0; b < RawRow<T, VPT>::WORDS; b++) {
+        const uint32_t u[4] = {r.w[b].x, r.w[b].y, r.w[b].z, r.w[b].w};
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&u[k]);
+                x[8 * b + 2 * k] = __low2float(h);
+                x[8 * b + 2 * k + 1] = __high2float(h);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                x[4 * b + k] = __uint_as_float(u[k]);
+        }
+    }
+}
+
 template <typename T, int VPT>
 __global__ void __launch_bounds__(256)
 norm_gate_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, int64_t ldu,
                  const float *__restrict__ gamma, const float *__restrict__ beta, float eps,
                  T *__restrict__ G, int64_t ldg, int64_t Trows)
 {
+    static_assert(VPT * sizeof(T) % 16 == 0, "16-byte words per lane");
     constexpr int F = 32 * VPT;
     const int lane = threadIdx.x & 31;
-    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (row >= Trows)
         return;
-    float x[VPT], u[VPT], ga[VPT], be[VPT];
+    float ga[VPT], be[VPT];
+    RawRow<T, VPT> o0, u0, o1, u1;  // this token's and the next one's rows
+    raw_load<T, VPT>(O + row * ldo + lane * VPT, o0);
+    raw_load<T, VPT>(U + row * ldu + lane * VPT, u0);
+    if (row + nwarps < Trows) {
+        raw_load<T, VPT>(O + (row + nwarps) * ldo + lane * VPT, o1);
+        raw_load<T, VPT>(U + (row + nwarps) * ldu + lane * VPT, u1);
+    }
+    load_vec<float, VPT>(gamma + lane * VPT, ga);
+    load_vec<float, VPT>(beta + lane * VPT, be);
+    for (; row < Trows; row += nwarps) {
+        float x[VPT], u[VPT];
+        raw_unpack<T, VPT>(o0, x);
+        raw_unpack<T, VPT>(u0, u);
+        o0 = o1;
+        u0 = u1;
+        const int64_t r2 = row + 2 * nwarps;  // the token after next
+        if (r2 < Trows) {
+            raw_load<T, VPT>(O + r2 * ldo + lane * VPT, o1);
+            raw_load<T, VPT>(U + r2 * ldu + lane * VPT, u1);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            sum += x[e];
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float mean = sum * (1.0f / F);
+        float var = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPT; e++) {
+            const float d = x[e] - mean;
+            var += d * d;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            var += __shfl_xor_sync(0xffffffffu, var, off);
+        const float rstd = rsqrtf(var * (1.0f / F) + eps);
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            x[e] = ((x[e] - mean) * rstd * ga[e] + be[e]) * u[e];
+        store_vec<T, VPT>(G + row * ldg + lane * VPT, x);
+    }
+}
+
+// The same for rows narrower than 16 bytes per lane (bf16 F <= 128, fp32 F = 64):
+// the next token's O and U are loaded as floats before this token is reduced.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256)
+norm_gate_narrow_kernel(const T *__restrict__ O, int64_t ldo, const T *__restrict__ U, int64_t ldu,
+                 const float *__restrict__ gamma, const float *__restrict__ beta, float eps,
+                 T *__restrict__ G, int64_t ldg, int64_t Trows)
+{
+    constexpr int F = 32 * VPT;
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (row >= Trows)
+        return;
+    float ga[VPT], be[VPT], x[VPT], u[VPT];
     load_vec<T, VPT>(O + row * ldo + lane * VPT, x);
     load_vec<T, VPT>(U + row * ldu + lane * VPT, u);
     load_vec<float, VPT>(gamma + lane * VPT, ga);
     load_vec<float, VPT>(beta + lane * VPT, be);
-    float sum = 0.f;
+    for (; row < Trows; row += nwarps) {
+        const int64_t nrow = row + nwarps;
+        float xn[VPT], un[VPT];
+        if (nrow < Trows) {
+            load_vec<T, VPT>(O + nrow * ldo + lane * VPT, xn);
+            load_vec<T, VPT>(U + nrow * ldu + lane * VPT, un);
+        }
+        float sum = 0.f;
 #pragma unroll
-    for (int e = 0; e < VPT; e++)
-        sum += x[e];
+        for (int e = 0; e < VPT; e++)
+            sum += x[e];
 #pragma unroll
-    for (int off = 16; off; off >>= 1)
-        sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float mean = sum * (1.0f / F);
-    float var = 0.f;
+        for (int off = 16; off; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float mean = sum * (1.0f / F);
+        float var = 0.f;
 #pragma unroll
-    for (int e = 0; e < VPT; e++) {
-        const float d = x[e] - mean;
-        var += d * d;
+        for (int e = 0; e < VPT; e++) {
+            const float d = x[e] - mean;
+            var += d * d;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            var += __shfl_xor_sync(0xffffffffu, var, off);
+        const float rstd = rsqrtf(var * (1.0f / F) + eps);
+        float y[VPT];
+#pragma unroll
+        for (int e = 0; e < VPT; e++)
+            y[e] = ((x[e] - mean) * rstd * ga[e] + be[e]) * u[e];
+        store_vec<T, VPT>(G + row * ldg + lane * VPT, y);
+        if (nrow < Trows) {
+#pragma unroll
+            for (int e = 0; e < VPT; e++) {
+                x[e] = xn[e];
+                u[e] = un[e];
+            }
+        }
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1)
-        var += __shfl_xor_sync(0xffffffffu, var, off);
-    const float rstd = rsqrtf(var * (1.0f / F) + eps);
-    float y[VPT];
-#pragma unroll
-    for (int e = 0; e < VPT; e++)
-        y[e] = ((x[e] - mean) * rstd * ga[e] + be[e]) * u[e];
-    store_vec<T, VPT>(G + row * ldg + lane * VPT, y);
 }
 
 template <typename T>
@@ -192,11 +307,17 @@ cudaError_t norm_gate_t(const T *O, int64_t ldo, const T *U, int64_t ldu, const 
                         const float *beta, float eps, T *G, int64_t ldg, int64_t Trows, int F,
                         cudaStream_t stream)
 {
-    const int64_t threads = Trows * 32;
-    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    // two resident blocks per SM, each warp walking a strided set of tokens
+    const int64_t want = (Trows * 32 + 255) / 256;
+    const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)device_info().sms * 2));
     switch (F) {
-    case 64: norm_gate_kernel<T, 2><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
-    case 128: norm_gate_kernel<T, 4><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 64: norm_gate_narrow_kernel<T, 2><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
+    case 128:
+        if constexpr (sizeof(T) == 2)
+            norm_gate_narrow_kernel<T, 4><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows);
+        else
+            norm_gate_kernel<T, 4><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows);
+        break;
     case 256: norm_gate_kernel<T, 8><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
     case 512: norm_gate_kernel<T, 16><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
     case 1024: norm_gate_kernel<T, 32><<<blocks, 256, 0, stream>>>(O, ldo, U, ldu, gamma, beta, eps, G, ldg, Trows); break;
