@@ -47,8 +47,8 @@ SEMI_LOCAL = (1024, 256)
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd -c 1
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
 # valid only for the kernel source it was taken on (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "f95cf640f241b868eba53bffc8f6f06bc29fcc154eff7e74d5dfb27f10f64d95",
-               "bytes": 616.24e6 + 355.64e6}
+BWD_TRAFFIC = {"source_sha256": "fbc70ed845f07d714ba8f77e92217c160344174709fc59de18fe000fd9d716fc",
+               "bytes": 630.78e6 + 364.78e6}
 
 
 def bwd_traffic():
