@@ -50,10 +50,11 @@ template <int BN, int EPI>
 struct GL {
     static constexpr int A = 0;
     static constexpr int B = A + GSTAGES * kRegA;
-    // output staging per epilogue warp: EPI_RED 2 x 4 KB fp32 boxes; otherwise one
-    // 2 KB bf16 box of 32 rows x 32 columns (64-byte swizzle) for a TMA store
+    // output staging per epilogue warp, two boxes used in turn (a box is rewritten
+    // once the TMA store two boxes back has read it): EPI_RED 4 KB fp32 boxes;
+    // otherwise 2 KB bf16 boxes of 32 rows x 32 columns (64-byte swizzle)
     static constexpr int STG = B + GSTAGES * BN * 128;
-    static constexpr int BAR = STG + kEpiWarpsG * (EPI == EPI_RED ? 2 * 4096 : 2048);
+    static constexpr int BAR = STG + kEpiWarpsG * (EPI == EPI_RED ? 2 * 4096 : 2 * 2048);
     static constexpr int NBAR = 2 * GSTAGES + 4;  // full, empty, acc_full[2], acc_empty[2]
     static constexpr int MISC = BAR + NBAR * 8;
     static constexpr int BYTES = MISC + 64;
@@ -326,9 +327,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 // this warp's 32 rows x 32 columns through shared memory and one TMA
                 // store (coalesced; rows past M are dropped by the tensor map)
-                unsigned char *stg = sm + LY::STG + ew * 2048;
-                if (lane == 0)
-                    bulk_wait_read0();  // the previous box has been read out
+                unsigned char *stg = sm + LY::STG + (ew * 2 + (nstage & 1)) * 2048;
+                if (lane == 0 && nstage >= 2)
+                    bulk_wait_read1();  // the box written two stores ago has been read out
+                nstage++;
                 __syncwarp();
 #pragma unroll
                 for (int u4 = 0; u4 < 4; u4++)
