@@ -60,6 +60,8 @@ def _load():
             lib.oracle_visible_sl.argtypes = [ctypes.c_int64] * 6
             lib.oracle_set_windows.restype = None
             lib.oracle_set_windows.argtypes = [ctypes.c_int64] * 2
+            lib.oracle_set_variants.restype = None
+            lib.oracle_set_variants.argtypes = [ctypes.c_int64] * 2
             _lib = lib
     return _lib
 
@@ -115,32 +117,54 @@ def visible_sl(i: int, j: int, L: int, n_t: int, local_window: int, global_windo
 
 
 def bias_pair_counts(seq_offsets, timestamps, num_targets, pos_lo, pos_hi, num_buckets,
-                     local_window=0, global_window=0, threads=None):
+                     local_window=0, global_window=0, threads=None, cand_own_index=False):
     """Visible pairs per rab_pos entry and per rab_time bucket, one head (int64
     arrays [pos_hi - pos_lo + 1] and [num_buckets]), with the attention's own
     visibility rule, windows and index functions."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     pc = np.zeros(int(pos_hi) - int(pos_lo) + 1, dtype=np.int64)
     tc = np.zeros(int(num_buckets), dtype=np.int64)
-    _load().oracle_bias_pair_counts(ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), _p(ts, _i64p),
-                                    ctypes.c_int(int(pos_lo)), ctypes.c_int(int(pos_hi)),
-                                    ctypes.c_int(int(num_buckets)), ctypes.c_int64(int(local_window)),
-                                    ctypes.c_int64(int(global_window)), _p(pc, _i64p), _p(tc, _i64p),
-                                    ctypes.c_int(threads or default_threads()))
+    with _Windows(0, 0, cand_own_index, False):
+        _load().oracle_bias_pair_counts(ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), _p(ts, _i64p),
+                                        ctypes.c_int(int(pos_lo)), ctypes.c_int(int(pos_hi)),
+                                        ctypes.c_int(int(num_buckets)), ctypes.c_int64(int(local_window)),
+                                        ctypes.c_int64(int(global_window)), _p(pc, _i64p), _p(tc, _i64p),
+                                        ctypes.c_int(threads or default_threads()))
     return pc, tc
 
 
 class _Windows:
-    """Semi-local windows applied by the oracle's attention for the duration of one call."""
+    """Readings applied by the oracle's attention for the duration of one call: the
+    semi-local windows, candidates at their own index instead of the shared slot
+    after the history, and one pair of bias tables per head instead of a shared pair."""
 
-    def __init__(self, local_window=0, global_window=0):
+    def __init__(self, local_window=0, global_window=0, cand_own_index=False, per_head_tables=False):
         self.w = (int(local_window), int(global_window))
+        self.v = (int(bool(cand_own_index)), int(bool(per_head_tables)))
 
     def __enter__(self):
         _load().oracle_set_windows(ctypes.c_int64(self.w[0]), ctypes.c_int64(self.w[1]))
+        _load().oracle_set_variants(ctypes.c_int64(self.v[0]), ctypes.c_int64(self.v[1]))
 
     def __exit__(self, *exc):
         _load().oracle_set_windows(ctypes.c_int64(0), ctypes.c_int64(0))
+        _load().oracle_set_variants(ctypes.c_int64(0), ctypes.c_int64(0))
+
+
+def _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi):
+    """(rab_pos, rab_time) flattened to float64, the bucket count, and whether the
+    tables are per head: 1-D tables are shared by the heads, 2-D ones are
+    [num_heads, entries]."""
+    rp, rt = np.asarray(rab_pos), np.asarray(rab_time)
+    if hasattr(rab_pos, "detach"):
+        rp = rab_pos.detach().cpu().double().numpy()
+    if hasattr(rab_time, "detach"):
+        rt = rab_time.detach().cpu().double().numpy()
+    per_head = rp.ndim == 2
+    assert rt.ndim == rp.ndim and (not per_head or (rp.shape[0] == rt.shape[0] == num_heads))
+    assert rp.shape[-1] == int(pos_hi) - int(pos_lo) + 1
+    return (np.ascontiguousarray(rp, dtype=np.float64).reshape(-1), np.ascontiguousarray(rt, dtype=np.float64).reshape(-1),
+            rt.shape[-1], per_head)
 
 
 class _Attn:
@@ -157,10 +181,9 @@ class _Attn:
         self.H = self.q.shape[1]
         self.dqk = self.q.shape[2]
         self.dv = self.v.shape[2]
-        self.rp, self.rt = _f64(rab_pos), _f64(rab_time)
         self.lo, self.hi = int(pos_lo), int(pos_hi)
-        assert len(self.rp) == self.hi - self.lo + 1
-        self.nb = len(self.rt)
+        self.rp, self.rt, self.nb, self.per_head = _tables(rab_pos, rab_time, self.H, self.lo, self.hi)
+        self.table_shapes = (np.shape(rab_pos), np.shape(rab_time))
         self.inv_n = float(inv_n)
 
     def head(self):
@@ -172,30 +195,32 @@ class _Attn:
 
 
 def attn_fwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
-             inv_n, threads=None, local_window=0, global_window=0):
-    """O[T, H, dv] of the jagged SiLU attention (float64)."""
+             inv_n, threads=None, local_window=0, global_window=0, cand_own_index=False):
+    """O[T, H, dv] of the jagged SiLU attention (float64).  Tables [H, entries]
+    are per head; cand_own_index puts each candidate at its own index."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     out = np.zeros((a.T, a.H, a.dv), dtype=np.float64)
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, a.per_head):
         _load().oracle_attn_fwd(*a.head(), _p(out, _f64p), ctypes.c_int(threads or default_threads()))
     return out
 
 
 def attn_fwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
-                  pos_hi, inv_n, rows, threads=None, local_window=0, global_window=0):
+                  pos_hi, inv_n, rows, threads=None, local_window=0, global_window=0, cand_own_index=False):
     """O rows for the given global token indices: [n, H, dv]."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     rows = _i64(rows)
     out = np.zeros((len(rows), a.H, a.dv), dtype=np.float64)
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, a.per_head):
         _load().oracle_attn_fwd_rows(*a.head(), ctypes.c_int64(len(rows)), _p(rows, _i64p),
                                      _p(out, _f64p), ctypes.c_int(threads or default_threads()))
     return out
 
 
 def attn_bwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi,
-             inv_n, dout, threads=None, local_window=0, global_window=0):
-    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
+             inv_n, dout, threads=None, local_window=0, global_window=0, cand_own_index=False):
+    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout); the table
+    gradients have the tables' shapes (per head for [H, entries] tables)."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     do = _f64(dout)
     dq = np.zeros_like(a.q)
@@ -203,14 +228,15 @@ def attn_bwd(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, p
     dv = np.zeros_like(a.v)
     drp = np.zeros_like(a.rp)
     drt = np.zeros_like(a.rt)
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, a.per_head):
         _load().oracle_attn_bwd(*a.head(), _p(do, _f64p), _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p),
                                 _p(drp, _f64p), _p(drt, _f64p), ctypes.c_int(threads or default_threads()))
-    return dq, dk, dv, drp, drt
+    return dq, dk, dv, drp.reshape(a.table_shapes[0]), drt.reshape(a.table_shapes[1])
 
 
 def attn_bwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo,
-                  pos_hi, inv_n, dout, q_rows, k_rows, threads=None, local_window=0, global_window=0):
+                  pos_hi, inv_n, dout, q_rows, k_rows, threads=None, local_window=0, global_window=0,
+                  cand_own_index=False):
     """dq for query rows `q_rows`; dk, dv for key rows `k_rows`."""
     a = _Attn(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_time, pos_lo, pos_hi, inv_n)
     do = _f64(dout)
@@ -218,7 +244,7 @@ def attn_bwd_rows(seq_offsets, timestamps, num_targets, q, k, v, rab_pos, rab_ti
     dq = np.zeros((len(qr), a.H, a.dqk))
     dk = np.zeros((len(kr), a.H, a.dqk))
     dv = np.zeros((len(kr), a.H, a.dv))
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, a.per_head):
         _load().oracle_attn_bwd_rows(*a.head(), _p(do, _f64p), ctypes.c_int64(len(qr)), _p(qr, _i64p),
                                      _p(dq, _f64p), ctypes.c_int64(len(kr)), _p(kr, _i64p),
                                      _p(dk, _f64p), _p(dv, _f64p),
@@ -249,47 +275,50 @@ def norm_gate(o, u, gamma, beta, eps=1e-5, threads=None):
 
 def layer_fwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, b2, ln_gamma, ln_beta,
               rab_pos, rab_time, pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, ln_eps=1e-5,
-              threads=None, want_intermediates=False, out_cat=False, local_window=0, global_window=0):
+              threads=None, want_intermediates=False, out_cat=False, local_window=0, global_window=0,
+              cand_own_index=False):
     """Y[T, D] of one transduction layer (and optionally uvqk, O).  out_cat: the
     output projection reads [U | O | G] (W2 is [3 H d_v, D]) instead of G;
     local_window / global_window: semi-local attention (see visible_sl)."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     x, w1, b1, w2, b2 = _f64(x), _f64(w1), _f64(b1), _f64(w2), _f64(b2)
-    g, be, rp, rt = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time)
+    g, be = _f64(ln_gamma), _f64(ln_beta)
+    rp, rt, nb, per_head = _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi)
     T, D = x.shape
     W = num_heads * (2 * d_v + 2 * d_qk)
     assert w2.shape == ((3 if out_cat else 1) * num_heads * d_v, D)
     y = np.zeros((T, D))
     uvqk = np.zeros((T, W)) if want_intermediates else None
     o = np.zeros((T, num_heads * d_v)) if want_intermediates else None
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, per_head):
         _layer_fwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, b2, g, be, ln_eps, ts, rp, pos_lo,
-                        pos_hi, rt, inv_n, y, uvqk, o, out_cat, threads)
+                        pos_hi, rt, nb, inv_n, y, uvqk, o, out_cat, threads)
     if want_intermediates:
         return y, uvqk, o
     return y
 
 
 def _layer_fwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, b2, g, be, ln_eps, ts, rp, pos_lo, pos_hi,
-                    rt, inv_n, y, uvqk, o, out_cat, threads):
+                    rt, nb, inv_n, y, uvqk, o, out_cat, threads):
     _load().oracle_layer_fwd(
         ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
         ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
         _p(b1, _f64p), _p(w2, _f64p), _p(b2, _f64p), _p(g, _f64p), _p(be, _f64p),
         ctypes.c_double(ln_eps), _p(ts, _i64p), _p(rp, _f64p), ctypes.c_int(int(pos_lo)),
-        ctypes.c_int(int(pos_hi)), _p(rt, _f64p), ctypes.c_int(len(rt)), ctypes.c_double(inv_n),
+        ctypes.c_int(int(pos_hi)), _p(rt, _f64p), ctypes.c_int(int(nb)), ctypes.c_double(inv_n),
         _p(y, _f64p), _p(uvqk, _f64p), _p(o, _f64p), ctypes.c_int(int(out_cat)),
         ctypes.c_int(threads or default_threads()))
 
 
 def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_beta, rab_pos, rab_time,
               pos_lo, pos_hi, inv_n, num_heads, d_qk, d_v, dy, ln_eps=1e-5, threads=None, out_cat=False,
-              local_window=0, global_window=0):
+              local_window=0, global_window=0, cand_own_index=False):
     """Gradients of sum(Y * dy) for one transduction layer: a dict with dx, dw1, db1,
     dw2, db2, d_ln_gamma, d_ln_beta, d_rab_pos, d_rab_time (out_cat as in layer_fwd)."""
     off, ts, nt = _i64(seq_offsets), _i64(timestamps), _i32_or_none(num_targets)
     x, w1, b1, w2 = _f64(x), _f64(w1), _f64(b1), _f64(w2)
-    g, be, rp, rt, dyy = _f64(ln_gamma), _f64(ln_beta), _f64(rab_pos), _f64(rab_time), _f64(dy)
+    g, be, dyy = _f64(ln_gamma), _f64(ln_beta), _f64(dy)
+    rp, rt, nb, per_head = _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi)
     T, D = x.shape
     hv = num_heads * d_v
     W = num_heads * (2 * d_v + 2 * d_qk)
@@ -298,20 +327,22 @@ def layer_bwd(seq_offsets, timestamps, num_targets, x, w1, b1, w2, ln_gamma, ln_
     out = {"dx": np.zeros((T, D)), "dw1": np.zeros((D, W)), "db1": np.zeros(W), "dw2": np.zeros((F, D)),
            "db2": np.zeros(D), "d_ln_gamma": np.zeros(hv), "d_ln_beta": np.zeros(hv),
            "d_rab_pos": np.zeros(len(rp)), "d_rab_time": np.zeros(len(rt))}
-    with _Windows(local_window, global_window):
+    with _Windows(local_window, global_window, cand_own_index, per_head):
         _layer_bwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, g, be, ln_eps, ts, rp, pos_lo, pos_hi,
-                        rt, inv_n, dyy, out, out_cat, threads)
+                        rt, nb, inv_n, dyy, out, out_cat, threads)
+    out["d_rab_pos"] = out["d_rab_pos"].reshape(np.shape(rab_pos))
+    out["d_rab_time"] = out["d_rab_time"].reshape(np.shape(rab_time))
     return out
 
 
 def _layer_bwd_call(off, nt, num_heads, d_qk, d_v, D, x, w1, b1, w2, g, be, ln_eps, ts, rp, pos_lo, pos_hi, rt,
-                    inv_n, dyy, out, out_cat, threads):
+                    nb, inv_n, dyy, out, out_cat, threads):
     _load().oracle_layer_bwd(
         ctypes.c_int(len(off) - 1), _p(off, _i64p), _p(nt, _i32p), ctypes.c_int(num_heads),
         ctypes.c_int(d_qk), ctypes.c_int(d_v), ctypes.c_int(D), _p(x, _f64p), _p(w1, _f64p),
         _p(b1, _f64p), _p(w2, _f64p), _p(g, _f64p), _p(be, _f64p), ctypes.c_double(ln_eps),
         _p(ts, _i64p), _p(rp, _f64p), ctypes.c_int(int(pos_lo)), ctypes.c_int(int(pos_hi)), _p(rt, _f64p),
-        ctypes.c_int(len(rt)), ctypes.c_double(inv_n), _p(dyy, _f64p), _p(out["dx"], _f64p),
+        ctypes.c_int(int(nb)), ctypes.c_double(inv_n), _p(dyy, _f64p), _p(out["dx"], _f64p),
         _p(out["dw1"], _f64p), _p(out["db1"], _f64p), _p(out["dw2"], _f64p), _p(out["db2"], _f64p),
         _p(out["d_ln_gamma"], _f64p), _p(out["d_ln_beta"], _f64p), _p(out["d_rab_pos"], _f64p),
         _p(out["d_rab_time"], _f64p), ctypes.c_int(int(out_cat)), ctypes.c_int(threads or default_threads()))

@@ -78,11 +78,29 @@ int oracle_pos_index(int64_t p_i, int64_t p_j, int pos_lo, int pos_hi)
     return (int)(d - pos_lo);
 }
 
+/*
+ * Readings selected per call (set by the caller, reset after it):
+ *  - g_cand_own_index: 0, the candidates of a sequence share the position
+ *    L - n_t, the slot appended after the history (the DLRMv4 page, "Model
+ *    Architecture": the candidate item is appended); 1, each candidate keeps its
+ *    own index i as its position;
+ *  - g_per_head_tables: 0, rab_pos and rab_time are shared by the heads; 1,
+ *    each head h has its own tables, rab_pos[h][e] and rab_time[h][k], and its
+ *    own table gradients.
+ */
+static int64_t g_cand_own_index = 0, g_per_head_tables = 0;
+
+void oracle_set_variants(int64_t cand_own_index, int64_t per_head_tables)
+{
+    g_cand_own_index = cand_own_index;
+    g_per_head_tables = per_head_tables;
+}
+
 /* Position of local token i in a sequence of length L with n_t candidates. */
 static int64_t token_pos(int64_t i, int64_t L, int64_t n_t)
 {
     int64_t hist = L - n_t;
-    return i < hist ? i : hist;
+    return (i < hist || g_cand_own_index) ? i : hist;
 }
 
 /* Is key j visible from query i (local indices)? */
@@ -156,7 +174,10 @@ static double score(const attn_args *a, const double *q, const double *k, int64_
         s += qi[c] * kj[c];
     int pi = oracle_pos_index(token_pos(i, L, n_t), token_pos(j, L, n_t), a->pos_lo, a->pos_hi);
     int bt = oracle_time_bucket(a->timestamps[s0 + i], a->timestamps[s0 + j], a->num_buckets);
-    return s + a->rab_pos[pi] + a->rab_time[bt];
+    /* per-head tables: head h's rows of rab_pos [H][npos] and rab_time [H][NB] */
+    const int64_t hp = g_per_head_tables ? (int64_t)h * (a->pos_hi - a->pos_lo + 1) : 0;
+    const int64_t ht = g_per_head_tables ? (int64_t)h * a->num_buckets : 0;
+    return s + a->rab_pos[hp + pi] + a->rab_time[ht + bt];
 }
 
 /* One output row: O[s0+i, h, :] = sum over visible j of SiLU(s_ij)/N * v_j. */
@@ -314,7 +335,8 @@ void oracle_bias_pair_counts(int num_seqs, const int64_t *seq_offsets, const int
  *   dP_ij = dO_i . v_j;  dS_ij = dP_ij * SiLU'(s_ij) / N on visible pairs;
  *   dQ_i = sum_j dS_ij k_j;  dK_j = sum_i dS_ij q_i;  dV_j = sum_i P_ij dO_i;
  *   d_rab_pos[idx(i,j)] and d_rab_time[bucket(i,j)] collect dS_ij over all
- *   pairs and heads.  Gradient outputs are overwritten, not accumulated.
+ *   pairs and heads (over the pairs of head h alone into head h's rows with
+ *   per-head tables).  Gradient outputs are overwritten, not accumulated.
  */
 void oracle_attn_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *num_targets,
                      int num_heads, int d_qk, int d_v, const double *q, const double *k,
@@ -369,15 +391,17 @@ void oracle_attn_bwd(int num_seqs, const int64_t *seq_offsets, const int32_t *nu
             }
         }
     }
-    for (int e = 0; e < npos; e++)
+    const int nh = g_per_head_tables ? num_heads : 1;
+    for (int64_t e = 0; e < (int64_t)nh * npos; e++)
         d_rab_pos[e] = 0.0;
-    for (int e = 0; e < num_buckets; e++)
+    for (int64_t e = 0; e < (int64_t)nh * num_buckets; e++)
         d_rab_time[e] = 0.0;
     for (int64_t task = 0; task < tasks; task++) {
+        const int64_t h = g_per_head_tables ? task % num_heads : 0;
         for (int e = 0; e < npos; e++)
-            d_rab_pos[e] += pos_part[task * npos + e];
+            d_rab_pos[h * npos + e] += pos_part[task * npos + e];
         for (int e = 0; e < num_buckets; e++)
-            d_rab_time[e] += time_part[task * num_buckets + e];
+            d_rab_time[h * num_buckets + e] += time_part[task * num_buckets + e];
     }
     free(pos_part);
     free(time_part);

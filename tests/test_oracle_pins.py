@@ -863,3 +863,182 @@ def test_bias_pair_counts_are_the_uniform_score_gradient():
         pc, tc = oracle.bias_pair_counts(off, ts, nts, lo, hi, nb, w, g)
         assert np.array_equal(drp, pc * (H * d * 0.5 * inv_n))
         assert np.array_equal(drt, tc * (H * d * 0.5 * inv_n))
+
+
+# ---- readings selected per call: candidates at their own index, per-head tables ----
+
+def dense_fwd_readings(c, own=False):
+    """Dense forward (numpy) with candidate positions at their own index when `own`
+    and per-head tables when rab_pos is [H, entries]."""
+    off, ts, nt = c["seq_offsets"], c["timestamps"], c["num_targets"]
+    q, k, v, lo, hi = c["q"], c["k"], c["v"], c["pos_lo"], c["pos_hi"]
+    T, H, dv = v.shape
+    rp, rt = np.asarray(c["rab_pos"]), np.asarray(c["rab_time"])
+    if rp.ndim == 1:
+        rp, rt = np.stack([rp] * H), np.stack([rt] * H)
+    nb = rt.shape[1]
+    out = np.zeros((T, H, dv))
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        hist = L - n_t
+        idx = np.arange(L)
+        p = idx if own else np.where(idx < hist, idx, hist)
+        rel = np.clip(p[:, None] - p[None, :], lo, hi) - lo
+        t = ts[s0:s1]
+        dt = np.maximum(t[:, None].astype(object) - t[None, :].astype(object), 0)
+        bkt = np.vectorize(lambda x: min(nb - 1, (int(x) + 1).bit_length() - 1), otypes=[np.int64])(dt)
+        I, J = idx[:, None], idx[None, :]
+        vis = np.where(I < hist, J <= I, (J < hist) | (J == I))
+        S = np.einsum("ihc,jhc->hij", q[s0:s1], k[s0:s1]) + np.stack([rp[h][rel] + rt[h][bkt] for h in range(H)])
+        P = S / (1.0 + np.exp(-S)) * c["inv_n"] * vis[None]
+        out[s0:s1] = np.einsum("hij,jhc->ihc", P, v[s0:s1])
+    return out
+
+
+def _per_head_case(rng, lengths, nt, H=3):
+    c = rand_case(rng, lengths, H=H, nt=nt)
+    c["rab_pos"] = rng.standard_normal((H, c["pos_hi"] - c["pos_lo"] + 1)) * 0.3
+    c["rab_time"] = rng.standard_normal((H, 5)) * 0.3
+    return c
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_own_index_candidates_match_dense(seed):
+    rng = np.random.default_rng(300 + seed)
+    lengths = [9, 6, 1, 11]
+    nt = [3, 6, 1, 4]
+    c = rand_case(rng, lengths, nt=nt, lo=-2, hi=12)
+    got = oracle.attn_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                          c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], cand_own_index=True)
+    np.testing.assert_allclose(got, dense_fwd_readings(c, own=True), rtol=0, atol=1e-12)
+    # the two readings differ only through the candidates' positions
+    shared = ofwd(c)
+    no_cand = dict(c, num_targets=None)
+    np.testing.assert_array_equal(oracle.attn_fwd(no_cand["seq_offsets"], no_cand["timestamps"], None, c["q"], c["k"],
+                                                  c["v"], c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"],
+                                                  c["inv_n"], cand_own_index=True), ofwd(no_cand))
+    assert np.abs(dense_fwd_readings(c, own=True) - shared).max() > 1e-6
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_per_head_tables_match_dense(seed):
+    rng = np.random.default_rng(320 + seed)
+    c = _per_head_case(rng, [7, 0, 10, 3], [2, 0, 0, 1])
+    got = oracle.attn_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                          c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+    np.testing.assert_allclose(got, dense_fwd_readings(c), rtol=0, atol=1e-12)
+
+
+def test_per_head_tables_identical_heads_are_the_shared_tables():
+    rng = np.random.default_rng(340)
+    c = rand_case(rng, [8, 5, 12], H=3, nt=[0, 2, 4])
+    H = 3
+    per = dict(c, rab_pos=np.stack([c["rab_pos"]] * H), rab_time=np.stack([c["rab_time"]] * H))
+    args = lambda d: (d["seq_offsets"], d["timestamps"], d["num_targets"], d["q"], d["k"], d["v"], d["rab_pos"],
+                      d["rab_time"], d["pos_lo"], d["pos_hi"], d["inv_n"])
+    np.testing.assert_array_equal(oracle.attn_fwd(*args(per)), oracle.attn_fwd(*args(c)))
+    dout = rng.standard_normal(c["v"].shape)
+    g_shared = oracle.attn_bwd(*args(c), dout)
+    g_per = oracle.attn_bwd(*args(per), dout)
+    for a, b in zip(g_per[:3], g_shared[:3]):
+        np.testing.assert_array_equal(a, b)
+    assert g_per[3].shape == (H, c["rab_pos"].size) and g_per[4].shape == (H, c["rab_time"].size)
+    np.testing.assert_allclose(g_per[3].sum(axis=0), g_shared[3], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g_per[4].sum(axis=0), g_shared[4], rtol=0, atol=1e-12)
+
+
+def test_per_head_tables_heads_are_independent():
+    # head h of a per-head problem is the one-head problem with head h's inputs and tables
+    rng = np.random.default_rng(350)
+    c = _per_head_case(rng, [9, 4], [2, 0])
+    dout = rng.standard_normal(c["v"].shape)
+    full = oracle.attn_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                           c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], dout)
+    fo = oracle.attn_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                         c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"])
+    for h in range(3):
+        sl = slice(h, h + 1)
+        one = oracle.attn_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"][:, sl], c["k"][:, sl],
+                              c["v"][:, sl], c["rab_pos"][h], c["rab_time"][h], c["pos_lo"], c["pos_hi"], c["inv_n"],
+                              dout[:, sl])
+        of = oracle.attn_fwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"][:, sl], c["k"][:, sl],
+                             c["v"][:, sl], c["rab_pos"][h], c["rab_time"][h], c["pos_lo"], c["pos_hi"], c["inv_n"])
+        np.testing.assert_array_equal(fo[:, sl], of)
+        for a, b in zip(full[:3], one[:3]):
+            np.testing.assert_array_equal(a[:, sl], b)
+        np.testing.assert_array_equal(full[3][h], one[3])
+        np.testing.assert_array_equal(full[4][h], one[4])
+
+
+def _torch_dense_loss_readings(c, dout, own):
+    off, nt = c["seq_offsets"], c["num_targets"]
+    q = torch.tensor(c["q"], requires_grad=True)
+    k = torch.tensor(c["k"], requires_grad=True)
+    v = torch.tensor(c["v"], requires_grad=True)
+    rp = torch.tensor(np.asarray(c["rab_pos"]), requires_grad=True)
+    rt = torch.tensor(np.asarray(c["rab_time"]), requires_grad=True)
+    H = c["q"].shape[1]
+    lo, hi = c["pos_lo"], c["pos_hi"]
+    loss = 0.0
+    for b in range(len(off) - 1):
+        s0, s1 = int(off[b]), int(off[b + 1])
+        L = s1 - s0
+        if L == 0:
+            continue
+        n_t = 0 if nt is None else int(nt[b])
+        hist = L - n_t
+        idx = np.arange(L)
+        p = idx if own else np.where(idx < hist, idx, hist)
+        rel = torch.tensor(np.clip(p[:, None] - p[None, :], lo, hi) - lo)
+        ts = c["timestamps"][s0:s1]
+        nb = rt.shape[-1]
+        bkt = torch.tensor([[min(nb - 1, (int(max(ts[i] - ts[j], 0)) + 1).bit_length() - 1)
+                             for j in range(L)] for i in range(L)])
+        I, J = idx[:, None], idx[None, :]
+        vis = torch.tensor(np.where(I < hist, J <= I, (J < hist) | (J == I)), dtype=torch.float64)
+        if rp.dim() == 2:
+            bias = torch.stack([rp[h][rel] + rt[h][bkt] for h in range(H)])
+        else:
+            bias = (rp[rel] + rt[bkt])[None]
+        S = torch.einsum("ihc,jhc->hij", q[s0:s1], k[s0:s1]) + bias
+        P = torch.nn.functional.silu(S) * c["inv_n"] * vis[None]
+        O = torch.einsum("hij,jhc->ihc", P, v[s0:s1])
+        loss = loss + (O * torch.tensor(dout[s0:s1])).sum()
+    loss.backward()
+    return [x.grad.numpy() for x in (q, k, v, rp, rt)]
+
+
+@pytest.mark.parametrize("own,per_head", [(True, False), (False, True), (True, True)])
+def test_readings_bwd_match_torch_autograd(own, per_head):
+    rng = np.random.default_rng(360 + 2 * own + per_head)
+    lengths, nt = [7, 3, 9], [2, 3, 4]
+    c = _per_head_case(rng, lengths, nt) if per_head else rand_case(rng, lengths, H=3, nt=nt)
+    dout = rng.standard_normal(c["v"].shape)
+    ours = oracle.attn_bwd(c["seq_offsets"], c["timestamps"], c["num_targets"], c["q"], c["k"], c["v"],
+                           c["rab_pos"], c["rab_time"], c["pos_lo"], c["pos_hi"], c["inv_n"], dout,
+                           cand_own_index=own)
+    ref = _torch_dense_loss_readings(c, dout, own)
+    for a, b in zip(ours, ref):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-11)
+
+
+def test_bias_pair_counts_own_index_candidates_closed_form():
+    # candidate i (own position i) sees every history key j at distance i - j and itself at 0
+    hist, nt = 20, 5
+    L = hist + nt
+    pc, tc = _counts([L], np.arange(L), nts=np.array([nt], dtype=np.int32), lo=0, hi=100, nb=10)
+    own = oracle.bias_pair_counts(np.array([0, L]), np.arange(L), np.array([nt], dtype=np.int32), 0, 100, 10,
+                                  cand_own_index=True)[0]
+    exp = np.zeros(101, dtype=np.int64)
+    for k in range(hist):
+        exp[k] += hist - k
+    for i in range(hist, L):
+        for j in range(hist):
+            exp[i - j] += 1
+        exp[0] += 1
+    np.testing.assert_array_equal(own, exp)
+    assert own.sum() == pc.sum()
