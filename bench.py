@@ -374,10 +374,10 @@ def config_timings(dev, stream, reps: int = 10):
     kw = dict(max_seq_len=inp.max_seq_len, inv_n=inp.inv_n, pos_lo=inp.pos_lo, pos_hi=inp.pos_hi)
     ws_f = ops.alloc_workspace(ops.hstu_attn_workspace_size(
         ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi,
-                            d["rab_time"]), False), dev)
+                            d["rab_pos"], d["rab_time"]), False), dev)
     ws_b = ops.alloc_workspace(ops.hstu_attn_workspace_size(
         ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi,
-                            d["rab_time"]), True), dev)
+                            d["rab_pos"], d["rab_time"]), True), dev)
     o = torch.empty_like(d["v"])
     f_ms = timed(lambda: ops.hstu_attn_fwd(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], None,
                                            d["rab_pos"], d["rab_time"], out=o, workspace=ws_f, stream=stream, **kw))
@@ -405,7 +405,7 @@ def config_timings(dev, stream, reps: int = 10):
     ro = torch.empty_like(r["v"])
     rws = ops.alloc_workspace(ops.hstu_attn_workspace_size(
         ops._attn_desc_from(r["q"], r["v"], r["seq_offsets"], att.max_seq_len, att.inv_n, att.pos_lo, att.pos_hi,
-                            r["rab_time"]), False), dev)
+                            r["rab_pos"], r["rab_time"]), False), dev)
     ra_ms = timed(lambda: ops.hstu_attn_fwd(r["q"], r["k"], r["v"], r["seq_offsets"], r["timestamps"],
                                             r["num_targets"], r["rab_pos"], r["rab_time"], out=ro, workspace=rws,
                                             stream=stream, **rkw))
@@ -780,7 +780,7 @@ def run_ours(args):
     # secondary: the same forward with Q K^T on E4M3 codes (q, k quantised inside the call)
     fp8s = None
     if not args.no_layer_stack:
-        desc8 = ops._attn_desc_from(q, v, off, inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi, rt, fp8_qk=True)
+        desc8 = ops._attn_desc_from(q, v, off, inp.max_seq_len, inp.inv_n, inp.pos_lo, inp.pos_hi, rp, rt, fp8_qk=True)
         ws8 = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc8, False), dev)
 
         def f8():

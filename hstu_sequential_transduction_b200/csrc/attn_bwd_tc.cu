@@ -224,7 +224,7 @@ __device__ __forceinline__ void warp_diagonals(const float *ds, int lane, float 
 
 // DH: head dim (64 or 128); SL: semi-local windows in use (otherwise every
 // window test compiles away)
-template <int DH, bool SL>
+template <int DH, bool SL, bool XB = false>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
@@ -379,8 +379,12 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
     } else {
         // ---------------- epilogue ----------------
         // time tables, filled while the first tiles load; only the epilogue warps use them
+        // offsets of this CTA's head's rows in per-head tables and their gradients
+        // (zero with shared tables)
+        const int hp = XB ? h * (int)p.pos_hstride : 0, ht = XB ? h * (int)p.time_hstride : 0;
+        const bool own = XB && p.cand_own != 0;
         for (int e = threadIdx.x - 64; e < 512; e += kEpiThreadsB)
-            E[e] = 0.5f * p.rab_time[exp_bucket(e, p.nb)];
+            E[e] = 0.5f * p.rab_time[ht + exp_bucket(e, p.nb)];
         named_bar(1, kEpiThreadsB);
         // Every warp handles a 32-key x NC-query block of each step on its own:
         // stamps, bias window, class and bias-table gradients are per warp, so
@@ -393,7 +397,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         const int lo = p.pos_lo, hi = p.pos_hi;
         const int64_t tb = p.timestamps[s0 + j0];
         const int64_t tj = krow_ok ? p.timestamps[s0 + j] : tb;
-        const int pj = token_pos(j, hist);
+        const int pj = token_pos(j, hist, own);
         const int64_t lim = (int64_t)1 << 24;
         const float tjf = (float)(tj - tb);
         const float gscale = 0.5f * p.inv_n;
@@ -505,8 +509,8 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
         auto prefetch = [&](int i) {
             const int iw0 = j0 + i * QB + NC * g;
             const int dw = iw0 - jw0;
-            wlo = 0.5f * p.rab_pos[clamp_idx(dw + lane - 31)];
-            whi = 0.5f * p.rab_pos[clamp_idx(dw + lane + 1)];
+            wlo = 0.5f * p.rab_pos[hp + clamp_idx(dw + lane - 31)];
+            whi = 0.5f * p.rab_pos[hp + clamp_idx(dw + lane + 1)];
             if (lane < NC)
                 tq = iw0 + lane < L ? p.timestamps[s0 + iw0 + lane] : tb;
         };
@@ -607,7 +611,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         else if (dd <= lo)
                             cl_lo += v;
                         else if (v != 0.f)
-                            red_add_global(p.d_rab_pos + (dd - lo), v * gscale);
+                            red_add_global(p.d_rab_pos + hp + (dd - lo), v * gscale);
                     };
                     diag_add(dw + lane, accP);
                     diag_add(dw + lane - 32, accN);
@@ -676,17 +680,17 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                         const int ii = iw0 + c + e;
                         pv[e] = 0.f;
                         dsv[e] = 0.f;
-                        if (krow_ok && ii < L && visible_w(ii, j, hist, lw, gw)) {
-                            const int idx = pos_index(token_pos(ii, hist), pj, lo, hi);
+                        if (krow_ok && ii < L && visible_w(ii, j, hist, lw, gw, own)) {
+                            const int idx = pos_index(token_pos(ii, hist, own), pj, lo, hi);
                             const int b = time_bucket(p.timestamps[s0 + ii], tj, p.nb);
-                            const float hh = 0.5f * (sv[c + e] + p.rab_pos[idx] + p.rab_time[b]);
+                            const float hh = 0.5f * (sv[c + e] + p.rab_pos[hp + idx] + p.rab_time[ht + b]);
                             const float t = tanh_approx(hh);
                             pv[e] = fmaf(hh, t, hh);
                             const float a = 1.f + t;
                             const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
                             dsv[e] = ds;
-                            red_add_global(p.d_rab_pos + idx, ds * gscale);
-                            red_add_global(p.d_rab_time + b, ds * gscale);
+                            red_add_global(p.d_rab_pos + hp + idx, ds * gscale);
+                            red_add_global(p.d_rab_time + ht + b, ds * gscale);
                         }
                     }
                     pk[c >> 1] = pack_bf16(pv[0], pv[1]);
@@ -721,13 +725,13 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
             ok = handle_dq(nq - 1);
         carry_flush(-1);
         if (hacc != 0.f)
-            red_add_global(p.d_rab_time + min(lane, p.nb - 1), hacc * gscale);
+            red_add_global(p.d_rab_time + ht + min(lane, p.nb - 1), hacc * gscale);
         {
             const float sh = warp_sum(cl_hi), sl = warp_sum(cl_lo);
             if (lane == 0 && sh != 0.f)
-                red_add_global(p.d_rab_pos + (hi - lo), sh * gscale);
+                red_add_global(p.d_rab_pos + hp + (hi - lo), sh * gscale);
             if (lane == 0 && sl != 0.f)
-                red_add_global(p.d_rab_pos, sl * gscale);
+                red_add_global(p.d_rab_pos + hp, sl * gscale);
         }
         if (ok && mbar_wait(bar(ACC_FULL), 0, abort_flag, p.hdr)) {
             tc_fence_after();
@@ -849,7 +853,11 @@ cudaError_t bwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     if (e != cudaSuccess)
         return e;
     const size_t bytes = BL<DH>::BYTES + 1024;
-    auto kern = p.lw > 0 ? attn_bwd_tc_kernel<DH, true> : attn_bwd_tc_kernel<DH, false>;
+    // the extended bias readings (candidates at their own index, per-head tables)
+    // are separate instantiations, so that the common case compiles without them
+    const bool xb = (p.num_targets && p.cand_own) || p.pos_hstride;
+    auto kern = xb ? (p.lw > 0 ? attn_bwd_tc_kernel<DH, true, true> : attn_bwd_tc_kernel<DH, false, true>)
+                   : (p.lw > 0 ? attn_bwd_tc_kernel<DH, true> : attn_bwd_tc_kernel<DH, false>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess)
         return e;

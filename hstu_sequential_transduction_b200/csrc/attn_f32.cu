@@ -71,7 +71,9 @@ __global__ void __launch_bounds__(TR) attn_fwd_f32_kernel(const AttnParams p)
         q[c] = row_ok ? gq[(s.s0 + i) * p.sq + (int64_t)h * D + c] : 0.f;
         o[c] = 0.f;
     }
-    const int pi = token_pos(i, s.hist);
+    const bool own = p.cand_own;
+    const float *rab_pos = p.rab_pos + h * p.pos_hstride, *rab_time = p.rab_time + h * p.time_hstride;
+    const int pi = token_pos(i, s.hist, own);
     const int64_t ti = row_ok ? p.timestamps[s.s0 + i] : 0;
     const int n = ntiles_fwd(qt, s);
     for (int idx = 0; idx < n; idx++) {
@@ -83,14 +85,14 @@ __global__ void __launch_bounds__(TR) attn_fwd_f32_kernel(const AttnParams p)
         __syncthreads();
         for (int jj = 0; jj < TR; jj++) {
             const int j = j0 + jj;
-            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw))
+            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw, own))
                 continue;
             float x = 0.f;
 #pragma unroll
             for (int c = 0; c < D; c++)
                 x = fmaf(q[c], sK[jj * D + c], x);
-            x += p.rab_pos[pos_index(pi, token_pos(j, s.hist), p.pos_lo, p.pos_hi)] +
-                 p.rab_time[time_bucket(ti, sT[jj], p.nb)];
+            x += rab_pos[pos_index(pi, token_pos(j, s.hist, own), p.pos_lo, p.pos_hi)] +
+                 rab_time[time_bucket(ti, sT[jj], p.nb)];
             const float w = silu_precise(x) * p.inv_n;
 #pragma unroll
             for (int c = 0; c < D; c++)
@@ -130,7 +132,9 @@ __global__ void __launch_bounds__(TR) attn_bwd_f32_kernel(const AttnParams p)
         dout[c] = row_ok ? gdo[(s.s0 + i) * p.sdo + (int64_t)h * D + c] : 0.f;
         dq[c] = 0.f;
     }
-    const int pi = token_pos(i, s.hist);
+    const bool own = p.cand_own;
+    const float *rab_pos = p.rab_pos + h * p.pos_hstride, *rab_time = p.rab_time + h * p.time_hstride;
+    const int pi = token_pos(i, s.hist, own);
     const int64_t ti = row_ok ? p.timestamps[s.s0 + i] : 0;
     const int n = ntiles_fwd(qt, s);
     for (int idx = 0; idx < n; idx++) {
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(TR) attn_bwd_f32_kernel(const AttnParams p)
         __syncthreads();
         for (int jj = 0; jj < TR; jj++) {
             const int j = j0 + jj;
-            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw))
+            if (!row_ok || j >= s.L || !visible_w(i, j, s.hist, p.lw, p.gw, own))
                 continue;
             float x = 0.f, dp = 0.f;
 #pragma unroll
@@ -150,9 +154,9 @@ __global__ void __launch_bounds__(TR) attn_bwd_f32_kernel(const AttnParams p)
                 x = fmaf(q[c], sK[jj * D + c], x);
                 dp = fmaf(dout[c], sV[jj * D + c], dp);
             }
-            const int pidx = pos_index(pi, token_pos(j, s.hist), p.pos_lo, p.pos_hi);
+            const int pidx = pos_index(pi, token_pos(j, s.hist, own), p.pos_lo, p.pos_hi);
             const int bkt = time_bucket(ti, sT[jj], p.nb);
-            x += p.rab_pos[pidx] + p.rab_time[bkt];
+            x += rab_pos[pidx] + rab_time[bkt];
             const float w = silu_precise(x) * p.inv_n;
             const float ds = dp * silu_grad_precise(x) * p.inv_n;
             float *dkr = gdk + (s.s0 + j) * p.sdk + (int64_t)h * D;
@@ -163,8 +167,8 @@ __global__ void __launch_bounds__(TR) attn_bwd_f32_kernel(const AttnParams p)
                 atomicAdd(dkr + c, ds * q[c]);
                 atomicAdd(dvr + c, w * dout[c]);
             }
-            atomicAdd(p.d_rab_pos + pidx, ds);
-            atomicAdd(p.d_rab_time + bkt, ds);
+            atomicAdd(p.d_rab_pos + h * p.pos_hstride + pidx, ds);
+            atomicAdd(p.d_rab_time + h * p.time_hstride + bkt, ds);
         }
     }
     if (row_ok) {

@@ -58,8 +58,10 @@ constexpr int kRegion = 16384;  // one 128-row x 128-byte swizzled region
 // K_*, V_*, S_FULL, P_FULL + b: the tile in stage / S buffer b;
 // P_FREE + b: P V of the tile in S buffer b has completed (buffer b is free);
 // O_FULL: a work item's O is complete in TMEM; O_FREE: the epilogue has read it.
+// E_DONE / E_READY: with per-head tables, every epilogue warp is done with the
+// previous head's time table / has filled its part of the next one.
 enum Bars { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10, S_FULL = 12,
-            P_FULL = 14, P_FREE = 16, O_FULL = 18, O_FREE = 19, NBARS = 20 };
+            P_FULL = 14, P_FREE = 16, O_FULL = 18, O_FREE = 19, E_DONE = 20, E_READY = 21, NBARS = 22 };
 
 // F8: Q and K tiles are E4M3 codes (one 128-byte region for D = 128)
 template <int D, bool F8 = false, bool CAND = false>
@@ -173,7 +175,7 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
 // at the sequence's stamps; jc0 is the key index of the thread's first column.
 template <bool F8>
 __device__ __noinline__ void p_tile_exact(uint32_t taddr, int i, bool row_ok, int jc0, int L, int hist, int lw,
-                                          int gw, int pi, int64_t ti, const int64_t *ts, const float *rab_pos,
+                                          int gw, bool own, int pi, int64_t ti, const int64_t *ts, const float *rab_pos,
                                           const float *rab_time, int pos_lo, int pos_hi, int nb, float rsq,
                                           const float *KSw)
 {
@@ -189,8 +191,8 @@ __device__ __noinline__ void p_tile_exact(uint32_t taddr, int i, bool row_ok, in
         for (int e = 0; e < 2; e++) {
             const int j = jc0 + c + e;
             pv[e] = 0.f;
-            if (row_ok && j < L && visible_w(i, j, hist, lw, gw)) {
-                const float bp = rab_pos[pos_index(pi, token_pos(j, hist), pos_lo, pos_hi)];
+            if (row_ok && j < L && visible_w(i, j, hist, lw, gw, own)) {
+                const float bp = rab_pos[pos_index(pi, token_pos(j, hist, own), pos_lo, pos_hi)];
                 const float bt = rab_time[time_bucket(ti, ts[j], nb)];
                 const float sr = F8 ? sv[c + e] * (2.f * rsq * KSw[c + e]) : sv[c + e];
                 const float hh = 0.5f * (sr + bp + bt);
@@ -237,7 +239,7 @@ __device__ __noinline__ void p_tile_own(uint32_t taddr, int cd, bool row_ok, flo
 // CAND: the batch has candidate rows (the candidates' own tiles take their own
 // path, O leaves through TMA stores); the instantiation without them keeps the
 // leaner tile loop
-template <int D, bool SL, bool F8 = false, bool CAND = false>
+template <int D, bool SL, bool F8 = false, bool CAND = false, bool XB = false>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -282,7 +284,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         U.lt0 = nfull;
         if (lw > 0) {
             U.gt = min(nfull, (gw + TBN - 1) / TBN);
-            U.lt0 = min(nfull, max(U.gt, max(0, token_pos(U.i0, U.hist) - lw + 1) / TBN));
+            U.lt0 = min(nfull, max(U.gt, max(0, token_pos(U.i0, U.hist, XB && p.cand_own) - lw + 1) / TBN));
         }
         U.nhist = U.gt + (nfull - U.lt0);
         U.ntiles = U.nhist + (U.qt >= nh ? 1 : 0);  // + the candidates' own tile
@@ -296,7 +298,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS; i++) {
-            const bool epi = (i == P_FULL || i == P_FULL + 1 || i == O_FREE);
+            const bool epi = (i == P_FULL || i == P_FULL + 1 || i == O_FREE || i == E_DONE || i == E_READY);
             mbar_init(bar(i), epi ? kEpiWarps : 1);
         }
         *abort_flag = 0;
@@ -440,11 +442,17 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         // ---------------- epilogue ----------------
         // expanded time table (index = sign:exponent of the fp32 (1 + dt)), filled
         // while the first tiles load; only the epilogue warps read it
-        for (int e = threadIdx.x - 64; e < 512; e += kEpiThreads) {
-            const int bkt = (e >= 256 || e < 127) ? 0 : min(e - 127, p.nb - 1);
-            E[e] = 0.5f * p.rab_time[bkt];
-        }
+        // per-head tables: the table of the head in E (refilled when the head changes)
+        auto fill_e = [&](int hh) {
+            const float *rt = p.rab_time + hh * (int)p.time_hstride;
+            for (int e = threadIdx.x - 64; e < 512; e += kEpiThreads) {
+                const int bkt = (e >= 256 || e < 127) ? 0 : min(e - 127, p.nb - 1);
+                E[e] = 0.5f * rt[bkt];
+            }
+        };
+        fill_e(0);
         named_bar(1, kEpiThreads);
+        int e_state = 0;  // head in E (bits 1..) and the refill barriers' phase (bit 0)
         const int ew = warp - 2, g = ew >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;
         bool ok = true;
@@ -453,12 +461,31 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         const Unit U = unit(w);
         const int64_t s0 = U.s0;
         const int L = U.L, hist = U.hist, i0 = U.i0, h = U.h, ntiles = U.ntiles;
+        const bool own = XB && p.cand_own != 0;
+        // this head's rows of per-head tables (0 if shared)
+        const int hp = XB ? h * (int)p.pos_hstride : 0, ht = XB ? h * (int)p.time_hstride : 0;
+        if (XB && p.time_hstride && h != (e_state >> 1)) {
+            // every epilogue warp reaches this unit: refill E once all are done with
+            // it, through bounded waits (a warp that gave up makes the others give up)
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(E_DONE));
+            if (!(ok = mbar_wait(bar(E_DONE), e_state & 1, abort_flag, p.hdr, p.wait_limit)))
+                break;
+            fill_e(h);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(E_READY));
+            if (!(ok = mbar_wait(bar(E_READY), e_state & 1, abort_flag, p.hdr, p.wait_limit)))
+                break;
+            e_state = (h << 1) | (~e_state & 1);
+        }
         auto tile_of = [&](int t) { return U.tile_of(t); };
         const int i = i0 + r;
         const bool row_ok = i < L;
         const int64_t tb = p.timestamps[s0 + i0];
         const int64_t ti = row_ok ? p.timestamps[s0 + i] : tb;
-        const int pi = token_pos(i, hist);
+        const int pi = token_pos(i, hist, own);
         const int64_t lim = (int64_t)1 << 24;
         const uint32_t full_mask = 0xffffffffu;
         const bool qbad = __any_sync(full_mask, (ti - tb + 1 >= lim) || (ti - tb + 1 <= -lim));
@@ -472,7 +499,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         float *KSw = Ww + 96;  // F8: half scales of the key columns
         // F8: this row's q scale
         const float rsq = F8 && row_ok ? p.sq8[(s0 + i) * p.H + h] : 0.f;
-        const int pw = token_pos(i0 + 32 * quarter, hist);
+        const int pw = token_pos(i0 + 32 * quarter, hist, own);
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         auto clamp_idx = [&](int d) { return (d < p.pos_lo ? p.pos_lo : (d > p.pos_hi ? p.pos_hi : d)) - p.pos_lo; };
 
@@ -484,9 +511,9 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
         auto prep = [&](int t) {
             const int jw = tile_of(t) * TBN + 64 * g;
             const int dbase = pw - jw - 63;
-            w0 = p.rab_pos[clamp_idx(dbase + lane)];
-            w1 = p.rab_pos[clamp_idx(dbase + lane + 32)];
-            w2 = p.rab_pos[clamp_idx(dbase + lane + 64)];
+            w0 = p.rab_pos[hp + clamp_idx(dbase + lane)];
+            w1 = p.rab_pos[hp + clamp_idx(dbase + lane + 32)];
+            w2 = p.rab_pos[hp + clamp_idx(dbase + lane + 64)];
             const int j = jw + 2 * lane;
             ta = tb;
             tc = tb;
@@ -519,7 +546,7 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 *reinterpret_cast<float2 *>(KSw + 2 * lane) = make_float2(0.5f * ka, 0.5f * kc);
             __syncwarp();
             // every pair of the tile inside the local window (or every key global)?
-            const bool band_all = lw <= 0 || token_pos(min(i0 + TBM, L) - 1, hist) - j0 < lw ||
+            const bool band_all = lw <= 0 || token_pos(min(i0 + TBM, L) - 1, hist, own) - j0 < lw ||
                                   j0 + TBN <= gw;
             const bool band_cut = !band_all;
             const bool full = (j0 + TBN <= hist) && (j0 + TBN - 1 <= i0) && band_all;
@@ -579,11 +606,11 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                 }
             } else if (CAND && i0 >= hist && j0 == i0) {
                 p_tile_own<F8>(trow + s * TBN + 64 * g, i - j0 - 64 * g, row_ok,
-                               p.rab_pos[pos_index(hist, hist, p.pos_lo, p.pos_hi)] + p.rab_time[0], rsq, KSw);
+                               p.rab_pos[hp + pos_index(0, 0, p.pos_lo, p.pos_hi)] + p.rab_time[ht], rsq, KSw);
                 stored = true;
             } else if (CAND) {
-                p_tile_exact<F8>(trow + s * TBN + 64 * g, i, row_ok, j0 + 64 * g, L, hist, lw, gw, pi, ti,
-                                 p.timestamps + s0, p.rab_pos, p.rab_time, p.pos_lo, p.pos_hi, p.nb, rsq, KSw);
+                p_tile_exact<F8>(trow + s * TBN + 64 * g, i, row_ok, j0 + 64 * g, L, hist, lw, gw, own, pi, ti,
+                                 p.timestamps + s0, p.rab_pos + hp, p.rab_time + ht, p.pos_lo, p.pos_hi, p.nb, rsq, KSw);
                 stored = true;
             } else {
 #pragma unroll
@@ -593,9 +620,9 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     for (int e = 0; e < 2; e++) {
                         const int j = j0 + 64 * g + c + e;
                         pv[e] = 0.f;
-                        if (row_ok && j < L && visible_w(i, j, hist, lw, gw)) {
-                            const float bp = p.rab_pos[pos_index(pi, token_pos(j, hist), p.pos_lo, p.pos_hi)];
-                            const float bt = p.rab_time[time_bucket(ti, p.timestamps[s0 + j], p.nb)];
+                        if (row_ok && j < L && visible_w(i, j, hist, lw, gw, own)) {
+                            const float bp = p.rab_pos[hp + pos_index(pi, token_pos(j, hist, own), p.pos_lo, p.pos_hi)];
+                            const float bt = p.rab_time[ht + time_bucket(ti, p.timestamps[s0 + j], p.nb)];
                             const float sr = F8 ? sv[c + e] * (2.f * rsq * KSw[c + e]) : sv[c + e];
                             const float hh = 0.5f * (sr + bp + bt);
                             pv[e] = fmaf(hh, tanh_approx(hh), hh);
@@ -698,7 +725,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-template <int D, bool SL, bool F8 = false, bool CAND = false>
+template <int D, bool SL, bool F8 = false, bool CAND = false, bool XB = false>
 cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stream)
 {
     CUtensorMap maps[3];
@@ -729,7 +756,7 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
                                     CU_TENSOR_MAP_SWIZZLE_64B) != cudaSuccess)
         o_tma = 0;
     const size_t bytes = FwdLayout<D, F8, CAND>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL, F8, CAND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, SL, F8, CAND, XB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess)
         return e;
@@ -737,8 +764,21 @@ cudaError_t fwd_tc_launch(const AttnParams &p, int grid_items, cudaStream_t stre
     const int sms = device_info().sms;
     const int64_t units = (int64_t)grid_items * p.H;
     const unsigned grid = (unsigned)std::min<int64_t>(units, sms);
-    attn_fwd_tc_kernel<D, SL, F8, CAND><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2], mo, o_tma);
+    attn_fwd_tc_kernel<D, SL, F8, CAND, XB><<<grid, kThreadsTc, bytes, stream>>>(p, maps[0], maps[1], maps[2], mo, o_tma);
     return cudaGetLastError();
+}
+
+// The semi-local windows and the extended bias readings (candidates at their own
+// index, per-head tables) are separate instantiations, so that the common case
+// compiles without their bookkeeping.
+template <int D, bool F8, bool CAND>
+cudaError_t fwd_tc_pick(const AttnParams &p, int grid_items, cudaStream_t stream)
+{
+    if ((CAND && p.cand_own) || p.pos_hstride)
+        return p.lw > 0 ? fwd_tc_launch<D, true, F8, CAND, true>(p, grid_items, stream)
+                        : fwd_tc_launch<D, false, F8, CAND, true>(p, grid_items, stream);
+    return p.lw > 0 ? fwd_tc_launch<D, true, F8, CAND>(p, grid_items, stream)
+                    : fwd_tc_launch<D, false, F8, CAND>(p, grid_items, stream);
 }
 
 }  // namespace
@@ -781,20 +821,13 @@ cudaError_t launch_attn_fwd_tc(const AttnParams &p, int grid_items, cudaStream_t
     const bool cand = p.num_targets != nullptr;  // FP8 scores keep the one instantiation
     switch (p.dqk) {
     case 64:
-        if (cand)
-            return p.lw > 0 ? fwd_tc_launch<64, true, false, true>(p, grid_items, stream)
-                            : fwd_tc_launch<64, false, false, true>(p, grid_items, stream);
-        return p.lw > 0 ? fwd_tc_launch<64, true>(p, grid_items, stream)
-                        : fwd_tc_launch<64, false>(p, grid_items, stream);
+        return cand ? fwd_tc_pick<64, false, true>(p, grid_items, stream)
+                    : fwd_tc_pick<64, false, false>(p, grid_items, stream);
     case 128:
         if (p.q8)  // FP8 scores
-            return p.lw > 0 ? fwd_tc_launch<128, true, true>(p, grid_items, stream)
-                            : fwd_tc_launch<128, false, true>(p, grid_items, stream);
-        if (cand)
-            return p.lw > 0 ? fwd_tc_launch<128, true, false, true>(p, grid_items, stream)
-                            : fwd_tc_launch<128, false, false, true>(p, grid_items, stream);
-        return p.lw > 0 ? fwd_tc_launch<128, true>(p, grid_items, stream)
-                        : fwd_tc_launch<128, false>(p, grid_items, stream);
+            return fwd_tc_pick<128, true, false>(p, grid_items, stream);
+        return cand ? fwd_tc_pick<128, false, true>(p, grid_items, stream)
+                    : fwd_tc_pick<128, false, false>(p, grid_items, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -70,6 +70,10 @@ struct AttnParams {
     int64_t sdq, sdk, sdv;
     float *dq_acc;  // fp32 [T, H, dqk] accumulator (bf16 mode)
     float *d_rab_pos, *d_rab_time;
+    int cand_own;  // candidates at their own index (else at the slot after the history)
+    // head strides of the bias tables and their gradients: 0 when the heads share
+    // one pair of tables, the table sizes when each head has its own
+    int64_t pos_hstride, time_hstride;
 };
 
 // floor(log2(1 + max(dt, 0))) capped at nb - 1, exact on int64 seconds.
@@ -88,8 +92,9 @@ __device__ __forceinline__ int pos_index(int p_i, int p_j, int lo, int hi)
     return d - lo;
 }
 
-// Local position of token i: candidates share the slot after the history.
-__device__ __forceinline__ int token_pos(int i, int hist) { return i < hist ? i : hist; }
+// Local position of token i: candidates share the slot after the history, or
+// (own) keep their own index.
+__device__ __forceinline__ int token_pos(int i, int hist, bool own) { return (i < hist || own) ? i : hist; }
 
 __device__ __forceinline__ bool visible(int i, int j, int hist)
 {
@@ -99,9 +104,9 @@ __device__ __forceinline__ bool visible(int i, int j, int hist)
 // visible() restricted to the semi-local windows: with lw > 0 the query must
 // be fewer than lw positions after the key, or the key among the first gw
 // tokens of the sequence.
-__device__ __forceinline__ bool visible_w(int i, int j, int hist, int lw, int gw)
+__device__ __forceinline__ bool visible_w(int i, int j, int hist, int lw, int gw, bool own)
 {
-    return visible(i, j, hist) && (lw <= 0 || token_pos(i, hist) - token_pos(j, hist) < lw || j < gw);
+    return visible(i, j, hist) && (lw <= 0 || token_pos(i, hist, own) - token_pos(j, hist, own) < lw || j < gw);
 }
 
 // SiLU and its derivative on the fp32 path (IEEE division, expf).

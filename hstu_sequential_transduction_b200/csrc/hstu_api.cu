@@ -40,6 +40,11 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
         return HSTU_ERR_INVALID_ARG;
     if (d->fp8_qk && (d->dtype != HSTU_BF16 || d->d_qk != 128))
         return HSTU_ERR_UNSUPPORTED;
+    if ((d->cand_positions != 0 && d->cand_positions != 1) ||
+        (d->per_head_tables != 0 && d->per_head_tables != 1))
+        return HSTU_ERR_INVALID_ARG;
+    if (d->per_head_tables && ((int64_t)d->pos_hi - d->pos_lo + 1) * d->num_heads > INT_MAX)
+        return HSTU_ERR_UNSUPPORTED;
     if (max_items(d->total_tokens, d->num_seqs, kMmaTile) > INT_MAX / 4 ||
         d->total_tokens * d->num_heads > ((int64_t)1 << 40))
         return HSTU_ERR_UNSUPPORTED;
@@ -114,12 +119,23 @@ AttnParams base_params(const hstu_attn_desc *d, const int64_t *off, const int64_
     p.nb = d->num_time_buckets;
     p.lw = d->local_window;
     p.gw = d->global_window;
+    p.cand_own = d->cand_positions;
+    p.pos_hstride = d->per_head_tables ? (int64_t)d->pos_hi - d->pos_lo + 1 : 0;
+    p.time_hstride = d->per_head_tables ? d->num_time_buckets : 0;
     p.hdr = static_cast<WsHeader *>(ws);
     const bool wait_test = d->debug_checks == HSTU_DEBUG_WAIT_TEST;
     p.wait_limit = wait_test ? kTestWaitLimitCycles : kWaitLimitCycles;
     p.withhold_first_k = wait_test ? 1 : 0;
     p.items = reinterpret_cast<const int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
     return p;
+}
+
+// The bias-table gradients are sums over pairs: zeroed before every backward.
+hstu_status zero_table_grads(const hstu_attn_desc *d, float *d_rab_pos, float *d_rab_time, cudaStream_t st)
+{
+    const size_t rows = d->per_head_tables ? (size_t)d->num_heads : 1;
+    HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * rows * (size_t)(d->pos_hi - d->pos_lo + 1), st));
+    return cuda_status(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * rows * d->num_time_buckets, st));
 }
 
 int grid_items(const hstu_attn_desc *d, int tile = kMmaTile)
@@ -169,9 +185,7 @@ hstu_status attn_bwd_strided(const hstu_attn_desc *desc, const void *q, int64_t 
                              const void *dout, int64_t sdo, void *dq, int64_t sdq, void *dk, int64_t sdk, void *dv,
                              int64_t sdv, float *d_rab_pos, float *d_rab_time, void *workspace, cudaStream_t st)
 {
-    const int npos = desc->pos_hi - desc->pos_lo + 1;
-    HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * npos, st));
-    HSTU_CUDA(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->num_time_buckets, st));
+    HSTU_TRY(zero_table_grads(desc, d_rab_pos, d_rab_time, st));
     const int64_t row = (int64_t)desc->num_heads * desc->d_qk;
     const size_t tensor_bytes = (size_t)desc->total_tokens * row * elem_bytes(desc);
     const bool bf16 = desc->dtype == HSTU_BF16;
@@ -534,8 +548,7 @@ hstu_status hstu_layer_bwd(const hstu_layer_desc *desc, const void *x, const voi
     HSTU_CUDA(cudaMemsetAsync(d_ln_gamma, 0, sizeof(float) * hv, st));
     HSTU_CUDA(cudaMemsetAsync(d_ln_beta, 0, sizeof(float) * hv, st));
     if (T == 0) {
-        HSTU_CUDA(cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (a->pos_hi - a->pos_lo + 1), st));
-        return cuda_status(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * a->num_time_buckets, st));
+        return zero_table_grads(a, d_rab_pos, d_rab_time, st);
     }
     char *cur = static_cast<char *>(workspace) + attn_ws(a, 1);
     auto take = [&](size_t bytes) {
@@ -720,8 +733,9 @@ hstu_status hstu_debug_bias_indices(const hstu_attn_desc *desc, const int64_t *s
     if (n < 0 || (n > 0 && (!seq_offsets || !timestamps || !rows || !pos_index || !bucket)))
         return HSTU_ERR_INVALID_ARG;
     return cuda_status(launch_debug_indices(seq_offsets, timestamps, num_targets, desc->num_seqs,
-                                            desc->pos_lo, desc->pos_hi, desc->num_time_buckets, rows,
-                                            n, pos_index, bucket, static_cast<cudaStream_t>(stream)));
+                                            desc->pos_lo, desc->pos_hi, desc->num_time_buckets,
+                                            desc->cand_positions != 0, rows, n, pos_index, bucket,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 hstu_status hstu_debug_schedule(const hstu_attn_desc *desc, const int64_t *seq_offsets,

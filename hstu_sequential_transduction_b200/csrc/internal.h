@@ -26,7 +26,7 @@ cudaError_t launch_schedule(const int64_t *off, const int32_t *nt, int B, int64_
                             int32_t *count_out, cudaStream_t stream);
 
 cudaError_t launch_debug_indices(const int64_t *off, const int64_t *ts, const int32_t *nt, int B,
-                                 int lo, int hi, int nb, const int64_t *rows, int64_t n,
+                                 int lo, int hi, int nb, bool own, const int64_t *rows, int64_t n,
                                  int32_t *pos_out, int32_t *bkt_out, cudaStream_t stream);
 
 // bf16 attention on tcgen05 / TMA (sm_100a), 128-row tiles, head dims 64 and 128.

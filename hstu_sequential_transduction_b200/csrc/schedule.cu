@@ -159,7 +159,7 @@ schedule_kernel(const int64_t *__restrict__ off, const int32_t *__restrict__ nt,
 }
 
 __global__ void debug_indices_kernel(const int64_t *__restrict__ off, const int64_t *__restrict__ ts,
-                                     const int32_t *__restrict__ nt, int B, int lo, int hi, int nb,
+                                     const int32_t *__restrict__ nt, int B, int lo, int hi, int nb, bool own,
                                      const int64_t *__restrict__ rows, int64_t n,
                                      int32_t *__restrict__ pos_out, int32_t *__restrict__ bkt_out)
 {
@@ -191,7 +191,7 @@ __global__ void debug_indices_kernel(const int64_t *__restrict__ off, const int6
     int L = (int)(s1 - s0);
     int hist = L - (nt ? nt[b] : 0);
     int i = (int)(gi - s0), j = (int)(gj - s0);
-    pos_out[e] = pos_index(token_pos(i, hist), token_pos(j, hist), lo, hi);
+    pos_out[e] = pos_index(token_pos(i, hist, own), token_pos(j, hist, own), lo, hi);
     bkt_out[e] = time_bucket(ts[gi], ts[gj], nb);
 }
 
@@ -208,14 +208,14 @@ cudaError_t launch_schedule(const int64_t *off, const int32_t *nt, int B, int64_
 }
 
 cudaError_t launch_debug_indices(const int64_t *off, const int64_t *ts, const int32_t *nt, int B,
-                                 int lo, int hi, int nb, const int64_t *rows, int64_t n,
+                                 int lo, int hi, int nb, bool own, const int64_t *rows, int64_t n,
                                  int32_t *pos_out, int32_t *bkt_out, cudaStream_t stream)
 {
     if (n == 0)
         return cudaSuccess;
     int threads = 256;
     int64_t blocks = (n + threads - 1) / threads;
-    debug_indices_kernel<<<(unsigned)blocks, threads, 0, stream>>>(off, ts, nt, B, lo, hi, nb, rows,
+    debug_indices_kernel<<<(unsigned)blocks, threads, 0, stream>>>(off, ts, nt, B, lo, hi, nb, own, rows,
                                                                    n, pos_out, bkt_out);
     return cudaGetLastError();
 }

@@ -45,7 +45,8 @@ class hstu_attn_desc(ctypes.Structure):
                 ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("inv_n", ctypes.c_float), ("pos_lo", ctypes.c_int32), ("pos_hi", ctypes.c_int32),
                 ("num_time_buckets", ctypes.c_int32), ("debug_checks", ctypes.c_int32),
-                ("local_window", ctypes.c_int32), ("global_window", ctypes.c_int32), ("fp8_qk", ctypes.c_int32)]
+                ("local_window", ctypes.c_int32), ("global_window", ctypes.c_int32), ("fp8_qk", ctypes.c_int32),
+                ("cand_positions", ctypes.c_int32), ("per_head_tables", ctypes.c_int32)]
 
 
 class hstu_layer_desc(ctypes.Structure):
@@ -120,10 +121,11 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
 
 def make_attn_desc(num_seqs, max_seq_len, total_tokens, num_heads, d_qk, d_v, dtype, inv_n,
                    pos_lo, pos_hi, num_time_buckets, local_window=0, global_window=0,
-                   fp8_qk=False) -> hstu_attn_desc:
+                   fp8_qk=False, cand_own_index=False, per_head_tables=False) -> hstu_attn_desc:
     return hstu_attn_desc(int(num_seqs), int(max_seq_len), int(total_tokens), int(num_heads),
                           int(d_qk), int(d_v), int(dtype), float(inv_n), int(pos_lo), int(pos_hi),
-                          int(num_time_buckets), 0, int(local_window), int(global_window), int(bool(fp8_qk)))
+                          int(num_time_buckets), 0, int(local_window), int(global_window), int(bool(fp8_qk)),
+                          int(bool(cand_own_index)), int(bool(per_head_tables)))
 
 
 def hstu_status_string(status: int) -> str:
@@ -153,20 +155,36 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window=0,
-                    global_window=0, fp8_qk=False):
+def _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi):
+    """(num_time_buckets, per_head) of a pair of bias tables: both 1-D (shared by
+    the heads) or both [num_heads, n] (one row per head)."""
+    npos = int(pos_hi) - int(pos_lo) + 1
+    if rab_pos.dim() != rab_time.dim() or rab_pos.dim() not in (1, 2):
+        raise ValueError("rab_pos and rab_time must both be 1-D or both [num_heads, n]")
+    per_head = rab_pos.dim() == 2
+    if per_head and (rab_pos.shape[0] != num_heads or rab_time.shape[0] != num_heads):
+        raise ValueError(f"per-head tables need {num_heads} rows")
+    if rab_pos.shape[-1] != npos:
+        raise ValueError(f"rab_pos has {rab_pos.shape[-1]} entries for distances {pos_lo}..{pos_hi}")
+    return rab_time.shape[-1], per_head
+
+
+def _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_pos, rab_time, local_window=0,
+                    global_window=0, fp8_qk=False, cand_own_index=False):
+    nb, per_head = _tables(rab_pos, rab_time, q.shape[1], pos_lo, pos_hi)
     return make_attn_desc(seq_offsets.numel() - 1, max_seq_len, q.shape[0], q.shape[1], q.shape[2],
-                          v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window,
-                          global_window, fp8_qk)
+                          v.shape[2], _dtype_code(q), inv_n, pos_lo, pos_hi, nb, local_window,
+                          global_window, fp8_qk, cand_own_index, per_head)
 
 
 def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, *,
                   max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, out=None,
                   workspace=None, stream=None, local_window: int = 0, global_window: int = 0,
-                  fp8_qk: bool = False):
+                  fp8_qk: bool = False, cand_own_index: bool = False):
     """O = jagged SiLU attention; q, k [T, H, d_qk], v [T, H, d_v] on CUDA.
     local_window > 0 applies the semi-local mask; fp8_qk computes Q K^T on E4M3
-    codes of q and k (see hstu_attn_desc)."""
+    codes of q and k; cand_own_index puts candidate i at position i; 2-D tables
+    [H, n] give each head its own (see hstu_attn_desc)."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         _dev(t, name, q.dtype)
     _dev(seq_offsets, "seq_offsets", torch.int64)
@@ -174,8 +192,8 @@ def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
     _dev(num_targets, "num_targets", torch.int32)
     _dev(rab_pos, "rab_pos", torch.float32)
     _dev(rab_time, "rab_time", torch.float32)
-    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window,
-                           global_window, fp8_qk)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_pos, rab_time, local_window,
+                           global_window, fp8_qk, cand_own_index)
     if out is None:
         out = torch.empty_like(v)
     _dev(out, "out", q.dtype)
@@ -190,11 +208,13 @@ def hstu_attn_fwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_ti
 
 
 def hstu_attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, out,
-                          *, max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, stream=None):
+                          *, max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, stream=None,
+                          cand_own_index: bool = False):
     """hstu_attn_fwd without a workspace: the library keeps the scheduler's
     scratch in a static device array (for callers that cannot allocate).
     `out` must be preallocated; nothing is allocated here either."""
-    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_pos, rab_time,
+                           cand_own_index=cand_own_index)
     _check("hstu_attn_fwd_noalloc", load_library().hstu_attn_fwd_noalloc(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(timestamps),
         _ptr(num_targets), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _stream(stream)))
@@ -203,15 +223,17 @@ def hstu_attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, num_targets, rab_pos
 
 def hstu_attn_bwd(q, k, v, seq_offsets, timestamps, num_targets, rab_pos, rab_time, dout, *,
                   max_seq_len: int, inv_n: float, pos_lo: int, pos_hi: int, grads=None,
-                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0):
-    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout)."""
+                  workspace=None, stream=None, local_window: int = 0, global_window: int = 0,
+                  cand_own_index: bool = False):
+    """(dq, dk, dv, d_rab_pos, d_rab_time) for the loss sum(O * dout); the table
+    gradients have the tables' shapes."""
     for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
         _dev(t, name, q.dtype)
     _dev(seq_offsets, "seq_offsets", torch.int64)
     _dev(timestamps, "timestamps", torch.int64)
     _dev(num_targets, "num_targets", torch.int32)
-    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_time, local_window,
-                           global_window)
+    desc = _attn_desc_from(q, v, seq_offsets, max_seq_len, inv_n, pos_lo, pos_hi, rab_pos, rab_time, local_window,
+                           global_window, cand_own_index=cand_own_index)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
                  torch.empty_like(rab_pos), torch.empty_like(rab_time))
@@ -230,7 +252,8 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
                    rab_pos, rab_time, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, y=None,
                    saved_uvqk=None, saved_o=None, workspace=None, stream=None, output_concat: bool = False,
-                   fp8_projections: bool = False, local_window: int = 0, global_window: int = 0):
+                   fp8_projections: bool = False, local_window: int = 0, global_window: int = 0,
+                   cand_own_index: bool = False):
     """Y = f2(LayerNorm(attention(SiLU(f1(X)))) * U) for one layer; with
     output_concat, f2 reads [U | O | G] and w2 is [3 H d_v, D]; with
     fp8_projections, w1 and w2 are E4M3 weight packs (quantize_weight_e4m3)."""
@@ -242,8 +265,10 @@ def hstu_layer_fwd(x, w1, b1, w2, b2, ln_gamma, ln_beta, seq_offsets, timestamps
     _dev(ln_gamma, "ln_gamma", torch.float32)
     _dev(ln_beta, "ln_beta", torch.float32)
     T, D = x.shape
+    nb, per_head = _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi)
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
-                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window, global_window)
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, nb, local_window, global_window,
+                          False, cand_own_index, per_head)
     desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)), int(bool(fp8_projections)))
     if fp8_projections:
         W = num_heads * (2 * d_v + 2 * d_qk)
@@ -274,10 +299,11 @@ def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc) -> int:
 def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
                    saved_uvqk, saved_o, dy, *, num_heads: int, d_qk: int, d_v: int, max_seq_len: int,
                    inv_n: float, pos_lo: int, pos_hi: int, ln_eps: float = 1e-5, workspace=None, stream=None,
-                   output_concat: bool = False, local_window: int = 0, global_window: int = 0):
+                   output_concat: bool = False, local_window: int = 0, global_window: int = 0,
+                   cand_own_index: bool = False):
     """Gradients of sum(Y * dy) for one layer (bf16): a dict with dx (bf16) and the
     float32 parameter gradients dw1, db1, dw2, db2, d_ln_gamma, d_ln_beta,
-    d_rab_pos, d_rab_time (output_concat as in hstu_layer_fwd)."""
+    d_rab_pos, d_rab_time (the tables' shapes; output_concat as in hstu_layer_fwd)."""
     for name, t in (("x", x), ("w1", w1), ("b1", b1), ("w2", w2), ("saved_uvqk", saved_uvqk),
                     ("saved_o", saved_o), ("dy", dy)):
         _dev(t, name, x.dtype)
@@ -286,8 +312,10 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
     T, D = x.shape
     W = w1.shape[1]
     hv = num_heads * d_v
+    nb, per_head = _tables(rab_pos, rab_time, num_heads, pos_lo, pos_hi)
     attn = make_attn_desc(seq_offsets.numel() - 1, max_seq_len, T, num_heads, d_qk, d_v,
-                          _dtype_code(x), inv_n, pos_lo, pos_hi, rab_time.numel(), local_window, global_window)
+                          _dtype_code(x), inv_n, pos_lo, pos_hi, nb, local_window, global_window,
+                          False, cand_own_index, per_head)
     desc = hstu_layer_desc(attn, int(D), float(ln_eps), int(bool(output_concat)))
     F = (3 if output_concat else 1) * hv
     if w2.shape[0] != F:
@@ -297,7 +325,7 @@ def hstu_layer_bwd(x, w1, b1, w2, ln_gamma, ln_beta, seq_offsets, timestamps, nu
     out = {"dx": torch.empty((T, D), dtype=x.dtype, device=dev), "dw1": torch.empty((D, W), **f32),
            "db1": torch.empty(W, **f32), "dw2": torch.empty((F, D), **f32), "db2": torch.empty(D, **f32),
            "d_ln_gamma": torch.empty(hv, **f32), "d_ln_beta": torch.empty(hv, **f32),
-           "d_rab_pos": torch.empty(rab_pos.numel(), **f32), "d_rab_time": torch.empty(rab_time.numel(), **f32)}
+           "d_rab_pos": torch.empty(rab_pos.shape, **f32), "d_rab_time": torch.empty(rab_time.shape, **f32)}
     if workspace is None:
         workspace = alloc_workspace(hstu_layer_bwd_workspace_size(desc), dev)
     _check("hstu_layer_bwd", load_library().hstu_layer_bwd(

@@ -15,7 +15,8 @@
  *   visibility: with n_t = num_targets[b] (0 when num_targets is NULL) the last
  *   n_t tokens are candidates; history rows see j <= i, candidate rows see the
  *   whole history and themselves.  p_i = i for history tokens and
- *   L_b - n_t for candidates.  Timestamps are integer seconds.
+ *   L_b - n_t for candidates (i with hstu_attn_desc.cand_positions = 1).
+ *   Timestamps are integer seconds.
  *
  *   Layer: [U | V | Q | K] = SiLU(X W1 + b1) (column blocks in that order, each
  *   [T, H, d] with d fastest); O = attention(Q, K, V);
@@ -30,7 +31,8 @@
  *    hstu_check_device_flag.
  *  - Layouts: values are row-major jagged [T, H, d] (T = seq_offsets[B]),
  *    seq_offsets int64 [B+1], timestamps int64 [T], num_targets int32 [B] or
- *    NULL, rab_pos float32 [pos_hi - pos_lo + 1], rab_time float32 [NB].
+ *    NULL, rab_pos float32 [pos_hi - pos_lo + 1], rab_time float32 [NB] (one
+ *    row per head, [H, ...], with hstu_attn_desc.per_head_tables).
  *    Weights are row-major.  dtype HSTU_BF16 means bf16 values/weights with
  *    fp32 accumulation (P is rounded to bf16 before P V); HSTU_F32 is fp32
  *    throughout.
@@ -103,6 +105,20 @@ typedef struct {
      * otherwise); the backward, the layer calls and hstu_attn_fwd_noalloc reject
      * it.  0: bf16 scores. */
     int32_t fp8_qk;
+    /* Where the candidates sit on the positional axis (the pages fix p_i = i
+     * for history tokens; they do not say where a candidate sits).  0: every
+     * candidate of sequence b at position L_b - n_t, the first position after
+     * the history (candidates are a set, not a continuation of each other).
+     * 1: candidate i at its own index i.  Visibility is the same in both: a
+     * candidate sees the whole history and itself.  The semi-local window
+     * measures distances on the same axis. */
+    int32_t cand_positions;
+    /* 0: one rab_pos [pos_hi - pos_lo + 1] and one rab_time [NB] table, shared
+     * by all heads.  1: one table per head, rab_pos [H, pos_hi - pos_lo + 1]
+     * and rab_time [H, NB] row-major, head h adding row h; the bias-table
+     * gradients then have the same [H, ...] shapes (each head's pairs summed
+     * into its own row). */
+    int32_t per_head_tables;
 } hstu_attn_desc;
 
 typedef struct {
@@ -155,7 +171,7 @@ hstu_status hstu_attn_fwd(const hstu_attn_desc *desc, const void *q, const void 
  * Attention backward for the loss sum(O * dout): dq, dk [T, H, d_qk],
  * dv [T, H, d_v] (desc->dtype) and the float32 bias-table gradients
  * d_rab_pos [pos_hi - pos_lo + 1], d_rab_time [NB], summed over all pairs and
- * heads.  Every output is overwritten, not accumulated.  The pair
+ * heads ([H, ...], each head's pairs in its own row, with per_head_tables).  Every output is overwritten, not accumulated.  The pair
  * gradient is dS_ij = (dout_i . v_j) * SiLU'(s_ij) * inv_n.
  */
 hstu_status hstu_attn_bwd(const hstu_attn_desc *desc, const void *q, const void *k,
@@ -196,7 +212,7 @@ hstu_status hstu_layer_bwd_workspace_size(const hstu_layer_desc *desc, size_t *b
  * output, as hstu_layer_fwd keeps them; dy [T, D] (bf16).
  * Outputs (all overwritten): dx [T, D] (bf16); dw1 [D, W], db1 [W],
  * dw2 [H d_v, D] ([3 H d_v, D] with output_concat), db2 [D], d_ln_gamma,
- * d_ln_beta [H d_v], d_rab_pos [pos_hi - pos_lo + 1], d_rab_time [NB] (all
+ * d_ln_beta [H d_v], d_rab_pos and d_rab_time shaped as the tables (all
  * float32; W = H(2 d_v + 2 d_qk)).
  * The pre-activation X W1 + b1 is recomputed (its SiLU derivative is applied
  * in that GEMM's epilogue), and G = LayerNorm(O) U from saved_o and U.

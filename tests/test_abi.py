@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from hstu_sequential_transduction_b200 import ops
 
@@ -43,14 +44,17 @@ def test_struct_layout_matches_header(tmp_path):
         ' offsetof(hstu_attn_desc,debug_checks), sizeof(hstu_layer_desc),'
         ' offsetof(hstu_layer_desc,ln_eps)); printf("%zu %zu\\n", offsetof(hstu_attn_desc,local_window),'
         ' offsetof(hstu_attn_desc,global_window)); printf("%zu\\n", offsetof(hstu_layer_desc,output_concat));'
-        ' printf("%zu\\n", offsetof(hstu_attn_desc,fp8_qk)); return 0;}\n')
+        ' printf("%zu\\n", offsetof(hstu_attn_desc,fp8_qk));'
+        ' printf("%zu %zu\\n", offsetof(hstu_attn_desc,cand_positions), offsetof(hstu_attn_desc,per_head_tables));'
+        ' printf("%zu\\n", offsetof(hstu_layer_desc,fp8_projections)); return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
     D, L = ops.hstu_attn_desc, ops.hstu_layer_desc
     assert got == [ctypes.sizeof(D), D.total_tokens.offset, D.inv_n.offset, D.debug_checks.offset,
                    ctypes.sizeof(L), L.ln_eps.offset, D.local_window.offset, D.global_window.offset,
-                   L.output_concat.offset, D.fp8_qk.offset]
+                   L.output_concat.offset, D.fp8_qk.offset, D.cand_positions.offset, D.per_head_tables.offset,
+                   L.fp8_projections.offset]
 
 
 def test_status_strings_and_version():
@@ -74,12 +78,34 @@ def _desc(**kw):
     # bf16 runs on the tcgen05 kernels only (head dims 64, 128); fp32 takes 32 and 64
     (dict(d_qk=32, d_v=32), 2), (dict(dtype=ops.HSTU_F32, d_qk=32, d_v=32), 0),
     (dict(d_qk=128, d_v=128), 0),
+    # the two readings of the bias are switches; per-head tables must stay indexable
+    (dict(cand_own_index=True, per_head_tables=True), 0),
+    (dict(pos_lo=-(1 << 23), pos_hi=(1 << 23) - 1, num_heads=256, per_head_tables=True), 2),
 ])
 def test_bad_descriptors_rejected(kw, status):
     lib = ops.load_library()
     n = ctypes.c_size_t(0)
     d = _desc(**kw)
     assert lib.hstu_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == status
+
+
+@pytest.mark.parametrize("field", ["cand_positions", "per_head_tables"])
+def test_bias_switches_take_zero_or_one(field):
+    lib = ops.load_library()
+    n = ctypes.c_size_t(0)
+    d = _desc()
+    setattr(d, field, 2)
+    assert lib.hstu_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == 1
+
+
+def test_table_shapes_checked_in_binding():
+    from hstu_sequential_transduction_b200.ops import _tables
+    assert _tables(torch.zeros(17), torch.zeros(16), 2, -8, 8) == (16, False)
+    assert _tables(torch.zeros(2, 17), torch.zeros(2, 16), 2, -8, 8) == (16, True)
+    for rp, rt in ((torch.zeros(2, 17), torch.zeros(16)), (torch.zeros(3, 17), torch.zeros(3, 16)),
+                   (torch.zeros(16), torch.zeros(16))):
+        with pytest.raises(ValueError):
+            _tables(rp, rt, 2, -8, 8)
 
 
 def test_wait_test_hook_is_forward_only():

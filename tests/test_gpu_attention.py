@@ -147,7 +147,7 @@ def test_bounded_wait_runs_out_without_fault(cuda_device):
     inp = _small([700, 300, 513], H=2, d=64, seed=77)
     d = dev_attn(inp, cuda_device)
     desc = ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo,
-                               inp.pos_hi, d["rab_time"])
+                               inp.pos_hi, d["rab_pos"], d["rab_time"])
     desc.debug_checks = ops.HSTU_DEBUG_WAIT_TEST
     ws = ops.alloc_workspace(ops.hstu_attn_workspace_size(desc, False), cuda_device)
     out = torch.zeros_like(d["v"])

@@ -32,21 +32,36 @@ from hstu_sequential_transduction_b200 import flops, ops, workloads
 pytestmark = pytest.mark.gpu
 
 H = 2
-# (pos_lo, pos_hi, num_time_buckets, candidates, local_window, global_window)
+# (pos_lo, pos_hi, num_time_buckets, candidates, local_window, global_window,
+#  candidates at their own index, one table pair per head)
 VARIANTS = {
     # clamp at 300 inside full tiles, 20 buckets (saturated by the 2^14 and 2^15 gaps)
-    "causal": (-500, 300, 20, False, 0, 0),
+    "causal": (-500, 300, 20, False, 0, 0, False, False),
     # candidates; lower clamp above 0 (distances 0..3 share an entry), upper at 129
-    "candidates": (3, 129, 32, True, 0, 0),
+    "candidates": (3, 129, 32, True, 0, 0, False, False),
     # semi-local windows, no clamp
-    "windows": (0, 1400, 26, False, 300, 70),
+    "windows": (0, 1400, 26, False, 300, 70, False, False),
     # both
-    "candidates_windows": (-64, 2000, 24, True, 150, 33),
+    "candidates_windows": (-64, 2000, 24, True, 150, 33, False, False),
+    # the same with candidates at their own index
+    "candidates_own": (3, 129, 32, True, 0, 0, True, False),
+    "candidates_windows_own": (-64, 2000, 24, True, 150, 33, True, False),
+    # per-head tables
+    "causal_per_head": (-500, 300, 20, False, 0, 0, False, True),
+    "candidates_windows_own_per_head": (-64, 2000, 24, True, 150, 33, True, True),
 }
 
 
-def _desc_kw(lo, hi, max_len, inv_n, lw, gw):
-    return dict(max_seq_len=max_len, inv_n=inv_n, pos_lo=lo, pos_hi=hi, local_window=lw, global_window=gw)
+def _tables(lo, hi, nb, seed, per_head):
+    if not per_head:
+        return bias_patterns.readout_tables(lo, hi, nb, seed=seed)
+    ts = [bias_patterns.readout_tables(lo, hi, nb, seed=seed + 97 * h) for h in range(H)]
+    return torch.stack([t[0] for t in ts]), torch.stack([t[1] for t in ts])
+
+
+def _desc_kw(lo, hi, max_len, inv_n, lw, gw, own):
+    return dict(max_seq_len=max_len, inv_n=inv_n, pos_lo=lo, pos_hi=hi, local_window=lw, global_window=gw,
+                cand_own_index=own)
 
 
 def _dev(t, dev):
@@ -65,20 +80,20 @@ def _assert_readout(gpu, ref, what):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("variant", list(VARIANTS))
 def test_fwd_bias_single_pair_readout(cuda_device, d, variant):
-    lo, hi, nb, cand, lw, gw = VARIANTS[variant]
+    lo, hi, nb, cand, lw, gw, own, ph = VARIANTS[variant]
     ps = bias_patterns.patterns(seed=10, candidates=cand)
     b, v1 = bias_patterns.readout_batch(ps, H, d, "v")
-    rp, rt = bias_patterns.readout_tables(lo, hi, nb, seed=11)
+    rp, rt = _tables(lo, hi, nb, 11, ph)
     T = b.timestamps.numel()
     z = torch.zeros((T, H, d), dtype=torch.bfloat16)
     dev = cuda_device
     zd = z.to(dev)
     out = ops.hstu_attn_fwd(zd, zd, v1.to(dev), _dev(b.seq_offsets, dev), _dev(b.timestamps, dev),
                             _dev(b.num_targets, dev), rp.to(dev), rt.to(dev),
-                            **_desc_kw(lo, hi, b.max_seq_len, 1.0, lw, gw))
+                            **_desc_kw(lo, hi, b.max_seq_len, 1.0, lw, gw, own))
     torch.cuda.synchronize()
     ref = oracle.attn_fwd(b.seq_offsets, b.timestamps, b.num_targets, z, z, v1, rp, rt, lo, hi, 1.0,
-                          local_window=lw, global_window=gw)
+                          local_window=lw, global_window=gw, cand_own_index=own)
     _assert_readout(out, ref, f"forward readout d={d} {variant}")
 
 
@@ -87,20 +102,20 @@ def test_fwd_bias_single_pair_readout(cuda_device, d, variant):
 def test_bwd_recomputed_bias_single_pair_readout(cuda_device, d, variant):
     # v = 0 and dO one-hot per query block: dV_j = P^T dO reads P of one pair per
     # element, while dP = 0 leaves every other gradient exactly zero
-    lo, hi, nb, cand, lw, gw = VARIANTS[variant]
+    lo, hi, nb, cand, lw, gw, own, ph = VARIANTS[variant]
     ps = bias_patterns.patterns(seed=20, candidates=cand)
     b, do1 = bias_patterns.readout_batch(ps, H, d, "dout")
-    rp, rt = bias_patterns.readout_tables(lo, hi, nb, seed=21)
+    rp, rt = _tables(lo, hi, nb, 21, ph)
     T = b.timestamps.numel()
     z = torch.zeros((T, H, d), dtype=torch.bfloat16)
     dev = cuda_device
     zd = z.to(dev)
     dq, dk, dv, drp, drt = ops.hstu_attn_bwd(zd, zd, zd, _dev(b.seq_offsets, dev), _dev(b.timestamps, dev),
                                              _dev(b.num_targets, dev), rp.to(dev), rt.to(dev), do1.to(dev),
-                                             **_desc_kw(lo, hi, b.max_seq_len, 1.0, lw, gw))
+                                             **_desc_kw(lo, hi, b.max_seq_len, 1.0, lw, gw, own))
     torch.cuda.synchronize()
     _, _, rdv, _, _ = oracle.attn_bwd(b.seq_offsets, b.timestamps, b.num_targets, z, z, z, rp, rt, lo, hi, 1.0,
-                                      do1, local_window=lw, global_window=gw)
+                                      do1, local_window=lw, global_window=gw, cand_own_index=own)
     _assert_readout(dv, rdv, f"backward dV readout d={d} {variant}")
     for name, t in (("dq", dq), ("dk", dk), ("d_rab_pos", drp), ("d_rab_time", drt)):
         assert not bool(t.any()), f"{name} should be exactly zero"
@@ -109,7 +124,7 @@ def test_bwd_recomputed_bias_single_pair_readout(cuda_device, d, variant):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("variant", list(VARIANTS))
 def test_bwd_bias_grad_histogram_exact(cuda_device, d, variant):
-    lo, hi, nb, cand, lw, gw = VARIANTS[variant]
+    lo, hi, nb, cand, lw, gw, own, ph = VARIANTS[variant]
     ps = bias_patterns.patterns(seed=30, candidates=cand)
     b = bias_patterns.plain_batch(ps)
     T = b.timestamps.numel()
@@ -117,21 +132,29 @@ def test_bwd_bias_grad_histogram_exact(cuda_device, d, variant):
     dev = cuda_device
     zd = torch.zeros((T, H, d), dtype=torch.bfloat16, device=dev)
     one = torch.ones((T, H, d), dtype=torch.bfloat16, device=dev)
-    zp = torch.zeros(hi - lo + 1, dtype=torch.float32, device=dev)
-    zt = torch.zeros(nb, dtype=torch.float32, device=dev)
+    rows = (H,) if ph else ()
+    zp = torch.zeros(rows + (hi - lo + 1,), dtype=torch.float32, device=dev)
+    zt = torch.zeros(rows + (nb,), dtype=torch.float32, device=dev)
     _, _, _, drp, drt = ops.hstu_attn_bwd(zd, zd, one, _dev(b.seq_offsets, dev), _dev(b.timestamps, dev),
                                           _dev(b.num_targets, dev), zp, zt, one,
-                                          **_desc_kw(lo, hi, b.max_seq_len, inv_n, lw, gw))
+                                          **_desc_kw(lo, hi, b.max_seq_len, inv_n, lw, gw, own))
     torch.cuda.synchronize()
-    pc, tc = oracle.bias_pair_counts(b.seq_offsets, b.timestamps, b.num_targets, lo, hi, nb, lw, gw)
-    unit = H * d * 0.5 * inv_n
+    pc, tc = oracle.bias_pair_counts(b.seq_offsets, b.timestamps, b.num_targets, lo, hi, nb, lw, gw,
+                                     cand_own_index=own)
+    # each head's pairs land in its own row with per-head tables, in the one row otherwise
+    unit = (1 if ph else H) * d * 0.5 * inv_n
     assert pc.sum() * H < 2**24  # every partial sum exact in fp32
-    got_p = drp.cpu().double().numpy()
-    got_t = drt.cpu().double().numpy()
+    if ph:
+        pc, tc = np.tile(pc, (H, 1)), np.tile(tc, (H, 1))
+    got_p = drp.cpu().double().numpy().reshape(pc.shape)
+    got_t = drt.cpu().double().numpy().reshape(tc.shape)
+    assert tuple(drp.shape) == tuple(zp.shape) and tuple(drt.shape) == tuple(zt.shape)
+    got_p, got_t, pc, tc = got_p.reshape(-1), got_t.reshape(-1), pc.reshape(-1), tc.reshape(-1)
     bad_p = np.flatnonzero(got_p != pc * unit)
     bad_t = np.flatnonzero(got_t != tc * unit)
-    assert bad_p.size == 0, f"rab_pos entries {bad_p[:10] + lo} (distance): gpu {got_p[bad_p[:10]] / unit} " \
-                            f"pairs vs {pc[bad_p[:10]]}"
+    npos = hi - lo + 1
+    assert bad_p.size == 0, f"rab_pos entries {bad_p[:10] % npos + lo} (distance; head {bad_p[:10] // npos}): " \
+                            f"gpu {got_p[bad_p[:10]] / unit} pairs vs {pc[bad_p[:10]]}"
     assert bad_t.size == 0, f"rab_time buckets {bad_t[:10]}: gpu {got_t[bad_t[:10]] / unit} pairs vs {tc[bad_t[:10]]}"
 
 

@@ -190,7 +190,7 @@ def test_fp8_score_attention_rejections(cuda_device):
                           fp8_qk=True, **kw)
     # the backward rejects the option
     desc = ops._attn_desc_from(d["q"], d["v"], d["seq_offsets"], inp.max_seq_len, inp.inv_n, inp.pos_lo,
-                               inp.pos_hi, d["rab_time"], fp8_qk=True)
+                               inp.pos_hi, d["rab_pos"], d["rab_time"], fp8_qk=True)
     n = ctypes.c_size_t(0)
     assert ops.load_library().hstu_attn_workspace_size(ctypes.byref(desc), 1, ctypes.byref(n)) == 0
     ws = ops.alloc_workspace(n.value, dev)
