@@ -4,6 +4,7 @@ Each rank takes its LPT shard of a small jagged batch, runs the oracle
 backward on it, and sums the bias-table gradients with the same all-reduce
 the GPU step uses; the result must equal the oracle on the whole batch."""
 
+import dataclasses
 import os
 import socket
 
@@ -21,14 +22,18 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _batch():
+def _batch(per_head=False):
     rng = np.random.default_rng(31)
-    return workloads.make_attn_inputs(rng, [9, 3, 14, 1, 7, 0, 12], 2, 4, 4, 30.0, -6, 6, 5, 16,
-                                      torch.float32, num_targets=[2, 0, 3, 0, 0, 0, 1],
-                                      with_dout=True)
+    inp = workloads.make_attn_inputs(rng, [9, 3, 14, 1, 7, 0, 12], 2, 4, 4, 30.0, -6, 6, 5, 16,
+                                     torch.float32, num_targets=[2, 0, 3, 0, 0, 0, 1],
+                                     with_dout=True)
+    if per_head:  # one table pair per head: the all-reduce keeps the [H, entries] shapes
+        inp = dataclasses.replace(inp, rab_pos=torch.stack([inp.rab_pos, 0.5 - inp.rab_pos]),
+                                  rab_time=torch.stack([inp.rab_time, 2.0 * inp.rab_time]))
+    return inp
 
 
-def _worker(rank, world, port, out_dir):
+def _worker(rank, world, port, out_dir, per_head=False, own=False):
     import torch.distributed as dist
 
     import oracle
@@ -36,19 +41,18 @@ def _worker(rank, world, port, out_dir):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        inp = _batch()
+        inp = _batch(per_head)
         costs = parallel.sequence_costs(inp.lengths, inp.num_targets.numpy())
         mine = parallel.lpt_partition(costs, world)[rank]
         sh = parallel.shard_attn_inputs(inp, mine)
         if sh.total_tokens:
             dq, dk, dv, drp, drt = oracle.attn_bwd(sh.seq_offsets, sh.timestamps, sh.num_targets, sh.q,
                                                    sh.k, sh.v, sh.rab_pos, sh.rab_time, sh.pos_lo,
-                                                   sh.pos_hi, sh.inv_n, sh.dout, threads=1)
+                                                   sh.pos_hi, sh.inv_n, sh.dout, threads=1, cand_own_index=own)
         else:
             dq = dk = dv = np.zeros((0,))
-            drp, drt = np.zeros(inp.rab_pos.numel()), np.zeros(inp.rab_time.numel())
-        buf = torch.from_numpy(np.concatenate([drp, drt]))
-        gp, gt = buf[:drp.size], buf[drp.size:]
+            drp, drt = np.zeros(tuple(inp.rab_pos.shape)), np.zeros(tuple(inp.rab_time.shape))
+        gp, gt = torch.from_numpy(drp.copy()), torch.from_numpy(drt.copy())
         parallel.allreduce_bias_grads(gp, gt)
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), seqs=np.array(mine), dq=dq, dk=dk, dv=dv,
                  drp=gp.numpy(), drt=gt.numpy())
@@ -71,17 +75,18 @@ def test_sequence_costs_are_visible_pairs():
     assert list(parallel.sequence_costs([4, 5], [0, 2])) == [10, 6 + 2 * 4]
 
 
-def test_dp_shards_reproduce_full_batch_gradients(tmp_path):
+@pytest.mark.parametrize("per_head,own", [(False, False), (True, True)])
+def test_dp_shards_reproduce_full_batch_gradients(tmp_path, per_head, own):
     import oracle
     oracle.build()
     world = 2
     port = _free_port()
-    mp.start_processes(_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+    mp.start_processes(_worker, args=(world, port, str(tmp_path), per_head, own), nprocs=world, join=True,
                        start_method="spawn")
-    inp = _batch()
+    inp = _batch(per_head)
     full = oracle.attn_bwd(inp.seq_offsets, inp.timestamps, inp.num_targets, inp.q, inp.k, inp.v,
                            inp.rab_pos, inp.rab_time, inp.pos_lo, inp.pos_hi, inp.inv_n, inp.dout,
-                           threads=1)
+                           threads=1, cand_own_index=own)
     off = inp.seq_offsets.numpy()
     covered = []
     for rank in range(world):
