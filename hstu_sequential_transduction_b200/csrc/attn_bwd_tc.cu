@@ -135,7 +135,10 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
     o.b1 = MODE == BK_ONE ? o.b0 : exp_offset(ti[l], tjf);
     const float E0 = MODE == BK_ONE ? 0.f : *reinterpret_cast<const float *>(Eb + o.b0);
     const float E1 = MODE == BK_ONE ? 0.f : *reinterpret_cast<const float *>(Eb + o.b1);
-    const float thr = __uint_as_float(o.b1 << 21);  // 2^(bucket of b1), exact
+    // BK_TWO: a column is in bucket b1 when RZ(ti - tj) >= 2^(bucket of b1); the
+    // stamps are integers and the threshold a power of two, so that is ti >= tj + 2^k
+    // in exact arithmetic, i.e. ti >= RU(tj + 2^k): one compare per column
+    const float lim = __fadd_ru(tjf, __uint_as_float(o.b1 << 21));
     o.mid = false;
     float upf[NC];  // 1 where the column is in bucket b1
 #pragma unroll
@@ -156,7 +159,7 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
                 bt = 0.f;  // the block's one time bias is folded into bp by the caller
                 upf[c] = 0.f;
             } else if (MODE == BK_TWO) {
-                const bool up = __fsub_rz(tv[e], tjf) >= thr;
+                const bool up = tv[e] >= lim;
                 upf[c] = up ? 1.f : 0.f;
                 bt = up ? E1 : E0;
             } else {
@@ -183,8 +186,9 @@ __device__ __forceinline__ RowOut bwd_row(float *sv, float *dv, const float *ti,
             const int cc = c + e;
             const float hh = sv[cc], t = th[cc];
             float pval = fmaf(hh, t, hh);
-            const float a = 1.f + t;
-            float ds = dv[cc] * fmaf(a, fmaf(-hh, t, hh), a);
+            // (1 + t)(1 + h (1 - t)) = 1 + t + h (1 - t^2)
+            const float y = fmaf(hh, fmaf(-t, t, 1.f), t);
+            float ds = fmaf(dv[cc], y, dv[cc]);
             if (MASK) {
                 const bool vis = cc >= c_lo && cc < c_hi;
                 pval = vis ? pval : 0.f;

@@ -95,16 +95,16 @@ __device__ __forceinline__ float time_bias_fast(float ti1, float tj, const float
 
 // P for the 64 key columns one thread owns (one query row), packed to bf16.
 // wr[-c]: positional bias / 2 of column c; tj[c]: rebased key stamp.
-// MASK: only columns c_lo <= c < c_lim are visible.  TWO: the row's columns fall in
-// at most two time buckets (hi for columns whose difference reaches `thr`).
+// MASK: only columns c_lo <= c < c_lim are visible.
 // MODE: 0 time bucket looked up per column, 1 one bucket for the whole row
-// (e_hi), 2 two buckets split at thr.  CONSTB: the positional index is clamped
+// (e_hi), 2 two buckets: e_hi for the columns whose key stamp is at most klim
+// (those whose difference reaches the upper bucket), e_lo for the others.  CONSTB: the positional index is clamped
 // for every column, so the positional bias is wr[0].
 // F8: the raw score is dec(q) . dec(k) without the row scales; column c's half
 // scale is ks[c] and the row's scale rsq, so h = s rsq ks[c] + bias / 2.
 template <bool MASK, int MODE, bool CONSTB, bool F8 = false>
 __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float *tj, float ti1,
-                                        const float *E, float e_hi, float e_lo, float thr, int c_lo, int c_lim,
+                                        const float *E, float e_hi, float e_lo, float klim, int c_lo, int c_lim,
                                         uint32_t *pk, const float *ks = nullptr, float rsq = 0.f)
 {
     const float bconst = CONSTB ? wr[0] + (MODE == 1 ? e_hi : 0.f) : 0.f;
@@ -141,7 +141,7 @@ __device__ __forceinline__ void fwd_row(float *sv, const float *wr, const float 
                 if (MODE == 1)
                     bt = e_hi;
                 else if (MODE == 2)
-                    bt = __fsub_rz(ti1, tv[e]) >= thr ? e_hi : e_lo;
+                    bt = tv[e] <= klim ? e_hi : e_lo;
                 else
                     bt = time_bias_fast(ti1, tv[e], E);
                 sv[cc] = fmaf(sv[cc], sc, CONSTB ? wr[0] : wr[-cc]) + bt;
@@ -583,7 +583,11 @@ attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tq,
                     const int dnear = pi - (j0 + 64 * g + 63), dfar = pi - (j0 + 64 * g);
                     const bool cst = __all_sync(0xffffffffu, !row_ok || dnear >= p.pos_hi || dfar <= p.pos_lo);
                     const float e_hi = time_bias_fast(ti1f, tj[0], E), e_lo = time_bias_fast(ti1f, tj[63], E);
-                    const float thr = __uint_as_float(bh << 23);
+                    // two buckets: a column is in the upper one when RZ(ti - tj) >= 2^k
+                    // (k = the bucket of the first column); stamps are integers and
+                    // 2^k a power of two, so that is tj <= ti - 2^k exactly, i.e.
+                    // tj <= RD(ti - 2^k): one compare per column
+                    const float thr = __fsub_rd(ti1f, __uint_as_float(bh << 23));
                     if (one) {
                         if (cst)
                             fwd_row<false, 1, true, F8>(sv, wr, tj, ti1f, E, e_hi, e_lo, thr, 0, 64, pk, KSw, rsq);

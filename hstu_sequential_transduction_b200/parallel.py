@@ -47,6 +47,27 @@ def lpt_partition(costs: Sequence[int], world: int) -> List[List[int]]:
     return [sorted(b) for b in bins]
 
 
+def dp_shard_inputs(w, world: int, rank: int):
+    """This rank's share of a global batch of `world` x `w.num_seqs` sequences of
+    workload `w` (a `workloads.Workload` without layers), for weak scaling: the
+    global lengths come from the workload's seed, `lpt_partition` assigns whole
+    sequences to ranks by cost, and the rank draws its own sequences' values from
+    its own seed.  The bias tables, parameters shared by every rank, come from
+    one seed, so all ranks hold the same tables."""
+    from . import workloads
+    gw = dataclasses.replace(w, num_seqs=w.num_seqs * world)
+    lengths = workloads.draw_lengths(gw, np.random.default_rng(w.seed))
+    mine = lengths[lpt_partition(sequence_costs(lengths), world)[rank]]
+    dt = workloads.torch_dtype(w)
+    inp = workloads.make_attn_inputs(np.random.default_rng(w.seed + 1 + rank), mine, w.num_heads, w.d_qk, w.d_v,
+                                     w.gap_mean_s, w.pos_lo, w.pos_hi, w.num_time_buckets, w.n_scale, dt,
+                                     value_std=w.value_std, table_std=w.table_std, with_dout=w.has_bwd)
+    tables = workloads.make_attn_inputs(np.random.default_rng(w.seed), [1], w.num_heads, w.d_qk, w.d_v,
+                                        w.gap_mean_s, w.pos_lo, w.pos_hi, w.num_time_buckets, w.n_scale, dt,
+                                        table_std=w.table_std, with_values=False)
+    return dataclasses.replace(inp, rab_pos=tables.rab_pos, rab_time=tables.rab_time)
+
+
 def shard_attn_inputs(inp, seqs: Sequence[int]):
     """The sequences `seqs` of a `workloads.AttnInputs` as a new jagged batch."""
     off = inp.seq_offsets.numpy()

@@ -300,6 +300,29 @@ def test_bwd_long_history_full_size_sampled(cuda_device):
     assert abs(tp - tt) <= 1e-3 * max(abs(tp), float(drp.abs().sum())), (tp, tt)
 
 
+def test_bwd_long_history_full_size_tables_element_wise(cuda_device):
+    """The full-size long-history backward (the bench's launch) with dout zero outside
+    one sequence: every pair's score gradient is linear in dout_i, so the bias-table
+    gradients hold that sequence's pairs alone and are compared element-wise with
+    the oracle run on that sequence; every gradient row of the other sequences
+    must be exactly zero."""
+    w = workloads.WORKLOADS["long_history_bf16"]
+    inp = workloads.generate(w)
+    off = inp.seq_offsets.numpy()
+    s = int(np.argmin(np.diff(off)))
+    a, b = int(off[s]), int(off[s + 1])
+    dout = torch.zeros_like(inp.dout)
+    dout[a:b] = inp.dout[a:b]
+    inp = dataclasses.replace(inp, dout=dout)
+    dq, dk, dv, drp, drt = gpu_bwd(inp, cuda_device)
+    ref = _oracle_bwd(sub_batch(inp, [s]))
+    assert_bf16_close(drp, ref[3], what="full-size d_rab_pos")
+    assert_bf16_close(drt, ref[4], what="full-size d_rab_time")
+    for name, g, r in (("dq", dq, ref[0]), ("dk", dk, ref[1]), ("dv", dv, ref[2])):
+        assert_bf16_close(g[a:b], r, what=f"full-size {name} of the sequence")
+        assert not bool(g[:a].any()) and not bool(g[b:].any()), f"{name} outside the sequence"
+
+
 def test_bwd_long_history_bias_grads_one_sequence(cuda_device):
     # full bias-table gradients of one long sequence (clamps at +-4096)
     w = workloads.WORKLOADS["long_history_bf16"]

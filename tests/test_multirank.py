@@ -71,6 +71,22 @@ def test_lpt_partition_balances_and_is_deterministic():
     assert parallel.lpt_partition([], 3) == [[], [], []]
 
 
+def test_dp_shards_of_a_global_batch():
+    # the multi-GPU bench's inputs: every global sequence on exactly one rank,
+    # ranks balanced by visible pairs, one set of bias tables for all
+    w = workloads.WORKLOADS["attn_bf16_short"]
+    world = 4
+    gw = dataclasses.replace(w, num_seqs=w.num_seqs * world)
+    glob = workloads.draw_lengths(gw, np.random.default_rng(w.seed))
+    shards = [parallel.dp_shard_inputs(w, world, r) for r in range(world)]
+    assert sorted(sum((list(s.lengths) for s in shards), [])) == sorted(glob.tolist())
+    loads = [int(parallel.sequence_costs(s.lengths).sum()) for s in shards]
+    assert max(loads) - min(loads) <= int(parallel.sequence_costs(glob).max())
+    for s in shards:
+        assert torch.equal(s.rab_pos, shards[0].rab_pos) and torch.equal(s.rab_time, shards[0].rab_time)
+        assert s.inv_n == shards[0].inv_n and s.q.shape[0] == s.total_tokens
+
+
 def test_sequence_costs_are_visible_pairs():
     assert list(parallel.sequence_costs([4, 5], [0, 2])) == [10, 6 + 2 * 4]
 
