@@ -690,8 +690,7 @@ attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                             const float hh = 0.5f * (sv[c + e] + p.rab_pos[hp + idx] + p.rab_time[ht + b]);
                             const float t = tanh_approx(hh);
                             pv[e] = fmaf(hh, t, hh);
-                            const float a = 1.f + t;
-                            const float ds = dv[c + e] * fmaf(a, fmaf(-hh, t, hh), a);
+                            const float ds = fmaf(dv[c + e], fmaf(hh, fmaf(-t, t, 1.f), t), dv[c + e]);
                             dsv[e] = ds;
                             red_add_global(p.d_rab_pos + hp + idx, ds * gscale);
                             red_add_global(p.d_rab_time + ht + b, ds * gscale);
