@@ -250,6 +250,28 @@ def layer_stack_timing(dev, stream, reps: int = 3):
     e1.record(stream)
     torch.cuda.synchronize()
     bwd_ms = e0.elapsed_time(e1) / reps
+
+    # the attention forward alone on the first layer's own Q, K, V (the column
+    # blocks of SiLU(X W1 + b1), copied out contiguous): warm, CUDA events
+    hv_, hq_ = w.num_heads * w.d_v, w.num_heads * w.d_qk
+    qa = uvqk[:, 2 * hv_:2 * hv_ + hq_].contiguous().view(T, w.num_heads, w.d_qk)
+    ka = uvqk[:, 2 * hv_ + hq_:2 * hv_ + 2 * hq_].contiguous().view(T, w.num_heads, w.d_qk)
+    va = uvqk[:, hv_:2 * hv_].contiguous().view(T, w.num_heads, w.d_v)
+    oa = torch.empty_like(va)
+    ws_a = ops.alloc_workspace(ops.hstu_attn_workspace_size(attn0, False), dev)
+
+    def attn_only():
+        ops.hstu_attn_fwd(qa, ka, va, off, ts, None, rp, rt, out=oa, workspace=ws_a, stream=stream,
+                          max_seq_len=a.max_seq_len, inv_n=a.inv_n, pos_lo=a.pos_lo, pos_hi=a.pos_hi)
+
+    attn_only()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        attn_only()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    attn_ms = e0.elapsed_time(e1) / reps
     # the first layer again with the output projection over [U | O | G] (3 H d_v wide)
     hv = w.num_heads * w.d_v
     gen_w = torch.Generator(device="cpu").manual_seed(2025)
@@ -332,6 +354,8 @@ def layer_stack_timing(dev, stream, reps: int = 3):
             "ms_per_forward": ms, "tflops": total / (ms * 1e-3) / 1e12,
             "gflop_per_layer": {"attention": attn_fl / 1e9, "f1_f2": gemm_fl / 1e9},
             "gate_bytes_per_layer": flops.gate_bytes(T, w.num_heads, w.d_v),
+            "attn_fwd": {"what": "the attention forward alone on the first layer's Q, K, V",
+                         "ms": attn_ms, "tflops": attn_fl / (attn_ms * 1e-3) / 1e12},
             "layer_bwd": {"ms": bwd_ms, "gflop": bwd_fl / 1e9, "tflops": bwd_fl / (bwd_ms * 1e-3) / 1e12},
             "fp8_projections": {
                 "what": "the stack forward with E4M3 f1 and f2 (per-row activation, per-column weight scales)",
@@ -842,6 +866,7 @@ def run_ours(args):
             "e2e": e2e,
         }
         if layer is not None:
+            layer["attn_fwd"]["pct_of_bf16_peak"] = 100 * layer["attn_fwd"]["tflops"] / burst
             line["layer_stack"] = layer
         if semi is not None:
             line["semi_local"] = semi
