@@ -186,6 +186,33 @@ def test_fwd_all_empty(cuda_device):
     assert out.shape[0] == 0
 
 
+def test_fwd_bwd_no_sequences(cuda_device):
+    # B = 0, T = 0: every call is legal, launches nothing that touches rows, and
+    # still zeroes the bias-table gradients
+    dev = cuda_device
+    z = torch.zeros((0, 2, 64), dtype=torch.bfloat16, device=dev)
+    off = torch.zeros(1, dtype=torch.int64, device=dev)
+    ts = torch.zeros(0, dtype=torch.int64, device=dev)
+    rp = torch.randn(17, device=dev)
+    rt = torch.randn(8, device=dev)
+    kw = dict(max_seq_len=0, inv_n=1.0, pos_lo=-8, pos_hi=8)
+    out = ops.hstu_attn_fwd(z, z, z, off, ts, None, rp, rt, **kw)
+    grads = (torch.empty_like(z), torch.empty_like(z), torch.empty_like(z),
+             torch.full_like(rp, 7.0), torch.full_like(rt, 7.0))
+    g = ops.hstu_attn_bwd(z, z, z, off, ts, None, rp, rt, z, grads=grads, **kw)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 2, 64)
+    assert not bool(g[3].any()) and not bool(g[4].any())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_bwd_eight_heads(cuda_device, d):
+    # more heads than the workloads use: the head index walks every per-head offset
+    inp = _small([1, 130, 64, 257], H=8, d=d, nt=[0, 9, 0, 0], seed=70 + d)
+    assert_bf16_close(gpu_fwd(inp, cuda_device), _oracle_fwd(inp), what=f"fwd H=8 d={d}")
+    _check_bwd(gpu_bwd(inp, cuda_device), _oracle_bwd(inp), assert_bf16_close, f"bwd H=8 d={d}")
+
+
 def test_fwd_attn_bf16_short_full(cuda_device):
     w = workloads.WORKLOADS["attn_bf16_short"]
     inp = workloads.generate(w)
