@@ -13,7 +13,7 @@ namespace hstu {
 
 namespace {
 
-constexpr int TR = kMmaTile;  // rows per tile (query and key)
+constexpr int TR = kF32Tile;  // rows per tile (query and key)
 
 struct SeqV {
     int64_t s0;

@@ -45,7 +45,7 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
         return HSTU_ERR_INVALID_ARG;
     if (d->per_head_tables && ((int64_t)d->pos_hi - d->pos_lo + 1) * d->num_heads > INT_MAX)
         return HSTU_ERR_UNSUPPORTED;
-    if (max_items(d->total_tokens, d->num_seqs, kMmaTile) > INT_MAX / 4 ||
+    if (max_items(d->total_tokens, d->num_seqs, kF32Tile) > INT_MAX / 4 ||
         d->total_tokens * d->num_heads > ((int64_t)1 << 40))
         return HSTU_ERR_UNSUPPORTED;
     return HSTU_OK;
@@ -55,7 +55,7 @@ size_t elem_bytes(const hstu_attn_desc *d) { return d->dtype == HSTU_BF16 ? 2 : 
 
 size_t items_bytes(const hstu_attn_desc *d)
 {
-    return align256(sizeof(int2) * (size_t)max_items(d->total_tokens, d->num_seqs, kMmaTile));
+    return align256(sizeof(int2) * (size_t)max_items(d->total_tokens, d->num_seqs, kF32Tile));
 }
 
 size_t attn_ws(const hstu_attn_desc *d, int is_bwd)
@@ -138,14 +138,14 @@ hstu_status zero_table_grads(const hstu_attn_desc *d, float *d_rab_pos, float *d
     return cuda_status(cudaMemsetAsync(d_rab_time, 0, sizeof(float) * rows * d->num_time_buckets, st));
 }
 
-int grid_items(const hstu_attn_desc *d, int tile = kMmaTile)
+int grid_items(const hstu_attn_desc *d, int tile = kF32Tile)
 {
     return (int)max_items(d->total_tokens, d->num_seqs, tile);
 }
 
 // The work list always has room for the 64-row bound, the largest of all tilings.
 hstu_status schedule(const hstu_attn_desc *d, const int64_t *off, const int32_t *nt, int is_bwd,
-                     void *ws, cudaStream_t stream, int tile = kMmaTile)
+                     void *ws, cudaStream_t stream, int tile = kF32Tile)
 {
     int2 *items = reinterpret_cast<int2 *>(static_cast<char *>(ws) + sizeof(WsHeader));
     return cuda_status(launch_schedule(off, nt, d->num_seqs, d->total_tokens, d->max_seq_len,

@@ -17,8 +17,10 @@ struct DeviceInfo {
 };
 DeviceInfo device_info();
 
-// Tile rows of the work items each attention implementation consumes.
-constexpr int kMmaTile = 64;
+// Tile rows of the work items each attention implementation consumes: 64 for
+// the fp32 kernels (the work list is always sized for this, the finer tiling),
+// 128 for the tcgen05 kernels.
+constexpr int kF32Tile = 64;
 constexpr int kTcTile = 128;
 
 cudaError_t launch_schedule(const int64_t *off, const int32_t *nt, int B, int64_t T, int max_len,
