@@ -48,7 +48,7 @@ SEMI_LOCAL = (1024, 256)
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:attn_bwd -c 1
 #       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-layer-stack
 # valid only for the kernel source it was taken on (else the line reports null)
-BWD_TRAFFIC = {"source_sha256": "209cb182945f4f00441e8d0b21a50de88cd973721c6e505954fec9fcd1dc9971",
+BWD_TRAFFIC = {"source_sha256": "73a20430600d938de794a814b070c61d59221bfcc1f41cf865348a33abca1a54",
                "bytes": 630.22e6 + 364.91e6}
 
 

@@ -1,10 +1,11 @@
-// HSTU jagged attention backward on sm_100a: TMA + tcgen05 (TMEM), head dim 128.
+// HSTU jagged attention backward on sm_100a: TMA + tcgen05 (TMEM), head dims 64
+// and 128.
 //
 // Exact derivatives of the forward (the DLRMv4 page, text under Table 7: the
 // backward produces dQ, dK and dV through about five GEMMs), plus the
-// gradients of the shared relative-bias tables.  Per work item (sequence,
-// 128-row key tile, head) the CTA keeps K and V resident and walks the query
-// rows that see the tile in steps of 64:
+// gradients of the relative-bias tables.  Per work item (sequence, 128-row key
+// tile, head) the CTA keeps K and V resident and walks the query rows that see
+// the tile in steps of 64:
 //   S^T  = K Q^T,  dP^T = V dO^T               (TMEM, 64 columns each)
 //   P = SiLU(s), dS' = dP * 2 SiLU'(s)          (epilogue, s = score + bias)
 //   dV += P^T dO,  dK += dS'^T Q                (TMEM accumulators, 128 cols each)
@@ -12,21 +13,23 @@
 //        TMA bulk reduce-add into an fp32 dQ accumulator in global memory
 // The constant factors (inv_n for P, inv_n / 2 for dS) are applied once at
 // the end.  With h = s / 2 and t = tanh(h):
-//   SiLU(s) = h (1 + t),  SiLU'(s) = (1 + t)(1 + h (1 - t)) / 2.
+//   SiLU(s) = h (1 + t),  2 SiLU'(s) = (1 + t)(1 + h (1 - t)) = 1 + t + h (1 - t^2).
 // Bias-table gradients without per-pair atomics: the positional index of a
 // pair is query - key, constant along diagonals, so each warp reduces its
 // 32 x 32 block of dS' along the 63 diagonals with one shuffle per column and
-// stores them to per-warp slots that are summed and flushed per step (one
-// global reduction per touched index); a step on one clamped index is a plain
-// sum.  Time buckets are monotone along a key row of sorted stamps: each step
-// splits a row into at most two buckets (else a per-column fallback), and the
-// running bucket sum is carried across steps, so shared-memory atomics happen
-// only when a row changes bucket.  Candidate rows and stamps spanning more
-// than 2^24 s take a general per-pair path.
+// adds each diagonal sum to the table with one global reduction; the two
+// clamped entries, which most far blocks land on, are summed in registers per
+// thread and reduced once per warp and CTA.  Time buckets are monotone along a
+// key row of sorted stamps: lane k of a warp holds the warp's sum for bucket
+// k; blocks within two adjacent buckets add to per-thread carries, reduced
+// across the warp only when the bucket moves; other blocks write their rows'
+// bucket runs to a lane-private shared row that lane k sums by column.
+// Candidate rows, unsorted stamps and stamps spanning more than 2^24 s take an
+// exact per-pair path.
 //
 // Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
 // warps 2-9 epilogue (lane quarter = warp % 4 selects the TMEM rows, the two
-// warpgroups split each step's 64 query columns).
+// groups of four warps split each step's 64 query columns).
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,320), dP^T [320,384),
 // dQ^T [384,448), and the bf16 P^T [448,480) and dS'^T [480,512) of a step,
 // which the dV and dK MMAs read as their A operands straight from TMEM.

@@ -1,39 +1,46 @@
 // HSTU jagged attention forward on sm_100a: TMA + tcgen05 (TMEM) kernel.
 //
-// Computes, per (sequence, 128-row query tile, head) work item,
+// Computes, per (sequence, 128-row query tile, head) work unit,
 //   O = inv_n * sum_j SiLU(Q K_j^T + rab_pos + rab_time) V_j
-// Persistent: one CTA per SM walks a share of the work items, so the next
-// item's query and first key tiles load and its first S MMAs run while the
-// epilogue still writes out the previous item's O.
 // over the visible 128-row key tiles j (the pointwise attention of the
 // "HSTU Architecture" section; causal block with appended candidates of the
 // DLRMv4 page's "Model Architecture" section).  No score matrix reaches HBM.
+// Persistent: one CTA per SM walks a share of the units, so the next unit's
+// query and first key tiles load and its first S MMAs run while the epilogue
+// still writes out the previous unit's O.
 //
 // Warp roles (320 threads):
-//   warp 0     TMA producer: Q of each item into one of two buffers, then K_j
+//   warp 0     TMA producer: Q of each unit into one of two buffers, then K_j
 //              and V_j into two-stage rings (separate K and V rings, so K_{j+2}
 //              loads as soon as S_j is done);
 //   warp 1     owns TMEM (512 columns) and issues every tcgen05.mma from one
 //              thread: S_j = Q K_j^T into one of two S buffers, O += P_j V_j;
-//   warps 2-9  epilogue: two warpgroups, each takes 64 of the 128 key columns
-//              of every S tile: tcgen05.ld, relative bias, SiLU, bf16 pack, and
-//              tcgen05.st of P over the first 32 of its own S columns, where the
-//              P V MMA reads it as its A operand; at the end they read O from
-//              TMEM and write it out.
+//   warps 2-9  epilogue: two groups of four warps (one per TMEM lane quarter),
+//              each taking 64 of the 128 key columns of every S tile:
+//              tcgen05.ld, relative bias, SiLU, bf16 pack, and tcgen05.st of P
+//              over the first 32 of its own S columns, where the P V MMA reads
+//              it as its A operand; at the end of a unit they read O from TMEM
+//              and write it out.
 // TMEM columns: S buffers [0,128) and [128,256), O [256, 256 + D).  S_{j+2}
 // reuses buffer j % 2 once P_j V_j has completed.
 //
-// Epilogue arithmetic on full tiles (every pair visible, timestamps of the
-// tile within 2^24 s of the query tile's first stamp):
+// Epilogue arithmetic (stamps rebased to the query tile's first stamp, within
+// 2^24 s, and sorted within the warp's key columns):
 //   h = s/2 + rab_pos/2 + rab_time/2       (tables pre-halved, exact)
 //   SiLU(x) = x sigma(x) = h (1 + tanh h)  (one MUFU tanh per score)
-// The positional term reads a per-tile 256-entry window of the clamped table
-// (index p_i - p_j, contiguous per row).  The temporal bucket
-// floor(log2(1 + dt)) is the exponent of the fp32 difference (t_i + 1) - t_j
-// of rebased stamps, computed with round-toward-zero so the exponent is exact,
-// and a 512-entry table indexed by sign+exponent maps it to rab_time/2.
-// Diagonal, ragged and candidate tiles, and tiles whose stamps span more than
-// 2^24 s, take the general path (per-pair visibility, exact int64 bucket).
+// The positional term reads the warp's 96-entry window of the clamped table
+// (index p_i - p_j, contiguous along a row), or one constant when every
+// column of the block is past a clamp.  The temporal bucket
+// floor(log2(1 + dt)) is the exponent of the fp32 difference (t_i + 1) - t_j,
+// computed with round-toward-zero so the exponent is exact; a row whose
+// columns fall in one bucket adds that bucket's bias, a row spanning two picks
+// one of two by comparing the key stamp against a per-row limit, and any other
+// row maps the exponent through a 512-entry table to rab_time/2.  Diagonal and
+// ragged tiles without candidate rows keep this arithmetic under a per-column
+// mask; candidate rows (their own tile, and tiles mixing them with history
+// rows), unsorted stamps and stamps more than 2^24 s apart take out-of-line
+// exact per-pair paths (int64 bucket).  The candidate-position and per-head
+// table options compile into separate instantiations.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
