@@ -20,8 +20,8 @@
 // projection over [U | O | G]).  The E4M3 instantiation (F8) takes K-major A
 // and B codes in slices of 128 and kind::f8f6f4 MMAs of K = 32.
 // Epilogues (the chunk's bias, scales and dSiLU factors are fetched while its
-// TMEM load is in flight; bf16 outputs leave through a per-warp 32 x 32
-// swizzled box and a TMA store):
+// TMEM load is in flight; bf16 outputs leave through 32 x 32 swizzled boxes,
+// two per warp used in turn, and TMA stores):
 //   EPI_ACT    bf16 out = acc (x row scale x column scale for F8) + bias,
 //              optionally SiLU as h (1 + tanh h), h = x / 2 (forward projections);
 //   EPI_DSILU  bf16 out = aux * SiLU'(acc + bias) (the SiLU backward fused into

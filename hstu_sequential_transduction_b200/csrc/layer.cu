@@ -6,7 +6,8 @@
 //   f1:   [U | V | Q | K] = SiLU(X W1 + b1)   (bias + SiLU fused in the epilogue;
 //         the four blocks are column ranges of one output, so the attention
 //         reads Q, K, V in place through row strides: no split copies)
-//   gate: G = LayerNorm(O) * U                 (one warp per token, fp32 stats)
+//   gate: G = LayerNorm(O) * U                 (fp32 stats; each warp walks a strided
+//         set of tokens with the next tokens' O and U rows already in flight)
 //   f2:   Y = G W2 + b2
 #include <algorithm>
 
