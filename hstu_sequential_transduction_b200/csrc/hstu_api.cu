@@ -43,7 +43,9 @@ hstu_status check_attn_desc(const hstu_attn_desc *d)
     if ((d->cand_positions != 0 && d->cand_positions != 1) ||
         (d->per_head_tables != 0 && d->per_head_tables != 1))
         return HSTU_ERR_INVALID_ARG;
-    if (d->per_head_tables && ((int64_t)d->pos_hi - d->pos_lo + 1) * d->num_heads > INT_MAX)
+    // per-head tables are indexed with 32-bit offsets
+    if (d->per_head_tables && (((int64_t)d->pos_hi - d->pos_lo + 1) * d->num_heads > INT_MAX ||
+                               (int64_t)d->num_time_buckets * d->num_heads > INT_MAX))
         return HSTU_ERR_UNSUPPORTED;
     if (max_items(d->total_tokens, d->num_seqs, kF32Tile) > INT_MAX / 4 ||
         d->total_tokens * d->num_heads > ((int64_t)1 << 40))

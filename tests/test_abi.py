@@ -81,6 +81,7 @@ def _desc(**kw):
     # the two readings of the bias are switches; per-head tables must stay indexable
     (dict(cand_own_index=True, per_head_tables=True), 0),
     (dict(pos_lo=-(1 << 23), pos_hi=(1 << 23) - 1, num_heads=256, per_head_tables=True), 2),
+    (dict(num_time_buckets=1 << 24, num_heads=256, per_head_tables=True), 2),
 ])
 def test_bad_descriptors_rejected(kw, status):
     lib = ops.load_library()
